@@ -1,0 +1,346 @@
+#!/usr/bin/env python3
+"""Benchmark of the B200 routed-MoE layer: one JSON line on rank 0.
+
+A step is one pass of the whole layer (route -> bucket -> gate/up -> down ->
+combine) over one batch of synthetic tokens.  Default workload: the
+full-shape decode layer (d=2048, 512 experts, top-10 + 1 shared, f=768,
+2-bit), 4 tokens per step (one token plus three draft tokens verified
+together).  Inputs are larger than L2: the step rotates through R distinct
+layers (R * 756 MB of packed weights) with fresh activations, so the touched
+experts of a layer are evicted before it comes round again.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode|chain48|prefill|sweep|tiny]
+                  [--tokens T] [--bits B] [--impl ours|reference]
+
+Multi-GPU (torchrun): independent replicas, one per GPU (weak scaling); the
+time is the max over ranks of the device-timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "routed-MoE layer tokens/s (decode 1-4 tok, 8K prefill); % of HBM/TC roofline"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="decode", choices=["decode", "chain48", "prefill", "sweep", "tiny"])
+    p.add_argument("--tokens", type=int, default=None)
+    p.add_argument("--bits", type=int, default=2)
+    p.add_argument("--rotate", type=int, default=8, help="distinct layers cycled through (decode/sweep)")
+    p.add_argument("--flags", default="", help="extra forward flags: gemv|gemm")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU-baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------- workload description
+def workload(args):
+    from synth import WORKLOADS, MoeShape
+    wl = WORKLOADS[args.workload]
+    sh = wl.shape
+    if args.workload == "sweep":
+        sh = MoeShape(sh.d, sh.f, sh.E, sh.k, sh.n_shared, args.bits)
+    T = args.tokens or {"decode": 4, "chain48": 1, "prefill": 8192, "sweep": 4, "tiny": 8}[args.workload]
+    layers = 48 if args.workload == "chain48" else (1 if args.workload == "tiny" else max(1, args.rotate))
+    return wl, sh, T, layers
+
+
+def expert_bytes(sh):
+    n = sh.f * sh.d
+    return 3 * n * sh.bits // 8 + 3 * (n // 32) * 2
+
+
+def mat_bytes(sh):
+    n = sh.f * sh.d
+    return n * sh.bits // 8 + (n // 32) * 2
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        if not self.out:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), d.get("bf16_tflops_sustained", 1400.0), \
+            "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------- oracle CPU baseline
+def oracle_sample(sh, wl, T, seconds, steps=None, warmup=0, layer_of=lambda i: 0):
+    """Time the fp64 oracle on batches of T tokens of the workload; returns (tok/s, tokens, secs, threads)."""
+    import numpy as np
+
+    import oracle
+    import synth
+    threads = oracle.threads()
+    routers = {}
+    done_tok, spent, i = 0, 0.0, 0
+    while True:
+        if steps is not None and i >= steps + warmup:
+            break
+        if steps is None and spent >= seconds:
+            break
+        layer = layer_of(i)
+        if layer not in routers:
+            routers[layer] = synth.router_host(sh, wl.master, layer, wl.zipf)
+        wr, bias = routers[layer]
+        x = synth.x_host(sh, wl.master, 50000 + i, T)
+        ids, _ = oracle.route(sh, x, wr, bias)
+        need = sorted(set(ids.ravel().tolist()) | ({sh.E} if sh.n_shared else set()))
+        codes = [None] * sh.n_experts_total
+        scales = [None] * sh.n_experts_total
+        for e in need:
+            codes[e], scales[e] = synth.expert_host(sh, wl.master, layer, e)
+        t0 = time.perf_counter()
+        oracle.layer(sh, x, wr, bias, codes, scales)
+        dt = time.perf_counter() - t0
+        if i >= warmup:
+            spent += dt
+            done_tok += T
+        i += 1
+    return done_tok / spent, done_tok, spent, threads
+
+
+def reference_arm(args):
+    """The oracle as the reference arm: rank 0 alone, on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl, sh, T, layers = workload(args)
+    Tref = min(T, 16)  # oracle batches: each is a bounded sample of the workload
+    steps = max(1, args.steps if args.steps <= 20 else 20)
+    tps, ntok, secs, threads = oracle_sample(sh, wl, Tref, None, steps=steps, warmup=min(args.warmup, 1),
+                                             layer_of=lambda i: i % layers)
+    line = {"metric": METRIC, "value": tps, "unit": "tok/s", "n_gpus": 0, "steps": steps, "warmup": min(args.warmup, 1),
+            "ms_per_step": 1000.0 * secs / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.workload, "tokens_per_step": Tref, "bits": sh.bits, "d": sh.d, "f": sh.f,
+                       "experts": sh.E, "top_k": sh.k, "shared": sh.n_shared},
+            "cpu_baseline": {"value": tps, "unit": "tok/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{ntok} tokens in {steps} batches of {Tref} (fp64 C oracle)"},
+            "e2e": {"value": tps, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+def ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import bit_expert_ffn_gemv_b200 as moe
+    from bit_expert_ffn_gemv_b200 import build
+    from synth import gpu as sgpu
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    build.build()
+    wl, sh, T, layers = workload(args)
+    flags = {"": 0, "gemv": moe.MOE_FORCE_GEMV, "gemm": moe.MOE_FORCE_GEMM}[args.flags]
+
+    # ---- setup: layers generated on the device, one handle holding all of them
+    h = moe.MoeLayer(sh.d, sh.f, sh.E, sh.k, sh.n_shared, layers, sh.bits, T)
+    weights = []
+    for l in range(layers):
+        w = sgpu.layer_device(sh, wl.master + 1000 * rank, l, wl.zipf)
+        h.load_layer(l, *w)
+        weights.append(w)
+    n_x = 16
+    xs = [sgpu.x_device(sh, wl.master + 1000 * rank, 10000 + i, T) for i in range(n_x)]
+    chain = args.workload == "chain48"
+    resid = [torch.empty_like(xs[0]) for _ in range(2)]
+
+    def step(i, stream=None):
+        if chain:
+            # x_{l+1} = x_l + layer_l(x_l), in place in the residual buffer
+            r = resid[i & 1]
+            r.copy_(xs[i % n_x])
+            for l in range(layers):
+                h.forward(l, r, r, flags=flags | moe.MOE_ACCUMULATE, stream=stream)
+            return r
+        return h.forward(i % layers, xs[i % n_x], ys[i & 1], flags=flags, stream=stream)
+
+    ys = [torch.empty(T, sh.d, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    torch.cuda.synchronize()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    launches0 = h.stats()["launches"]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        ev0.record()
+        for i in range(args.steps):
+            step(args.warmup + i)
+        ev1.record()
+        torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    launches = h.stats()["launches"] - launches0
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    tok_per_step = T
+    value = tok_per_step * args.steps * world / (ms / 1000.0)
+
+    # ---- per-kernel device time (events on the library's launch stream), separate pass
+    h.profile(True)
+    alg_bytes = {"gemv_gateup": 0.0, "gemv_down": 0.0, "layer": 0.0}
+    nprof = min(args.steps, 64)
+    for i in range(nprof):
+        step(args.warmup + i)
+        st = h.stats()
+        D = st["active_experts"]
+        nl = layers if chain else 1
+        alg_bytes["gemv_gateup"] += nl * (D + sh.n_shared) * 2 * mat_bytes(sh)
+        alg_bytes["gemv_down"] += nl * (D + sh.n_shared) * mat_bytes(sh)
+        alg_bytes["layer"] += nl * (sh.E * sh.d * 2 + (D + sh.n_shared) * expert_bytes(sh) + 4 * T * sh.d)
+    prof = h.profile_read()
+    h.profile(False)
+    hbm, tc_burst, tc_sus, peak_kind = measured_peaks()
+    dom = max(prof.items(), key=lambda kv: kv[1][0])[0] if prof else None
+    roof = None
+    if dom in ("gemv_gateup", "gemv_down"):
+        dom_ms = prof[dom][0]
+        ach = alg_bytes[dom] / (dom_ms / 1000.0) / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                "traffic": None, "peak_kind": peak_kind,
+                "bytes_per_launch": alg_bytes[dom] / max(1, prof[dom][1]),
+                "avg_launch_us": 1000.0 * dom_ms / max(1, prof[dom][1])}
+    layer_time = sum(v[0] for v in prof.values())
+    layer_gbs = alg_bytes["layer"] / (layer_time / 1000.0) / 1e9 if layer_time else None
+
+    # ---- end to end through the host-buffer entry point (pinned memory)
+    e2e = None
+    if not args.no_e2e and not chain:
+        xh = [x.cpu().pin_memory() for x in xs]
+        yh = torch.empty(T, sh.d, dtype=torch.bfloat16).pin_memory()
+        for i in range(3):
+            h.forward_host(i % layers, xh[i % n_x], yh, flags=flags)
+        torch.cuda.synchronize()
+        k2 = min(args.steps, 100)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(k2):
+            h.forward_host(i % layers, xh[i % n_x], yh, flags=flags)
+        e1.record()
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": T * k2 * world / (ems / 1000.0), "unit": "tok/s", "h2d_bytes_per_step": T * sh.d * 2,
+               "d2h_bytes_per_step": T * sh.d * 2}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        Tc = min(T, 16)
+        tps, ntok, secs, threads = oracle_sample(sh, wl, Tc, args.cpu_seconds, layer_of=lambda i: 0)
+        cpu = {"value": tps, "unit": "tok/s", "cores": threads, "kind": "oracle",
+               "sample": f"{ntok} tokens in batches of {Tc}, {secs:.1f} s of fp64 C oracle work"}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": args.workload, "tokens_per_step": T, "d": sh.d, "f": sh.f, "experts": sh.E,
+                           "top_k": sh.k, "shared": sh.n_shared, "bits": sh.bits, "layers": layers,
+                           "l2": ("inputs larger than L2: 48 layers x 756 MB per step" if chain else
+                                  f"inputs larger than L2: {layers} distinct layers cycled, {n_x} fresh inputs"),
+                           "parallelism": f"replicas x{world}"},
+                "roofline": roof, "layer_hbm_gbs": layer_gbs,
+                "kernels_ms_per_step": {k: v[0] / nprof for k, v in prof.items()},
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    h.close()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,256 @@
+"""Thin Python binding of libmoe.so, the B200 routed-MoE layer (C ABI in include/moe.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the CUDA stream.  There is no
+CPU fallback: if the library is missing, importing the binding's functions
+raises.
+
+Module-level functions carry the C names (moe_layer_init, moe_load_layer,
+moe_route, moe_forward, moe_forward_host, moe_destroy, moe_debug_dequant,
+moe_check_status, moe_get_stats, moe_status_string); ``MoeLayer`` wraps a
+handle for torch tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = ["MoeError", "MoeConfig", "MoeLayerWeights", "MoeLayer", "lib", "library_path", "MOE_OUT_FP32",
+           "MOE_ACCUMULATE", "MOE_FORCE_GEMV", "MOE_FORCE_GEMM", "STATUS", "moe_layer_init", "moe_load_layer",
+           "moe_route", "moe_forward", "moe_forward_host", "moe_destroy", "moe_debug_dequant", "moe_check_status",
+           "moe_get_stats", "moe_status_string", "moe_profile", "moe_profile_read", "moe_kernel_name", "MoeStats"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libmoe.so")
+
+MOE_OUT_FP32 = 0x1
+MOE_ACCUMULATE = 0x2
+MOE_FORCE_GEMV = 0x4
+MOE_FORCE_GEMM = 0x8
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_CUDA", 3: "MOE_ERR_OOM", 4: "MOE_ERR_NOT_LOADED",
+          5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_BOUNDS"}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({_status_text(status)})")
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [("d", ctypes.c_int32), ("f", ctypes.c_int32), ("n_experts", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("n_layers", ctypes.c_int32),
+                ("bits", ctypes.c_int32), ("max_tokens", ctypes.c_int32)]
+
+
+class MoeStats(ctypes.Structure):
+    _fields_ = [("fixup_tokens", ctypes.c_int64), ("active_experts", ctypes.c_int64), ("max_group", ctypes.c_int64),
+                ("launches", ctypes.c_int64)]
+
+
+MOE_KERNEL_COUNT = 9
+
+
+class MoeLayerWeights(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("router_w", ctypes.c_void_p),
+                ("router_bias", ctypes.c_void_p)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so (built by bit_expert_ffn_gemv_b200.build); raise if it is absent."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(library_path):
+                raise ImportError(f"{library_path} is missing: build it with `python -m bit_expert_ffn_gemv_b200.build`"
+                                  " (there is no CPU fallback)")
+            L = ctypes.CDLL(library_path)
+            vp, i32, u32, st = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint32, ctypes.c_int
+            L.moe_layer_init.restype = st
+            L.moe_layer_init.argtypes = [ctypes.POINTER(MoeConfig), ctypes.POINTER(vp)]
+            L.moe_load_layer.restype = st
+            L.moe_load_layer.argtypes = [vp, i32, ctypes.POINTER(MoeLayerWeights)]
+            L.moe_route.restype = st
+            L.moe_route.argtypes = [vp, i32, vp, i32, vp, vp, vp]
+            L.moe_forward.restype = st
+            L.moe_forward.argtypes = [vp, i32, vp, i32, vp, u32, vp]
+            L.moe_forward_host.restype = st
+            L.moe_forward_host.argtypes = [vp, i32, vp, i32, vp, u32, vp]
+            L.moe_destroy.restype = st
+            L.moe_destroy.argtypes = [vp]
+            L.moe_debug_dequant.restype = st
+            L.moe_debug_dequant.argtypes = [vp, i32, i32, i32, vp, vp]
+            L.moe_check_status.restype = st
+            L.moe_check_status.argtypes = [vp]
+            L.moe_get_stats.restype = st
+            L.moe_get_stats.argtypes = [vp, ctypes.POINTER(MoeStats)]
+            L.moe_profile.restype = st
+            L.moe_profile.argtypes = [vp, i32]
+            L.moe_profile_read.restype = st
+            L.moe_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
+            L.moe_kernel_name.restype = ctypes.c_char_p
+            L.moe_kernel_name.argtypes = [i32]
+            L.moe_status_string.restype = ctypes.c_char_p
+            L.moe_status_string.argtypes = [st]
+            _lib = L
+    return _lib
+
+
+def _status_text(s: int) -> str:
+    try:
+        return lib().moe_status_string(s).decode()
+    except Exception:  # pragma: no cover - library not loadable
+        return "?"
+
+
+def _check(s: int, what: str):
+    if s != 0:
+        raise MoeError(s, what)
+
+
+# ---------------------------------------------------------------- C-named wrappers
+def moe_layer_init(cfg: MoeConfig) -> int:
+    h = ctypes.c_void_p()
+    _check(lib().moe_layer_init(ctypes.byref(cfg), ctypes.byref(h)), "moe_layer_init")
+    return h.value
+
+
+def moe_load_layer(handle: int, layer: int, w: MoeLayerWeights) -> None:
+    _check(lib().moe_load_layer(handle, layer, ctypes.byref(w)), "moe_load_layer")
+
+
+def moe_route(handle: int, layer: int, x_ptr: int, T: int, ids_ptr: int, w_ptr: int, stream: int) -> None:
+    _check(lib().moe_route(handle, layer, x_ptr, T, ids_ptr, w_ptr, stream), "moe_route")
+
+
+def moe_forward(handle: int, layer: int, x_ptr: int, T: int, y_ptr: int, flags: int, stream: int) -> None:
+    _check(lib().moe_forward(handle, layer, x_ptr, T, y_ptr, flags, stream), "moe_forward")
+
+
+def moe_forward_host(handle: int, layer: int, x_host: int, T: int, y_host: int, flags: int, stream: int) -> None:
+    _check(lib().moe_forward_host(handle, layer, x_host, T, y_host, flags, stream), "moe_forward_host")
+
+
+def moe_destroy(handle: int) -> None:
+    _check(lib().moe_destroy(handle), "moe_destroy")
+
+
+def moe_debug_dequant(handle: int, layer: int, expert: int, mat: int, out_ptr: int, stream: int) -> None:
+    _check(lib().moe_debug_dequant(handle, layer, expert, mat, out_ptr, stream), "moe_debug_dequant")
+
+
+def moe_check_status(handle: int) -> int:
+    return int(lib().moe_check_status(handle))
+
+
+def moe_get_stats(handle: int):
+    st = MoeStats()
+    _check(lib().moe_get_stats(handle, ctypes.byref(st)), "moe_get_stats")
+    return {f: int(getattr(st, f)) for f, _ in MoeStats._fields_}
+
+
+def moe_profile(handle: int, enable: bool) -> None:
+    _check(lib().moe_profile(handle, 1 if enable else 0), "moe_profile")
+
+
+def moe_profile_read(handle: int):
+    """{kernel name: (total ms, launches)} of kernels launched since moe_profile(h, True)."""
+    ms = (ctypes.c_double * MOE_KERNEL_COUNT)()
+    n = (ctypes.c_int64 * MOE_KERNEL_COUNT)()
+    _check(lib().moe_profile_read(handle, ms, n), "moe_profile_read")
+    return {moe_kernel_name(i): (ms[i], n[i]) for i in range(MOE_KERNEL_COUNT) if n[i]}
+
+
+def moe_kernel_name(i: int) -> str:
+    return lib().moe_kernel_name(i).decode()
+
+
+def moe_status_string(s: int) -> str:
+    return lib().moe_status_string(s).decode()
+
+
+# ---------------------------------------------------------------- torch convenience
+def _stream_ptr(stream) -> int:
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+class MoeLayer:
+    """A handle holding up to n_layers routed-MoE layers (weights borrowed from torch tensors)."""
+
+    def __init__(self, d, f, n_experts, top_k, n_shared=1, n_layers=1, bits=2, max_tokens=64):
+        self.cfg = MoeConfig(d, f, n_experts, top_k, n_shared, n_layers, bits, max_tokens)
+        self.handle = moe_layer_init(self.cfg)
+        self._keep = {}
+
+    def load_layer(self, layer, codes, scales, router_w, router_bias=None):
+        """codes (uint8), scales (fp16 bits as int16/uint16/float16), router_w (bf16 bits or bf16), bias fp32."""
+        for t in (codes, scales, router_w) + ((router_bias,) if router_bias is not None else ()):
+            if not t.is_cuda or not t.is_contiguous():
+                raise ValueError("weights must be contiguous CUDA tensors")
+        w = MoeLayerWeights(codes.data_ptr(), scales.data_ptr(), router_w.data_ptr(),
+                            router_bias.data_ptr() if router_bias is not None else None)
+        moe_load_layer(self.handle, layer, w)
+        self._keep[layer] = (codes, scales, router_w, router_bias)
+
+    def route(self, layer, x, ids=None, w=None, stream=None):
+        import torch
+        T = x.shape[0]
+        if ids is None:
+            ids = torch.empty((T, self.cfg.top_k), dtype=torch.int32, device=x.device)
+        if w is None:
+            w = torch.empty((T, self.cfg.top_k), dtype=torch.float32, device=x.device)
+        moe_route(self.handle, layer, x.data_ptr(), T, ids.data_ptr(), w.data_ptr(), _stream_ptr(stream))
+        return ids, w
+
+    def forward(self, layer, x, y=None, flags=0, stream=None):
+        import torch
+        T = x.shape[0]
+        if y is None:
+            dt = torch.float32 if flags & MOE_OUT_FP32 else torch.bfloat16
+            y = torch.empty((T, self.cfg.d), dtype=dt, device=x.device)
+        moe_forward(self.handle, layer, x.data_ptr(), T, y.data_ptr(), flags, _stream_ptr(stream))
+        return y
+
+    def forward_host(self, layer, x_host, y_host, flags=0, stream=None):
+        moe_forward_host(self.handle, layer, x_host.data_ptr(), x_host.shape[0], y_host.data_ptr(), flags,
+                         _stream_ptr(stream))
+        return y_host
+
+    def debug_dequant(self, layer, expert, mat, out=None, stream=None):
+        import torch
+        N, K = (self.cfg.f, self.cfg.d) if mat < 2 else (self.cfg.d, self.cfg.f)
+        if out is None:
+            out = torch.empty((N, K), dtype=torch.float32, device="cuda")
+        moe_debug_dequant(self.handle, layer, expert, mat, out.data_ptr(), _stream_ptr(stream))
+        return out
+
+    def check_status(self) -> int:
+        return moe_check_status(self.handle)
+
+    def stats(self):
+        return moe_get_stats(self.handle)
+
+    def profile(self, enable: bool):
+        moe_profile(self.handle, enable)
+
+    def profile_read(self):
+        return moe_profile_read(self.handle)
+
+    def close(self):
+        if self.handle:
+            moe_destroy(self.handle)
+            self.handle = None
+            self._keep = {}
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,408 @@
+// api.cu -- the C ABI (include/moe.h): handle, scratch, argument checks and the
+// order in which the kernels of one routed-MoE layer are enqueued.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "moe.h"
+
+static const char* const kKernelNames[MOE_KERNEL_COUNT] = {
+    "router_logits", "topk", "bucket", "gemv_gateup", "gemv_down", "combine", "gemm_gateup", "gemm_down",
+    "router_gemm"};
+
+struct moe_layer_state {
+    const uint8_t* codes = nullptr;
+    const uint16_t* scales = nullptr;
+    const void* router_w = nullptr;
+    const float* bias = nullptr;
+    float* wnorm = nullptr;  // owned
+    bool loaded = false;
+};
+
+struct moe_handle {
+    moe_config cfg{};
+    int device = 0;
+    std::vector<moe_layer_state> layers;
+    void* arena = nullptr;
+    size_t arena_bytes = 0;
+    // views into the arena
+    float* logits = nullptr;
+    int32_t* ids = nullptr;
+    float* w = nullptr;
+    int32_t* offsets = nullptr;
+    int32_t* pairs = nullptr;
+    int32_t* inv = nullptr;
+    int32_t* active = nullptr;
+    moe::Meta* meta = nullptr;
+    uint32_t* status = nullptr;
+    __half* h = nullptr;
+    float* obuf = nullptr;
+    void* x_stage = nullptr;
+    void* y_stage = nullptr;
+    // launch accounting and optional per-kernel event timing
+    int64_t launches = 0;
+    bool prof_on = false;
+    std::vector<cudaEvent_t> ev;    // pairs (start, stop)
+    std::vector<int> ev_kernel;     // kernel id of each recorded pair
+    double prof_ms[MOE_KERNEL_COUNT] = {};
+    int64_t prof_n[MOE_KERNEL_COUNT] = {};
+};
+
+namespace {
+
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+// Enqueue one kernel (via `f`), counting it and, when profiling is on,
+// bracketing it with a pair of events on the same stream.
+template <class F>
+cudaError_t run(moe_handle* h, int kernel, cudaStream_t s, F&& f) {
+    h->launches++;
+    if (!h->prof_on) return f();
+    const size_t i = 2 * h->ev_kernel.size();
+    while (h->ev.size() < i + 2) {
+        cudaEvent_t e;
+        if (cudaEventCreate(&e) != cudaSuccess) return cudaErrorMemoryAllocation;
+        h->ev.push_back(e);
+    }
+    cudaError_t e = cudaEventRecord(h->ev[i], s);
+    if (e != cudaSuccess) return e;
+    e = f();
+    if (e != cudaSuccess) return e;
+    e = cudaEventRecord(h->ev[i + 1], s);
+    h->ev_kernel.push_back(kernel);
+    return e;
+}
+
+moe_status check_layer(moe_handle* h, int32_t layer) {
+    if (!h || layer < 0 || layer >= h->cfg.n_layers) return MOE_ERR_INVALID_ARG;
+    if (!h->layers[layer].loaded) return MOE_ERR_NOT_LOADED;
+    return MOE_OK;
+}
+
+// router -> certified top-k; writes ids / w (device)
+moe_status do_route(moe_handle* h, int32_t layer, const void* x, int32_t T, int32_t* ids, float* w,
+                    cudaStream_t s) {
+    const moe_layer_state& L = h->layers[layer];
+    cudaError_t e = cudaMemsetAsync(h->meta, 0, sizeof(moe::Meta), s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    moe::RouteArgs ra;
+    ra.x = x;
+    ra.T = T;
+    ra.d = h->cfg.d;
+    ra.E = h->cfg.n_experts;
+    ra.k = h->cfg.top_k;
+    ra.wr = L.router_w;
+    ra.bias = L.bias;
+    ra.wnorm = L.wnorm;
+    ra.logits = h->logits;
+    ra.ids = ids;
+    ra.w = w;
+    ra.meta = h->meta;
+    e = run(h, MOE_K_ROUTER_LOGITS, s, [&] { return moe::launch_router_logits(ra, s); });
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    return cuda_status(run(h, MOE_K_TOPK, s, [&] { return moe::launch_topk(ra, s); }));
+}
+
+moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, void* y, uint32_t flags,
+                      cudaStream_t s) {
+    const moe_config& c = h->cfg;
+    moe_status st = do_route(h, layer, x, T, h->ids, h->w, s);
+    if (st != MOE_OK) return st;
+    moe::BucketArgs ba;
+    ba.ids = h->ids;
+    ba.T = T;
+    ba.k = c.top_k;
+    ba.E = c.n_experts;
+    ba.offsets = h->offsets;
+    ba.pairs = h->pairs;
+    ba.inv = h->inv;
+    ba.active = h->active;
+    ba.meta = h->meta;
+    ba.status = h->status;
+    cudaError_t e = run(h, MOE_K_BUCKET, s, [&] { return moe::launch_bucket(ba, s); });
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+
+    const moe_layer_state& L = h->layers[layer];
+    moe::ExpertArgs ea;
+    ea.T = T;
+    ea.d = c.d;
+    ea.f = c.f;
+    ea.E = c.n_experts;
+    ea.k = c.top_k;
+    ea.n_shared = c.n_shared;
+    ea.bits = c.bits;
+    ea.codes = L.codes;
+    ea.scales = L.scales;
+    ea.x = x;
+    ea.offsets = h->offsets;
+    ea.pairs = h->pairs;
+    ea.active = h->active;
+    ea.meta = h->meta;
+    ea.h = h->h;
+    ea.obuf = h->obuf;
+    ea.status = h->status;
+    e = run(h, MOE_K_GEMV_GATEUP, s, [&] { return moe::launch_gemv_gateup(ea, s); });
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    e = run(h, MOE_K_GEMV_DOWN, s, [&] { return moe::launch_gemv_down(ea, s); });
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+
+    moe::CombineArgs ca;
+    ca.T = T;
+    ca.d = c.d;
+    ca.k = c.top_k;
+    ca.n_shared = c.n_shared;
+    ca.obuf = h->obuf;
+    ca.inv = h->inv;
+    ca.w = h->w;
+    ca.y = y;
+    ca.out_fp32 = (flags & MOE_OUT_FP32) != 0;
+    ca.accumulate = (flags & MOE_ACCUMULATE) != 0;
+    return cuda_status(run(h, MOE_K_COMBINE, s, [&] { return moe::launch_combine(ca, s); }));
+}
+
+moe_status check_forward_args(moe_handle* h, int32_t layer, const void* x, int32_t T, const void* y,
+                              uint32_t flags) {
+    moe_status st = check_layer(h, layer);
+    if (st != MOE_OK) return st;
+    if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (flags & ~(MOE_OUT_FP32 | MOE_ACCUMULATE | MOE_FORCE_GEMV | MOE_FORCE_GEMM)) return MOE_ERR_INVALID_ARG;
+    if ((flags & MOE_FORCE_GEMV) && (flags & MOE_FORCE_GEMM)) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !y || !aligned16(x) || !aligned16(y))) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
+    if (!out) return MOE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!cfg) return MOE_ERR_INVALID_ARG;
+    const moe_config c = *cfg;
+    if (c.d <= 0 || c.f <= 0 || c.d % 128 || c.f % 128 || c.n_experts < 1 || c.n_experts > 1024 || c.top_k < 1 ||
+        c.top_k > c.n_experts || c.top_k > 32 || (c.n_shared != 0 && c.n_shared != 1) || c.n_layers < 1 ||
+        c.n_layers > 4096 || c.bits < 2 || c.bits > 4 || c.max_tokens < 1 || c.max_tokens > (1 << 20))
+        return MOE_ERR_INVALID_ARG;
+    moe_handle* h = new (std::nothrow) moe_handle();
+    if (!h) return MOE_ERR_OOM;
+    h->cfg = c;
+    if (cudaGetDevice(&h->device) != cudaSuccess) {
+        delete h;
+        return MOE_ERR_CUDA;
+    }
+    h->layers.resize(c.n_layers);
+
+    const size_t T = (size_t)c.max_tokens, E = (size_t)c.n_experts, k = (size_t)c.top_k;
+    const size_t rows = T * k + T * (size_t)c.n_shared;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += round256(bytes);
+        return o;
+    };
+    const size_t o_logits = take(sizeof(float) * T * E);
+    const size_t o_ids = take(sizeof(int32_t) * T * k);
+    const size_t o_w = take(sizeof(float) * T * k);
+    const size_t o_off = take(sizeof(int32_t) * (E + 1));
+    const size_t o_pairs = take(sizeof(int32_t) * T * k);
+    const size_t o_inv = take(sizeof(int32_t) * T * k);
+    const size_t o_active = take(sizeof(int32_t) * E);
+    const size_t o_meta = take(sizeof(moe::Meta));
+    const size_t o_status = take(sizeof(uint32_t) * 4);
+    const size_t o_h = take(sizeof(__half) * rows * (size_t)c.f);
+    const size_t o_obuf = take(sizeof(float) * rows * (size_t)c.d);
+    const size_t o_xs = take(sizeof(uint16_t) * T * (size_t)c.d);
+    const size_t o_ys = take(sizeof(float) * T * (size_t)c.d);
+    const size_t o_norms = take(sizeof(float) * E * (size_t)c.n_layers);
+    h->arena_bytes = off;
+    cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        delete h;
+        return e == cudaErrorMemoryAllocation ? MOE_ERR_OOM : MOE_ERR_CUDA;
+    }
+    char* base = static_cast<char*>(h->arena);
+    h->logits = reinterpret_cast<float*>(base + o_logits);
+    h->ids = reinterpret_cast<int32_t*>(base + o_ids);
+    h->w = reinterpret_cast<float*>(base + o_w);
+    h->offsets = reinterpret_cast<int32_t*>(base + o_off);
+    h->pairs = reinterpret_cast<int32_t*>(base + o_pairs);
+    h->inv = reinterpret_cast<int32_t*>(base + o_inv);
+    h->active = reinterpret_cast<int32_t*>(base + o_active);
+    h->meta = reinterpret_cast<moe::Meta*>(base + o_meta);
+    h->status = reinterpret_cast<uint32_t*>(base + o_status);
+    h->h = reinterpret_cast<__half*>(base + o_h);
+    h->obuf = reinterpret_cast<float*>(base + o_obuf);
+    h->x_stage = base + o_xs;
+    h->y_stage = base + o_ys;
+    for (int l = 0; l < c.n_layers; ++l) h->layers[l].wnorm = reinterpret_cast<float*>(base + o_norms) + E * l;
+    if (cudaMemset(h->arena, 0, h->arena_bytes) != cudaSuccess) {
+        cudaFree(h->arena);
+        delete h;
+        return MOE_ERR_CUDA;
+    }
+    *out = h;
+    return MOE_OK;
+}
+
+moe_status moe_load_layer(moe_handle* h, int32_t layer, const moe_layer_weights* w) {
+    if (!h || !w || layer < 0 || layer >= h->cfg.n_layers) return MOE_ERR_INVALID_ARG;
+    if (!w->codes || !w->scales || !w->router_w) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(w->codes) || !aligned16(w->scales) || !aligned16(w->router_w) ||
+        (w->router_bias && (reinterpret_cast<uintptr_t>(w->router_bias) & 3u)))
+        return MOE_ERR_INVALID_ARG;
+    moe_layer_state& L = h->layers[layer];
+    L.loaded = false;
+    L.codes = static_cast<const uint8_t*>(w->codes);
+    L.scales = static_cast<const uint16_t*>(w->scales);
+    L.router_w = w->router_w;
+    L.bias = w->router_bias;
+    cudaError_t e = moe::launch_router_norms(L.router_w, h->cfg.n_experts, h->cfg.d, L.wnorm, 0);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(0);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    L.loaded = true;
+    return MOE_OK;
+}
+
+moe_status moe_route(moe_handle* h, int32_t layer, const void* x, int32_t T, int32_t* ids, float* w,
+                     void* stream) {
+    moe_status st = check_layer(h, layer);
+    if (st != MOE_OK) return st;
+    if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !ids || !w || !aligned16(x) || !aligned16(ids) || !aligned16(w)) return MOE_ERR_INVALID_ARG;
+    return do_route(h, layer, x, T, ids, w, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, void* y, uint32_t flags,
+                       void* stream) {
+    moe_status st = check_forward_args(h, layer, x, T, y, flags);
+    if (st != MOE_OK || T == 0) return st;
+    return do_forward(h, layer, x, T, y, flags, static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_forward_host(moe_handle* h, int32_t layer, const void* x_host, int32_t T, void* y_host,
+                            uint32_t flags, void* stream) {
+    moe_status st = check_layer(h, layer);
+    if (st != MOE_OK) return st;
+    if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x_host || !y_host) return MOE_ERR_INVALID_ARG;
+    if (flags & ~(MOE_OUT_FP32 | MOE_ACCUMULATE | MOE_FORCE_GEMV | MOE_FORCE_GEMM)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t xb = sizeof(uint16_t) * (size_t)T * h->cfg.d;
+    const size_t yb = ((flags & MOE_OUT_FP32) ? sizeof(float) : sizeof(uint16_t)) * (size_t)T * h->cfg.d;
+    if (cudaMemcpyAsync(h->x_stage, x_host, xb, cudaMemcpyHostToDevice, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((flags & MOE_ACCUMULATE) &&
+        cudaMemcpyAsync(h->y_stage, y_host, yb, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    st = do_forward(h, layer, h->x_stage, T, h->y_stage, flags, s);
+    if (st != MOE_OK) return st;
+    if (cudaMemcpyAsync(y_host, h->y_stage, yb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+    return cuda_status(cudaStreamSynchronize(s));
+}
+
+moe_status moe_destroy(moe_handle* h) {
+    if (!h) return MOE_OK;
+    cudaError_t e = cudaSuccess;
+    if (h->arena) e = cudaFree(h->arena);
+    for (cudaEvent_t ev : h->ev) cudaEventDestroy(ev);
+    delete h;
+    return cuda_status(e);
+}
+
+moe_status moe_debug_dequant(moe_handle* h, int32_t layer, int32_t expert, int32_t mat, float* out, void* stream) {
+    moe_status st = check_layer(h, layer);
+    if (st != MOE_OK) return st;
+    const moe_config& c = h->cfg;
+    if (expert < 0 || expert >= c.n_experts + c.n_shared || mat < 0 || mat > 2 || !out || !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    const moe_layer_state& L = h->layers[layer];
+    const int64_t mc = (int64_t)c.f * c.d * c.bits / 8, ms = (int64_t)c.f * c.d / 32;
+    const int N = mat < 2 ? c.f : c.d, K = mat < 2 ? c.d : c.f;
+    return cuda_status(moe::launch_dequant(L.codes + (expert * 3 + mat) * mc, L.scales + (expert * 3 + mat) * ms, N,
+                                           K, c.bits, out, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_check_status(moe_handle* h) {
+    if (!h) return MOE_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, h->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemset(h->status, 0, sizeof(uint32_t)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (v & moe::kStatusTimeout) return MOE_ERR_TIMEOUT;
+    if (v & moe::kStatusBounds) return MOE_ERR_BOUNDS;
+    return MOE_OK;
+}
+
+moe_status moe_get_stats(moe_handle* h, moe_stats* out) {
+    if (!h || !out) return MOE_ERR_INVALID_ARG;
+    moe::Meta m;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpy(&m, h->meta, sizeof(m), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    out->fixup_tokens = m.n_fixup;
+    out->active_experts = m.n_active;
+    out->max_group = m.max_count;
+    out->launches = h->launches;
+    return MOE_OK;
+}
+
+moe_status moe_profile(moe_handle* h, int32_t enable) {
+    if (!h) return MOE_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    h->prof_on = enable != 0;
+    h->ev_kernel.clear();
+    for (int i = 0; i < MOE_KERNEL_COUNT; ++i) {
+        h->prof_ms[i] = 0.0;
+        h->prof_n[i] = 0;
+    }
+    return MOE_OK;
+}
+
+moe_status moe_profile_read(moe_handle* h, double* total_ms, int64_t* launches) {
+    if (!h || !total_ms || !launches) return MOE_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    for (size_t j = 0; j < h->ev_kernel.size(); ++j) {
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, h->ev[2 * j], h->ev[2 * j + 1]) != cudaSuccess) return MOE_ERR_CUDA;
+        h->prof_ms[h->ev_kernel[j]] += ms;
+        h->prof_n[h->ev_kernel[j]] += 1;
+    }
+    h->ev_kernel.clear();
+    for (int i = 0; i < MOE_KERNEL_COUNT; ++i) {
+        total_ms[i] = h->prof_ms[i];
+        launches[i] = h->prof_n[i];
+    }
+    return MOE_OK;
+}
+
+const char* moe_kernel_name(int32_t kernel) {
+    return (kernel >= 0 && kernel < MOE_KERNEL_COUNT) ? kKernelNames[kernel] : "unknown";
+}
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_CUDA: return "CUDA runtime error";
+        case MOE_ERR_OOM: return "out of device memory";
+        case MOE_ERR_NOT_LOADED: return "layer weights not loaded";
+        case MOE_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+        case MOE_ERR_BOUNDS: return "a device-side index was out of range";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

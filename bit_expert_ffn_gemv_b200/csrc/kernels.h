@@ -1,0 +1,68 @@
+// kernels.h -- host-side launchers of the routed-MoE kernels (internal).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+struct Meta;
+
+struct RouteArgs {
+    const void* x;      // bf16 [T x d]
+    int T, d, E, k;
+    const void* wr;     // bf16 [E x d]
+    const float* bias;  // [E] or null
+    const float* wnorm; // [E] ||W_r,e||_2, rounded up
+    float* logits;      // scratch [T x E]
+    int32_t* ids;       // [T x k]
+    float* w;           // [T x k]
+    Meta* meta;
+};
+
+// Bucketing of the T*k (token, slot) pairs by expert.
+struct BucketArgs {
+    const int32_t* ids;  // [T x k]
+    int T, k, E;
+    int32_t* offsets;    // [E + 1] start of each expert's group in `pairs`
+    int32_t* pairs;      // [T*k] t*k + r, grouped by expert, ascending t within a group
+    int32_t* inv;        // [T*k] position of pair t*k + r in `pairs`
+    int32_t* active;     // [E] experts with >= 1 pair, ascending
+    Meta* meta;
+    uint32_t* status;
+};
+
+// Grouped GEMV/GEMM problem description shared by the expert kernels.
+struct ExpertArgs {
+    int T, d, f, E, k, n_shared, bits;
+    const uint8_t* codes;   // layer codes, expert-major (gate, up, down)
+    const uint16_t* scales; // layer scales, same order
+    const void* x;          // bf16 [T x d]
+    const int32_t* offsets; // [E + 1]
+    const int32_t* pairs;   // [T*k]
+    const int32_t* active;  // [E]
+    const Meta* meta;
+    void* h;                // fp16 [(T*k + T*n_shared) x f]
+    float* obuf;            // fp32 [(T*k + T*n_shared) x d]
+    uint32_t* status;
+};
+
+struct CombineArgs {
+    int T, d, k, n_shared;
+    const float* obuf;
+    const int32_t* inv;
+    const float* w;         // [T x k]
+    void* y;                // bf16 or fp32 [T x d]
+    bool out_fp32, accumulate;
+};
+
+cudaError_t launch_router_norms(const void* wr, int E, int d, float* out, cudaStream_t s);
+cudaError_t launch_router_logits(const RouteArgs& a, cudaStream_t s);
+cudaError_t launch_topk(const RouteArgs& a, cudaStream_t s);
+cudaError_t launch_bucket(const BucketArgs& a, cudaStream_t s);
+cudaError_t launch_gemv_gateup(const ExpertArgs& a, cudaStream_t s);
+cudaError_t launch_gemv_down(const ExpertArgs& a, cudaStream_t s);
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+cudaError_t launch_dequant(const uint8_t* codes, const uint16_t* scales, int N, int K, int bits, float* out,
+                           cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,271 @@
+// route.cu -- router logits, certified top-k selection and renormalisation.
+//
+// The router the Strata pages place on the GPU (discuss.pytorch.kr post,
+// section "Strata's operating principle": the GPU runs the router and writes
+// the numbers of the 10 selected experts), with the formulas of the tiny-layer
+// workload definition: logits l = W_r x + bias, softmax over the E experts,
+// top-k with ties to the lower index, weights renormalised over the k chosen.
+//
+// Exact selection.  Logits are accumulated in fp32 from exact bf16 x bf16
+// products; every logit carries the bound |l32 - l| <= delta_e with
+//   delta_e = 2 * D * 2^-24 * (||W_r,e||_2 ||x||_2 + |bias_e|)
+// (D = longest chain of fp32 roundings in the logits kernel).  When the fp32
+// order of the top k+1 is not certified by these intervals, the token's
+// candidate experts (those whose interval reaches the k-th one's) are re-ranked
+// from fp64 logits, whose sums of bf16 products are exact in practice, so the
+// result is the exact ranking.
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- logits (CUDA cores)
+// One warp per expert row, tokens in chunks of 4 held in shared memory as
+// fp32.  Each lane accumulates d/32 products serially, then a 5-level shuffle
+// tree, then the bias: D = d/32 + 6.
+constexpr int kLogitTok = 4;
+
+__global__ void __launch_bounds__(256) router_logits_kernel(const __nv_bfloat16* __restrict__ x, int T, int d,
+                                                            const __nv_bfloat16* __restrict__ wr,
+                                                            const float* __restrict__ bias, int E,
+                                                            float* __restrict__ logits) {
+    extern __shared__ float xs[];  // [kLogitTok][d]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nwarps = blockDim.x >> 5;
+    for (int t0 = 0; t0 < T; t0 += kLogitTok) {
+        const int nt = min(kLogitTok, T - t0);
+        __syncthreads();
+        for (int i = threadIdx.x; i < kLogitTok * d; i += blockDim.x) {
+            int tt = i / d;
+            xs[i] = tt < nt ? __bfloat162float(x[(int64_t)(t0 + tt) * d + (i - tt * d)]) : 0.0f;
+        }
+        __syncthreads();
+        for (int e = blockIdx.x * nwarps + warp; e < E; e += gridDim.x * nwarps) {
+            const __nv_bfloat16* row = wr + (int64_t)e * d;
+            float acc[kLogitTok] = {0.f, 0.f, 0.f, 0.f};
+            for (int i = lane * 8; i < d; i += 256) {
+                uint4 v = __ldg(reinterpret_cast<const uint4*>(row + i));
+                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float w0 = __uint_as_float(wv[q] << 16), w1 = __uint_as_float(wv[q] & 0xFFFF0000u);
+#pragma unroll
+                    for (int tt = 0; tt < kLogitTok; ++tt) {
+                        acc[tt] = fmaf(w0, xs[tt * d + i + 2 * q], acc[tt]);
+                        acc[tt] = fmaf(w1, xs[tt * d + i + 2 * q + 1], acc[tt]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int tt = 0; tt < kLogitTok; ++tt) {
+                float v = acc[tt];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == 0 && tt < nt) logits[(int64_t)(t0 + tt) * E + e] = v + (bias ? bias[e] : 0.0f);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- row norms
+__global__ void router_norms_kernel(const __nv_bfloat16* __restrict__ wr, int E, int d, float* __restrict__ out) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (warp >= E) return;
+    double acc = 0.0;
+    for (int i = lane; i < d; i += 32) {
+        double v = (double)__bfloat162float(wr[(int64_t)warp * d + i]);
+        acc += v * v;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    // round up so the bound stays a bound
+    if (lane == 0) out[warp] = __double2float_ru(sqrt(acc) * (1.0 + 1e-12));
+}
+
+// ---------------------------------------------------------------- top-k
+// (value desc, index asc) with NaN ranked as -inf
+MOE_DEV bool better(float va, int ia, float vb, int ib) {
+    va = isnan(va) ? -INFINITY : va;
+    vb = isnan(vb) ? -INFINITY : vb;
+    return va > vb || (va == vb && ia < ib);
+}
+MOE_DEV bool better64(double va, int ia, double vb, int ib) {
+    va = isnan(va) ? -INFINITY : va;
+    vb = isnan(vb) ? -INFINITY : vb;
+    return va > vb || (va == vb && ia < ib);
+}
+
+constexpr int kTopkWarps = 4;
+constexpr int kMaxK = 32;
+
+// One warp per token.  Shared memory per warp: E floats (fp32 logits),
+// E floats (bounds), E doubles (fp64 logits of candidates).
+__global__ void __launch_bounds__(kTopkWarps * 32)
+    topk_kernel(const float* __restrict__ logits, const __nv_bfloat16* __restrict__ x, int T, int d, int E, int k,
+                const __nv_bfloat16* __restrict__ wr, const float* __restrict__ bias,
+                const float* __restrict__ wnorm, float depth, int32_t* __restrict__ ids_out,
+                float* __restrict__ w_out, Meta* __restrict__ meta) {
+    extern __shared__ unsigned char smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * kTopkWarps + warp;
+    double* lg64 = reinterpret_cast<double*>(smem_raw) + (size_t)warp * E;
+    float* lv = reinterpret_cast<float*>(smem_raw + sizeof(double) * (size_t)kTopkWarps * E) + (size_t)warp * 2 * E;
+    float* dv = lv + E;
+    if (t >= T) return;
+
+    // ||x_t||_2 (fp32, inflated to stay an upper bound)
+    const __nv_bfloat16* xt = x + (int64_t)t * d;
+    float ss = 0.f;
+    for (int i = lane; i < d; i += 32) {
+        float v = __bfloat162float(xt[i]);
+        ss = fmaf(v, v, ss);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float xn = sqrtf(ss) * (1.0f + 1e-5f);
+    const float c = 2.0f * depth * 5.9604645e-8f * (1.0f + 1e-5f);
+
+    for (int e = lane; e < E; e += 32) {
+        float v = logits[(int64_t)t * E + e];
+        lv[e] = v;
+        dv[e] = c * (wnorm[e] * xn + (bias ? fabsf(bias[e]) : 0.0f));
+    }
+    __syncwarp();
+
+    // top-(k+1) by repeated warp argmax; `taken` bit j <-> element lane + 32 j
+    uint32_t taken = 0;
+    int sel[kMaxK + 1];
+    const int kk = min(k + 1, E);
+    for (int r = 0; r < kk; ++r) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+        for (int j = 0, e = lane; e < E; ++j, e += 32)
+            if (!((taken >> j) & 1u) && (bi == 0x7fffffff || better(lv[e], e, bv, bi))) {
+                bv = lv[e];
+                bi = e;
+            }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (oi != 0x7fffffff && (bi == 0x7fffffff || better(ov, oi, bv, bi))) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        sel[r] = bi;
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    }
+
+    // certification of the fp32 order
+    bool ok = true;
+    for (int r = 0; r + 1 < k; ++r) {
+        int a = sel[r], b = sel[r + 1];
+        if (!(lv[a] - dv[a] > lv[b] + dv[b])) ok = false;
+    }
+    const float lower_k = lv[sel[k - 1]] - dv[sel[k - 1]];
+    int n_cand = 0;
+    for (int e = lane; e < E; e += 32) n_cand += (isnan(lv[e]) ? false : (lv[e] + dv[e] >= lower_k)) ? 1 : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n_cand += __shfl_xor_sync(0xffffffffu, n_cand, o);
+    if (n_cand != k) ok = false;
+    if (isnan(lower_k)) ok = false;
+
+    float wsel[kMaxK];
+    if (ok) {
+        for (int r = 0; r < k; ++r) wsel[r] = lv[sel[r]];
+    } else {
+        // fp64 logits of every candidate, then exact ranking among them
+        for (int e = 0; e < E; ++e) {
+            bool cand = isnan(lower_k) || isnan(lv[e]) || (lv[e] + dv[e] >= lower_k);
+            if (!cand) {
+                if (lane == 0) lg64[e] = -INFINITY;
+                continue;
+            }
+            double acc = 0.0;
+            const __nv_bfloat16* row = wr + (int64_t)e * d;
+            for (int i = lane; i < d; i += 32)
+                acc = fma((double)__bfloat162float(row[i]), (double)__bfloat162float(xt[i]), acc);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (lane == 0) lg64[e] = acc + (bias ? (double)bias[e] : 0.0);
+        }
+        __syncwarp();
+        uint32_t tk = 0;
+        for (int r = 0; r < k; ++r) {
+            double bv = -INFINITY;
+            int bi = 0x7fffffff;
+            for (int j = 0, e = lane; e < E; ++j, e += 32)
+                if (!((tk >> j) & 1u) && (bi == 0x7fffffff || better64(lg64[e], e, bv, bi))) {
+                    bv = lg64[e];
+                    bi = e;
+                }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (oi != 0x7fffffff && (bi == 0x7fffffff || better64(ov, oi, bv, bi))) {
+                    bv = ov;
+                    bi = oi;
+                }
+            }
+            sel[r] = bi;
+            wsel[r] = (float)bv;
+            if ((bi & 31) == lane) tk |= 1u << (bi >> 5);
+        }
+        if (lane == 0) atomicAdd(&meta->n_fixup, 1);
+    }
+
+    // renormalised weights = softmax over the k selected logits
+    if (lane == 0) {
+        float m = wsel[0];
+        float z = 0.f;
+        float ex[kMaxK];
+        for (int r = 0; r < k; ++r) {
+            ex[r] = expf(wsel[r] - m);
+            z += ex[r];
+        }
+        const float inv = 1.0f / z;
+        for (int r = 0; r < k; ++r) {
+            ids_out[(int64_t)t * k + r] = sel[r];
+            w_out[(int64_t)t * k + r] = ex[r] * inv;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- launchers
+cudaError_t launch_router_norms(const void* wr, int E, int d, float* out, cudaStream_t s) {
+    router_norms_kernel<<<(E * 32 + 255) / 256, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(wr), E, d, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_logits(const RouteArgs& a, cudaStream_t s) {
+    const size_t smem_l = sizeof(float) * kLogitTok * a.d;
+    if (smem_l > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(router_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem_l);
+        if (e != cudaSuccess) return e;
+    }
+    int grid = (a.E + 7) / 8;
+    router_logits_kernel<<<grid, 256, smem_l, s>>>(static_cast<const __nv_bfloat16*>(a.x), a.T, a.d,
+                                                  static_cast<const __nv_bfloat16*>(a.wr), a.bias, a.E, a.logits);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_topk(const RouteArgs& a, cudaStream_t s) {
+    const size_t smem_t = (size_t)kTopkWarps * a.E * (sizeof(double) + 2 * sizeof(float));
+    if (smem_t > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_t);
+        if (e != cudaSuccess) return e;
+    }
+    const float depth = (float)(a.d / 32 + 6);
+    topk_kernel<<<(a.T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, smem_t, s>>>(
+        a.logits, static_cast<const __nv_bfloat16*>(a.x), a.T, a.d, a.E, a.k,
+        static_cast<const __nv_bfloat16*>(a.wr), a.bias, a.wnorm, depth, a.ids, a.w, a.meta);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

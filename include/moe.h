@@ -1,0 +1,219 @@
+/*
+ * moe.h -- C ABI of the B200 routed Mixture-of-Experts layer.
+ *
+ * One routed-MoE layer of a Qwen3.8-Flash-Next-shaped model: per token, a
+ * router picks k of E experts (10 of 512 per layer), each a SwiGLU FFN with
+ * 2-4-bit block-quantised weights, plus one shared expert that every token
+ * uses; the GPU combines the results before the next layer.  The operation is
+ * the one the Strata pages describe -- discuss.pytorch.kr post, section
+ * "Strata's operating principle / experts split across VRAM, RAM and SSD"
+ * ("the GPU runs the router and writes the numbers of the 10 selected
+ * experts ... the GPU combines each result, then moves to the next layer"),
+ * and tech.okbari.net guide, section "Strata, Qwen and GSQ-RCO are different
+ * components" (48 layers, 10 of 512 routed experts plus 1 shared expert
+ * active per MoE layer).  The formulas are those of the tiny-layer workload
+ * definition:
+ *   logits  l = W_r x + bias             (W_r bf16 [E x d], bias fp32 or none)
+ *   p       = softmax(l) over the E experts
+ *   ids     = top-k of l, ties to the lower expert index, in rank order
+ *   w_r     = p[ids_r] / sum_r' p[ids_r']
+ *   expert  o_e = W_d,e (silu(W_g,e x) * W_u,e x),  silu(a) = a / (1 + e^-a)
+ *   y       = o_shared + sum_r w_r o_{ids_r}
+ * with What = q * s: b-bit codes q in [-2^(b-1), 2^(b-1)-1] and one fp16
+ * scale s per block of 32 weights along the input dimension.
+ *
+ * Conventions
+ *   - Every call returns a moe_status; no exception crosses the ABI.
+ *   - All tensor pointers are DEVICE pointers on the handle's device unless
+ *     a function says otherwise, and must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream); work is
+ *     enqueued asynchronously on it.
+ *   - A handle is not thread-safe: use one handle per stream.
+ *   - Device-side anomalies (an expert id out of range, a bounded wait that
+ *     ran out) set a status word in device memory; moe_check_status()
+ *     synchronises and reports it.
+ *
+ * Packed weight layout of one layer (memory owned by the caller, borrowed):
+ *   codes : expert-major; expert e (the shared expert is e = E) holds
+ *           gate [f x d], up [f x d], down [d x f], each f*d*b/8 bytes
+ *   scales: same order, each matrix f*d/32 fp16 values
+ * Each matrix W[N x K] is tiled into 16 x 128 super-tiles stored at
+ * (n/16)*(K/128) + k/128, 256*b code bytes and 64 fp16 scales each.  Inside
+ * a super-tile, with r = n%16 and j = k%128:
+ *   kb = j/32, ks = (j%32)/16, m = j%16,
+ *   lane = 4*(r%8) + (m%8)/2, pair p = 4*ks + 2*(m/8) + r/8, elem e = m%2
+ *   b=2: u = bits [2p+16e, +1] of the 32-bit LE word at byte 16*lane + 4*kb
+ *   b=3: same two bits = u%4, plus bit (p+8e) of the 16-bit LE word at
+ *        byte 512 + 8*lane + 2*kb = u/4
+ *   b=4: u = bits [4(p%4)+16e, +3] of the 32-bit LE word at byte
+ *        512*(p/4) + 16*lane + 4*kb
+ *   q = u - 2^(b-1); the block scale is fp16 number 8*(r%8) + 2*kb + r/8 of
+ *   the super-tile's 64.
+ * (lane and p follow the A-operand registers of a 16x8x16 warp-level MMA, so
+ * each thread of a warp loads exactly the codes it multiplies.)
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_handle moe_handle;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* a bad argument; nothing was enqueued */
+    MOE_ERR_CUDA = 2,        /* a CUDA runtime call failed */
+    MOE_ERR_OOM = 3,         /* device allocation failed */
+    MOE_ERR_NOT_LOADED = 4,  /* the layer has no weights loaded */
+    MOE_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up */
+    MOE_ERR_BOUNDS = 6       /* a device-side index was out of range */
+} moe_status;
+
+typedef struct {
+    int32_t d;          /* hidden size, multiple of 128 */
+    int32_t f;          /* expert intermediate size, multiple of 128 */
+    int32_t n_experts;  /* routed experts E, 1..1024 */
+    int32_t top_k;      /* experts per token k, 1..min(E, 32) */
+    int32_t n_shared;   /* shared experts, 0 or 1 */
+    int32_t n_layers;   /* layers this handle can hold, >= 1 */
+    int32_t bits;       /* code width b: 2, 3 or 4 */
+    int32_t max_tokens; /* largest T a call may pass, >= 1 */
+} moe_config;
+
+typedef struct {
+    const void* codes;       /* device, packed codes of all E + n_shared experts */
+    const void* scales;      /* device, fp16 block scales, same order */
+    const void* router_w;    /* device, bf16 [E x d] row-major */
+    const float* router_bias;/* device, fp32 [E], or NULL for no bias */
+} moe_layer_weights;
+
+/* forward flags */
+#define MOE_OUT_FP32 0x1u   /* y is fp32 [T x d] (default: bf16) */
+#define MOE_ACCUMULATE 0x2u /* y += layer output (default: y = layer output) */
+#define MOE_FORCE_GEMV 0x4u /* use the grouped-GEMV path whatever T is */
+#define MOE_FORCE_GEMM 0x8u /* use the grouped-GEMM path whatever T is */
+
+/*
+ * Create a handle on the current CUDA device.  Checks the configuration and
+ * allocates all library-owned scratch for up to cfg->max_tokens tokens.
+ * Errors: INVALID_ARG (bad field, NULL pointer), OOM, CUDA.  *out is set to
+ * NULL on error.
+ */
+moe_status moe_layer_init(const moe_config* cfg, moe_handle** out);
+
+/*
+ * Attach layer `layer`'s weights (device pointers, layout above).  The memory
+ * stays owned by the caller and must outlive the handle or the next load of
+ * the same layer.  Precomputes the router row norms used to certify the
+ * expert selection (synchronous on the legacy default stream).
+ * Errors: INVALID_ARG (NULL handle/weights/pointer, layer out of range,
+ * misaligned pointer), CUDA, OOM.
+ */
+moe_status moe_load_layer(moe_handle* h, int32_t layer, const moe_layer_weights* w);
+
+/*
+ * Routing only: ids [T x k] int32 (rank order) and renormalised weights
+ * w [T x k] fp32 for bf16 activations x [T x d].  The selection equals the
+ * exact (fp64) ranking: tokens whose fp32 logits leave the order uncertain
+ * are re-ranked from fp64 logits.  T = 0 is a no-op.
+ * Errors: INVALID_ARG (T < 0 or > max_tokens, NULL or misaligned pointer),
+ * NOT_LOADED, CUDA.
+ */
+moe_status moe_route(moe_handle* h, int32_t layer, const void* x, int32_t T, int32_t* ids, float* w,
+                     void* stream);
+
+/*
+ * The whole layer for bf16 activations x [T x d]: writes (or, with
+ * MOE_ACCUMULATE, adds to) y [T x d], bf16 or (MOE_OUT_FP32) fp32.  x and y
+ * must not overlap, except y == x (bf16) with MOE_ACCUMULATE, which updates a
+ * residual stream in place (x += layer(x)): every read of x is enqueued
+ * before the final write of y.  T = 0 is a no-op.
+ * Errors: INVALID_ARG, NOT_LOADED, CUDA.
+ */
+moe_status moe_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, void* y, uint32_t flags,
+                       void* stream);
+
+/*
+ * moe_forward for HOST buffers: copies x_host (bf16 [T x d]) to the device,
+ * runs the layer and copies y back into y_host ([T x d], bf16 or fp32 per
+ * flags), all on `stream`; returns after the result is in y_host.  Pinned
+ * host memory makes the copies asynchronous DMA; pageable memory works but is
+ * staged by the driver.  MOE_ACCUMULATE adds to the values already in y_host.
+ * Errors: as moe_forward.
+ */
+moe_status moe_forward_host(moe_handle* h, int32_t layer, const void* x_host, int32_t T, void* y_host,
+                            uint32_t flags, void* stream);
+
+/* Free the handle's own memory (never the borrowed weights).  NULL is a no-op. */
+moe_status moe_destroy(moe_handle* h);
+
+/*
+ * Debug: the fp32 values q * s of matrix `mat` (0 gate [f x d], 1 up [f x d],
+ * 2 down [d x f]) of expert `expert` (E = shared) of a loaded layer, written
+ * row-major to out (device).  Exact: |q| <= 8 and s is fp16.
+ */
+moe_status moe_debug_dequant(moe_handle* h, int32_t layer, int32_t expert, int32_t mat, float* out,
+                             void* stream);
+
+/*
+ * Synchronise the device and return the first device-side error recorded
+ * since the last call (then clear it): MOE_ERR_TIMEOUT, MOE_ERR_BOUNDS or
+ * MOE_OK; MOE_ERR_CUDA if the synchronisation itself failed.
+ */
+moe_status moe_check_status(moe_handle* h);
+
+/* Counters (moe_get_stats). */
+typedef struct {
+    int64_t fixup_tokens;   /* tokens of the last routing re-ranked from fp64 logits */
+    int64_t active_experts; /* distinct routed experts of the last moe_forward */
+    int64_t max_group;      /* largest expert group of the last moe_forward */
+    int64_t launches;       /* kernels this handle has launched since moe_layer_init */
+} moe_stats;
+
+/* Synchronise the device and read the counters. */
+moe_status moe_get_stats(moe_handle* h, moe_stats* out);
+
+/* Kernel ids for the per-kernel timing of moe_profile_read. */
+enum {
+    MOE_K_ROUTER_LOGITS = 0,
+    MOE_K_TOPK = 1,
+    MOE_K_BUCKET = 2,
+    MOE_K_GEMV_GATEUP = 3,
+    MOE_K_GEMV_DOWN = 4,
+    MOE_K_COMBINE = 5,
+    MOE_K_GEMM_GATEUP = 6,
+    MOE_K_GEMM_DOWN = 7,
+    MOE_K_ROUTER_GEMM = 8,
+    MOE_KERNEL_COUNT = 9
+};
+
+/*
+ * Per-kernel timing.  moe_profile(h, 1) synchronises, clears the totals and
+ * from then on brackets every kernel the handle launches with a pair of CUDA
+ * events on the launching stream; moe_profile(h, 0) stops.  Events add a
+ * little time between kernels, so time throughput with profiling off.
+ */
+moe_status moe_profile(moe_handle* h, int32_t enable);
+
+/*
+ * Synchronise and add up the recorded events: total_ms[i] and launches[i]
+ * (arrays of MOE_KERNEL_COUNT) receive the summed device time and the launch
+ * count of kernel i since moe_profile(h, 1).
+ */
+moe_status moe_profile_read(moe_handle* h, double* total_ms, int64_t* launches);
+
+/* Static name of kernel id i ("unknown" when out of range). */
+const char* moe_kernel_name(int32_t kernel);
+
+/* Static text for a status code. */
+const char* moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

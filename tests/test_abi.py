@@ -1,0 +1,70 @@
+"""The C-ABI library loads and exports what include/moe.h declares (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import bit_expert_ffn_gemv_b200 as moe
+from bit_expert_ffn_gemv_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", src))
+    return names
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return moe.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert {"moe_layer_init", "moe_load_layer", "moe_route", "moe_forward", "moe_destroy"} <= names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for s, name in moe.STATUS.items():
+        assert moe.moe_status_string(s)
+    assert moe.moe_status_string(99) == "unknown status"
+
+
+def _cfg(**kw):
+    base = dict(d=256, f=128, n_experts=16, top_k=2, n_shared=1, n_layers=1, bits=2, max_tokens=8)
+    base.update(kw)
+    return moe.MoeConfig(**base)
+
+
+@pytest.mark.parametrize("bad", [dict(d=200), dict(f=100), dict(n_experts=0), dict(n_experts=2000),
+                                 dict(top_k=0), dict(top_k=17), dict(n_shared=2), dict(bits=1), dict(bits=5),
+                                 dict(max_tokens=0), dict(n_layers=0), dict(top_k=33, n_experts=64)])
+def test_init_rejects_bad_config_before_touching_the_gpu(L, bad):
+    h = ctypes.c_void_p(1234)
+    s = L.moe_layer_init(ctypes.byref(_cfg(**bad)), ctypes.byref(h))
+    assert s == 1 and h.value is None  # MOE_ERR_INVALID_ARG, *out cleared
+
+
+def test_null_arguments(L):
+    assert L.moe_layer_init(None, None) == 1
+    assert L.moe_destroy(None) == 0
+    assert L.moe_route(None, 0, None, 1, None, None, None) == 1
+    assert L.moe_forward(None, 0, None, 1, None, 0, None) == 1
+    assert L.moe_forward_host(None, 0, None, 1, None, 0, None) == 1
+    assert L.moe_load_layer(None, 0, None) == 1
+    assert L.moe_debug_dequant(None, 0, 0, 0, None, None) == 1
+    assert L.moe_check_status(None) == 1
+    assert L.moe_get_stats(None, None) == 1
+    assert L.moe_profile(None, 1) == 1
+    assert L.moe_profile_read(None, None, None) == 1
+    assert moe.moe_kernel_name(0) == "router_logits" and moe.moe_kernel_name(99) == "unknown"
