@@ -18,7 +18,7 @@ import threading
 
 __all__ = ["MoeError", "MoeConfig", "MoeLayerWeights", "MoeLayer", "lib", "library_path", "MOE_OUT_FP32",
            "MOE_ACCUMULATE", "MOE_FORCE_GEMV", "MOE_FORCE_GEMM", "STATUS", "moe_layer_init", "moe_load_layer",
-           "moe_route", "moe_forward", "moe_forward_host", "moe_destroy", "moe_debug_dequant", "moe_check_status",
+           "moe_route", "moe_route_noalloc", "moe_forward", "moe_forward_host", "moe_destroy", "moe_debug_dequant", "moe_check_status",
            "moe_get_stats", "moe_status_string", "moe_profile", "moe_profile_read", "moe_kernel_name", "MoeStats"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -95,6 +95,8 @@ def lib() -> ctypes.CDLL:
             L.moe_profile_read.argtypes = [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
             L.moe_kernel_name.restype = ctypes.c_char_p
             L.moe_kernel_name.argtypes = [i32]
+            L.moe_route_noalloc.restype = st
+            L.moe_route_noalloc.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]
             L.moe_status_string.restype = ctypes.c_char_p
             L.moe_status_string.argtypes = [st]
             _lib = L
@@ -134,6 +136,13 @@ def moe_forward(handle: int, layer: int, x_ptr: int, T: int, y_ptr: int, flags: 
 
 def moe_forward_host(handle: int, layer: int, x_host: int, T: int, y_host: int, flags: int, stream: int) -> None:
     _check(lib().moe_forward_host(handle, layer, x_host, T, y_host, flags, stream), "moe_forward_host")
+
+
+def moe_route_noalloc(x_ptr: int, T: int, d: int, n_experts: int, top_k: int, router_w_ptr: int, bias_ptr,
+                      ids_ptr: int, w_ptr: int, stream: int) -> None:
+    """Routing for callers that cannot allocate device memory (no handle; fixed in-library scratch)."""
+    _check(lib().moe_route_noalloc(x_ptr, T, d, n_experts, top_k, router_w_ptr, bias_ptr, ids_ptr, w_ptr, stream),
+           "moe_route_noalloc")
 
 
 def moe_destroy(handle: int) -> None:

@@ -148,6 +148,31 @@ moe_status moe_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, v
 moe_status moe_forward_host(moe_handle* h, int32_t layer, const void* x_host, int32_t T, void* y_host,
                             uint32_t flags, void* stream);
 
+/*
+ * Routing without any device allocation (the Strata pages have no counterpart
+ * of this call; it exists for callers of this library that cannot allocate:
+ * code running while a CUDA graph is captured, plug-ins whose host framework
+ * owns all device memory, loops that cannot pay for cudaMalloc's implicit
+ * synchronisation).  Same result as moe_route() -- ids [T x k] int32 and
+ * weights w [T x k] fp32 -- but without a handle: the caller passes the router
+ * weights (bf16 [n_experts x d], 16-byte aligned), the bias (fp32 [n_experts]
+ * or NULL) and the activations x (bf16 [T x d]).  All device pointers.
+ *
+ * Intermediates live in one fixed device array inside the library (about
+ * 260 KB, held by every GPU that loads the library until the process exits):
+ * T * n_experts must not exceed 65536 and n_experts not 1024, else
+ * MOE_ERR_INVALID_ARG and nothing is enqueued.  d must be a multiple of 128,
+ * 1 <= top_k <= min(n_experts, 32).  The first call on each device looks the
+ * array's address up on the current device; make that first call before any
+ * stream capture.  All calls share the array: two calls whose work overlaps
+ * on the GPU (different streams, no ordering between them) race and give
+ * wrong results -- order them on one stream.
+ * Errors: INVALID_ARG, CUDA.
+ */
+moe_status moe_route_noalloc(const void* x, int32_t T, int32_t d, int32_t n_experts, int32_t top_k,
+                             const void* router_w, const float* router_bias, int32_t* ids, float* w,
+                             void* stream);
+
 /* Free the handle's own memory (never the borrowed weights).  NULL is a no-op. */
 moe_status moe_destroy(moe_handle* h);
 
