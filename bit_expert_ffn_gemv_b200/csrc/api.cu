@@ -5,6 +5,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <algorithm>
 #include <new>
 #include <vector>
 
@@ -14,7 +15,7 @@
 
 static const char* const kKernelNames[MOE_KERNEL_COUNT] = {
     "router_logits", "topk", "bucket", "gemv_gateup", "gemv_down", "combine", "gemm_gateup", "gemm_down",
-    "router_gemm"};
+    "router_gemm", "decode_fused"};
 
 struct moe_layer_state {
     const uint8_t* codes = nullptr;
@@ -43,6 +44,8 @@ struct moe_handle {
     uint32_t* status = nullptr;
     __half* h = nullptr;
     float* obuf = nullptr;
+    double* logits64 = nullptr;
+    int* sync = nullptr;
     void* x_stage = nullptr;
     void* y_stage = nullptr;
     // launch accounting and optional per-kernel event timing
@@ -56,6 +59,8 @@ struct moe_handle {
 
 namespace {
 
+
+constexpr uint32_t kAllFlags = MOE_OUT_FP32 | MOE_ACCUMULATE | MOE_FORCE_GEMV | MOE_FORCE_GEMM | MOE_FORCE_UNFUSED;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -114,9 +119,48 @@ moe_status do_route(moe_handle* h, int32_t layer, const void* x, int32_t T, int3
     return cuda_status(run(h, MOE_K_TOPK, s, [&] { return moe::launch_topk(ra, s); }));
 }
 
+moe_status do_decode(moe_handle* h, int32_t layer, const void* x, int32_t T, void* y, uint32_t flags,
+                     cudaStream_t s) {
+    const moe_config& c = h->cfg;
+    const moe_layer_state& L = h->layers[layer];
+    moe::DecodeLaunch d;
+    d.T = T;
+    d.d = c.d;
+    d.f = c.f;
+    d.E = c.n_experts;
+    d.k = c.top_k;
+    d.n_shared = c.n_shared;
+    d.bits = c.bits;
+    d.x = x;
+    d.y = y;
+    d.out_fp32 = (flags & MOE_OUT_FP32) ? 1 : 0;
+    d.accumulate = (flags & MOE_ACCUMULATE) ? 1 : 0;
+    d.codes = L.codes;
+    d.scales = L.scales;
+    d.wr = L.router_w;
+    d.bias = L.bias;
+    d.wnorm = L.wnorm;
+    d.logits = h->logits;
+    d.logits64 = h->logits64;
+    d.ids = h->ids;
+    d.w = h->w;
+    d.offsets = h->offsets;
+    d.pairs = h->pairs;
+    d.inv = h->inv;
+    d.active = h->active;
+    d.meta = h->meta;
+    d.status = h->status;
+    d.h = h->h;
+    d.obuf = h->obuf;
+    d.sync = h->sync;
+    return cuda_status(run(h, MOE_K_DECODE, s, [&] { return moe::launch_decode(d, s); }));
+}
+
 moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, void* y, uint32_t flags,
                       cudaStream_t s) {
     const moe_config& c = h->cfg;
+    if (T <= moe::kDecodeMaxTokens && !(flags & (MOE_FORCE_GEMM | MOE_FORCE_UNFUSED)))
+        return do_decode(h, layer, x, T, y, flags, s);
     moe_status st = do_route(h, layer, x, T, h->ids, h->w, s);
     if (st != MOE_OK) return st;
     moe::BucketArgs ba;
@@ -176,7 +220,7 @@ moe_status check_forward_args(moe_handle* h, int32_t layer, const void* x, int32
     moe_status st = check_layer(h, layer);
     if (st != MOE_OK) return st;
     if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
-    if (flags & ~(MOE_OUT_FP32 | MOE_ACCUMULATE | MOE_FORCE_GEMV | MOE_FORCE_GEMM)) return MOE_ERR_INVALID_ARG;
+    if (flags & ~kAllFlags) return MOE_ERR_INVALID_ARG;
     if ((flags & MOE_FORCE_GEMV) && (flags & MOE_FORCE_GEMM)) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!x || !y || !aligned16(x) || !aligned16(y))) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
@@ -226,6 +270,9 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     const size_t o_xs = take(sizeof(uint16_t) * T * (size_t)c.d);
     const size_t o_ys = take(sizeof(float) * T * (size_t)c.d);
     const size_t o_norms = take(sizeof(float) * E * (size_t)c.n_layers);
+    const size_t o_l64 = take(sizeof(double) * std::min<size_t>(T, moe::kDecodeMaxTokens) * E);
+    const size_t o_sync =
+        take(sizeof(int) * moe::decode_sync_words(std::min(c.max_tokens, moe::kDecodeMaxTokens), c.n_experts, c.d));
     h->arena_bytes = off;
     cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
     if (e != cudaSuccess) {
@@ -245,6 +292,8 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     h->status = reinterpret_cast<uint32_t*>(base + o_status);
     h->h = reinterpret_cast<__half*>(base + o_h);
     h->obuf = reinterpret_cast<float*>(base + o_obuf);
+    h->logits64 = reinterpret_cast<double*>(base + o_l64);
+    h->sync = reinterpret_cast<int*>(base + o_sync);
     h->x_stage = base + o_xs;
     h->y_stage = base + o_ys;
     for (int l = 0; l < c.n_layers; ++l) h->layers[l].wnorm = reinterpret_cast<float*>(base + o_norms) + E * l;
@@ -300,7 +349,8 @@ moe_status moe_forward_host(moe_handle* h, int32_t layer, const void* x_host, in
     if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x_host || !y_host) return MOE_ERR_INVALID_ARG;
-    if (flags & ~(MOE_OUT_FP32 | MOE_ACCUMULATE | MOE_FORCE_GEMV | MOE_FORCE_GEMM)) return MOE_ERR_INVALID_ARG;
+    if (flags & ~kAllFlags) return MOE_ERR_INVALID_ARG;
+    if ((flags & MOE_FORCE_GEMV) && (flags & MOE_FORCE_GEMM)) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t xb = sizeof(uint16_t) * (size_t)T * h->cfg.d;
     const size_t yb = ((flags & MOE_OUT_FP32) ? sizeof(float) : sizeof(uint16_t)) * (size_t)T * h->cfg.d;

@@ -55,6 +55,35 @@ struct CombineArgs {
     bool out_fp32, accumulate;
 };
 
+// Whole layer for up to kDecodeMaxTokens tokens in one persistent kernel.
+constexpr int kDecodeMaxTokens = 64;
+struct DecodeLaunch {
+    int T, d, f, E, k, n_shared, bits;
+    const void* x;
+    void* y;
+    int out_fp32, accumulate;
+    const uint8_t* codes;
+    const uint16_t* scales;
+    const void* wr;
+    const float* bias;
+    const float* wnorm;
+    float* logits;
+    double* logits64;
+    int32_t* ids;
+    float* w;
+    int32_t* offsets;
+    int32_t* pairs;
+    int32_t* inv;
+    int32_t* active;
+    Meta* meta;
+    uint32_t* status;
+    void* h;
+    float* obuf;
+    int* sync;  // zeroed once; the kernel leaves it zeroed
+};
+cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t s);
+size_t decode_sync_words(int max_tokens, int E, int d);
+
 cudaError_t launch_router_norms(const void* wr, int E, int d, float* out, cudaStream_t s);
 cudaError_t launch_router_logits(const RouteArgs& a, cudaStream_t s);
 cudaError_t launch_topk(const RouteArgs& a, cudaStream_t s);

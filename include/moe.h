@@ -96,6 +96,7 @@ typedef struct {
 #define MOE_ACCUMULATE 0x2u /* y += layer output (default: y = layer output) */
 #define MOE_FORCE_GEMV 0x4u /* use the grouped-GEMV path whatever T is */
 #define MOE_FORCE_GEMM 0x8u /* use the grouped-GEMM path whatever T is */
+#define MOE_FORCE_UNFUSED 0x10u /* small T: one kernel per step instead of the fused persistent kernel */
 
 /*
  * Create a handle on the current CUDA device.  Checks the configuration and
@@ -213,7 +214,8 @@ enum {
     MOE_K_GEMM_GATEUP = 6,
     MOE_K_GEMM_DOWN = 7,
     MOE_K_ROUTER_GEMM = 8,
-    MOE_KERNEL_COUNT = 9
+    MOE_K_DECODE = 9,
+    MOE_KERNEL_COUNT = 10
 };
 
 /*

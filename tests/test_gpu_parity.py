@@ -156,8 +156,34 @@ def decode_layer(torch_cuda):
     h.close()
 
 
-@pytest.mark.parametrize("T", [1, 4, 16, 64, 7])
+@pytest.mark.parametrize("T", [1, 4, 16, 64, 7, 33])
 def test_decode_layer(torch_cuda, decode_layer, T):
     wl, L, h = decode_layer
     x = synth.x_host(wl.shape, wl.master, 200 + T, T)
     _check_layer(torch_cuda, h, wl.shape, L, x, label="decode")
+
+
+@pytest.mark.parametrize("T", [1, 4, 64])
+def test_decode_layer_unfused(torch_cuda, decode_layer, T):
+    """The one-kernel-per-step path meets the same bar, and agrees with the fused kernel to fp32 rounding."""
+    import bit_expert_ffn_gemv_b200 as moe
+    wl, L, h = decode_layer
+    xb = synth.x_host(wl.shape, wl.master, 400 + T, T)
+    _check_layer(torch_cuda, h, wl.shape, L, xb, flags_extra=moe.MOE_FORCE_UNFUSED, label="decode-unfused")
+    x = x_to_device(xb)
+    a = h.forward(0, x, flags=moe.MOE_OUT_FP32)
+    b = h.forward(0, x, flags=moe.MOE_OUT_FP32 | moe.MOE_FORCE_UNFUSED)
+    torch_cuda.cuda.synchronize()
+    assert rel_l2(y_to_f64(a), y_to_f64(b)) < 1e-5
+
+
+def test_inplace_residual(torch_cuda, decode_layer):
+    """y == x with MOE_ACCUMULATE updates a residual stream in place."""
+    import bit_expert_ffn_gemv_b200 as moe
+    wl, L, h = decode_layer
+    x = x_to_device(synth.x_host(wl.shape, wl.master, 77, 4))
+    ref = (x.float() + h.forward(0, x, flags=moe.MOE_OUT_FP32)).to(torch_cuda.bfloat16)
+    r = x.clone()
+    h.forward(0, r, r, flags=moe.MOE_ACCUMULATE)
+    torch_cuda.cuda.synchronize()
+    assert torch_cuda.equal(r, ref)
