@@ -18,7 +18,7 @@ import threading
 
 __all__ = ["MoeError", "MoeConfig", "MoeLayerWeights", "MoeLayer", "lib", "library_path", "MOE_OUT_FP32",
            "MOE_ACCUMULATE", "MOE_FORCE_GEMV", "MOE_FORCE_GEMM", "MOE_FORCE_UNFUSED", "STATUS", "moe_layer_init", "moe_load_layer",
-           "moe_route", "moe_route_noalloc", "moe_forward", "moe_forward_host", "moe_destroy", "moe_debug_dequant", "moe_check_status",
+           "moe_route", "moe_route_noalloc", "moe_forward", "moe_forward_host", "moe_destroy", "moe_debug_dequant", "moe_debug_last_routing", "moe_check_status",
            "moe_get_stats", "moe_status_string", "moe_profile", "moe_profile_read", "moe_kernel_name", "MoeStats"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
             L.moe_destroy.argtypes = [vp]
             L.moe_debug_dequant.restype = st
             L.moe_debug_dequant.argtypes = [vp, i32, i32, i32, vp, vp]
+            L.moe_debug_last_routing.restype = st
+            L.moe_debug_last_routing.argtypes = [vp, i32, vp, vp, vp]
             L.moe_check_status.restype = st
             L.moe_check_status.argtypes = [vp]
             L.moe_get_stats.restype = st
@@ -152,6 +154,10 @@ def moe_destroy(handle: int) -> None:
 
 def moe_debug_dequant(handle: int, layer: int, expert: int, mat: int, out_ptr: int, stream: int) -> None:
     _check(lib().moe_debug_dequant(handle, layer, expert, mat, out_ptr, stream), "moe_debug_dequant")
+
+
+def moe_debug_last_routing(handle: int, T: int, ids_ptr: int, w_ptr: int, stream: int) -> None:
+    _check(lib().moe_debug_last_routing(handle, T, ids_ptr, w_ptr, stream), "moe_debug_last_routing")
 
 
 def moe_check_status(handle: int) -> int:
@@ -240,6 +246,14 @@ class MoeLayer:
             out = torch.empty((N, K), dtype=torch.float32, device="cuda")
         moe_debug_dequant(self.handle, layer, expert, mat, out.data_ptr(), _stream_ptr(stream))
         return out
+
+    def last_routing(self, T, stream=None):
+        """(ids, w) the last forward computed internally for its T tokens."""
+        import torch
+        ids = torch.empty((T, self.cfg.top_k), dtype=torch.int32, device="cuda")
+        w = torch.empty((T, self.cfg.top_k), dtype=torch.float32, device="cuda")
+        moe_debug_last_routing(self.handle, T, ids.data_ptr(), w.data_ptr(), _stream_ptr(stream))
+        return ids, w
 
     def check_status(self) -> int:
         return moe_check_status(self.handle)

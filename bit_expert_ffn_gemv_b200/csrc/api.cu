@@ -386,6 +386,16 @@ moe_status moe_debug_dequant(moe_handle* h, int32_t layer, int32_t expert, int32
                                            K, c.bits, out, static_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_debug_last_routing(moe_handle* h, int32_t T, int32_t* ids, float* w, void* stream) {
+    if (!h || T < 0 || T > h->cfg.max_tokens || (T > 0 && (!ids || !w))) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t n = (size_t)T * h->cfg.top_k;
+    if (cudaMemcpyAsync(ids, h->ids, n * sizeof(int32_t), cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return cuda_status(cudaMemcpyAsync(w, h->w, n * sizeof(float), cudaMemcpyDeviceToDevice, s));
+}
+
 moe_status moe_check_status(moe_handle* h) {
     if (!h) return MOE_ERR_INVALID_ARG;
     if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;

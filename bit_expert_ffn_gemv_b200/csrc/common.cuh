@@ -140,6 +140,69 @@ MOE_DEV void load_tile(const uint8_t* __restrict__ codes, const __half* __restri
     t.sc[3] = s.w;
 }
 
+// The calling lane's part of one super-tile already staged in shared memory:
+// `code` points at the super-tile's 256*BITS code bytes, `scale` at its 64
+// fp16 scales.
+template <int BITS>
+MOE_DEV void load_tile_smem(const uint8_t* code, const uint8_t* scale, int lane, TileRegs<BITS>& t) {
+    const uint4 w = *reinterpret_cast<const uint4*>(code + 16 * lane);
+    t.lo[0] = w.x;
+    t.lo[1] = w.y;
+    t.lo[2] = w.z;
+    t.lo[3] = w.w;
+    if (BITS == 3) {
+        const uint2 hv = *reinterpret_cast<const uint2*>(code + 512 + 8 * lane);
+        t.hi[0] = hv.x & 0xFFFFu;
+        t.hi[1] = hv.x >> 16;
+        t.hi[2] = hv.y & 0xFFFFu;
+        t.hi[3] = hv.y >> 16;
+    } else if (BITS == 4) {
+        const uint4 w2 = *reinterpret_cast<const uint4*>(code + 512 + 16 * lane);
+        t.hi[0] = w2.x;
+        t.hi[1] = w2.y;
+        t.hi[2] = w2.z;
+        t.hi[3] = w2.w;
+    } else {
+        t.hi[0] = t.hi[1] = t.hi[2] = t.hi[3] = 0;
+    }
+    const uint4 sv = *reinterpret_cast<const uint4*>(scale + 16 * (lane >> 2));
+    t.sc[0] = sv.x;
+    t.sc[1] = sv.y;
+    t.sc[2] = sv.z;
+    t.sc[3] = sv.w;
+}
+
+// ---------------------------------------------------------------- bulk copies (TMA, 1-D) and mbarriers
+MOE_DEV uint32_t smem_addr(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+
+MOE_DEV void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
+}
+// one arrival that also announces `bytes` of transactions still to land
+MOE_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+MOE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// global -> shared copy completed on `bar` (16-byte aligned, bytes % 16 == 0)
+MOE_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst)),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+}
+// order earlier generic-proxy accesses before later async-proxy (bulk copy) ones
+MOE_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+MOE_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
 MOE_DEV float silu(float g) { return g / (1.0f + __expf(-g)); }
 
 MOE_DEV float bf16_bits_to_float(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }

@@ -7,7 +7,7 @@
 // of weights per token-layer, a few microseconds of HBM time, so separate
 // launches per step would dominate.  Here one launch does everything.  CTAs
 // pull tasks from a global queue in dependency order:
-//   1. router rows (8 experts per CTA, fp32 logits with a rounding bound)
+//   1. router rows (8 experts per CTA, exact fp64 logits)
 //   2. shared-expert gate/up tiles (no routing dependency: overlap the router)
 //   3. certified top-k (8 tokens per CTA; the last one also buckets the pairs)
 //   4. shared-expert down tiles
@@ -21,7 +21,17 @@
 // on tasks claimed before it, so any grid size makes progress; every wait is
 // bounded and, if one gives up, sets the status word and an abort flag that
 // ends all other waits.  The last CTA to leave resets the counters.
+//
+// Every task that multiplies weights stages them in shared memory with 1-D
+// bulk copies (TMA, one elected thread, completion on an mbarrier): a gate/up
+// tile is 2 x 16 contiguous super-tiles, a down task 8 row-tiles x f/128
+// contiguous super-tiles, a router task 8 contiguous W_r rows.  The activation
+// rows (or h rows) it multiplies are staged the same way into padded rows, so
+// warps read their MMA operands from shared memory without bank conflicts and
+// hold no weights in registers.
 #include <cuda_runtime.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -30,17 +40,25 @@ namespace moe {
 
 constexpr int kDecWarps = 8;
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr uint32_t kSpinLimit = 1u << 21;  // x >= 100 ns per spin: >= 0.2 s
+constexpr uint32_t kSpinLimit = 1u << 21;  // spins of >= 32 ns (mostly 256 ns): >= 0.5 s
+constexpr int kPad = 8;                    // 16-bit elements of padding per staged row
+constexpr int kRouterRows = 4;             // router rows per task (two warps per row)
 
-// sync block (int32 words)
-enum { SY_HEAD = 0, SY_ROUTER = 1, SY_TOPK = 2, SY_BUCKET = 3, SY_EXIT = 4, SY_ABORT = 5, SY_FIXUP = 6,
-       SY_SLOTS = 16 };
+// sync block (int32 words); each scalar counter has a 128-byte line of its own
+enum { SY_HEAD = 0, SY_ROUTER = 32, SY_TOPK = 64, SY_BUCKET = 96, SY_EXIT = 128, SY_ABORT = 160, SY_FIXUP = 192,
+       SY_SLOTS = 224 };
 
 MOE_DEV int ld_acquire(const int* p) {
     int v;
     asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+MOE_DEV int ld_relaxed(const int* p) {
+    int v;
+    asm volatile("ld.relaxed.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+MOE_DEV void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 MOE_DEV int atom_add_acqrel(int* p, int v) {
     int old;
     asm volatile("atom.add.acq_rel.gpu.global.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
@@ -52,16 +70,23 @@ MOE_DEV void red_add_release(int* p, int v) {
 MOE_DEV void st_release(int* p, int v) { asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory"); }
 
 // Wait until *p >= target.  False if the wait gave up (timeout or abort).
+// Polls with relaxed loads and a growing sleep (hundreds of CTAs may wait on
+// one flag), then fences once so later reads see what the release published.
 MOE_DEV bool wait_geq(const int* p, int target, int* sync, uint32_t* status) {
+    uint32_t ns = 32;
     for (uint32_t it = 0;; ++it) {
-        if (ld_acquire(p) >= target) return true;
-        if (ld_acquire(sync + SY_ABORT)) return false;
+        if (ld_relaxed(p) >= target) {
+            fence_acq_rel_gpu();
+            return true;
+        }
+        if ((it & 7) == 7 && ld_relaxed(sync + SY_ABORT)) return false;
         if (it > kSpinLimit) {
             flag_status(status, kStatusTimeout);
             st_release(sync + SY_ABORT, 1);
             return false;
         }
-        __nanosleep(128);
+        __nanosleep(ns);
+        if (ns < 256) ns <<= 1;
     }
 }
 
@@ -88,6 +113,9 @@ struct DecodeArgs {
     __half* h;
     float* obuf;
     int* sync;
+    int red_bytes;  // shared memory: [red_bytes] reductions | 2 x [buf_bytes] staging buffers
+    int buf_bytes;  //   each buffer: [w_bytes] weights | activations
+    int w_bytes;
 };
 
 struct TaskMap {
@@ -97,7 +125,7 @@ struct TaskMap {
 
 MOE_DEV TaskMap task_map(const DecodeArgs& a) {
     TaskMap m;
-    m.nRt = (a.E + kDecWarps - 1) / kDecWarps;
+    m.nRt = (a.E + kRouterRows - 1) / kRouterRows;
     m.FT = a.f / 16;
     m.nSG = a.n_shared ? m.FT : 0;
     m.nTK = (a.T + kDecWarps - 1) / kDecWarps;
@@ -145,6 +173,8 @@ MOE_DEV int slot_tok(const DecodeArgs& a, const Slot& s, int i) { return s.share
 
 MOE_DEV float h_lo(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v & 0xFFFFu))); }
 MOE_DEV float h_hi(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v >> 16))); }
+MOE_DEV float bf_lo(uint32_t v) { return __uint_as_float(v << 16); }
+MOE_DEV float bf_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 
 MOE_DEV void acc_scaled(float (&acc)[4], const float (&t)[4], uint32_t sc) {
     const float slo = h_lo(sc), shi = h_hi(sc);
@@ -165,243 +195,324 @@ MOE_DEV bool better64d(double va, int ia, double vb, int ib) {
     return va > vb || (va == vb && ia < ib);
 }
 
-// ---------------------------------------------------------------- 1. router row
-// logits[t][e] for all T tokens; lane covers columns lane*4 + 128 j.  Each
-// lane's sum is a serial FMA chain of d/32 terms, then 5 shuffle levels, then
-// the bias: at most d/32 + 6 roundings.
-MOE_DEV void router_row(const DecodeArgs& a, int e, int lane) {
-    const uint16_t* row = a.wr + (int64_t)e * a.d;
-    const float b = a.bias ? a.bias[e] : 0.0f;
-    for (int t0 = 0; t0 < a.T; t0 += 8) {
-        float acc[8];
+// ---------------------------------------------------------------- 1. router rows (CTA)
+// logits64[t][e] = sum_i double(W_r[e,i]) * double(x[t,i]) + double(bias_e).
+// A task covers kRouterRows experts; warp w takes expert w/2 and half w%2 of
+// the columns (lane: columns half*d/2 + lane*8 + 256 j, j while < d/2).  A bf16 x bf16
+// product is exact in fp32, and it and every partial sum are exact in fp64
+// (their bits span far less than 53), so the logits are the exact fp64 values
+// of the plain definition in any summation order: ranking them is the exact
+// ranking.  part: [kRouterRows][2][8] doubles of shared memory.
+MOE_DEV void router_compute(const DecodeArgs& a, int e0, int nrow, int t0, int nt, const uint16_t* W,
+                            const uint16_t* xs, double* part, int warp, int lane) {
+    const int d = a.d, stride = d + kPad;
+    const int r = warp >> 1, half = warp & 1;
+    if (r < nrow) {
+        const uint16_t* wrow = W + r * d + half * (d / 2);
+        const uint16_t* xh = xs + half * (d / 2);
+        double acc[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-        for (int p = lane * 4; p < a.d; p += 128) {
-            const uint2 wv = *reinterpret_cast<const uint2*>(row + p);
-            const float w0 = __uint_as_float(wv.x << 16), w1 = __uint_as_float(wv.x & 0xFFFF0000u);
-            const float w2 = __uint_as_float(wv.y << 16), w3 = __uint_as_float(wv.y & 0xFFFF0000u);
+        for (int q = 0; q < 8; ++q) acc[q] = 0.0;
+        for (int c0 = lane * 8; c0 < d / 2; c0 += 256) {
+            const uint4 wv = *reinterpret_cast<const uint4*>(wrow + c0);
+            const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-                if (t0 + q < a.T) {
-                    const uint2 xv = *reinterpret_cast<const uint2*>(a.x + (int64_t)(t0 + q) * a.d + p);
-                    acc[q] = fmaf(w0, __uint_as_float(xv.x << 16), acc[q]);
-                    acc[q] = fmaf(w1, __uint_as_float(xv.x & 0xFFFF0000u), acc[q]);
-                    acc[q] = fmaf(w2, __uint_as_float(xv.y << 16), acc[q]);
-                    acc[q] = fmaf(w3, __uint_as_float(xv.y & 0xFFFF0000u), acc[q]);
+                if (q >= nt) break;
+                const uint4 xv = *reinterpret_cast<const uint4*>(xh + q * stride + c0);
+                const uint32_t x4[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    acc[q] += (double)(bf_lo(w4[u]) * bf_lo(x4[u]));  // exact product, exact sum
+                    acc[q] += (double)(bf_hi(w4[u]) * bf_hi(x4[u]));
                 }
             }
         }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-            float v = acc[q];
+            if (q >= nt) break;
+            double v = acc[q];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0 && t0 + q < a.T) a.logits[(int64_t)(t0 + q) * a.E + e] = v + b;
+            if (lane == 0) part[(r * 2 + half) * 8 + q] = v;
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < nrow * 8) {
+        const int rr = threadIdx.x >> 3, q = threadIdx.x & 7;
+        if (q < nt) {
+            const int e = e0 + rr;
+            const double b = a.bias ? (double)a.bias[e] : 0.0;
+            a.logits64[(int64_t)(t0 + q) * a.E + e] = part[(rr * 2) * 8 + q] + part[(rr * 2 + 1) * 8 + q] + b;
         }
     }
 }
 
-// ---------------------------------------------------------------- 3. certified top-k of one token
-MOE_DEV void topk_token(const DecodeArgs& a, int t, int lane, float* v) {
-    const int E = a.E, k = a.k, d = a.d;
-    const uint16_t* xt = a.x + (int64_t)t * d;
-    float ss = 0.f;
-    for (int i = lane; i < d; i += 32) {
-        const float xv = __uint_as_float((uint32_t)xt[i] << 16);
-        ss = fmaf(xv, xv, ss);
+// ---------------------------------------------------------------- 3. exact top-k of one token (warp)
+// Order (l desc, e asc), NaN ranked as -inf: a 64-bit key that orders like the
+// double (with -0 == +0), compared together with the expert index.
+MOE_DEV uint64_t order_key(double v) {
+    if (isnan(v)) v = -INFINITY;
+    v = v + 0.0;  // -0 -> +0
+    const uint64_t b = (uint64_t)__double_as_longlong(v);
+    return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+MOE_DEV bool key_better(uint64_t ka, int ia, uint64_t kb, int ib) { return ka > kb || (ka == kb && ia < ib); }
+
+// v: this warp's E-double shared-memory buffer.  For E <= 512 each lane sorts
+// its (up to) 16 elements e = lane + 32 j in registers with a bitonic network,
+// then every round is one warp argmax over the lanes' heads and the winning
+// lane shifts its list; larger E falls back to rescanning the winner's lane.
+// ids_s: the token's k ids are also left here (shared memory) for bucketing.
+constexpr int kTopkLane = 16;
+
+MOE_DEV void ce_desc(uint64_t& ka, int& ia, uint64_t& kb, int& ib, bool desc) {
+    const bool swap = desc ? key_better(kb, ib, ka, ia) : key_better(ka, ia, kb, ib);
+    if (swap) {
+        const uint64_t tk = ka;
+        ka = kb;
+        kb = tk;
+        const int ti = ia;
+        ia = ib;
+        ib = ti;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float xn = sqrtf(ss) * (1.0f + 1e-5f);
-    const float c = 2.0f * (float)(d / 32 + 6) * 5.9604645e-8f * (1.0f + 1e-5f);
-    const float* lg = a.logits + (int64_t)t * E;
-    auto bound = [&](int e) { return c * (a.wnorm[e] * xn + (a.bias ? fabsf(a.bias[e]) : 0.0f)); };
-    for (int e = lane; e < E; e += 32) v[e] = lg[e];  // this warp's shared-memory copy
+}
+
+MOE_DEV void topk_token(const DecodeArgs& a, int t, int lane, double* v, int* ids_s) {
+    const int E = a.E, k = a.k;
+    const double* lg = a.logits64 + (int64_t)t * E;
+#pragma unroll 8
+    for (int e = lane; e < E; e += 32) v[e] = lg[e];
     __syncwarp();
-
-    int sel[33];
-    uint32_t taken = 0;
-    const int kk = min(k + 1, E);
-    for (int r = 0; r < kk; ++r) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-        for (int j = 0, e = lane; e < E; ++j, e += 32) {
-            const float ve = v[e];
-            if (!((taken >> j) & 1u) && (bi == 0x7fffffff || better32(ve, e, bv, bi))) {
-                bv = ve;
-                bi = e;
-            }
-        }
+    int sel = -1;     // lane r < k keeps ids[r]
+    double lsel = 0;  //   and its logit
+    double top = 0;
+    if (E <= 32 * kTopkLane) {
+        uint64_t kk[kTopkLane];
+        int ii[kTopkLane];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (oi != 0x7fffffff && (bi == 0x7fffffff || better32(ov, oi, bv, bi))) {
-                bv = ov;
-                bi = oi;
-            }
+        for (int j = 0; j < kTopkLane; ++j) {
+            const int e = lane + 32 * j;
+            kk[j] = e < E ? order_key(v[e]) : 0ull;
+            ii[j] = e < E ? e : 0x7fffffff;
         }
-        sel[r] = bi;
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    }
-    bool ok = true;
-    for (int r = 0; r + 1 < k; ++r) {
-        const int p = sel[r], q = sel[r + 1];
-        if (!(lg[p] - bound(p) > lg[q] + bound(q))) ok = false;
-    }
-    const float lower_k = lg[sel[k - 1]] - bound(sel[k - 1]);
-    int ncand = 0;
-    for (int e = lane; e < E; e += 32)
-        if (!isnan(v[e]) && v[e] + bound(e) >= lower_k) ++ncand;
+        // bitonic sort, best first
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ncand += __shfl_xor_sync(0xffffffffu, ncand, o);
-    if (ncand != k || isnan(lower_k)) ok = false;
-
-    float wsel[32];
-    if (ok) {
-        for (int r = 0; r < k; ++r) wsel[r] = lg[sel[r]];
-    } else {
-        // fp64 logits of the candidates (exact sums of bf16 products), then exact ranking
-        double* l64 = a.logits64 + (int64_t)t * E;
-        const uint16_t* wr = a.wr;
-        for (int e = 0; e < E; ++e) {
-            const float ve = lg[e];
-            const bool cand = isnan(lower_k) || isnan(ve) || (ve + bound(e) >= lower_k);
-            double acc = 0.0;
-            if (cand) {
-                for (int i = lane; i < d; i += 32)
-                    acc = fma((double)__uint_as_float((uint32_t)wr[(int64_t)e * d + i] << 16),
-                              (double)__uint_as_float((uint32_t)xt[i] << 16), acc);
+        for (int size = 2; size <= kTopkLane; size <<= 1)
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-                acc += a.bias ? (double)a.bias[e] : 0.0;
-            }
-            if (lane == 0) l64[e] = cand ? acc : -INFINITY;
-        }
-        __syncwarp();
-        uint32_t tk = 0;
-        for (int r = 0; r < k; ++r) {
-            double bv = -INFINITY;
-            int bi = 0x7fffffff;
-            for (int j = 0, e = lane; e < E; ++j, e += 32) {
-                const double ve = l64[e];
-                if (!((tk >> j) & 1u) && (bi == 0x7fffffff || better64d(ve, e, bv, bi))) {
-                    bv = ve;
-                    bi = e;
+            for (int stride = size >> 1; stride > 0; stride >>= 1)
+#pragma unroll
+                for (int i = 0; i < kTopkLane; ++i) {
+                    const int jx = i ^ stride;
+                    if (jx > i) ce_desc(kk[i], ii[i], kk[jx], ii[jx], (i & size) == 0);
                 }
-            }
+        for (int r = 0; r < k; ++r) {
+            uint64_t bk = kk[0];
+            int bi = ii[0];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
-                const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const uint64_t ok = __shfl_xor_sync(0xffffffffu, bk, o);
                 const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (oi != 0x7fffffff && (bi == 0x7fffffff || better64d(ov, oi, bv, bi))) {
-                    bv = ov;
+                if (oi != 0x7fffffff && (bi == 0x7fffffff || key_better(ok, oi, bk, bi))) {
+                    bk = ok;
                     bi = oi;
                 }
             }
-            sel[r] = bi;
-            wsel[r] = (float)bv;
-            if ((bi & 31) == lane) tk |= 1u << (bi >> 5);
+            const double lv = v[bi];
+            if (lane == r) {
+                sel = bi;
+                lsel = lv;
+            }
+            if (r == 0) top = lv;
+            if ((bi & 31) == lane) {  // the winner's list moves up by one
+#pragma unroll
+                for (int j = 0; j + 1 < kTopkLane; ++j) {
+                    kk[j] = kk[j + 1];
+                    ii[j] = ii[j + 1];
+                }
+                kk[kTopkLane - 1] = 0ull;
+                ii[kTopkLane - 1] = 0x7fffffff;
+            }
         }
-        if (lane == 0) atomicAdd(a.sync + SY_FIXUP, 1);
+    } else {
+        uint32_t taken = 0;
+        auto local_best = [&](uint64_t& bk, int& bi) {
+            bk = 0;
+            bi = 0x7fffffff;
+            for (int j = 0, e = lane; e < E; ++j, e += 32) {
+                if ((taken >> j) & 1u) continue;
+                const uint64_t ke = order_key(v[e]);
+                if (bi == 0x7fffffff || key_better(ke, e, bk, bi)) {
+                    bk = ke;
+                    bi = e;
+                }
+            }
+        };
+        uint64_t mk;
+        int mi;
+        local_best(mk, mi);
+        for (int r = 0; r < k; ++r) {
+            uint64_t bk = mk;
+            int bi = mi;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const uint64_t ok = __shfl_xor_sync(0xffffffffu, bk, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (oi != 0x7fffffff && (bi == 0x7fffffff || key_better(ok, oi, bk, bi))) {
+                    bk = ok;
+                    bi = oi;
+                }
+            }
+            const double lv = v[bi];
+            if (lane == r) {
+                sel = bi;
+                lsel = lv;
+            }
+            if (r == 0) top = lv;
+            if ((bi & 31) == lane) {
+                taken |= 1u << (bi >> 5);
+                local_best(mk, mi);
+            }
+        }
     }
-    if (lane == 0) {
-        const float m = wsel[0];
-        float z = 0.f;
-        for (int r = 0; r < k; ++r) {
-            wsel[r] = expf(wsel[r] - m);
-            z += wsel[r];
-        }
-        const float inv = 1.0f / z;
-        for (int r = 0; r < k; ++r) {
-            a.ids[(int64_t)t * k + r] = sel[r];
-            a.w[(int64_t)t * k + r] = wsel[r] * inv;
-        }
+    // renormalised weights: softmax over the k selected logits (fp32)
+    const float ex = lane < k ? expf((float)(lsel - top)) : 0.0f;
+    float z = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane < k) {
+        a.ids[(int64_t)t * k + lane] = sel;
+        a.w[(int64_t)t * k + lane] = ex / z;
+        ids_s[lane] = sel;
     }
 }
 
-// ---------------------------------------------------------------- bucketing (one warp)
+// ---------------------------------------------------------------- bucketing (CTA)
 // Counting sort of the T*k pairs by expert, stable in token order.
-MOE_DEV void bucket_warp(const DecodeArgs& a, int lane, int* sm) {
+// sm: cnt[E] | off[E + 1] | ids[T*k] | wtot[3 * kDecWarps]
+MOE_DEV void bucket_cta(const DecodeArgs& a, int* sm, const int* ids_local) {
     const int E = a.E, k = a.k, n = a.T * a.k;
-    int* cnt = sm;          // [E]
-    int* off = sm + E;      // [E + 1]
-    for (int e = lane; e < E; e += 32) cnt[e] = 0;
-    __syncwarp();
-    for (int i = lane; i < n; i += 32) {
-        const int e = a.ids[i];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int* cnt = sm;
+    int* off = sm + E;
+    int* ids = off + E + 1;
+    int* wtot = ids + n;
+    for (int e = threadIdx.x; e < E; e += kDecThreads) cnt[e] = 0;
+    for (int i = threadIdx.x; i < n; i += kDecThreads) ids[i] = ids_local ? ids_local[i] : a.ids[i];
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kDecThreads) {
+        const int e = ids[i];
         if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
         else flag_status(a.status, kStatusBounds);
     }
-    __syncwarp();
-    int base = 0, nact = 0, mx = 0;
-    for (int e0 = 0; e0 < E; e0 += 32) {
+    __syncthreads();
+    // block-wide exclusive scan of cnt and of the active flags: warp w owns a
+    // contiguous chunk of experts, 32 per step
+    const int chunk = ((E + kDecWarps - 1) / kDecWarps + 31) & ~31;
+    const int e_begin = warp * chunk, e_end = min(E, e_begin + chunk);
+    int run = 0, runa = 0, mx = 0;
+    for (int e0 = e_begin; e0 < e_end; e0 += 32) {
         const int e = e0 + lane;
-        const int cv = e < E ? cnt[e] : 0;
+        const int cv = e < e_end ? cnt[e] : 0;
         int inc = cv;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int u = __shfl_up_sync(0xffffffffu, inc, o);
             if (lane >= o) inc += u;
         }
-        if (e < E) {
-            off[e] = base + inc - cv;
-            a.offsets[e] = base + inc - cv;
+        if (e < e_end) off[e] = run + inc - cv;  // chunk-local for now
+        run += __shfl_sync(0xffffffffu, inc, 31);
+        runa += __popc(__ballot_sync(0xffffffffu, cv > 0));
+        mx = max(mx, cv);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) {
+        wtot[warp] = run;
+        wtot[kDecWarps + warp] = runa;
+        wtot[2 * kDecWarps + warp] = mx;
+    }
+    __syncthreads();
+    int base = 0, abase = 0;
+    for (int w = 0; w < warp; ++w) {
+        base += wtot[w];
+        abase += wtot[kDecWarps + w];
+    }
+    for (int e0 = e_begin; e0 < e_end; e0 += 32) {
+        const int e = e0 + lane;
+        const int cv = e < e_end ? cnt[e] : 0;
+        if (e < e_end) {
+            off[e] += base;
+            a.offsets[e] = off[e];
         }
         const unsigned bal = __ballot_sync(0xffffffffu, cv > 0);
-        if (cv > 0) a.active[nact + __popc(bal & ((1u << lane) - 1u))] = e;
-        nact += __popc(bal);
-        int m = cv;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-        mx = max(mx, m);
-        base += __shfl_sync(0xffffffffu, inc, 31);
+        if (cv > 0) a.active[abase + __popc(bal & ((1u << lane) - 1u))] = e;
+        abase += __popc(bal);
     }
-    if (lane == 0) {
-        a.offsets[E] = base;
-        a.meta->n_active = nact;
-        a.meta->max_count = mx;
-        a.meta->n_fixup = ld_acquire(a.sync + SY_FIXUP);
-    }
-    __syncwarp();
-    for (int t = 0; t < a.T; ++t) {
-        if (lane < k) {
-            const int e = a.ids[(int64_t)t * k + lane];
-            if (e >= 0 && e < E) {
-                const int pos = off[e]++;
-                a.pairs[pos] = t * k + lane;
-                a.inv[(int64_t)t * k + lane] = pos;
-            } else {
-                a.inv[(int64_t)t * k + lane] = -1;
-            }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int tot = 0, nact = 0, big = 0;
+        for (int w = 0; w < kDecWarps; ++w) {
+            tot += wtot[w];
+            nact += wtot[kDecWarps + w];
+            big = max(big, wtot[2 * kDecWarps + w]);
         }
-        __syncwarp();
+        a.offsets[E] = tot;
+        a.meta->n_active = nact;
+        a.meta->max_count = big;
+        a.meta->n_fixup = 0;  // the fp64 logits need no re-ranking
+    }
+    __syncthreads();
+    // stable scatter by warp 0, token by token (a token's k experts are distinct)
+    if (warp == 0) {
+        for (int t = 0; t < a.T; ++t) {
+            if (lane < k) {
+                const int e = ids[t * k + lane];
+                if (e >= 0 && e < E) {
+                    const int pos = off[e]++;
+                    a.pairs[pos] = t * k + lane;
+                    a.inv[(int64_t)t * k + lane] = pos;
+                } else {
+                    a.inv[(int64_t)t * k + lane] = -1;
+                }
+            }
+            __syncwarp();
+        }
     }
 }
 
 // ---------------------------------------------------------------- gate/up tile (CTA)
-// h[hbase + i][jt*16 .. +15] = silu(g) * u for the slot's tokens i; the 8
-// warps split the input dimension into 128-wide super-tiles.
-template <int BITS, int NT>
-MOE_DEV void gateup_tile(const DecodeArgs& a, const Slot& s, int jt, float* red, int warp, int lane) {
+// h[hbase + i][jt*16 .. +15] = silu(g) * u for the slot's tokens i.  W holds
+// the 16-row tile's gate codes (KT super-tiles), gate scales, up codes, up
+// scales; with STAGE, xs holds the slot's activation rows (padded).  The 8
+// warps split the KT super-tiles of the input dimension.
+template <int BITS, int NT, bool STAGE>
+MOE_DEV void gateup_compute(const DecodeArgs& a, const Slot& s, int jt, float* red, const uint8_t* W,
+                            const uint16_t* xs, int warp, int lane) {
+    constexpr int TB = 256 * BITS;
     const int g = lane >> 2, c = lane & 3;
     const int KT = a.d / 128;
-    const int64_t mc = (int64_t)a.f * a.d * BITS / 8, ms = (int64_t)a.f * a.d / 32;
-    const uint8_t* cg = a.codes + (int64_t)s.expert * 3 * mc;
-    const uint8_t* cu = cg + mc;
-    const __half* sg = reinterpret_cast<const __half*>(a.scales) + (int64_t)s.expert * 3 * ms;
-    const __half* su = sg + ms;
+    const int xstride = a.d + kPad;
+    const uint8_t* gc = W;
+    const uint8_t* gs = gc + KT * TB;
+    const uint8_t* uc = gs + KT * 128;
+    const uint8_t* us = uc + KT * TB;
     const int nrem = s.count;
     int tok[NT];
+    if (!STAGE) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) tok[nt] = (nt * 8 + g < nrem) ? slot_tok(a, s, nt * 8 + g) : -1;
+        for (int nt = 0; nt < NT; ++nt) tok[nt] = (nt * 8 + g < nrem) ? slot_tok(a, s, nt * 8 + g) : -1;
+    }
     float accg[NT][4], accu[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) accg[nt][i] = accu[nt][i] = 0.f;
 
-    auto process = [&](const TileRegs<BITS>& tg, const TileRegs<BITS>& tu, int kt) {
+    for (int kt = warp; kt < KT; kt += kDecWarps) {
+        TileRegs<BITS> tg, tu;
+        load_tile_smem<BITS>(gc + kt * TB, gs + kt * 128, lane, tg);
+        load_tile_smem<BITS>(uc + kt * TB, us + kt * 128, lane, tu);
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {
             const int k0 = kt * 128 + kb * 32 + 2 * c;
@@ -409,8 +520,14 @@ MOE_DEV void gateup_tile(const DecodeArgs& a, const Slot& s, int jt, float* red,
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 b[nt][0] = b[nt][1] = b[nt][2] = b[nt][3] = 0u;
-                if (tok[nt] >= 0) {
-                    const uint16_t* xr = a.x + (int64_t)tok[nt] * a.d + k0;
+                const int i = nt * 8 + g;
+                const uint16_t* xr = nullptr;
+                if (STAGE) {
+                    if (i < nrem) xr = xs + i * xstride + k0;
+                } else if (tok[nt] >= 0) {
+                    xr = a.x + (int64_t)tok[nt] * a.d + k0;
+                }
+                if (xr) {
                     b[nt][0] = *reinterpret_cast<const uint32_t*>(xr);
                     b[nt][1] = *reinterpret_cast<const uint32_t*>(xr + 8);
                     b[nt][2] = *reinterpret_cast<const uint32_t*>(xr + 16);
@@ -418,44 +535,32 @@ MOE_DEV void gateup_tile(const DecodeArgs& a, const Slot& s, int jt, float* red,
                 }
             }
             {
-                uint32_t ag[8];
-                decode_block<false, BITS>(tg.lo[kb], tg.hi[kb], ag);
-                const uint32_t g0[4] = {ag[0], ag[1], ag[2], ag[3]}, g1[4] = {ag[4], ag[5], ag[6], ag[7]};
+                uint32_t q[8];
+                decode_block<false, BITS>(tg.lo[kb], tg.hi[kb], q);
+                const uint32_t q0[4] = {q[0], q[1], q[2], q[3]}, q1[4] = {q[4], q[5], q[6], q[7]};
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     if (nt * 8 >= nrem) break;
                     float t4[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_bf16(t4, g0, b[nt][0], b[nt][1], t4);
-                    mma_bf16(t4, g1, b[nt][2], b[nt][3], t4);
+                    mma_bf16(t4, q0, b[nt][0], b[nt][1], t4);
+                    mma_bf16(t4, q1, b[nt][2], b[nt][3], t4);
                     acc_scaled(accg[nt], t4, tg.sc[kb]);
                 }
             }
             {
-                uint32_t au[8];
-                decode_block<false, BITS>(tu.lo[kb], tu.hi[kb], au);
-                const uint32_t u0[4] = {au[0], au[1], au[2], au[3]}, u1[4] = {au[4], au[5], au[6], au[7]};
+                uint32_t q[8];
+                decode_block<false, BITS>(tu.lo[kb], tu.hi[kb], q);
+                const uint32_t q0[4] = {q[0], q[1], q[2], q[3]}, q1[4] = {q[4], q[5], q[6], q[7]};
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     if (nt * 8 >= nrem) break;
                     float t4[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_bf16(t4, u0, b[nt][0], b[nt][1], t4);
-                    mma_bf16(t4, u1, b[nt][2], b[nt][3], t4);
+                    mma_bf16(t4, q0, b[nt][0], b[nt][1], t4);
+                    mma_bf16(t4, q1, b[nt][2], b[nt][3], t4);
                     acc_scaled(accu[nt], t4, tu.sc[kb]);
                 }
             }
         }
-    };
-    for (int kt0 = warp; kt0 < KT; kt0 += 2 * kDecWarps) {
-        const int kt1 = kt0 + kDecWarps;
-        TileRegs<BITS> g0, u0, g1, u1;
-        load_tile<BITS>(cg, sg, (int64_t)jt * KT + kt0, lane, g0);
-        load_tile<BITS>(cu, su, (int64_t)jt * KT + kt0, lane, u0);
-        if (kt1 < KT) {
-            load_tile<BITS>(cg, sg, (int64_t)jt * KT + kt1, lane, g1);
-            load_tile<BITS>(cu, su, (int64_t)jt * KT + kt1, lane, u1);
-        }
-        process(g0, u0, kt0);
-        if (kt1 < KT) process(g1, u1, kt1);
     }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
@@ -470,14 +575,36 @@ MOE_DEV void gateup_tile(const DecodeArgs& a, const Slot& s, int jt, float* red,
         const int m = (ln >> 2) + 8 * (i >> 1);
         const int n = nt * 8 + 2 * (ln & 3) + (i & 1);
         if (n >= nrem) continue;
-        float gs = 0.f, us = 0.f;
+        float gsum = 0.f, usum = 0.f;
 #pragma unroll
         for (int w = 0; w < kDecWarps; ++w) {
-            gs += red[(((w * 2 + 0) * NT + nt) * 4 + i) * 32 + ln];
-            us += red[(((w * 2 + 1) * NT + nt) * 4 + i) * 32 + ln];
+            gsum += red[(((w * 2 + 0) * NT + nt) * 4 + i) * 32 + ln];
+            usum += red[(((w * 2 + 1) * NT + nt) * 4 + i) * 32 + ln];
         }
-        a.h[(int64_t)(s.hbase + n) * a.f + jt * 16 + m] = __float2half_rn(silu(gs) * us);
+        a.h[(int64_t)(s.hbase + n) * a.f + jt * 16 + m] = __float2half_rn(silu(gsum) * usum);
     }
+}
+
+// Thread 0: issue the bulk copies of one gate/up task (weights of tile jt of
+// the slot's expert; with STAGE its activation rows too).  Returns the bytes.
+template <int BITS, bool STAGE>
+MOE_DEV uint32_t gateup_issue(const DecodeArgs& a, const Slot& s, int jt, uint8_t* W, uint16_t* xs, uint64_t* bar) {
+    constexpr int TB = 256 * BITS;
+    const int KT = a.d / 128;
+    const int64_t mc = (int64_t)a.f * a.d * BITS / 8, msb = (int64_t)a.f * a.d / 16;  // bytes per matrix
+    const uint8_t* cbase = a.codes + (int64_t)s.expert * 3 * mc;
+    const uint8_t* sbase = reinterpret_cast<const uint8_t*>(a.scales) + (int64_t)s.expert * 3 * msb;
+    const uint32_t cb = KT * TB, sb = KT * 128;
+    const uint32_t xb = STAGE ? (uint32_t)s.count * a.d * 2 : 0;
+    mbar_arrive_expect_tx(bar, 2 * (cb + sb) + xb);
+    bulk_g2s(W, cbase + (int64_t)jt * cb, cb, bar);
+    bulk_g2s(W + cb, sbase + (int64_t)jt * sb, sb, bar);
+    bulk_g2s(W + cb + sb, cbase + mc + (int64_t)jt * cb, cb, bar);
+    bulk_g2s(W + 2 * cb + sb, sbase + msb + (int64_t)jt * sb, sb, bar);
+    if (STAGE)
+        for (int i = 0; i < s.count; ++i)
+            bulk_g2s(xs + i * (a.d + kPad), a.x + (int64_t)slot_tok(a, s, i) * a.d, a.d * 2, bar);
+    return 2 * (cb + sb) + xb;
 }
 
 // ---------------------------------------------------------------- combine of one (token, 16-row tile)
@@ -499,53 +626,54 @@ MOE_DEV void combine_tile(const DecodeArgs& a, int t, int rt, int lane) {
     }
 }
 
-// ---------------------------------------------------------------- down tile (warp)
-// o for the slot's tokens on output rows rt*16 .. +15, then per-token
-// completion counting; the warp that completes a (token, tile) combines it.
-template <int BITS, int NT>
-MOE_DEV void down_tile(const DecodeArgs& a, const Slot& s, int rt, int lane) {
+// ---------------------------------------------------------------- down tiles (CTA: one 16-row tile per warp)
+// o for the slot's tokens on output rows rt*16 .. +15 (rt = 8 rtg + warp),
+// then per-token completion counting; the warp that completes a (token, tile)
+// combines it.  W holds the CTA's 8 row-tiles x KTd super-tiles of codes, then
+// their scales; with STAGE, hs holds the slot's h rows (padded).
+template <int BITS, int NT, bool STAGE>
+MOE_DEV void down_compute(const DecodeArgs& a, const Slot& s, int rtg, int RT16, const uint8_t* W,
+                          const uint16_t* hs, int warp, int lane) {
+    constexpr int TB = 256 * BITS;
     const int g = lane >> 2, c = lane & 3;
-    const int KT = a.f / 128;
-    const int64_t mc = (int64_t)a.f * a.d * BITS / 8, ms = (int64_t)a.f * a.d / 32;
-    const uint8_t* cd = a.codes + (int64_t)s.expert * 3 * mc + 2 * mc;
-    const __half* sd = reinterpret_cast<const __half*>(a.scales) + (int64_t)s.expert * 3 * ms + 2 * ms;
+    const int KTd = a.f / 128;
+    const int rt = rtg * kDecWarps + warp;
+    if (rt >= RT16) return;
+    const int hstride = a.f + kPad;
+    const uint8_t* wc = W + warp * KTd * TB;
+    const uint8_t* ws = W + kDecWarps * KTd * TB + warp * KTd * 128;
     const int nrem = s.count;
     float acc[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-    constexpr int G = 3;  // super-tiles in flight per warp
-    for (int kt0 = 0; kt0 < KT; kt0 += G) {
-        TileRegs<BITS> td[G];
+    for (int kt = 0; kt < KTd; ++kt) {
+        TileRegs<BITS> td;
+        load_tile_smem<BITS>(wc + kt * TB, ws + kt * 128, lane, td);
 #pragma unroll
-        for (int q = 0; q < G; ++q)
-            if (kt0 + q < KT) load_tile<BITS>(cd, sd, (int64_t)rt * KT + kt0 + q, lane, td[q]);
+        for (int kb = 0; kb < 4; ++kb) {
+            uint32_t q[8];
+            decode_block<true, BITS>(td.lo[kb], td.hi[kb], q);
+            const int k0 = kt * 128 + kb * 32 + 2 * c;
+            const uint32_t a0[4] = {q[0], q[1], q[2], q[3]}, a1[4] = {q[4], q[5], q[6], q[7]};
 #pragma unroll
-        for (int q = 0; q < G; ++q) {
-            if (kt0 + q >= KT) break;
-#pragma unroll
-            for (int kb = 0; kb < 4; ++kb) {
-                uint32_t ad[8];
-                decode_block<true, BITS>(td[q].lo[kb], td[q].hi[kb], ad);
-                const int k0 = (kt0 + q) * 128 + kb * 32 + 2 * c;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    if (nt * 8 >= nrem) break;
-                    uint32_t b[4] = {0u, 0u, 0u, 0u};
-                    if (nt * 8 + g < nrem) {
-                        const __half* hr = a.h + (int64_t)(s.hbase + nt * 8 + g) * a.f + k0;
-                        b[0] = *reinterpret_cast<const uint32_t*>(hr);
-                        b[1] = *reinterpret_cast<const uint32_t*>(hr + 8);
-                        b[2] = *reinterpret_cast<const uint32_t*>(hr + 16);
-                        b[3] = *reinterpret_cast<const uint32_t*>(hr + 24);
-                    }
-                    const uint32_t a0[4] = {ad[0], ad[1], ad[2], ad[3]}, a1[4] = {ad[4], ad[5], ad[6], ad[7]};
-                    float t4[4] = {0.f, 0.f, 0.f, 0.f};
-                    mma_f16(t4, a0, b[0], b[1], t4);
-                    mma_f16(t4, a1, b[2], b[3], t4);
-                    acc_scaled(acc[nt], t4, td[q].sc[kb]);
+            for (int nt = 0; nt < NT; ++nt) {
+                if (nt * 8 >= nrem) break;
+                uint32_t b[4] = {0u, 0u, 0u, 0u};
+                if (nt * 8 + g < nrem) {
+                    const uint16_t* hr = STAGE ? hs + (nt * 8 + g) * hstride + k0
+                                               : reinterpret_cast<const uint16_t*>(a.h) +
+                                                     (int64_t)(s.hbase + nt * 8 + g) * a.f + k0;
+                    b[0] = *reinterpret_cast<const uint32_t*>(hr);
+                    b[1] = *reinterpret_cast<const uint32_t*>(hr + 8);
+                    b[2] = *reinterpret_cast<const uint32_t*>(hr + 16);
+                    b[3] = *reinterpret_cast<const uint32_t*>(hr + 24);
                 }
+                float t4[4] = {0.f, 0.f, 0.f, 0.f};
+                mma_f16(t4, a0, b[0], b[1], t4);
+                mma_f16(t4, a1, b[2], b[3], t4);
+                acc_scaled(acc[nt], t4, td.sc[kb]);
             }
         }
     }
@@ -579,84 +707,285 @@ MOE_DEV void down_tile(const DecodeArgs& a, const Slot& s, int rt, int lane) {
     }
 }
 
+// Thread 0: announce and issue the weight copies of a down task.
+template <int BITS>
+MOE_DEV uint32_t down_weight_bytes(const DecodeArgs& a, int rtg, int RT16) {
+    const int nrt = min(kDecWarps, RT16 - rtg * kDecWarps);
+    return (uint32_t)nrt * (a.f / 128) * (256 * BITS + 128);
+}
+template <int BITS>
+MOE_DEV void down_issue_weights(const DecodeArgs& a, const Slot& s, int rtg, int RT16, uint8_t* W, uint64_t* bar) {
+    constexpr int TB = 256 * BITS;
+    const int KTd = a.f / 128;
+    const int nrt = min(kDecWarps, RT16 - rtg * kDecWarps);
+    const int64_t mc = (int64_t)a.f * a.d * BITS / 8, msb = (int64_t)a.f * a.d / 16;
+    const uint8_t* cbase = a.codes + (int64_t)s.expert * 3 * mc + 2 * mc;
+    const uint8_t* sbase = reinterpret_cast<const uint8_t*>(a.scales) + (int64_t)s.expert * 3 * msb + 2 * msb;
+    const int64_t st0 = (int64_t)rtg * kDecWarps * KTd;
+    bulk_g2s(W, cbase + st0 * TB, (uint32_t)nrt * KTd * TB, bar);
+    bulk_g2s(W + kDecWarps * KTd * TB, sbase + st0 * 128, (uint32_t)nrt * KTd * 128, bar);
+}
+// All threads: copy the slot's h rows (written by other CTAs, published by the
+// release the caller acquired) into shared memory with padded rows.
+MOE_DEV void stage_h_rows(const DecodeArgs& a, const Slot& s, uint16_t* hs) {
+    const int vpr = a.f / 8, stride = a.f + kPad;
+    const uint16_t* h = reinterpret_cast<const uint16_t*>(a.h);
+    for (int v = threadIdx.x; v < s.count * vpr; v += kDecThreads) {
+        const int r = v / vpr, c = v - r * vpr;
+        *reinterpret_cast<uint4*>(hs + r * stride + 8 * c) =
+            *reinterpret_cast<const uint4*>(h + (int64_t)(s.hbase + r) * a.f + 8 * c);
+    }
+}
+
 // ---------------------------------------------------------------- the kernel
+// Wait for a buffer's staged copies (all threads).  On a timeout: flag it,
+// stop every other wait, give the copies in flight a second bounded wait, and
+// report failure.
+MOE_DEV bool stage_wait(uint64_t* bar, uint32_t& phase, const DecodeArgs& a) {
+    for (uint32_t it = 0; it <= kSpinLimit; ++it)
+        if (mbar_try_wait(bar, phase)) {
+            phase ^= 1u;
+            return true;
+        }
+    if (threadIdx.x == 0) {
+        flag_status(a.status, kStatusTimeout);
+        st_release(a.sync + SY_ABORT, 1);
+    }
+    for (uint32_t it = 0; it <= kSpinLimit; ++it)
+        if (mbar_try_wait(bar, phase)) {
+            phase ^= 1u;
+            break;
+        }
+    return false;
+}
+
+enum { K_ROUTER, K_SGU, K_TOPK, K_SDN, K_RGU, K_RDN };
+
+struct Task {
+    int kind, slot, sidx, idx;  // idx: jt (gate/up), rtg (down), router task or top-k task index
+};
+
+MOE_DEV Task decode_task(const TaskMap& m, int task) {
+    Task t;
+    t.slot = 0;
+    t.sidx = 0;
+    if (task < m.b1) {
+        t.kind = K_ROUTER;
+        t.idx = task;
+    } else if (task < m.b2) {
+        t.kind = K_SGU;
+        t.idx = task - m.b1;
+    } else if (task < m.b3) {
+        t.kind = K_TOPK;
+        t.idx = task - m.b2;
+    } else if (task < m.b4) {
+        t.kind = K_SDN;
+        t.idx = task - m.b3;
+    } else if (task < m.b5) {
+        t.kind = K_RGU;
+        t.sidx = (task - m.b4) / m.FT;
+        t.idx = (task - m.b4) % m.FT;
+    } else {
+        t.kind = K_RDN;
+        t.sidx = (task - m.b5) / m.nRTG;
+        t.idx = (task - m.b5) % m.nRTG;
+    }
+    return t;
+}
+
+// Per-CTA pipeline: buffer b holds the running task's staged operands while
+// the next task's weights land in buffer 1 - b.
+struct Pipe {
+    uint8_t* R[2];     // staging regions: [weights W | activations A]
+    int w_bytes;       // size of the W part
+    uint64_t* bar;     // [2]
+    uint32_t phase[2];
+};
+
+// Thread 0: issue the copies a task can start now (routed tasks need the
+// bucketing, which the caller has checked).  Returns 1 if copies were issued.
+template <int BITS, bool STAGE>
+MOE_DEV int issue_task(const DecodeArgs& a, const TaskMap& m, const Task& t, Pipe& p, int buf) {
+    uint8_t* W = p.R[buf];
+    uint16_t* A = reinterpret_cast<uint16_t*>(p.R[buf] + p.w_bytes);
+    uint64_t* bar = p.bar + buf;
+    fence_proxy_async_smem();  // earlier generic use of this buffer happens before the copies
+    switch (t.kind) {
+        case K_ROUTER: {
+            const int e0 = t.idx * kRouterRows, nrow = min(kRouterRows, a.E - e0), nt = min(8, a.T);
+            mbar_arrive_expect_tx(bar, (uint32_t)(nrow + nt) * a.d * 2);
+            bulk_g2s(W, a.wr + (int64_t)e0 * a.d, (uint32_t)nrow * a.d * 2, bar);
+            for (int q = 0; q < nt; ++q) bulk_g2s(A + q * (a.d + kPad), a.x + (int64_t)q * a.d, a.d * 2, bar);
+            return 1;
+        }
+        case K_SGU:
+            gateup_issue<BITS, STAGE>(a, make_slot(a, 0), t.idx, W, A, bar);
+            return 1;
+        case K_SDN:
+            mbar_arrive_expect_tx(bar, down_weight_bytes<BITS>(a, t.idx, m.RT16));
+            down_issue_weights<BITS>(a, make_slot(a, 0), t.idx, m.RT16, W, bar);
+            return 1;
+        case K_RGU:
+            if (t.sidx >= a.meta->n_active) return 0;
+            gateup_issue<BITS, STAGE>(a, make_slot(a, a.n_shared + t.sidx), t.idx, W, A, bar);
+            return 1;
+        case K_RDN:
+            if (t.sidx >= a.meta->n_active) return 0;
+            mbar_arrive_expect_tx(bar, down_weight_bytes<BITS>(a, t.idx, m.RT16));
+            down_issue_weights<BITS>(a, make_slot(a, a.n_shared + t.sidx), t.idx, m.RT16, W, bar);
+            return 1;
+        default:
+            return 0;
+    }
+}
+
 template <int BITS, int NT>
-__global__ void __launch_bounds__(kDecThreads, NT <= 2 ? 2 : 1) decode_kernel(const DecodeArgs a) {
-    extern __shared__ float smem[];
-    __shared__ int s_task, s_flag;
+__global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecodeArgs a) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ __align__(8) uint64_t bars[2];
+    __shared__ int s_claim, s_flag, s_issued[2];
+    constexpr bool STAGE = NT <= 2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const TaskMap m = task_map(a);
     int* sync = a.sync;
     int* slot_done = sync + SY_SLOTS;  // [1 + E] (slot index)
+    float* red = reinterpret_cast<float*>(smem_raw);  // gate/up partial sums, router partials
+    Pipe p;
+    p.R[0] = smem_raw + a.red_bytes;
+    p.R[1] = p.R[0] + a.buf_bytes;
+    p.w_bytes = a.w_bytes;
+    p.bar = bars;
+    p.phase[0] = p.phase[1] = 0;
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        fence_proxy_async_smem();
+    }
+    __syncthreads();
 
-    for (;;) {
-        if (threadIdx.x == 0) s_task = atomicAdd(sync + SY_HEAD, 1);
+    auto claim = [&]() {
+        if (threadIdx.x == 0) s_claim = ld_relaxed(sync + SY_ABORT) ? m.total : atomicAdd(sync + SY_HEAD, 1);
         __syncthreads();
-        const int task = s_task;
+        const int v = s_claim;
         __syncthreads();
-        if (task >= m.total) break;
-
-        if (task < m.b1) {  // router rows
-            const int e = task * kDecWarps + warp;
-            if (e < a.E) router_row(a, e, lane);
-            __threadfence();
-            __syncthreads();
-            if (threadIdx.x == 0) red_add_release(sync + SY_ROUTER, 1);
-        } else if (task < m.b2) {  // shared gate/up
-            const int jt = task - m.b1;
-            const Slot s = make_slot(a, 0);
-            gateup_tile<BITS, NT>(a, s, jt, smem, warp, lane);
-            __threadfence();
-            __syncthreads();
-            if (threadIdx.x == 0) red_add_release(slot_done + 0, 1);
-        } else if (task < m.b3) {  // top-k (+ bucketing by the last)
-            if (threadIdx.x == 0) s_flag = wait_geq(sync + SY_ROUTER, m.nRt, sync, a.status) ? 1 : 0;
-            __syncthreads();
-            const int t = (task - m.b2) * kDecWarps + warp;
-            if (s_flag && t < a.T) topk_token(a, t, lane, smem + warp * a.E);
-            __threadfence();
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                const int ntok = min(kDecWarps, a.T - (task - m.b2) * kDecWarps);
-                s_flag = (atom_add_acqrel(sync + SY_TOPK, ntok) + ntok == a.T) ? 1 : 0;
+        return v;
+    };
+    // Stage a task's operands into buffer `buf`.  blocking: wait for the
+    // bucketing if the task needs it; otherwise give up (return false) when it
+    // is not published yet.
+    auto prepare = [&](int task, int buf, bool blocking) {
+        const Task t = decode_task(m, task);
+        if (threadIdx.x == 0) {
+            int ok = 1;
+            if (t.kind == K_RGU || t.kind == K_RDN) {
+                if (blocking) ok = wait_geq(sync + SY_BUCKET, 1, sync, a.status) ? 1 : 0;
+                else if (ld_relaxed(sync + SY_BUCKET) >= 1) fence_acq_rel_gpu();
+                else ok = -1;
             }
-            __syncthreads();
-            if (s_flag) {
-                if (warp == 0) bucket_warp(a, lane, reinterpret_cast<int*>(smem));
+            s_flag = ok;
+            s_issued[buf] = ok == 1 ? issue_task<BITS, STAGE>(a, m, t, p, buf) : 0;
+        }
+        __syncthreads();
+        const bool done = s_flag != -1;
+        __syncthreads();
+        return done;
+    };
+    auto run = [&](int task, int buf) {
+        const Task t = decode_task(m, task);
+        uint8_t* W = p.R[buf];
+        uint16_t* A = reinterpret_cast<uint16_t*>(p.R[buf] + p.w_bytes);
+        const bool staged = s_issued[buf] != 0;
+        bool ok = true;
+        if (staged) ok = stage_wait(&p.bar[buf], p.phase[buf], a);
+        switch (t.kind) {
+            case K_ROUTER: {
+                const int e0 = t.idx * kRouterRows, nrow = min(kRouterRows, a.E - e0);
+                double* part = reinterpret_cast<double*>(red);
+                for (int t0 = 0; t0 < a.T; t0 += 8) {
+                    const int nt = min(8, a.T - t0);
+                    if (t0 > 0) {  // next chunk of activation rows
+                        __syncthreads();
+                        if (threadIdx.x == 0) {
+                            fence_proxy_async_smem();
+                            mbar_arrive_expect_tx(&p.bar[buf], (uint32_t)nt * a.d * 2);
+                            for (int q = 0; q < nt; ++q)
+                                bulk_g2s(A + q * (a.d + kPad), a.x + (int64_t)(t0 + q) * a.d, a.d * 2, &p.bar[buf]);
+                        }
+                        ok = stage_wait(&p.bar[buf], p.phase[buf], a) && ok;
+                    }
+                    if (ok) router_compute(a, e0, nrow, t0, nt, reinterpret_cast<const uint16_t*>(W), A, part, warp,
+                                           lane);
+                    __syncthreads();
+                }
                 __threadfence();
                 __syncthreads();
-                if (threadIdx.x == 0) st_release(sync + SY_BUCKET, 1);
+                if (threadIdx.x == 0) red_add_release(sync + SY_ROUTER, 1);
+                break;
             }
-        } else if (task < m.b4) {  // shared down
-            if (threadIdx.x == 0) s_flag = wait_geq(slot_done + 0, m.FT, sync, a.status) ? 1 : 0;
-            __syncthreads();
-            const int rt = (task - m.b3) * kDecWarps + warp;
-            if (threadIdx.x == 0 && s_flag) s_flag = wait_geq(sync + SY_BUCKET, 1, sync, a.status) ? 1 : 0;
-            __syncthreads();
-            if (s_flag && rt < m.RT16) down_tile<BITS, NT>(a, make_slot(a, 0), rt, lane);
-        } else if (task < m.b5) {  // routed gate/up
-            const int sidx = (task - m.b4) / m.FT, jt = (task - m.b4) % m.FT;
-            if (threadIdx.x == 0) s_flag = wait_geq(sync + SY_BUCKET, 1, sync, a.status) ? 1 : 0;
-            __syncthreads();
-            if (s_flag && sidx < a.meta->n_active) {
-                const Slot s = make_slot(a, a.n_shared + sidx);
-                gateup_tile<BITS, NT>(a, s, jt, smem, warp, lane);
+            case K_SGU:
+            case K_RGU: {
+                if (!staged) break;  // an expert slot beyond the active ones
+                const int slot = t.kind == K_SGU ? 0 : a.n_shared + t.sidx;
+                const Slot sl = make_slot(a, slot);
+                if (ok) gateup_compute<BITS, NT, STAGE>(a, sl, t.idx, red, W, A, warp, lane);
                 __threadfence();
                 __syncthreads();
-                if (threadIdx.x == 0) red_add_release(slot_done + a.n_shared + sidx, 1);
+                if (threadIdx.x == 0) red_add_release(slot_done + slot, 1);
+                break;
             }
-        } else {  // routed down
-            const int sidx = (task - m.b5) / m.nRTG, rtg = (task - m.b5) % m.nRTG;
-            if (threadIdx.x == 0) s_flag = wait_geq(sync + SY_BUCKET, 1, sync, a.status) ? 1 : 0;
-            __syncthreads();
-            if (s_flag && sidx < a.meta->n_active) {
-                if (threadIdx.x == 0) s_flag = wait_geq(slot_done + a.n_shared + sidx, m.FT, sync, a.status) ? 1 : 0;
+            case K_TOPK: {
+                if (threadIdx.x == 0) s_flag = wait_geq(sync + SY_ROUTER, m.nRt, sync, a.status) ? 1 : 0;
                 __syncthreads();
-                const int rt = rtg * kDecWarps + warp;
-                if (s_flag && rt < m.RT16) down_tile<BITS, NT>(a, make_slot(a, a.n_shared + sidx), rt, lane);
+                const int tk = t.idx * kDecWarps + warp;
+                int* ids_s = reinterpret_cast<int*>(red);  // [8 x k] ids of this CTA's tokens
+                if (s_flag && tk < a.T)
+                    topk_token(a, tk, lane, reinterpret_cast<double*>(p.R[buf]) + warp * a.E, ids_s + warp * a.k);
+                __threadfence();
+                __syncthreads();
+                if (threadIdx.x == 0) {
+                    const int ntok = min(kDecWarps, a.T - t.idx * kDecWarps);
+                    s_flag = (atom_add_acqrel(sync + SY_TOPK, ntok) + ntok == a.T) ? 1 : 0;
+                }
+                __syncthreads();
+                if (s_flag) {
+                    bucket_cta(a, reinterpret_cast<int*>(p.R[buf]), a.T <= kDecWarps ? ids_s : nullptr);
+                    __threadfence();
+                    __syncthreads();
+                    if (threadIdx.x == 0) st_release(sync + SY_BUCKET, 1);
+                }
+                break;
+            }
+            default: {  // K_SDN, K_RDN
+                if (!staged) break;
+                const int slot = t.kind == K_SDN ? 0 : a.n_shared + t.sidx;
+                if (threadIdx.x == 0) {
+                    s_flag = wait_geq(slot_done + slot, m.FT, sync, a.status) ? 1 : 0;
+                    if (s_flag && t.kind == K_SDN) s_flag = wait_geq(sync + SY_BUCKET, 1, sync, a.status) ? 1 : 0;
+                }
+                __syncthreads();
+                const Slot sl = make_slot(a, slot);
+                if (STAGE && s_flag) {
+                    stage_h_rows(a, sl, A);
+                    __syncthreads();
+                }
+                if (ok && s_flag) down_compute<BITS, NT, STAGE>(a, sl, t.idx, m.RT16, W, A, warp, lane);
+                break;
             }
         }
         __syncthreads();
+    };
+
+    int b = 0;
+    int cur = claim();
+    if (cur < m.total) prepare(cur, b, true);
+    while (cur < m.total) {
+        const int nxt = claim();
+        bool ready = false;
+        if (nxt < m.total) ready = prepare(nxt, b ^ 1, false);
+        run(cur, b);
+        if (nxt < m.total && !ready) prepare(nxt, b ^ 1, true);
+        cur = nxt;
+        b ^= 1;
     }
 
     // leave; the last CTA resets the counters for the next launch
@@ -672,26 +1001,56 @@ __global__ void __launch_bounds__(kDecThreads, NT <= 2 ? 2 : 1) decode_kernel(co
 }
 
 // ---------------------------------------------------------------- launcher
+// Shared memory: [gate/up reduction] [staged weights: max of router rows,
+// gate/up tile, down task] [activations: max of router x chunk, gate/up x rows,
+// down h rows, top-k buffers (8 warps x 2E floats), bucket (2E + 1 + T*k ints)].
+static size_t round128(size_t n) { return (n + 127) & ~size_t(127); }
+
+static size_t decode_smem(int BITS, int NT, int d, int f, int E, int T, int k, int* red_b, int* buf_b, int* w_b) {
+    const bool stage = NT <= 2;
+    const size_t tb = 256 * (size_t)BITS + 128;
+    const size_t red = round128(std::max((size_t)NT * kDecWarps * 2 * 4 * 32 * 4, (size_t)kRouterRows * 2 * 8 * 8));
+    size_t w = (size_t)kRouterRows * d * 2;
+    w = std::max(w, 2 * (size_t)(d / 128) * tb);
+    w = std::max(w, (size_t)kDecWarps * (f / 128) * tb);
+    w = round128(w);
+    const size_t rows = (size_t)std::min(T, 8 * NT);
+    size_t act = (size_t)std::min(T, 8) * (d + kPad) * 2;  // router chunk
+    if (stage) {
+        act = std::max(act, rows * (d + kPad) * 2);
+        act = std::max(act, rows * (f + kPad) * 2);
+    }
+    size_t buf = w + round128(act);
+    buf = std::max(buf, (size_t)kDecWarps * E * 8);                          // top-k
+    buf = std::max(buf, (size_t)(2 * E + 1 + T * k + 3 * kDecWarps) * 4);    // bucket
+    buf = round128(buf);
+    *red_b = (int)red;
+    *buf_b = (int)buf;
+    *w_b = (int)w;
+    return red + 2 * buf;
+}
+
 template <int BITS, int NT>
 static cudaError_t decode_bits_nt(const DecodeLaunch& L, cudaStream_t st) {
     auto kern = decode_kernel<BITS, NT>;
-    const int E = L.E;
-    // union: gate/up partials | per-warp top-k logits | bucket counters
-    const size_t smem = (size_t)max(max(NT * kDecWarps * 2 * 4 * 32, kDecWarps * E), 2 * E + 1) * sizeof(float);
-    static int blocks_per_sm[64] = {};  // per device, looked up once
+    int red_b = 0, buf_b = 0, w_b = 0;
+    const size_t smem = decode_smem(BITS, NT, L.d, L.f, L.E, L.T, L.k, &red_b, &buf_b, &w_b);
+    static int blocks_per_sm[64] = {};  // per device, looked up once per shared-memory size
+    static size_t smem_seen[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (smem > 48 * 1024) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    if (blocks_per_sm[dev] == 0) {
+    if (smem != smem_seen[dev]) {
+        if (smem > 48 * 1024) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
         int nb = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kDecThreads, smem);
         if (e != cudaSuccess) return e;
         blocks_per_sm[dev] = nb > 0 ? nb : 1;
+        smem_seen[dev] = smem;
     }
     int sms = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -725,6 +1084,9 @@ static cudaError_t decode_bits_nt(const DecodeLaunch& L, cudaStream_t st) {
     a.h = static_cast<__half*>(L.h);
     a.obuf = L.obuf;
     a.sync = L.sync;
+    a.red_bytes = red_b;
+    a.buf_bytes = buf_b;
+    a.w_bytes = w_b;
     const int grid = blocks_per_sm[dev] * sms;
     kern<<<grid, kDecThreads, smem, st>>>(a);
     return cudaGetLastError();

@@ -186,6 +186,13 @@ moe_status moe_debug_dequant(moe_handle* h, int32_t layer, int32_t expert, int32
                              void* stream);
 
 /*
+ * Debug: copy the routing the last moe_forward computed internally (rank-order
+ * ids [T x k] int32 and weights [T x k] fp32, device pointers) for its T
+ * tokens.  Enqueued on `stream` after that forward.  Errors: INVALID_ARG.
+ */
+moe_status moe_debug_last_routing(moe_handle* h, int32_t T, int32_t* ids, float* w, void* stream);
+
+/*
  * Synchronise the device and return the first device-side error recorded
  * since the last call (then clear it): MOE_ERR_TIMEOUT, MOE_ERR_BOUNDS or
  * MOE_OK; MOE_ERR_CUDA if the synchronisation itself failed.

@@ -64,6 +64,7 @@ def test_null_arguments(L):
     assert L.moe_load_layer(None, 0, None) == 1
     assert L.moe_debug_dequant(None, 0, 0, 0, None, None) == 1
     assert L.moe_check_status(None) == 1
+    assert L.moe_debug_last_routing(None, 1, None, None, None) == 1
     assert L.moe_get_stats(None, None) == 1
     assert L.moe_profile(None, 1) == 1
     assert L.moe_profile_read(None, None, None) == 1

@@ -36,7 +36,10 @@ def _check_layer(torch, h, shape, L, x_bits, layer=0, flags_extra=0, label=""):
     assert np.allclose(w.cpu().numpy(), w_ref, rtol=2e-6, atol=1e-7), label
     y16 = h.forward(layer, x, flags=flags_extra)
     y32 = h.forward(layer, x, flags=moe.MOE_OUT_FP32 | flags_extra)
+    ids_f, w_f = h.last_routing(T)
     torch.cuda.synchronize()
+    assert np.array_equal(ids_f.cpu().numpy(), ids_ref), f"{label}: forward's expert selection differs"
+    assert np.allclose(w_f.cpu().numpy(), w_ref, rtol=2e-6, atol=1e-7), label
     assert h.check_status() == 0
     g16, g32 = y_to_f64(y16), y_to_f64(y32)
     r16, m16, r32 = rel_l2(g16, y_ref), max_abs(g16, y_ref), rel_l2(g32, y_ref)
