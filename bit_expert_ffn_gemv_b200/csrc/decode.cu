@@ -259,22 +259,65 @@ MOE_DEV uint64_t order_key(double v) {
 }
 MOE_DEV bool key_better(uint64_t ka, int ia, uint64_t kb, int ib) { return ka > kb || (ka == kb && ia < ib); }
 
-// v: this warp's E-double shared-memory buffer.  For E <= 512 each lane sorts
-// its (up to) 16 elements e = lane + 32 j in registers with a bitonic network,
-// then every round is one warp argmax over the lanes' heads and the winning
-// lane shifts its list; larger E falls back to rescanning the winner's lane.
-// ids_s: the token's k ids are also left here (shared memory) for bucketing.
+// v: this warp's E-double shared-memory buffer.
+// Fast path (E <= 512, k <= 15): 32-bit keys = an order-preserving image of
+// fp32(l) with the low 10 bits replaced by (1023 - e).  A strictly larger key
+// prefix means a strictly larger logit, so the exact top-k lies among the
+// elements whose prefix is >= the k-th key's prefix.  Each lane sorts its 16
+// keys (bitonic, min/max), a 5-level butterfly merges the sorted lists so every
+// lane holds the global top 16, and those candidates are ranked exactly by
+// (fp64 logit desc, index asc) with pairwise comparisons.  If the candidates do
+// not fit in 16 (ties in the key prefix) or E, k are larger, a slow exact scan
+// runs instead.  ids_s: the token's k ids are also left here for bucketing.
 constexpr int kTopkLane = 16;
 
-MOE_DEV void ce_desc(uint64_t& ka, int& ia, uint64_t& kb, int& ib, bool desc) {
-    const bool swap = desc ? key_better(kb, ib, ka, ia) : key_better(ka, ia, kb, ib);
-    if (swap) {
-        const uint64_t tk = ka;
-        ka = kb;
-        kb = tk;
-        const int ti = ia;
-        ia = ib;
-        ib = ti;
+MOE_DEV uint32_t key32(double v, int e) {
+    float f = (float)(isnan(v) ? -INFINITY : v);
+    f = f + 0.0f;  // -0 -> +0
+    const uint32_t b = __float_as_uint(f);
+    const uint32_t o = (b >> 31) ? ~b : (b | 0x80000000u);
+    return (o & 0xFFFFFC00u) | (uint32_t)(1023 - e);
+}
+
+MOE_DEV void topk_exact_scan(const double* v, int E, int k, int lane, int& sel, double& lsel, double& top) {
+    uint32_t taken = 0;
+    auto local_best = [&](uint64_t& bk, int& bi) {
+        bk = 0;
+        bi = 0x7fffffff;
+        for (int j = 0, e = lane; e < E; ++j, e += 32) {
+            if ((taken >> j) & 1u) continue;
+            const uint64_t ke = order_key(v[e]);
+            if (bi == 0x7fffffff || key_better(ke, e, bk, bi)) {
+                bk = ke;
+                bi = e;
+            }
+        }
+    };
+    uint64_t mk;
+    int mi;
+    local_best(mk, mi);
+    for (int r = 0; r < k; ++r) {
+        uint64_t bk = mk;
+        int bi = mi;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const uint64_t ok = __shfl_xor_sync(0xffffffffu, bk, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (oi != 0x7fffffff && (bi == 0x7fffffff || key_better(ok, oi, bk, bi))) {
+                bk = ok;
+                bi = oi;
+            }
+        }
+        const double lv = v[bi];
+        if (lane == r) {
+            sel = bi;
+            lsel = lv;
+        }
+        if (r == 0) top = lv;
+        if ((bi & 31) == lane) {
+            taken |= 1u << (bi >> 5);
+            local_best(mk, mi);
+        }
     }
 }
 
@@ -287,16 +330,15 @@ MOE_DEV void topk_token(const DecodeArgs& a, int t, int lane, double* v, int* id
     int sel = -1;     // lane r < k keeps ids[r]
     double lsel = 0;  //   and its logit
     double top = 0;
-    if (E <= 32 * kTopkLane) {
-        uint64_t kk[kTopkLane];
-        int ii[kTopkLane];
+    bool done = false;
+    if (E <= 32 * kTopkLane && k < kTopkLane) {
+        uint32_t kk[kTopkLane];
 #pragma unroll
         for (int j = 0; j < kTopkLane; ++j) {
             const int e = lane + 32 * j;
-            kk[j] = e < E ? order_key(v[e]) : 0ull;
-            ii[j] = e < E ? e : 0x7fffffff;
+            kk[j] = e < E ? key32(v[e], e) : 0u;
         }
-        // bitonic sort, best first
+        // sort descending (bitonic network on registers)
 #pragma unroll
         for (int size = 2; size <= kTopkLane; size <<= 1)
 #pragma unroll
@@ -304,77 +346,67 @@ MOE_DEV void topk_token(const DecodeArgs& a, int t, int lane, double* v, int* id
 #pragma unroll
                 for (int i = 0; i < kTopkLane; ++i) {
                     const int jx = i ^ stride;
-                    if (jx > i) ce_desc(kk[i], ii[i], kk[jx], ii[jx], (i & size) == 0);
+                    if (jx > i) {
+                        const uint32_t lo = min(kk[i], kk[jx]), hi = max(kk[i], kk[jx]);
+                        const bool desc = (i & size) == 0;
+                        kk[i] = desc ? hi : lo;
+                        kk[jx] = desc ? lo : hi;
+                    }
                 }
-        for (int r = 0; r < k; ++r) {
-            uint64_t bk = kk[0];
-            int bi = ii[0];
+        // butterfly: merge with the partner's sorted list, keep the top 16, re-sort
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const uint64_t ok = __shfl_xor_sync(0xffffffffu, bk, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (oi != 0x7fffffff && (bi == 0x7fffffff || key_better(ok, oi, bk, bi))) {
-                    bk = ok;
-                    bi = oi;
-                }
-            }
-            const double lv = v[bi];
-            if (lane == r) {
-                sel = bi;
-                lsel = lv;
-            }
-            if (r == 0) top = lv;
-            if ((bi & 31) == lane) {  // the winner's list moves up by one
+        for (int o = 1; o < 32; o <<= 1) {
 #pragma unroll
-                for (int j = 0; j + 1 < kTopkLane; ++j) {
-                    kk[j] = kk[j + 1];
-                    ii[j] = ii[j + 1];
-                }
-                kk[kTopkLane - 1] = 0ull;
-                ii[kTopkLane - 1] = 0x7fffffff;
+            for (int j = 0; j < kTopkLane; ++j) {
+                const uint32_t other = __shfl_xor_sync(0xffffffffu, kk[kTopkLane - 1 - j], o);
+                kk[j] = max(kk[j], other);  // bitonic: top 16 of the two lists
             }
+#pragma unroll
+            for (int stride = kTopkLane >> 1; stride > 0; stride >>= 1)
+#pragma unroll
+                for (int i = 0; i < kTopkLane; ++i) {
+                    const int jx = i ^ stride;
+                    if (jx > i) {
+                        const uint32_t lo = min(kk[i], kk[jx]), hi = max(kk[i], kk[jx]);
+                        kk[i] = hi;
+                        kk[jx] = lo;
+                    }
+                }
         }
-    } else {
-        uint32_t taken = 0;
-        auto local_best = [&](uint64_t& bk, int& bi) {
-            bk = 0;
-            bi = 0x7fffffff;
-            for (int j = 0, e = lane; e < E; ++j, e += 32) {
-                if ((taken >> j) & 1u) continue;
-                const uint64_t ke = order_key(v[e]);
-                if (bi == 0x7fffffff || key_better(ke, e, bk, bi)) {
-                    bk = ke;
-                    bi = e;
-                }
-            }
-        };
-        uint64_t mk;
-        int mi;
-        local_best(mk, mi);
-        for (int r = 0; r < k; ++r) {
-            uint64_t bk = mk;
-            int bi = mi;
+        // candidates: key prefix >= the k-th key's prefix (a sorted prefix of kk)
+        const uint32_t pk = kk[k - 1] & 0xFFFFFC00u;
+        if ((kk[kTopkLane - 1] & 0xFFFFFC00u) < pk) {
+            int m = 0;
+            uint32_t mine = 0;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const uint64_t ok = __shfl_xor_sync(0xffffffffu, bk, o);
-                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                if (oi != 0x7fffffff && (bi == 0x7fffffff || key_better(ok, oi, bk, bi))) {
-                    bk = ok;
-                    bi = oi;
+            for (int j = 0; j < kTopkLane; ++j) {
+                if ((kk[j] & 0xFFFFFC00u) >= pk) ++m;
+                if (j == lane) mine = kk[j];
+            }
+            const int my_e = 1023 - (int)(mine & 0x3FFu);
+            const double my_v = lane < m ? v[my_e] : 0.0;
+            const uint64_t my_k = order_key(my_v);
+            int rank = 0;
+            for (int j = 0; j < m; ++j) {
+                const uint64_t ok = __shfl_sync(0xffffffffu, my_k, j);
+                const int oe = __shfl_sync(0xffffffffu, my_e, j);
+                if (j != lane && key_better(ok, oe, my_k, my_e)) ++rank;
+            }
+            // lane r < k fetches the candidate of rank r
+            for (int j = 0; j < m; ++j) {
+                const int rj = __shfl_sync(0xffffffffu, rank, j);
+                const int ej = __shfl_sync(0xffffffffu, my_e, j);
+                const double vj = __shfl_sync(0xffffffffu, my_v, j);
+                if (rj == lane) {
+                    sel = ej;
+                    lsel = vj;
                 }
+                if (rj == 0) top = vj;
             }
-            const double lv = v[bi];
-            if (lane == r) {
-                sel = bi;
-                lsel = lv;
-            }
-            if (r == 0) top = lv;
-            if ((bi & 31) == lane) {
-                taken |= 1u << (bi >> 5);
-                local_best(mk, mi);
-            }
+            done = true;
         }
     }
+    if (!done) topk_exact_scan(v, E, k, lane, sel, lsel, top);
     // renormalised weights: softmax over the k selected logits (fp32)
     const float ex = lane < k ? expf((float)(lsel - top)) : 0.0f;
     float z = ex;
