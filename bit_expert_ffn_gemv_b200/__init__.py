@@ -19,7 +19,8 @@ import threading
 __all__ = ["MoeError", "MoeConfig", "MoeLayerWeights", "MoeLayer", "lib", "library_path", "MOE_OUT_FP32",
            "MOE_ACCUMULATE", "MOE_FORCE_GEMV", "MOE_FORCE_GEMM", "MOE_FORCE_UNFUSED", "STATUS", "moe_layer_init", "moe_load_layer",
            "moe_route", "moe_route_noalloc", "moe_forward", "moe_forward_host", "moe_destroy", "moe_debug_dequant", "moe_debug_last_routing", "moe_check_status",
-           "moe_get_stats", "moe_status_string", "moe_profile", "moe_profile_read", "moe_kernel_name", "MoeStats"]
+           "moe_get_stats", "moe_status_string", "moe_profile", "moe_profile_read", "moe_kernel_name", "MoeStats",
+           "moe_debug_router_logits", "moe_router_error_depth"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libmoe.so")
@@ -30,7 +31,7 @@ MOE_FORCE_GEMV = 0x4
 MOE_FORCE_GEMM = 0x8
 MOE_FORCE_UNFUSED = 0x10
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_CUDA", 3: "MOE_ERR_OOM", 4: "MOE_ERR_NOT_LOADED",
-          5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_BOUNDS"}
+          5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_BOUNDS", 7: "MOE_ERR_RANGE"}
 
 
 class MoeError(RuntimeError):
@@ -50,7 +51,7 @@ class MoeStats(ctypes.Structure):
                 ("launches", ctypes.c_int64)]
 
 
-MOE_KERNEL_COUNT = 10
+MOE_KERNEL_COUNT = 12
 
 
 class MoeLayerWeights(ctypes.Structure):
@@ -100,6 +101,10 @@ def lib() -> ctypes.CDLL:
             L.moe_kernel_name.argtypes = [i32]
             L.moe_route_noalloc.restype = st
             L.moe_route_noalloc.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp]
+            L.moe_debug_router_logits.restype = st
+            L.moe_debug_router_logits.argtypes = [vp, i32, vp, i32, vp, i32, vp]
+            L.moe_router_error_depth.restype = ctypes.c_float
+            L.moe_router_error_depth.argtypes = [i32, i32]
             L.moe_status_string.restype = ctypes.c_char_p
             L.moe_status_string.argtypes = [st]
             _lib = L
@@ -158,6 +163,16 @@ def moe_debug_dequant(handle: int, layer: int, expert: int, mat: int, out_ptr: i
 
 def moe_debug_last_routing(handle: int, T: int, ids_ptr: int, w_ptr: int, stream: int) -> None:
     _check(lib().moe_debug_last_routing(handle, T, ids_ptr, w_ptr, stream), "moe_debug_last_routing")
+
+
+def moe_debug_router_logits(handle: int, layer: int, x_ptr: int, T: int, logits_ptr: int, tensor_cores: bool,
+                            stream: int) -> None:
+    _check(lib().moe_debug_router_logits(handle, layer, x_ptr, T, logits_ptr, 1 if tensor_cores else 0, stream),
+           "moe_debug_router_logits")
+
+
+def moe_router_error_depth(d: int, tensor_cores: bool) -> float:
+    return float(lib().moe_router_error_depth(d, 1 if tensor_cores else 0))
 
 
 def moe_check_status(handle: int) -> int:
@@ -254,6 +269,14 @@ class MoeLayer:
         w = torch.empty((T, self.cfg.top_k), dtype=torch.float32, device="cuda")
         moe_debug_last_routing(self.handle, T, ids.data_ptr(), w.data_ptr(), _stream_ptr(stream))
         return ids, w
+
+    def router_logits(self, layer, x, tensor_cores=True, stream=None):
+        """fp32 logits [T x E] from one of the two router kernels (for bound checks)."""
+        import torch
+        out = torch.empty((x.shape[0], self.cfg.n_experts), dtype=torch.float32, device=x.device)
+        moe_debug_router_logits(self.handle, layer, x.data_ptr(), x.shape[0], out.data_ptr(), tensor_cores,
+                                _stream_ptr(stream))
+        return out
 
     def check_status(self) -> int:
         return moe_check_status(self.handle)

@@ -15,7 +15,7 @@
 
 static const char* const kKernelNames[MOE_KERNEL_COUNT] = {
     "router_logits", "topk", "bucket", "gemv_gateup", "gemv_down", "combine", "gemm_gateup", "gemm_down",
-    "router_gemm", "decode_fused"};
+    "router_gemm", "decode_fused", "to_f16", "tile_list"};
 
 struct moe_layer_state {
     const uint8_t* codes = nullptr;
@@ -48,6 +48,8 @@ struct moe_handle {
     int* sync = nullptr;
     void* x_stage = nullptr;
     void* y_stage = nullptr;
+    void* xh = nullptr;        // fp16 copy of x for the tensor-core path
+    int32_t* tiles = nullptr;  // gate/up and down tile lists
     // launch accounting and optional per-kernel event timing
     int64_t launches = 0;
     bool prof_on = false;
@@ -95,8 +97,14 @@ moe_status check_layer(moe_handle* h, int32_t layer) {
     return MOE_OK;
 }
 
+// Large token counts take the tensor-core router (bf16 tcgen05 GEMM).
+bool use_tensor_cores(int32_t T, uint32_t flags) {
+    if (flags & (MOE_FORCE_GEMV | MOE_FORCE_UNFUSED)) return false;
+    return T > moe::kDecodeMaxTokens || (flags & MOE_FORCE_GEMM);
+}
+
 // router -> certified top-k; writes ids / w (device)
-moe_status do_route(moe_handle* h, int32_t layer, const void* x, int32_t T, int32_t* ids, float* w,
+moe_status do_route(moe_handle* h, int32_t layer, const void* x, int32_t T, int32_t* ids, float* w, bool tc,
                     cudaStream_t s) {
     const moe_layer_state& L = h->layers[layer];
     cudaError_t e = cudaMemsetAsync(h->meta, 0, sizeof(moe::Meta), s);
@@ -114,7 +122,12 @@ moe_status do_route(moe_handle* h, int32_t layer, const void* x, int32_t T, int3
     ra.ids = ids;
     ra.w = w;
     ra.meta = h->meta;
-    e = run(h, MOE_K_ROUTER_LOGITS, s, [&] { return moe::launch_router_logits(ra, s); });
+    if (tc) {
+        ra.depth = moe::router_gemm_depth(ra.d);
+        e = run(h, MOE_K_ROUTER_GEMM, s, [&] { return moe::launch_router_gemm(ra, h->status, s); });
+    } else {
+        e = run(h, MOE_K_ROUTER_LOGITS, s, [&] { return moe::launch_router_logits(ra, s); });
+    }
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     return cuda_status(run(h, MOE_K_TOPK, s, [&] { return moe::launch_topk(ra, s); }));
 }
@@ -161,7 +174,14 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     const moe_config& c = h->cfg;
     if (T <= moe::kDecodeMaxTokens && !(flags & (MOE_FORCE_GEMM | MOE_FORCE_UNFUSED)))
         return do_decode(h, layer, x, T, y, flags, s);
-    moe_status st = do_route(h, layer, x, T, h->ids, h->w, s);
+    const bool tc = use_tensor_cores(T, flags);
+    cudaError_t e;
+    if (tc) {
+        e = run(h, MOE_K_TO_F16, s,
+                [&] { return moe::launch_to_f16(x, h->xh, (int64_t)T * c.d, h->status, s); });
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    moe_status st = do_route(h, layer, x, T, h->ids, h->w, tc, s);
     if (st != MOE_OK) return st;
     moe::BucketArgs ba;
     ba.ids = h->ids;
@@ -174,7 +194,7 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     ba.active = h->active;
     ba.meta = h->meta;
     ba.status = h->status;
-    cudaError_t e = run(h, MOE_K_BUCKET, s, [&] { return moe::launch_bucket(ba, s); });
+    e = run(h, MOE_K_BUCKET, s, [&] { return moe::launch_bucket(ba, s); });
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 
     const moe_layer_state& L = h->layers[layer];
@@ -196,10 +216,20 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     ea.h = h->h;
     ea.obuf = h->obuf;
     ea.status = h->status;
-    e = run(h, MOE_K_GEMV_GATEUP, s, [&] { return moe::launch_gemv_gateup(ea, s); });
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
-    e = run(h, MOE_K_GEMV_DOWN, s, [&] { return moe::launch_gemv_down(ea, s); });
-    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (tc) {
+        e = run(h, MOE_K_TILE_LIST, s, [&] { return moe::launch_build_tiles(ea, h->tiles, s); });
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        e = run(h, MOE_K_GEMM_GATEUP, s, [&] { return moe::launch_gemm_gateup(ea, h->xh, h->tiles, s); });
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        // the fp16 partial outputs reuse the fp32 partial-output buffer
+        e = run(h, MOE_K_GEMM_DOWN, s, [&] { return moe::launch_gemm_down(ea, h->w, h->obuf, h->tiles, s); });
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    } else {
+        e = run(h, MOE_K_GEMV_GATEUP, s, [&] { return moe::launch_gemv_gateup(ea, s); });
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        e = run(h, MOE_K_GEMV_DOWN, s, [&] { return moe::launch_gemv_down(ea, s); });
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
+    }
 
     moe::CombineArgs ca;
     ca.T = T;
@@ -212,6 +242,7 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     ca.y = y;
     ca.out_fp32 = (flags & MOE_OUT_FP32) != 0;
     ca.accumulate = (flags & MOE_ACCUMULATE) != 0;
+    if (tc) return cuda_status(run(h, MOE_K_COMBINE, s, [&] { return moe::launch_combine_f16(ca, h->obuf, s); }));
     return cuda_status(run(h, MOE_K_COMBINE, s, [&] { return moe::launch_combine(ca, s); }));
 }
 
@@ -271,6 +302,8 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     const size_t o_ys = take(sizeof(float) * T * (size_t)c.d);
     const size_t o_norms = take(sizeof(float) * E * (size_t)c.n_layers);
     const size_t o_l64 = take(sizeof(double) * std::min<size_t>(T, moe::kDecodeMaxTokens) * E);
+    const size_t o_xh = take(sizeof(uint16_t) * T * (size_t)c.d);
+    const size_t o_tiles = take(sizeof(int32_t) * moe::tile_list_words(c.n_experts));
     const size_t o_sync =
         take(sizeof(int) * moe::decode_sync_words(std::min(c.max_tokens, moe::kDecodeMaxTokens), c.n_experts, c.d));
     h->arena_bytes = off;
@@ -296,6 +329,8 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     h->sync = reinterpret_cast<int*>(base + o_sync);
     h->x_stage = base + o_xs;
     h->y_stage = base + o_ys;
+    h->xh = base + o_xh;
+    h->tiles = reinterpret_cast<int32_t*>(base + o_tiles);
     for (int l = 0; l < c.n_layers; ++l) h->layers[l].wnorm = reinterpret_cast<float*>(base + o_norms) + E * l;
     if (cudaMemset(h->arena, 0, h->arena_bytes) != cudaSuccess) {
         cudaFree(h->arena);
@@ -332,7 +367,38 @@ moe_status moe_route(moe_handle* h, int32_t layer, const void* x, int32_t T, int
     if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x || !ids || !w || !aligned16(x) || !aligned16(ids) || !aligned16(w)) return MOE_ERR_INVALID_ARG;
-    return do_route(h, layer, x, T, ids, w, static_cast<cudaStream_t>(stream));
+    return do_route(h, layer, x, T, ids, w, use_tensor_cores(T, 0), static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_debug_router_logits(moe_handle* h, int32_t layer, const void* x, int32_t T, float* logits,
+                                   int32_t tensor_cores, void* stream) {
+    moe_status st = check_layer(h, layer);
+    if (st != MOE_OK) return st;
+    if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !logits || !aligned16(x) || !aligned16(logits)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const moe_layer_state& L = h->layers[layer];
+    moe::RouteArgs ra;
+    ra.x = x;
+    ra.T = T;
+    ra.d = h->cfg.d;
+    ra.E = h->cfg.n_experts;
+    ra.k = h->cfg.top_k;
+    ra.wr = L.router_w;
+    ra.bias = L.bias;
+    ra.wnorm = L.wnorm;
+    ra.logits = logits;
+    ra.ids = nullptr;
+    ra.w = nullptr;
+    ra.meta = h->meta;
+    cudaError_t e = tensor_cores ? moe::launch_router_gemm(ra, h->status, s) : moe::launch_router_logits(ra, s);
+    return cuda_status(e);
+}
+
+float moe_router_error_depth(int32_t d, int32_t tensor_cores) {
+    if (d <= 0) return 0.0f;
+    return tensor_cores ? moe::router_gemm_depth(d) : (float)(d / 32 + 6);
 }
 
 moe_status moe_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, void* y, uint32_t flags,
@@ -404,6 +470,7 @@ moe_status moe_check_status(moe_handle* h) {
     if (cudaMemset(h->status, 0, sizeof(uint32_t)) != cudaSuccess) return MOE_ERR_CUDA;
     if (v & moe::kStatusTimeout) return MOE_ERR_TIMEOUT;
     if (v & moe::kStatusBounds) return MOE_ERR_BOUNDS;
+    if (v & moe::kStatusRange) return MOE_ERR_RANGE;
     return MOE_OK;
 }
 
@@ -461,6 +528,7 @@ const char* moe_status_string(moe_status s) {
         case MOE_ERR_NOT_LOADED: return "layer weights not loaded";
         case MOE_ERR_TIMEOUT: return "a bounded device-side wait gave up";
         case MOE_ERR_BOUNDS: return "a device-side index was out of range";
+        case MOE_ERR_RANGE: return "a value left the range of an internal fp16 operand";
         default: return "unknown status";
     }
 }

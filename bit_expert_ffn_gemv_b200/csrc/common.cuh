@@ -11,9 +11,11 @@
 namespace moe {
 
 // ---------------------------------------------------------------- status word
-// bit 0: a bounded wait gave up; bit 1: an index was out of range.
+// bit 0: a bounded wait gave up; bit 1: an index was out of range;
+// bit 2: a value did not fit an fp16 operand.
 constexpr uint32_t kStatusTimeout = 1u;
 constexpr uint32_t kStatusBounds = 2u;
+constexpr uint32_t kStatusRange = 4u;
 
 MOE_DEV void flag_status(uint32_t* status, uint32_t bit) { atomicOr(status, bit); }
 

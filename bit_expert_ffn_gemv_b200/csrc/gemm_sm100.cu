@@ -1,0 +1,657 @@
+// gemm_sm100.cu -- tcgen05 (5th-generation tensor core) GEMMs for large token counts.
+//
+// Prefill chunks (thousands of tokens; the pages read prompts in chunks of up
+// to 8192 tokens -- molayo1419.me summary, section "Distributed model
+// execution across the PC") turn the layer into three dense contractions:
+//   router    logits[t, e] = x_t . W_r[e] + bias_e           (bf16 x bf16)
+//   gate/up   h[p, j] = silu(Wg_e[j] . x_t) * (Wu_e[j] . x_t)   per expert group
+//   down      o[p, n] = w_p * (Wd_e[n] . h_p)                  per expert group
+// (p: an expert slot's (token, rank) pair, or the token for the shared expert.)
+//
+// Each CTA owns one tile at a time: 128 weight rows (the MMA's M, "swap AB")
+// by up to 256 tokens (the MMA's N, rounded up to a multiple of 16 for small
+// expert groups), accumulated in tensor memory (TMEM) over K in steps of 64.
+// A 3- or 4-stage cp.async pipeline brings in the tokens' activation rows and
+// the packed weight codes; the CTA's threads turn codes into fp16(q * s) and
+// write them straight into the 128-byte-swizzled K-major layout the MMA reads;
+// one thread issues tcgen05.mma (kind::f16, fp32 accumulate) and commits each
+// step to an mbarrier, so dequantising step s overlaps the MMAs of step s - 1.
+// The epilogue reads TMEM with tcgen05.ld.  Every wait is bounded.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace tc {
+
+constexpr uint32_t kSpin = 1u << 20;
+
+MOE_DEV uint64_t sdesc(uint32_t addr) {
+    // K-major, 128-byte swizzle: 8-row atoms of 1024 B, 16-B LBO, SM100 version 1
+    return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
+           (2ull << 61);
+}
+// byte offset of element (r, k) in a [rows x 64] 16-bit tile, K-major SW128
+MOE_DEV uint32_t sw128(int r, int k) {
+    return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((((k >> 3) ^ (r & 7)) & 7) << 4) + (k & 7) * 2);
+}
+// 16-byte chunk c (8 elements) of row r
+MOE_DEV uint32_t sw128_chunk(int r, int c) { return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + (((c ^ r) & 7) << 4)); }
+
+MOE_DEV uint32_t idesc_f16(int M, int N, bool bf16) {
+    return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+MOE_DEV void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(slot)), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+MOE_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+MOE_DEV void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+MOE_DEV void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+MOE_DEV void mma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+            d_tmem),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+MOE_DEV void commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+MOE_DEV void ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+MOE_DEV void cp16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+MOE_DEV void cp8(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+MOE_DEV void cp4(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+MOE_DEV void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+MOE_DEV void cp_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// bounded wait on an mbarrier phase; false if it gave up
+MOE_DEV bool bar_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
+    for (uint32_t it = 0; it < kSpin; ++it)
+        if (mbar_try_wait(bar, parity)) return true;
+    flag_status(status, kStatusTimeout);
+    return false;
+}
+
+}  // namespace tc
+
+constexpr int kGemmThreads = 256;
+constexpr int kTileM = 128;  // weight rows per tile (the MMA's M)
+constexpr int kStepK = 64;   // K per pipeline step (one SW128 atom of 16-bit values)
+constexpr int kExpertTileN = 256;  // tokens per expert tile (at most; the MMA's N)
+constexpr int kRouterTileN = 128;  // tokens per router tile
+
+// ---------------------------------------------------------------- tile list
+// tile_gu[s] / tile_dn[s] = first gate/up / down tile of slot s (slot 0 = the
+// shared expert if any, then the active routed experts in ascending order);
+// a slot holds ceil(count / kExpertTileN) token tiles x the row-tiles of the
+// weight; entry n_slots is the total.
+__global__ void build_tiles_kernel(const ExpertArgs a, int jt_gateup, int jt_down, int32_t* tile_gu, int32_t* tile_dn) {
+    if (threadIdx.x != 0) return;
+    const int n_slots = a.n_shared + a.meta->n_active;
+    int g = 0, dn = 0;
+    for (int s = 0; s < n_slots; ++s) {
+        int count;
+        if (s < a.n_shared) count = a.T;
+        else {
+            const int e = a.active[s - a.n_shared];
+            count = a.offsets[e + 1] - a.offsets[e];
+        }
+        const int tt = (count + kExpertTileN - 1) / kExpertTileN;
+        tile_gu[s] = g;
+        tile_dn[s] = dn;
+        g += tt * jt_gateup;
+        dn += tt * jt_down;
+    }
+    tile_gu[n_slots] = g;
+    tile_dn[n_slots] = dn;
+}
+
+struct GemmArgs {
+    ExpertArgs e;
+    const uint16_t* xh;    // fp16 activations [T x d]
+    const float* w;        // routing weights [T x k]
+    __half* o;             // fp16 weighted expert outputs [rows x d]
+    const int32_t* tiles;  // tile prefix per slot
+};
+
+struct TileInfo {
+    int slot, expert, count, hbase, pair0, tt, jt, n;  // n: tokens in this tile
+    bool shared;
+};
+
+MOE_DEV bool find_tile(const GemmArgs& g, int tile, int JT, TileInfo& ti) {
+    const ExpertArgs& a = g.e;
+    const int n_slots = a.n_shared + a.meta->n_active;
+    if (tile >= g.tiles[n_slots]) return false;
+    int lo = 0, hi = n_slots - 1;  // last slot with tiles[s] <= tile
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (g.tiles[mid] <= tile) lo = mid;
+        else hi = mid - 1;
+    }
+    ti.slot = lo;
+    ti.shared = lo < a.n_shared;
+    if (ti.shared) {
+        ti.expert = a.E;
+        ti.count = a.T;
+        ti.hbase = a.T * a.k;
+        ti.pair0 = 0;
+    } else {
+        ti.expert = a.active[lo - a.n_shared];
+        ti.pair0 = a.offsets[ti.expert];
+        ti.count = a.offsets[ti.expert + 1] - ti.pair0;
+        ti.hbase = ti.pair0;
+    }
+    const int local = tile - g.tiles[lo];
+    ti.tt = local / JT;
+    ti.jt = local % JT;
+    ti.n = min(kExpertTileN, ti.count - ti.tt * kExpertTileN);
+    return true;
+}
+
+// ---------------------------------------------------------------- grouped expert GEMM
+// GATEUP: A0 = W_g rows, A1 = W_u rows (row-tile jt of f), B = x rows of the
+// slot's tokens; epilogue h = silu(g) * u -> fp16.  Otherwise: A0 = W_d rows
+// (row-tile jt of d), B = h rows; epilogue o = w_p * acc -> fp16.
+template <int BITS, bool GATEUP>
+struct GemmCfg {
+    static constexpr int kN = kExpertTileN;
+    static constexpr int kStages = GATEUP ? 3 : 4;
+    static constexpr int kMats = GATEUP ? 2 : 1;
+    static constexpr int kCodeBytes = 4096;  // [8 row-tiles][32 lanes][16 B]
+    static constexpr int kScaleBytes = 512;  // [8 row-tiles][8 g][8 B]
+    static constexpr int kA = kTileM * 128, kB = kN * 128;
+    static constexpr int kStageRaw = kMats * kA + kB + kMats * (kCodeBytes + kScaleBytes);
+    static constexpr int kStageBytes = (kStageRaw + 1023) & ~1023;
+    static constexpr int kSmem = kStages * kStageBytes + 1024;  // + alignment slack
+    static constexpr int kTmemCols = GATEUP ? 2 * kN : kN;
+    static_assert(kSmem <= 227 * 1024, "shared memory");
+    static_assert(kTmemCols <= 512, "tensor memory");
+};
+
+template <int BITS, bool GATEUP>
+__global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(const GemmArgs g) {
+    using C = GemmCfg<BITS, GATEUP>;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t mma_bar[C::kStages];
+    __shared__ uint32_t tmem_slot;
+    const ExpertArgs& a = g.e;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    const int K = GATEUP ? a.d : a.f;  // contraction length
+    const int KS = K / kStepK;         // pipeline steps per tile
+    const int JT = (GATEUP ? a.f : a.d) / kTileM;
+    const int KT = K / 128;            // super-tiles along K
+    const int64_t mc = (int64_t)a.f * a.d * BITS / 8, ms = (int64_t)a.f * a.d / 32;
+
+    if (tid == 0) {
+        for (int i = 0; i < C::kStages; ++i) mbar_init(&mma_bar[i], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) tc::tmem_alloc(&tmem_slot, C::kTmemCols);
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = tmem_slot;
+
+    // gstep counts pipeline steps over all tiles of this CTA: step i uses stage
+    // i % S, and its MMAs complete phase i / S of that stage's barrier.
+    uint32_t gstep = 0;
+    bool ok = true;  // per thread: no wait has given up yet
+    bool all_ok = true;  // CTA-uniform copy, refreshed once per tile
+    for (int tile = blockIdx.x; all_ok; tile += gridDim.x) {
+        TileInfo ti;
+        if (!find_tile(g, tile, JT, ti)) break;
+        const int nmma = (ti.n + 15) & ~15;
+        const uint32_t idesc = tc::idesc_f16(kTileM, nmma, false);
+        const uint8_t* cbase = a.codes + ((int64_t)ti.expert * 3 + (GATEUP ? 0 : 2)) * mc;
+        const uint8_t* sbase =
+            reinterpret_cast<const uint8_t*>(a.scales) + ((int64_t)ti.expert * 3 + (GATEUP ? 0 : 2)) * ms * 2;
+
+        // cp.async copies of local step s into stage `st`
+        auto load_step = [&](int s, int st) {
+            uint8_t* sb = smem + st * C::kStageBytes;
+            uint8_t* Bs = sb + C::kMats * C::kA;
+            uint8_t* Cs = Bs + C::kB;
+            // B: nmma rows x 64 values = 8 chunks of 16 B per row; rows past the
+            // group repeat its last row (their columns are never stored)
+            for (int v = tid; v < nmma * 8; v += kGemmThreads) {
+                const int r = v >> 3, c = v & 7;
+                const int row = ti.tt * kExpertTileN + min(r, ti.n - 1);
+                const uint16_t* src;
+                if (GATEUP) {
+                    const int tok = ti.shared ? row : a.pairs[ti.pair0 + row] / a.k;
+                    src = g.xh + (int64_t)tok * a.d + s * kStepK + c * 8;
+                } else {
+                    src = reinterpret_cast<const uint16_t*>(a.h) + (int64_t)(ti.hbase + row) * a.f + s * kStepK +
+                          c * 8;
+                }
+                tc::cp16(Bs + tc::sw128_chunk(r, c), src);
+            }
+            // codes and scales: thread = (row-tile, lane); step s is half hs of super-tile kt
+            const int kt = s >> 1, hs = s & 1;
+            const int rt = tid >> 5, ln = tid & 31;
+#pragma unroll
+            for (int m = 0; m < C::kMats; ++m) {
+                uint8_t* cs = Cs + m * (C::kCodeBytes + C::kScaleBytes);
+                uint8_t* ss = cs + C::kCodeBytes;
+                const int64_t st_idx = (int64_t)(ti.jt * 8 + rt) * KT + kt;
+                const uint8_t* stile = cbase + m * mc + st_idx * (256 * BITS);
+                uint8_t* dst = cs + (rt * 32 + ln) * 16;
+                tc::cp8(dst, stile + ln * 16 + hs * 8);
+                if (BITS == 3) tc::cp4(dst + 8, stile + 512 + ln * 8 + hs * 4);
+                if (BITS == 4) tc::cp8(dst + 8, stile + 512 + ln * 16 + hs * 8);
+                if (ln < 8) tc::cp8(ss + rt * 64 + ln * 8, sbase + m * ms * 2 + st_idx * 128 + ln * 16 + hs * 8);
+            }
+        };
+        // codes of stage st -> fp16(q * s) in the SW128 A tiles of that stage
+        auto dequant_step = [&](int st) {
+            uint8_t* sb = smem + st * C::kStageBytes;
+            uint8_t* Cs = sb + C::kMats * C::kA + C::kB;
+            const int rt = tid >> 5, ln = tid & 31, gg = ln >> 2, c = ln & 3;
+#pragma unroll
+            for (int m = 0; m < C::kMats; ++m) {
+                uint8_t* A = sb + m * C::kA;
+                const uint8_t* cs = Cs + m * (C::kCodeBytes + C::kScaleBytes);
+                const uint8_t* src = cs + (rt * 32 + ln) * 16;
+                const uint2 lo = *reinterpret_cast<const uint2*>(src);
+                uint32_t hi0 = 0, hi1 = 0;
+                if (BITS == 3) {
+                    const uint32_t hv = *reinterpret_cast<const uint32_t*>(src + 8);
+                    hi0 = hv & 0xFFFFu;
+                    hi1 = hv >> 16;
+                } else if (BITS == 4) {
+                    const uint2 hv = *reinterpret_cast<const uint2*>(src + 8);
+                    hi0 = hv.x;
+                    hi1 = hv.y;
+                }
+                const uint2 sc = *reinterpret_cast<const uint2*>(cs + C::kCodeBytes + rt * 64 + gg * 8);
+                const uint32_t words[2] = {lo.x, lo.y}, his[2] = {hi0, hi1}, scs[2] = {sc.x, sc.y};
+#pragma unroll
+                for (int kbl = 0; kbl < 2; ++kbl) {
+                    uint32_t q[8];
+                    decode_block<true, BITS>(words[kbl], his[kbl], q);
+                    const __half2 s_lo = __half2half2(__ushort_as_half((unsigned short)(scs[kbl] & 0xFFFFu)));
+                    const __half2 s_hi = __half2half2(__ushort_as_half((unsigned short)(scs[kbl] >> 16)));
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        // pair p = 4 ks + 2 (m / 8) + r / 8 of the A-fragment layout
+                        const int ks = p >> 2, hi8 = (p >> 1) & 1, half = p & 1;
+                        const int r = rt * 16 + gg + 8 * half;
+                        const int kk = 32 * kbl + 16 * ks + 8 * hi8 + 2 * c;
+                        const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&q[p]), half ? s_hi : s_lo);
+                        *reinterpret_cast<__half2*>(A + tc::sw128(r, kk)) = v;
+                    }
+                }
+            }
+        };
+
+        // prologue: steps 0 .. S-2 in flight (all stages are free: the last
+        // tile ended by waiting for all of its MMAs)
+        const int P = C::kStages - 1;
+        for (int s = 0; s < P; ++s) {
+            if (s < KS) load_step(s, (gstep + s) % C::kStages);
+            tc::cp_commit();
+        }
+        for (int s = 0; s < KS; ++s) {
+            const uint32_t cur = gstep + s;
+            const int st = cur % C::kStages;
+            tc::cp_wait<C::kStages - 2>();  // this thread's copies of step s have landed
+            __syncthreads();                // ... and everyone's
+            dequant_step(st);
+            fence_proxy_async_smem();       // make the A and B tiles visible to the tensor core
+            // step s + P reuses the stage of step s - 1: wait for those MMAs first
+            if (s + P < KS) {
+                if (cur >= 1 && ok) {
+                    const uint32_t prev = cur - 1;
+                    ok = tc::bar_wait(&mma_bar[prev % C::kStages], (prev / C::kStages) & 1, a.status);
+                }
+                load_step(s + P, (cur + P) % C::kStages);
+            }
+            tc::cp_commit();
+            __syncthreads();
+            if (tid == 0) {
+                tc::fence_after();
+                uint8_t* sb = smem + st * C::kStageBytes;
+                const uint32_t b_addr = smem_addr(sb + C::kMats * C::kA);
+#pragma unroll
+                for (int kk = 0; kk < kStepK / 16; ++kk) {
+                    const uint64_t bd = tc::sdesc(b_addr + kk * 32);
+                    const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                    tc::mma(tmem, tc::sdesc(smem_addr(sb) + kk * 32), bd, idesc, acc);
+                    if (GATEUP) tc::mma(tmem + C::kN, tc::sdesc(smem_addr(sb + C::kA) + kk * 32), bd, idesc, acc);
+                }
+                tc::commit(&mma_bar[st]);
+            }
+        }
+        // the last commit tracks every MMA of the tile
+        if (ok) {
+            const uint32_t last = gstep + KS - 1;
+            ok = tc::bar_wait(&mma_bar[last % C::kStages], (last / C::kStages) & 1, a.status);
+        }
+        gstep += KS;
+        all_ok = __syncthreads_and(ok) != 0;
+        tc::fence_after();
+
+        // epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (= weight rows);
+        // warps 0-3 take the even 16-column chunks, warps 4-7 the odd ones
+        const int row = 32 * (warp & 3) + lane;
+        for (int c0 = 16 * (warp >> 2); c0 < nmma && all_ok; c0 += 32) {
+            const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c0;
+            uint32_t r0[16];
+            tc::ld16(ta, r0);
+            if (GATEUP) {
+                uint32_t r1[16];
+                tc::ld16(ta + C::kN, r1);
+                bool finite = true;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int tok = c0 + i;
+                    if (tok < ti.n) {
+                        const float hv = silu(__uint_as_float(r0[i])) * __uint_as_float(r1[i]);
+                        finite = finite && fabsf(hv) <= 65504.0f;
+                        static_cast<__half*>(a.h)[(int64_t)(ti.hbase + ti.tt * kExpertTileN + tok) * a.f +
+                                                  ti.jt * kTileM + row] = __float2half_rn(hv);
+                    }
+                }
+                if (!finite) flag_status(a.status, kStatusRange);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int tok = c0 + i;
+                    if (tok < ti.n) {
+                        const int prow = ti.tt * kExpertTileN + tok;
+                        const float wp = ti.shared ? 1.0f : g.w[a.pairs[ti.pair0 + prow]];
+                        g.o[(int64_t)(ti.hbase + prow) * a.d + ti.jt * kTileM + row] =
+                            __float2half_rn(wp * __uint_as_float(r0[i]));
+                    }
+                }
+            }
+        }
+        tc::fence_before();
+        __syncthreads();
+    }
+    tc::cp_wait<0>();
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, C::kTmemCols);
+}
+
+// ---------------------------------------------------------------- router GEMM
+// logits[t][e] = W_r[e] . x_t + bias_e for 128-expert x 128-token tiles, bf16
+// operands copied straight into the SW128 tiles.
+constexpr int kRouterStages = 4;
+constexpr int kRouterStage = kTileM * 128 + kRouterTileN * 128;
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    router_gemm_kernel(const uint16_t* __restrict__ x, int T, int d, const uint16_t* __restrict__ wr,
+                       const float* __restrict__ bias, int E, float* __restrict__ logits, uint32_t* status) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t mma_bar[kRouterStages];
+    __shared__ uint32_t tmem_slot;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+    const int KS = d / kStepK;
+    const int MT = (E + kTileM - 1) / kTileM, NT = (T + kRouterTileN - 1) / kRouterTileN;
+    if (tid == 0) {
+        for (int i = 0; i < kRouterStages; ++i) mbar_init(&mma_bar[i], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) tc::tmem_alloc(&tmem_slot, kRouterTileN);
+    tc::fence_before();
+    __syncthreads();
+    tc::fence_after();
+    const uint32_t tmem = tmem_slot;
+    uint32_t gstep = 0;
+    bool ok = true, all_ok = true;
+    for (int tile = blockIdx.x; tile < MT * NT && all_ok; tile += gridDim.x) {
+        const int mt = tile % MT, nt = tile / MT;
+        const int e0 = mt * kTileM, t0 = nt * kRouterTileN;
+        const int n = min(kRouterTileN, T - t0), nmma = (n + 15) & ~15;
+        const uint32_t idesc = tc::idesc_f16(kTileM, nmma, true);
+        auto load_step = [&](int s, int st) {
+            uint8_t* As = smem + st * kRouterStage;
+            uint8_t* Bs = As + kTileM * 128;
+            for (int v = tid; v < kTileM * 8; v += kGemmThreads) {
+                const int r = v >> 3, c = v & 7;
+                const int e = min(e0 + r, E - 1);
+                tc::cp16(As + tc::sw128_chunk(r, c), wr + (int64_t)e * d + s * kStepK + c * 8);
+            }
+            for (int v = tid; v < nmma * 8; v += kGemmThreads) {
+                const int r = v >> 3, c = v & 7;
+                const int t = t0 + min(r, n - 1);
+                tc::cp16(Bs + tc::sw128_chunk(r, c), x + (int64_t)t * d + s * kStepK + c * 8);
+            }
+        };
+        const int P = kRouterStages - 1;
+        for (int s = 0; s < P; ++s) {
+            if (s < KS) load_step(s, (gstep + s) % kRouterStages);
+            tc::cp_commit();
+        }
+        for (int s = 0; s < KS; ++s) {
+            const uint32_t cur = gstep + s;
+            const int st = cur % kRouterStages;
+            tc::cp_wait<kRouterStages - 2>();
+            fence_proxy_async_smem();
+            if (s + P < KS) {
+                if (cur >= 1 && ok) {
+                    const uint32_t prev = cur - 1;
+                    ok = tc::bar_wait(&mma_bar[prev % kRouterStages], (prev / kRouterStages) & 1, status);
+                }
+                load_step(s + P, (cur + P) % kRouterStages);
+            }
+            tc::cp_commit();
+            __syncthreads();
+            if (tid == 0) {
+                tc::fence_after();
+                const uint32_t a_addr = smem_addr(smem + st * kRouterStage), b_addr = a_addr + kTileM * 128;
+#pragma unroll
+                for (int kk = 0; kk < kStepK / 16; ++kk)
+                    tc::mma(tmem, tc::sdesc(a_addr + kk * 32), tc::sdesc(b_addr + kk * 32), idesc,
+                            (s > 0 || kk > 0) ? 1u : 0u);
+                tc::commit(&mma_bar[st]);
+            }
+        }
+        if (ok) {
+            const uint32_t last = gstep + KS - 1;
+            ok = tc::bar_wait(&mma_bar[last % kRouterStages], (last / kRouterStages) & 1, status);
+        }
+        gstep += KS;
+        all_ok = __syncthreads_and(ok) != 0;
+        tc::fence_after();
+        const int e = e0 + 32 * (warp & 3) + lane;
+        const float b = (bias && e < E) ? bias[e] : 0.0f;
+        for (int c0 = 16 * (warp >> 2); c0 < nmma && all_ok; c0 += 32) {
+            uint32_t r0[16];
+            tc::ld16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c0, r0);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (c0 + i < n && e < E) logits[(int64_t)(t0 + c0 + i) * E + e] = __uint_as_float(r0[i]) + b;
+        }
+        tc::fence_before();
+        __syncthreads();
+    }
+    tc::cp_wait<0>();
+    tc::fence_before();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tmem, kRouterTileN);
+}
+
+// ---------------------------------------------------------------- activations to fp16, combine
+__global__ void to_f16_kernel(const __nv_bfloat16* __restrict__ x, __half* __restrict__ xh, int64_t n,
+                              uint32_t* status) {
+    const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+    if (i >= n) return;
+    const uint4 v = *reinterpret_cast<const uint4*>(x + i);
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[4];
+    bool finite = true;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float lo = __uint_as_float(in[j] << 16), hi = __uint_as_float(in[j] & 0xFFFF0000u);
+        finite = finite && fabsf(lo) <= 65504.0f && fabsf(hi) <= 65504.0f;
+        const __half2 hv = __floats2half2_rn(lo, hi);
+        out[j] = *reinterpret_cast<const uint32_t*>(&hv);
+    }
+    *reinterpret_cast<uint4*>(xh + i) = make_uint4(out[0], out[1], out[2], out[3]);
+    if (!finite) flag_status(status, kStatusRange);
+}
+
+// y[t] = o[shared row of t] + sum_r o[row of (t, r)] (already weighted), fixed order
+__global__ void combine_f16_kernel(const CombineArgs a, const __half* __restrict__ o) {
+    const int t = blockIdx.y;
+    const int n = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+    if (n >= a.d) return;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    auto add_row = [&](int64_t row) {
+        const uint4 v = *reinterpret_cast<const uint4*>(o + row * a.d + n);
+        const __half2* h2 = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 f = __half22float2(h2[j]);
+            acc[2 * j] += f.x;
+            acc[2 * j + 1] += f.y;
+        }
+    };
+    if (a.n_shared) add_row((int64_t)a.T * a.k + t);
+    for (int r = 0; r < a.k; ++r) {
+        const int pos = a.inv[(int64_t)t * a.k + r];
+        if (pos >= 0) add_row(pos);
+    }
+    if (a.out_fp32) {
+        float* y = static_cast<float*>(a.y) + (int64_t)t * a.d + n;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) y[j] = a.accumulate ? y[j] + acc[j] : acc[j];
+    } else {
+        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(a.y) + (int64_t)t * a.d + n;
+        uint32_t out[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float v0 = acc[2 * j], v1 = acc[2 * j + 1];
+            if (a.accumulate) {
+                v0 += __bfloat162float(y[2 * j]);
+                v1 += __bfloat162float(y[2 * j + 1]);
+            }
+            const __nv_bfloat162 b = __floats2bfloat162_rn(v0, v1);
+            out[j] = *reinterpret_cast<const uint32_t*>(&b);
+        }
+        *reinterpret_cast<uint4*>(y) = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+}
+
+// ---------------------------------------------------------------- launchers
+static int num_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+    return sms;
+}
+
+template <int BITS, bool GATEUP>
+static cudaError_t gemm_bits(const GemmArgs& g, cudaStream_t s) {
+    using C = GemmCfg<BITS, GATEUP>;
+    auto kern = expert_gemm_kernel<BITS, GATEUP>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    if (e != cudaSuccess) return e;
+    kern<<<num_sms(), kGemmThreads, C::kSmem, s>>>(g);
+    return cudaGetLastError();
+}
+
+size_t tile_list_words(int E) { return 2 * (size_t)(E + 2); }
+
+cudaError_t launch_build_tiles(const ExpertArgs& a, int32_t* tiles, cudaStream_t s) {
+    build_tiles_kernel<<<1, 32, 0, s>>>(a, a.f / kTileM, a.d / kTileM, tiles, tiles + a.E + 2);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_gateup(const ExpertArgs& a, const void* xh, const int32_t* tiles, cudaStream_t s) {
+    GemmArgs g;
+    g.e = a;
+    g.xh = static_cast<const uint16_t*>(xh);
+    g.w = nullptr;
+    g.o = nullptr;
+    g.tiles = tiles;
+    switch (a.bits) {
+        case 2: return gemm_bits<2, true>(g, s);
+        case 3: return gemm_bits<3, true>(g, s);
+        case 4: return gemm_bits<4, true>(g, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_gemm_down(const ExpertArgs& a, const float* w, void* o, const int32_t* tiles, cudaStream_t s) {
+    GemmArgs g;
+    g.e = a;
+    g.xh = nullptr;
+    g.w = w;
+    g.o = static_cast<__half*>(o);
+    g.tiles = tiles + a.E + 2;
+    switch (a.bits) {
+        case 2: return gemm_bits<2, false>(g, s);
+        case 3: return gemm_bits<3, false>(g, s);
+        case 4: return gemm_bits<4, false>(g, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_router_gemm(const RouteArgs& a, uint32_t* status, cudaStream_t s) {
+    const int smem = kRouterStages * kRouterStage + 1024;
+    cudaError_t e = cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    const int tiles = ((a.E + kTileM - 1) / kTileM) * ((a.T + kRouterTileN - 1) / kRouterTileN);
+    router_gemm_kernel<<<min(tiles, num_sms()), kGemmThreads, smem, s>>>(
+        static_cast<const uint16_t*>(a.x), a.T, a.d, static_cast<const uint16_t*>(a.wr), a.bias, a.E, a.logits,
+        status);
+    return cudaGetLastError();
+}
+
+// Error bound of the tensor-core logits, in the units of the top-k kernel's
+// certificate delta = 2 * depth * 2^-24 * (||W_r,e|| ||x|| + |bias_e|).
+// Model: each MMA adds 16 exact bf16 x bf16 products to the fp32 accumulator;
+// aligning the 17 terms to the largest exponent and truncating costs at most
+// one fp32 ulp of that largest term per term, and every term is at most
+// sum_i |w_i x_i| <= ||w|| ||x||.  So a K = 16 step errs by at most
+// 17 * 2^-23 * ||w|| ||x||; doubled for margin and summed over d / 16 steps,
+// plus the fp32 bias add: depth = 34 * (d / 16) + 2.
+float router_gemm_depth(int d) { return 34.0f * (float)(d / 16) + 2.0f; }
+
+cudaError_t launch_to_f16(const void* x, void* xh, int64_t n, uint32_t* status, cudaStream_t s) {
+    const int64_t threads = n / 8;
+    to_f16_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
+                                                                    static_cast<__half*>(xh), n, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine_f16(const CombineArgs& a, const void* o, cudaStream_t s) {
+    dim3 grid((a.d / 8 + 127) / 128, a.T);
+    combine_f16_kernel<<<grid, 128, 0, s>>>(a, static_cast<const __half*>(o));
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -17,6 +17,7 @@ struct RouteArgs {
     int32_t* ids;       // [T x k]
     float* w;           // [T x k]
     Meta* meta;
+    float depth = 0.f;  // logits error bound (see launch_topk); 0: the CUDA-core logits kernel's
 };
 
 // Bucketing of the T*k (token, slot) pairs by expert.
@@ -91,6 +92,15 @@ cudaError_t launch_bucket(const BucketArgs& a, cudaStream_t s);
 cudaError_t launch_gemv_gateup(const ExpertArgs& a, cudaStream_t s);
 cudaError_t launch_gemv_down(const ExpertArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+// tcgen05 path (T > kDecodeMaxTokens)
+cudaError_t launch_to_f16(const void* x, void* xh, int64_t n, uint32_t* status, cudaStream_t s);
+cudaError_t launch_router_gemm(const RouteArgs& a, uint32_t* status, cudaStream_t s);
+float router_gemm_depth(int d);
+size_t tile_list_words(int E);
+cudaError_t launch_build_tiles(const ExpertArgs& a, int32_t* tiles, cudaStream_t s);
+cudaError_t launch_gemm_gateup(const ExpertArgs& a, const void* xh, const int32_t* tiles, cudaStream_t s);
+cudaError_t launch_gemm_down(const ExpertArgs& a, const float* w, void* o, const int32_t* tiles, cudaStream_t s);
+cudaError_t launch_combine_f16(const CombineArgs& a, const void* o, cudaStream_t s);
 cudaError_t launch_dequant(const uint8_t* codes, const uint16_t* scales, int N, int K, int bits, float* out,
                            cudaStream_t s);
 

@@ -261,7 +261,7 @@ cudaError_t launch_topk(const RouteArgs& a, cudaStream_t s) {
         cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_t);
         if (e != cudaSuccess) return e;
     }
-    const float depth = (float)(a.d / 32 + 6);
+    const float depth = a.depth > 0.f ? a.depth : (float)(a.d / 32 + 6);
     topk_kernel<<<(a.T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, smem_t, s>>>(
         a.logits, static_cast<const __nv_bfloat16*>(a.x), a.T, a.d, a.E, a.k,
         static_cast<const __nv_bfloat16*>(a.wr), a.bias, a.wnorm, depth, a.ids, a.w, a.meta);

@@ -70,7 +70,9 @@ typedef enum {
     MOE_ERR_OOM = 3,         /* device allocation failed */
     MOE_ERR_NOT_LOADED = 4,  /* the layer has no weights loaded */
     MOE_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up */
-    MOE_ERR_BOUNDS = 6       /* a device-side index was out of range */
+    MOE_ERR_BOUNDS = 6,      /* a device-side index was out of range */
+    MOE_ERR_RANGE = 7        /* a value left the range of an internal fp16
+                                operand (|x| or |h| above 65504, or NaN) */
 } moe_status;
 
 typedef struct {
@@ -193,9 +195,25 @@ moe_status moe_debug_dequant(moe_handle* h, int32_t layer, int32_t expert, int32
 moe_status moe_debug_last_routing(moe_handle* h, int32_t T, int32_t* ids, float* w, void* stream);
 
 /*
+ * Debug: the fp32 router logits l = W_r x + bias [T x n_experts] (device,
+ * row-major) of a loaded layer as one of the two router kernels computes
+ * them: tensor_cores != 0 the bf16 tcgen05 GEMM used for T > 64 tokens, else
+ * the CUDA-core kernel.  Each logit is within
+ *   delta_e = 2 * depth * 2^-24 * (||W_r,e||_2 ||x||_2 + |bias_e|)
+ * of the exact value, depth = moe_router_error_depth(d, tensor_cores); the
+ * top-k re-ranks every token whose order these intervals leave open.
+ * Errors: INVALID_ARG, NOT_LOADED, CUDA.
+ */
+moe_status moe_debug_router_logits(moe_handle* h, int32_t layer, const void* x, int32_t T, float* logits,
+                                   int32_t tensor_cores, void* stream);
+
+/* The `depth` of the logits error bound above for hidden size d (0 if d <= 0). */
+float moe_router_error_depth(int32_t d, int32_t tensor_cores);
+
+/*
  * Synchronise the device and return the first device-side error recorded
- * since the last call (then clear it): MOE_ERR_TIMEOUT, MOE_ERR_BOUNDS or
- * MOE_OK; MOE_ERR_CUDA if the synchronisation itself failed.
+ * since the last call (then clear it): MOE_ERR_TIMEOUT, MOE_ERR_BOUNDS,
+ * MOE_ERR_RANGE or MOE_OK; MOE_ERR_CUDA if the synchronisation itself failed.
  */
 moe_status moe_check_status(moe_handle* h);
 
@@ -222,7 +240,9 @@ enum {
     MOE_K_GEMM_DOWN = 7,
     MOE_K_ROUTER_GEMM = 8,
     MOE_K_DECODE = 9,
-    MOE_KERNEL_COUNT = 10
+    MOE_K_TO_F16 = 10,
+    MOE_K_TILE_LIST = 11,
+    MOE_KERNEL_COUNT = 12
 };
 
 /*
