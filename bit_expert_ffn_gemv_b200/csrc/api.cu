@@ -48,8 +48,11 @@ struct moe_handle {
     int* sync = nullptr;
     void* x_stage = nullptr;
     void* y_stage = nullptr;
-    void* xh = nullptr;        // fp16 copy of x for the tensor-core path
-    int32_t* tiles = nullptr;  // gate/up and down tile lists
+    void* xh = nullptr;          // fp16 copy of x for the tensor-core path
+    int4* desc_gu = nullptr;     // gate/up tile descriptors
+    int4* desc_dn = nullptr;     // down tile descriptors
+    int32_t* n_tiles = nullptr;  // [2] descriptor counts
+    float* wsorted = nullptr;    // routing weights in group order
     // launch accounting and optional per-kernel event timing
     int64_t launches = 0;
     bool prof_on = false;
@@ -194,6 +197,10 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     ba.active = h->active;
     ba.meta = h->meta;
     ba.status = h->status;
+    if (tc) {
+        ba.w = h->w;
+        ba.wsorted = h->wsorted;
+    }
     e = run(h, MOE_K_BUCKET, s, [&] { return moe::launch_bucket(ba, s); });
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -217,12 +224,15 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     ea.obuf = h->obuf;
     ea.status = h->status;
     if (tc) {
-        e = run(h, MOE_K_TILE_LIST, s, [&] { return moe::launch_build_tiles(ea, h->tiles, s); });
+        e = run(h, MOE_K_TILE_LIST, s,
+                [&] { return moe::launch_build_tiles(ea, h->desc_gu, h->desc_dn, h->n_tiles, s); });
         if (e != cudaSuccess) return MOE_ERR_CUDA;
-        e = run(h, MOE_K_GEMM_GATEUP, s, [&] { return moe::launch_gemm_gateup(ea, h->xh, h->tiles, s); });
+        e = run(h, MOE_K_GEMM_GATEUP, s,
+                [&] { return moe::launch_gemm_gateup(ea, h->xh, h->desc_gu, h->n_tiles, s); });
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         // the fp16 partial outputs reuse the fp32 partial-output buffer
-        e = run(h, MOE_K_GEMM_DOWN, s, [&] { return moe::launch_gemm_down(ea, h->w, h->obuf, h->tiles, s); });
+        e = run(h, MOE_K_GEMM_DOWN, s,
+                [&] { return moe::launch_gemm_down(ea, h->wsorted, h->obuf, h->desc_dn, h->n_tiles, s); });
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     } else {
         e = run(h, MOE_K_GEMV_GATEUP, s, [&] { return moe::launch_gemv_gateup(ea, s); });
@@ -303,7 +313,12 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     const size_t o_norms = take(sizeof(float) * E * (size_t)c.n_layers);
     const size_t o_l64 = take(sizeof(double) * std::min<size_t>(T, moe::kDecodeMaxTokens) * E);
     const size_t o_xh = take(sizeof(uint16_t) * T * (size_t)c.d);
-    const size_t o_tiles = take(sizeof(int32_t) * moe::tile_list_words(c.n_experts));
+    const size_t o_dgu = take(sizeof(int4) * moe::tile_desc_count(c.max_tokens, c.top_k, c.n_experts, c.n_shared,
+                                                                   c.f / 128));
+    const size_t o_ddn = take(sizeof(int4) * moe::tile_desc_count(c.max_tokens, c.top_k, c.n_experts, c.n_shared,
+                                                                   c.d / 128));
+    const size_t o_ntiles = take(sizeof(int32_t) * 2);
+    const size_t o_wsorted = take(sizeof(float) * T * k);
     const size_t o_sync =
         take(sizeof(int) * moe::decode_sync_words(std::min(c.max_tokens, moe::kDecodeMaxTokens), c.n_experts, c.d));
     h->arena_bytes = off;
@@ -330,7 +345,10 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     h->x_stage = base + o_xs;
     h->y_stage = base + o_ys;
     h->xh = base + o_xh;
-    h->tiles = reinterpret_cast<int32_t*>(base + o_tiles);
+    h->desc_gu = reinterpret_cast<int4*>(base + o_dgu);
+    h->desc_dn = reinterpret_cast<int4*>(base + o_ddn);
+    h->n_tiles = reinterpret_cast<int32_t*>(base + o_ntiles);
+    h->wsorted = reinterpret_cast<float*>(base + o_wsorted);
     for (int l = 0; l < c.n_layers; ++l) h->layers[l].wnorm = reinterpret_cast<float*>(base + o_norms) + E * l;
     if (cudaMemset(h->arena, 0, h->arena_bytes) != cudaSuccess) {
         cudaFree(h->arena);

@@ -3,8 +3,8 @@
 // Counting sort, stable in the token index: per-expert counts, an exclusive
 // scan over experts, and a scatter that keeps ascending token order inside
 // each expert's group (so the grouping, and everything computed from it, is
-// deterministic).  One CTA of 32 warps; warp w owns a contiguous token range,
-// which makes the per-warp counts a stable prefix.
+// deterministic).  One CTA of 32 warps; warp w owns a contiguous range of
+// (token, rank) pairs, which makes the per-warp counts a stable prefix.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -14,30 +14,44 @@ namespace moe {
 
 constexpr int kBucketWarps = 32;
 
+// Warp w owns the contiguous range of pair indices p = t*k + r in
+// [w*ppw, (w+1)*ppw); ascending p means ascending t, so per-warp counts and
+// in-warp ranks (lanes with equal expert, by lane order) give a stable order.
 __global__ void __launch_bounds__(kBucketWarps * 32)
     bucket_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int32_t* __restrict__ offsets,
                   int32_t* __restrict__ pairs, int32_t* __restrict__ inv, int32_t* __restrict__ active,
-                  Meta* __restrict__ meta, uint32_t* __restrict__ status) {
+                  Meta* __restrict__ meta, uint32_t* __restrict__ status, const float* __restrict__ w,
+                  float* __restrict__ wsorted) {
     extern __shared__ int32_t sm[];
     int32_t* cnt = sm;                          // [kBucketWarps][E]
     int32_t* total = sm + kBucketWarps * E;     // [E]
     int32_t* off_s = total + E;                 // [E + 1]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tpw = (T + kBucketWarps - 1) / kBucketWarps;
-    const int t_begin = min(T, warp * tpw), t_end = min(T, t_begin + tpw);
+    const int n_pairs = T * k;
+    const int ppw = ((n_pairs + kBucketWarps - 1) / kBucketWarps + 31) & ~31;
+    const int p_begin = min(n_pairs, warp * ppw), p_end = min(n_pairs, p_begin + ppw);
+    const uint32_t lt = (1u << lane) - 1u;
 
     for (int i = threadIdx.x; i < kBucketWarps * E; i += blockDim.x) cnt[i] = 0;
     __syncthreads();
 
-    // phase 1: per-warp counts
-    for (int t = t_begin; t < t_end; ++t) {
-        if (lane < k) {
-            int e = ids[(int64_t)t * k + lane];
-            if (e < 0 || e >= E) {
-                flag_status(status, kStatusBounds);
-            } else {
-                atomicAdd(&cnt[warp * E + e], 1);
-            }
+    // phase 1: per-warp counts (one smem update per distinct expert per 32
+    // pairs); ids are read 8 x 32 at a time so the loads overlap
+    for (int p0 = p_begin; p0 < p_end; p0 += 256) {
+        int ev[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int p = p0 + 32 * u + lane;
+            ev[u] = p < p_end ? __ldg(&ids[p]) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = ev[u];
+            const bool live = p0 + 32 * u + lane < p_end;
+            const bool valid = live && e >= 0 && e < E;
+            if (live && !valid) flag_status(status, kStatusBounds);
+            const uint32_t same = __match_any_sync(0xffffffffu, valid ? e : -1);
+            if (valid && (same & lt) == 0) cnt[warp * E + e] += __popc(same);
         }
     }
     __syncthreads();
@@ -68,7 +82,7 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
             }
             if (e < E) off_s[e] = base + inc - c;
             unsigned b = __ballot_sync(0xffffffffu, c > 0);
-            if (c > 0) active[nact + __popc(b & ((1u << lane) - 1u))] = e;
+            if (c > 0) active[nact + __popc(b & lt)] = e;
             nact += __popc(b);
             int m = c;
 #pragma unroll
@@ -85,20 +99,39 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
     __syncthreads();
     for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = off_s[e];
 
-    // phase 3: stable scatter (a token's k experts are distinct)
-    for (int t = t_begin; t < t_end; ++t) {
-        if (lane < k) {
-            int e = ids[(int64_t)t * k + lane];
-            if (e >= 0 && e < E) {
-                int pos = off_s[e] + cnt[warp * E + e];
-                cnt[warp * E + e] += 1;
-                pairs[pos] = t * k + lane;
-                inv[(int64_t)t * k + lane] = pos;
-            } else {
-                inv[(int64_t)t * k + lane] = -1;
+    // phase 3: stable scatter (and, if asked, the routing weights in group order)
+    for (int p0 = p_begin; p0 < p_end; p0 += 256) {
+        int ev[8];
+        float wv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int p = p0 + 32 * u + lane;
+            ev[u] = p < p_end ? __ldg(&ids[p]) : -1;
+            wv[u] = (wsorted && p < p_end) ? __ldg(&w[p]) : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int e = ev[u];
+            const int p = p0 + 32 * u + lane;
+            const bool live = p < p_end;
+            const bool valid = live && e >= 0 && e < E;
+            const uint32_t same = __match_any_sync(0xffffffffu, valid ? e : -1);
+            const int leader = __ffs(same) - 1;
+            int base = 0;
+            if (valid && lane == leader) {
+                base = off_s[e] + cnt[warp * E + e];
+                cnt[warp * E + e] += __popc(same);
+            }
+            base = __shfl_sync(0xffffffffu, base, leader);
+            if (valid) {
+                const int pos = base + __popc(same & lt);
+                pairs[pos] = p;
+                inv[p] = pos;
+                if (wsorted) wsorted[pos] = wv[u];
+            } else if (live) {
+                inv[p] = -1;
             }
         }
-        __syncwarp();
     }
 }
 
@@ -109,7 +142,7 @@ cudaError_t launch_bucket(const BucketArgs& a, cudaStream_t s) {
         if (e != cudaSuccess) return e;
     }
     bucket_kernel<<<1, kBucketWarps * 32, smem, s>>>(a.ids, a.T, a.k, a.E, a.offsets, a.pairs, a.inv, a.active,
-                                                     a.meta, a.status);
+                                                     a.meta, a.status, a.w, a.wsorted);
     return cudaGetLastError();
 }
 

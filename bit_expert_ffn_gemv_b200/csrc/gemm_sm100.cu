@@ -107,78 +107,126 @@ constexpr int kExpertTileN = 256;  // tokens per expert tile (at most; the MMA's
 constexpr int kRouterTileN = 128;  // tokens per router tile
 
 // ---------------------------------------------------------------- tile list
-// tile_gu[s] / tile_dn[s] = first gate/up / down tile of slot s (slot 0 = the
-// shared expert if any, then the active routed experts in ascending order);
-// a slot holds ceil(count / kExpertTileN) token tiles x the row-tiles of the
-// weight; entry n_slots is the total.
-__global__ void build_tiles_kernel(const ExpertArgs a, int jt_gateup, int jt_down, int32_t* tile_gu, int32_t* tile_dn) {
-    if (threadIdx.x != 0) return;
+// Slots: the shared expert (if any), then the active routed experts in
+// ascending order.  A slot with c tokens holds ceil(c / kExpertTileN) token
+// tiles; token tile q of the layer times the JT row-tiles of a weight gives
+// tiles q * JT .. q * JT + JT - 1, so CTAs that take consecutive tiles read
+// the same activation rows.  One descriptor per tile:
+//   x = expert (E for the shared one), y = row0 (h / partial-output row of
+//   the tile's first token = its first pair position), z = n | jt << 16,
+//   w = first token for the shared expert, -1 for a routed one (whose rows'
+//   tokens are pairs[row0 + r] / k).
+constexpr int kTileListThreads = 1024;
+constexpr int kMaxSlots = 1024 + 1;
+
+static inline int max_token_tiles(int T, int k, int E, int n_shared) {
+    return (T * k + kExpertTileN - 1) / kExpertTileN + E + n_shared * ((T + kExpertTileN - 1) / kExpertTileN) + 1;
+}
+
+__global__ void __launch_bounds__(kTileListThreads)
+    build_tiles_kernel(const ExpertArgs a, int jt_gateup, int jt_down, int4* __restrict__ desc_gu,
+                       int4* __restrict__ desc_dn, int32_t* __restrict__ counts) {
+    __shared__ int pre[kMaxSlots + 1];
+    __shared__ int wsum[kTileListThreads / 32];
+    __shared__ int carry_s;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int n_slots = a.n_shared + a.meta->n_active;
-    int g = 0, dn = 0;
-    for (int s = 0; s < n_slots; ++s) {
-        int count;
-        if (s < a.n_shared) count = a.T;
-        else {
-            const int e = a.active[s - a.n_shared];
-            count = a.offsets[e + 1] - a.offsets[e];
+    if (tid == 0) carry_s = 0;
+    __syncthreads();
+    for (int base = 0; base < n_slots; base += kTileListThreads) {
+        const int s = base + tid;
+        int tt = 0;
+        if (s < n_slots) {
+            int count;
+            if (s < a.n_shared) count = a.T;
+            else {
+                const int e = a.active[s - a.n_shared];
+                count = a.offsets[e + 1] - a.offsets[e];
+            }
+            tt = (count + kExpertTileN - 1) / kExpertTileN;
         }
-        const int tt = (count + kExpertTileN - 1) / kExpertTileN;
-        tile_gu[s] = g;
-        tile_dn[s] = dn;
-        g += tt * jt_gateup;
-        dn += tt * jt_down;
+        int inc = tt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        if (lane == 31) wsum[warp] = inc;
+        __syncthreads();
+        if (warp == 0) {
+            int v = wsum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
+            }
+            wsum[lane] = v;  // inclusive over warps
+        }
+        __syncthreads();
+        const int carry = carry_s;
+        if (s < n_slots) pre[s] = carry + (warp ? wsum[warp - 1] : 0) + inc - tt;
+        __syncthreads();
+        if (tid == 0) carry_s = carry + wsum[kTileListThreads / 32 - 1];
+        __syncthreads();
     }
-    tile_gu[n_slots] = g;
-    tile_dn[n_slots] = dn;
+    const int total_tt = carry_s;
+    if (tid == 0) {
+        pre[n_slots] = total_tt;
+        counts[0] = total_tt * jt_gateup;
+        counts[1] = total_tt * jt_down;
+    }
+    __syncthreads();
+    for (int q = tid; q < total_tt; q += kTileListThreads) {
+        int lo = 0, hi = n_slots - 1;  // last slot with pre[s] <= q
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (pre[mid] <= q) lo = mid;
+            else hi = mid - 1;
+        }
+        const int tt = q - pre[lo];
+        int expert, row0, count, tok0;
+        if (lo < a.n_shared) {
+            expert = a.E;
+            count = a.T;
+            row0 = a.T * a.k + tt * kExpertTileN;
+            tok0 = tt * kExpertTileN;
+        } else {
+            expert = a.active[lo - a.n_shared];
+            const int p0 = a.offsets[expert];
+            count = a.offsets[expert + 1] - p0;
+            row0 = p0 + tt * kExpertTileN;
+            tok0 = -1;
+        }
+        const int n = min(kExpertTileN, count - tt * kExpertTileN);
+        for (int jt = 0; jt < jt_gateup; ++jt) desc_gu[q * jt_gateup + jt] = make_int4(expert, row0, n | (jt << 16), tok0);
+        for (int jt = 0; jt < jt_down; ++jt) desc_dn[q * jt_down + jt] = make_int4(expert, row0, n | (jt << 16), tok0);
+    }
 }
 
 struct GemmArgs {
     ExpertArgs e;
-    const uint16_t* xh;    // fp16 activations [T x d]
-    const float* w;        // routing weights [T x k]
-    __half* o;             // fp16 weighted expert outputs [rows x d]
-    const int32_t* tiles;  // tile prefix per slot
+    const uint16_t* xh;      // fp16 activations [T x d]
+    const float* wsorted;    // routing weight of each pair, in group order [T*k]
+    __half* o;               // fp16 weighted expert outputs [rows x d]
+    const int4* desc;        // tile descriptors
+    const int32_t* n_tiles;  // number of descriptors
 };
-
-struct TileInfo {
-    int slot, expert, count, hbase, pair0, tt, jt, n;  // n: tokens in this tile
-    bool shared;
-};
-
-MOE_DEV bool find_tile(const GemmArgs& g, int tile, int JT, TileInfo& ti) {
-    const ExpertArgs& a = g.e;
-    const int n_slots = a.n_shared + a.meta->n_active;
-    if (tile >= g.tiles[n_slots]) return false;
-    int lo = 0, hi = n_slots - 1;  // last slot with tiles[s] <= tile
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (g.tiles[mid] <= tile) lo = mid;
-        else hi = mid - 1;
-    }
-    ti.slot = lo;
-    ti.shared = lo < a.n_shared;
-    if (ti.shared) {
-        ti.expert = a.E;
-        ti.count = a.T;
-        ti.hbase = a.T * a.k;
-        ti.pair0 = 0;
-    } else {
-        ti.expert = a.active[lo - a.n_shared];
-        ti.pair0 = a.offsets[ti.expert];
-        ti.count = a.offsets[ti.expert + 1] - ti.pair0;
-        ti.hbase = ti.pair0;
-    }
-    const int local = tile - g.tiles[lo];
-    ti.tt = local / JT;
-    ti.jt = local % JT;
-    ti.n = min(kExpertTileN, ti.count - ti.tt * kExpertTileN);
-    return true;
-}
 
 // ---------------------------------------------------------------- grouped expert GEMM
 // GATEUP: A0 = W_g rows, A1 = W_u rows (row-tile jt of f), B = x rows of the
 // slot's tokens; epilogue h = silu(g) * u -> fp16.  Otherwise: A0 = W_d rows
 // (row-tile jt of d), B = h rows; epilogue o = w_p * acc -> fp16.
+//
+// Warp roles (persistent; every role walks the same tile sequence
+// blockIdx.x, blockIdx.x + gridDim.x, ...):
+//   warps 0-7   producers: cp.async of codes, scales and B rows S-1 steps
+//               ahead; dequantise the codes of the current step into the A
+//               tiles; signal full[stage]
+//   warps 8-11  epilogue: wait for a finished accumulator, tcgen05.ld, SwiGLU
+//               or weighting, fp16 stores; signal acc_empty[buffer]
+//   warp 12     MMA issuer (one thread): wait full[stage], issue the K = 64
+//               step's MMAs, commit to empty[stage]; at the end of a tile
+//               commit to acc_full[buffer]
 template <int BITS, bool GATEUP>
 struct GemmCfg {
     static constexpr int kN = kExpertTileN;
@@ -190,78 +238,117 @@ struct GemmCfg {
     static constexpr int kStageRaw = kMats * kA + kB + kMats * (kCodeBytes + kScaleBytes);
     static constexpr int kStageBytes = (kStageRaw + 1023) & ~1023;
     static constexpr int kSmem = kStages * kStageBytes + 1024;  // + alignment slack
-    static constexpr int kTmemCols = GATEUP ? 2 * kN : kN;
+    static constexpr int kAccCols = kMats * kN;                 // one accumulator set
+    static constexpr int kAccBufs = 512 / kAccCols;             // 1 (gate/up) or 2 (down)
     static_assert(kSmem <= 227 * 1024, "shared memory");
-    static_assert(kTmemCols <= 512, "tensor memory");
+    static_assert(kAccBufs >= 1, "tensor memory");
 };
+constexpr int kProducerThreads = 256;
+constexpr int kEpilogueWarp0 = 8;
+constexpr int kMmaWarp = 12;
+constexpr int kExpertThreads = 13 * 32;
+
+MOE_DEV void producer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+// warp-uniform bounded wait (lane 0 polls)
+MOE_DEV bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
+    bool okw = true;
+    if ((threadIdx.x & 31) == 0) okw = tc::bar_wait(bar, parity, status);
+    return __shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0;
+}
+
+MOE_DEV int4 load_desc(const GemmArgs& g, int tile) { return __ldg(&g.desc[tile]); }
 
 template <int BITS, bool GATEUP>
-__global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(const GemmArgs g) {
+__global__ void __launch_bounds__(kExpertThreads, 1) expert_gemm_kernel(const GemmArgs g) {
     using C = GemmCfg<BITS, GATEUP>;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t mma_bar[C::kStages];
+    __shared__ __align__(8) uint64_t full_bar[C::kStages];
+    __shared__ __align__(8) uint64_t empty_bar[C::kStages];
+    __shared__ __align__(8) uint64_t accf_bar[C::kAccBufs];
+    __shared__ __align__(8) uint64_t acce_bar[C::kAccBufs];
     __shared__ uint32_t tmem_slot;
+    __shared__ float w_s[GATEUP ? 1 : kExpertTileN];  // routing weights of the epilogue's tile
     const ExpertArgs& a = g.e;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     const int K = GATEUP ? a.d : a.f;  // contraction length
     const int KS = K / kStepK;         // pipeline steps per tile
-    const int JT = (GATEUP ? a.f : a.d) / kTileM;
     const int KT = K / 128;            // super-tiles along K
     const int64_t mc = (int64_t)a.f * a.d * BITS / 8, ms = (int64_t)a.f * a.d / 32;
 
     if (tid == 0) {
-        for (int i = 0; i < C::kStages; ++i) mbar_init(&mma_bar[i], 1);
+        for (int i = 0; i < C::kStages; ++i) {
+            mbar_init(&full_bar[i], 1);
+            mbar_init(&empty_bar[i], 1);
+        }
+        for (int i = 0; i < C::kAccBufs; ++i) {
+            mbar_init(&accf_bar[i], 1);
+            mbar_init(&acce_bar[i], 128);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) tc::tmem_alloc(&tmem_slot, C::kTmemCols);
+    if (warp == kMmaWarp) tc::tmem_alloc(&tmem_slot, 512);
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = tmem_slot;
 
-    // gstep counts pipeline steps over all tiles of this CTA: step i uses stage
-    // i % S, and its MMAs complete phase i / S of that stage's barrier.
-    uint32_t gstep = 0;
-    bool ok = true;  // per thread: no wait has given up yet
-    bool all_ok = true;  // CTA-uniform copy, refreshed once per tile
-    for (int tile = blockIdx.x; all_ok; tile += gridDim.x) {
-        TileInfo ti;
-        if (!find_tile(g, tile, JT, ti)) break;
-        const int nmma = (ti.n + 15) & ~15;
-        const uint32_t idesc = tc::idesc_f16(kTileM, nmma, false);
-        const uint8_t* cbase = a.codes + ((int64_t)ti.expert * 3 + (GATEUP ? 0 : 2)) * mc;
-        const uint8_t* sbase =
-            reinterpret_cast<const uint8_t*>(a.scales) + ((int64_t)ti.expert * 3 + (GATEUP ? 0 : 2)) * ms * 2;
+    const int total_tiles = *g.n_tiles;
+    const int bid = (int)blockIdx.x, grid = (int)gridDim.x;
+    const int my_tiles = total_tiles > bid ? (total_tiles - 1 - bid) / grid + 1 : 0;
 
-        // cp.async copies of local step s into stage `st`
-        auto load_step = [&](int s, int st) {
+    if (warp < kEpilogueWarp0) {
+        // ======================= producers
+        const int total = my_tiles * KS;
+        constexpr int L = C::kStages - 1;  // steps loaded ahead
+        bool ok = true;
+        // load cursor: its tile's descriptor, the next one (prefetched), and this
+        // thread's 8 B-row sources (rows rb + 32 i, 16-byte chunk cb)
+        const int cb = tid & 7, rb = tid >> 3;
+        int lt_idx = -1;
+        int4 ld = make_int4(0, 0, 0, 0), nd = my_tiles > 0 ? load_desc(g, bid) : make_int4(0, 0, 0, 0);
+        const uint16_t* rowp[8];
+        int lt_nmma = 0;
+        auto load_step = [&](int j) {
+            const int ti_local = j / KS, s = j - ti_local * KS, st = j % C::kStages;
+            if (ti_local != lt_idx) {
+                lt_idx = ti_local;
+                ld = nd;
+                if (ti_local + 1 < my_tiles) nd = load_desc(g, bid + (ti_local + 1) * grid);
+                const int n = ld.z & 0xFFFF;
+                lt_nmma = (n + 15) & ~15;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int rr = min(rb + 32 * i, n - 1);  // rows past the group repeat its last row
+                    if (GATEUP) {
+                        const int tok = ld.w >= 0 ? ld.w + rr : __ldg(&a.pairs[ld.y + rr]) / a.k;
+                        rowp[i] = g.xh + (int64_t)tok * a.d;
+                    } else {
+                        rowp[i] = reinterpret_cast<const uint16_t*>(a.h) + (int64_t)(ld.y + rr) * a.f;
+                    }
+                }
+            }
             uint8_t* sb = smem + st * C::kStageBytes;
             uint8_t* Bs = sb + C::kMats * C::kA;
             uint8_t* Cs = Bs + C::kB;
-            // B: nmma rows x 64 values = 8 chunks of 16 B per row; rows past the
-            // group repeat its last row (their columns are never stored)
-            for (int v = tid; v < nmma * 8; v += kGemmThreads) {
-                const int r = v >> 3, c = v & 7;
-                const int row = ti.tt * kExpertTileN + min(r, ti.n - 1);
-                const uint16_t* src;
-                if (GATEUP) {
-                    const int tok = ti.shared ? row : a.pairs[ti.pair0 + row] / a.k;
-                    src = g.xh + (int64_t)tok * a.d + s * kStepK + c * 8;
-                } else {
-                    src = reinterpret_cast<const uint16_t*>(a.h) + (int64_t)(ti.hbase + row) * a.f + s * kStepK +
-                          c * 8;
-                }
-                tc::cp16(Bs + tc::sw128_chunk(r, c), src);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int r = rb + 32 * i;
+                if (r < lt_nmma) tc::cp16(Bs + tc::sw128_chunk(r, cb), rowp[i] + s * kStepK + cb * 8);
             }
             // codes and scales: thread = (row-tile, lane); step s is half hs of super-tile kt
+            const int expert = ld.x, jt = ld.z >> 16;
+            const uint8_t* cbase = a.codes + ((int64_t)expert * 3 + (GATEUP ? 0 : 2)) * mc;
+            const uint8_t* sbase =
+                reinterpret_cast<const uint8_t*>(a.scales) + ((int64_t)expert * 3 + (GATEUP ? 0 : 2)) * ms * 2;
             const int kt = s >> 1, hs = s & 1;
             const int rt = tid >> 5, ln = tid & 31;
 #pragma unroll
             for (int m = 0; m < C::kMats; ++m) {
                 uint8_t* cs = Cs + m * (C::kCodeBytes + C::kScaleBytes);
                 uint8_t* ss = cs + C::kCodeBytes;
-                const int64_t st_idx = (int64_t)(ti.jt * 8 + rt) * KT + kt;
+                const int64_t st_idx = (int64_t)(jt * 8 + rt) * KT + kt;
                 const uint8_t* stile = cbase + m * mc + st_idx * (256 * BITS);
                 uint8_t* dst = cs + (rt * 32 + ln) * 16;
                 tc::cp8(dst, stile + ln * 16 + hs * 8);
@@ -311,96 +398,114 @@ __global__ void __launch_bounds__(kGemmThreads, 1) expert_gemm_kernel(const Gemm
                 }
             }
         };
-
-        // prologue: steps 0 .. S-2 in flight (all stages are free: the last
-        // tile ended by waiting for all of its MMAs)
-        const int P = C::kStages - 1;
-        for (int s = 0; s < P; ++s) {
-            if (s < KS) load_step(s, (gstep + s) % C::kStages);
+        // the first S steps find their stages free
+        for (int j = 0; j < L; ++j) {
+            if (j < total) load_step(j);
             tc::cp_commit();
         }
-        for (int s = 0; s < KS; ++s) {
-            const uint32_t cur = gstep + s;
-            const int st = cur % C::kStages;
-            tc::cp_wait<C::kStages - 2>();  // this thread's copies of step s have landed
-            __syncthreads();                // ... and everyone's
+        for (int gs = 0; gs < total; ++gs) {
+            const int st = gs % C::kStages;
+            tc::cp_wait<L - 1>();  // this thread's copies of step gs have landed
+            producer_sync();       // ... and every producer's
             dequant_step(st);
-            fence_proxy_async_smem();       // make the A and B tiles visible to the tensor core
-            // step s + P reuses the stage of step s - 1: wait for those MMAs first
-            if (s + P < KS) {
-                if (cur >= 1 && ok) {
-                    const uint32_t prev = cur - 1;
-                    ok = tc::bar_wait(&mma_bar[prev % C::kStages], (prev / C::kStages) & 1, a.status);
-                }
-                load_step(s + P, (cur + P) % C::kStages);
+            fence_proxy_async_smem();  // A and B tiles visible to the tensor core
+            producer_sync();
+            if (tid == 0) mbar_arrive(&full_bar[st]);
+            const int j = gs + L;
+            if (j < total) {
+                if (j >= C::kStages && ok)  // the MMAs of step j - S have read the stage
+                    ok = tc::bar_wait(&empty_bar[j % C::kStages], ((j / C::kStages) - 1) & 1, a.status);
+                load_step(j);
             }
             tc::cp_commit();
-            __syncthreads();
-            if (tid == 0) {
+        }
+        tc::cp_wait<0>();
+    } else if (warp < kMmaWarp) {
+        // ======================= epilogue
+        const int q = warp & 3;  // TMEM lanes 32 q .. 32 q + 31 = weight rows
+        const int row = 32 * q + lane;
+        const int et = tid - 32 * kEpilogueWarp0;  // 0 .. 127
+        bool ok = true;
+        int4 nd = my_tiles > 0 ? load_desc(g, bid) : make_int4(0, 0, 0, 0);
+        for (int it = 0; it < my_tiles; ++it) {
+            const int4 ds = nd;
+            if (it + 1 < my_tiles) nd = load_desc(g, bid + (it + 1) * grid);
+            const int n = ds.z & 0xFFFF, jt = ds.z >> 16, nmma = (n + 15) & ~15;
+            if (!GATEUP) {
+                for (int i = et; i < n; i += 128) w_s[i] = ds.w >= 0 ? 1.0f : __ldg(&g.wsorted[ds.y + i]);
+                asm volatile("bar.sync 2, 128;" ::: "memory");
+            }
+            const int b = it % C::kAccBufs, use = it / C::kAccBufs;
+            if (ok) ok = warp_wait(&accf_bar[b], use & 1, a.status);
+            tc::fence_after();
+            const uint32_t tb = tmem + ((uint32_t)(32 * q) << 16) + b * C::kAccCols;
+            for (int c0 = 0; c0 < nmma && ok; c0 += 16) {
+                uint32_t r0[16];
+                tc::ld16(tb + c0, r0);
+                if (GATEUP) {
+                    uint32_t r1[16];
+                    tc::ld16(tb + C::kN + c0, r1);
+                    bool finite = true;
+                    __half* hrow = static_cast<__half*>(a.h) + (int64_t)ds.y * a.f + jt * kTileM + row;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int tok = c0 + i;
+                        if (tok < n) {
+                            const float hv = silu(__uint_as_float(r0[i])) * __uint_as_float(r1[i]);
+                            finite = finite && fabsf(hv) <= 65504.0f;
+                            hrow[(int64_t)tok * a.f] = __float2half_rn(hv);
+                        }
+                    }
+                    if (!finite) flag_status(a.status, kStatusRange);
+                } else {
+                    __half* orow = g.o + (int64_t)ds.y * a.d + jt * kTileM + row;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int tok = c0 + i;
+                        if (tok < n) orow[(int64_t)tok * a.d] = __float2half_rn(w_s[tok] * __uint_as_float(r0[i]));
+                    }
+                }
+            }
+            tc::fence_before();
+            mbar_arrive(&acce_bar[b]);
+            if (!GATEUP) asm volatile("bar.sync 2, 128;" ::: "memory");  // w_s reads done
+        }
+    } else if (lane == 0) {
+        // ======================= MMA issuer
+        bool ok = true;
+        int gs = 0;
+        int4 nd = my_tiles > 0 ? load_desc(g, bid) : make_int4(0, 0, 0, 0);
+        for (int it = 0; it < my_tiles; ++it) {
+            const int4 ds = nd;
+            if (it + 1 < my_tiles) nd = load_desc(g, bid + (it + 1) * grid);
+            const int nmma = ((ds.z & 0xFFFF) + 15) & ~15;
+            const uint32_t idesc = tc::idesc_f16(kTileM, nmma, false);
+            const int b = it % C::kAccBufs, use = it / C::kAccBufs;
+            if (use > 0 && ok) ok = tc::bar_wait(&acce_bar[b], (use - 1) & 1, a.status);
+            tc::fence_after();
+            const uint32_t acc_addr = tmem + b * C::kAccCols;
+            for (int s = 0; s < KS; ++s, ++gs) {
+                const int st = gs % C::kStages;
+                if (ok) ok = tc::bar_wait(&full_bar[st], (gs / C::kStages) & 1, a.status);
                 tc::fence_after();
                 uint8_t* sb = smem + st * C::kStageBytes;
-                const uint32_t b_addr = smem_addr(sb + C::kMats * C::kA);
+                const uint32_t a_addr = smem_addr(sb), b_addr = smem_addr(sb + C::kMats * C::kA);
 #pragma unroll
                 for (int kk = 0; kk < kStepK / 16; ++kk) {
                     const uint64_t bd = tc::sdesc(b_addr + kk * 32);
                     const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-                    tc::mma(tmem, tc::sdesc(smem_addr(sb) + kk * 32), bd, idesc, acc);
-                    if (GATEUP) tc::mma(tmem + C::kN, tc::sdesc(smem_addr(sb + C::kA) + kk * 32), bd, idesc, acc);
+                    tc::mma(acc_addr, tc::sdesc(a_addr + kk * 32), bd, idesc, acc);
+                    if (GATEUP) tc::mma(acc_addr + C::kN, tc::sdesc(a_addr + C::kA + kk * 32), bd, idesc, acc);
                 }
-                tc::commit(&mma_bar[st]);
+                tc::commit(&empty_bar[st]);
             }
+            tc::commit(&accf_bar[b]);
         }
-        // the last commit tracks every MMA of the tile
-        if (ok) {
-            const uint32_t last = gstep + KS - 1;
-            ok = tc::bar_wait(&mma_bar[last % C::kStages], (last / C::kStages) & 1, a.status);
-        }
-        gstep += KS;
-        all_ok = __syncthreads_and(ok) != 0;
-        tc::fence_after();
-
-        // epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31 (= weight rows);
-        // warps 0-3 take the even 16-column chunks, warps 4-7 the odd ones
-        const int row = 32 * (warp & 3) + lane;
-        for (int c0 = 16 * (warp >> 2); c0 < nmma && all_ok; c0 += 32) {
-            const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c0;
-            uint32_t r0[16];
-            tc::ld16(ta, r0);
-            if (GATEUP) {
-                uint32_t r1[16];
-                tc::ld16(ta + C::kN, r1);
-                bool finite = true;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int tok = c0 + i;
-                    if (tok < ti.n) {
-                        const float hv = silu(__uint_as_float(r0[i])) * __uint_as_float(r1[i]);
-                        finite = finite && fabsf(hv) <= 65504.0f;
-                        static_cast<__half*>(a.h)[(int64_t)(ti.hbase + ti.tt * kExpertTileN + tok) * a.f +
-                                                  ti.jt * kTileM + row] = __float2half_rn(hv);
-                    }
-                }
-                if (!finite) flag_status(a.status, kStatusRange);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int tok = c0 + i;
-                    if (tok < ti.n) {
-                        const int prow = ti.tt * kExpertTileN + tok;
-                        const float wp = ti.shared ? 1.0f : g.w[a.pairs[ti.pair0 + prow]];
-                        g.o[(int64_t)(ti.hbase + prow) * a.d + ti.jt * kTileM + row] =
-                            __float2half_rn(wp * __uint_as_float(r0[i]));
-                    }
-                }
-            }
-        }
-        tc::fence_before();
-        __syncthreads();
     }
-    tc::cp_wait<0>();
     tc::fence_before();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, C::kTmemCols);
+    tc::fence_after();
+    if (warp == kMmaWarp) tc::tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------- router GEMM
@@ -579,24 +684,29 @@ static cudaError_t gemm_bits(const GemmArgs& g, cudaStream_t s) {
     auto kern = expert_gemm_kernel<BITS, GATEUP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
-    kern<<<num_sms(), kGemmThreads, C::kSmem, s>>>(g);
+    kern<<<num_sms(), kExpertThreads, C::kSmem, s>>>(g);
     return cudaGetLastError();
 }
 
-size_t tile_list_words(int E) { return 2 * (size_t)(E + 2); }
+size_t tile_desc_count(int T, int k, int E, int n_shared, int jt) {
+    return (size_t)max_token_tiles(T, k, E, n_shared) * (size_t)jt;
+}
 
-cudaError_t launch_build_tiles(const ExpertArgs& a, int32_t* tiles, cudaStream_t s) {
-    build_tiles_kernel<<<1, 32, 0, s>>>(a, a.f / kTileM, a.d / kTileM, tiles, tiles + a.E + 2);
+cudaError_t launch_build_tiles(const ExpertArgs& a, int4* desc_gu, int4* desc_dn, int32_t* counts, cudaStream_t s) {
+    if (a.n_shared + a.E > kMaxSlots) return cudaErrorInvalidValue;
+    build_tiles_kernel<<<1, kTileListThreads, 0, s>>>(a, a.f / kTileM, a.d / kTileM, desc_gu, desc_dn, counts);
     return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_gateup(const ExpertArgs& a, const void* xh, const int32_t* tiles, cudaStream_t s) {
+cudaError_t launch_gemm_gateup(const ExpertArgs& a, const void* xh, const int4* desc, const int32_t* counts,
+                               cudaStream_t s) {
     GemmArgs g;
     g.e = a;
     g.xh = static_cast<const uint16_t*>(xh);
-    g.w = nullptr;
+    g.wsorted = nullptr;
     g.o = nullptr;
-    g.tiles = tiles;
+    g.desc = desc;
+    g.n_tiles = counts;
     switch (a.bits) {
         case 2: return gemm_bits<2, true>(g, s);
         case 3: return gemm_bits<3, true>(g, s);
@@ -605,13 +715,15 @@ cudaError_t launch_gemm_gateup(const ExpertArgs& a, const void* xh, const int32_
     }
 }
 
-cudaError_t launch_gemm_down(const ExpertArgs& a, const float* w, void* o, const int32_t* tiles, cudaStream_t s) {
+cudaError_t launch_gemm_down(const ExpertArgs& a, const float* wsorted, void* o, const int4* desc,
+                             const int32_t* counts, cudaStream_t s) {
     GemmArgs g;
     g.e = a;
     g.xh = nullptr;
-    g.w = w;
+    g.wsorted = wsorted;
     g.o = static_cast<__half*>(o);
-    g.tiles = tiles + a.E + 2;
+    g.desc = desc;
+    g.n_tiles = counts + 1;
     switch (a.bits) {
         case 2: return gemm_bits<2, false>(g, s);
         case 3: return gemm_bits<3, false>(g, s);

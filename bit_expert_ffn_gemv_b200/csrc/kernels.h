@@ -30,6 +30,8 @@ struct BucketArgs {
     int32_t* active;     // [E] experts with >= 1 pair, ascending
     Meta* meta;
     uint32_t* status;
+    const float* w = nullptr;  // [T x k] routing weights; with wsorted:
+    float* wsorted = nullptr;  // [T*k] w of pairs[pos] at pos (or null: not written)
 };
 
 // Grouped GEMV/GEMM problem description shared by the expert kernels.
@@ -96,10 +98,12 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 cudaError_t launch_to_f16(const void* x, void* xh, int64_t n, uint32_t* status, cudaStream_t s);
 cudaError_t launch_router_gemm(const RouteArgs& a, uint32_t* status, cudaStream_t s);
 float router_gemm_depth(int d);
-size_t tile_list_words(int E);
-cudaError_t launch_build_tiles(const ExpertArgs& a, int32_t* tiles, cudaStream_t s);
-cudaError_t launch_gemm_gateup(const ExpertArgs& a, const void* xh, const int32_t* tiles, cudaStream_t s);
-cudaError_t launch_gemm_down(const ExpertArgs& a, const float* w, void* o, const int32_t* tiles, cudaStream_t s);
+size_t tile_desc_count(int T, int k, int E, int n_shared, int jt);
+cudaError_t launch_build_tiles(const ExpertArgs& a, int4* desc_gu, int4* desc_dn, int32_t* counts, cudaStream_t s);
+cudaError_t launch_gemm_gateup(const ExpertArgs& a, const void* xh, const int4* desc, const int32_t* counts,
+                               cudaStream_t s);
+cudaError_t launch_gemm_down(const ExpertArgs& a, const float* wsorted, void* o, const int4* desc,
+                             const int32_t* counts, cudaStream_t s);
 cudaError_t launch_combine_f16(const CombineArgs& a, const void* o, cudaStream_t s);
 cudaError_t launch_dequant(const uint8_t* codes, const uint16_t* scales, int N, int K, int bits, float* out,
                            cudaStream_t s);

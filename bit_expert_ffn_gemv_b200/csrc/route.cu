@@ -116,22 +116,31 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
     float* dv = lv + E;
     if (t >= T) return;
 
-    // ||x_t||_2 (fp32, inflated to stay an upper bound)
+    // ||x_t||_2 (fp32, inflated to stay an upper bound); 8 values per lane per 256
     const __nv_bfloat16* xt = x + (int64_t)t * d;
     float ss = 0.f;
-    for (int i = lane; i < d; i += 32) {
-        float v = __bfloat162float(xt[i]);
-        ss = fmaf(v, v, ss);
+#pragma unroll 4
+    for (int i = lane * 8; i < d; i += 256) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(xt + i));
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float a = __uint_as_float(u[q] << 16), b = __uint_as_float(u[q] & 0xFFFF0000u);
+            ss = fmaf(a, a, ss);
+            ss = fmaf(b, b, ss);
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float xn = sqrtf(ss) * (1.0f + 1e-5f);
     const float c = 2.0f * depth * 5.9604645e-8f * (1.0f + 1e-5f);
 
+#pragma unroll 8
     for (int e = lane; e < E; e += 32) {
-        float v = logits[(int64_t)t * E + e];
+        const float v = __ldg(&logits[(int64_t)t * E + e]);
+        const float wn = __ldg(&wnorm[e]), b = bias ? fabsf(__ldg(&bias[e])) : 0.0f;
         lv[e] = v;
-        dv[e] = c * (wnorm[e] * xn + (bias ? fabsf(bias[e]) : 0.0f));
+        dv[e] = c * (wn * xn + b);
     }
     __syncwarp();
 
@@ -167,10 +176,19 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
         if (!(lv[a] - dv[a] > lv[b] + dv[b])) ok = false;
     }
     const float lower_k = lv[sel[k - 1]] - dv[sel[k - 1]];
+    // candidates: every expert whose interval reaches the k-th one's lower end,
+    // listed in ascending index order (reusing the bound array, no longer needed)
+    int* cand = reinterpret_cast<int*>(dv);
     int n_cand = 0;
-    for (int e = lane; e < E; e += 32) n_cand += (isnan(lv[e]) ? false : (lv[e] + dv[e] >= lower_k)) ? 1 : 0;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) n_cand += __shfl_xor_sync(0xffffffffu, n_cand, o);
+    for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        const bool is_c = e < E && (isnan(lower_k) || isnan(lv[e]) || lv[e] + dv[e] >= lower_k);
+        const uint32_t m = __ballot_sync(0xffffffffu, is_c);
+        __syncwarp();  // every lane has read dv[e0 .. e0+31] before it is overwritten
+        if (is_c) cand[n_cand + __popc(m & ((1u << lane) - 1u))] = e;
+        n_cand += __popc(m);
+    }
+    __syncwarp();
     if (n_cand != k) ok = false;
     if (isnan(lower_k)) ok = false;
 
@@ -178,43 +196,68 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
     if (ok) {
         for (int r = 0; r < k; ++r) wsel[r] = lv[sel[r]];
     } else {
-        // fp64 logits of every candidate, then exact ranking among them
-        for (int e = 0; e < E; ++e) {
-            bool cand = isnan(lower_k) || isnan(lv[e]) || (lv[e] + dv[e] >= lower_k);
-            if (!cand) {
-                if (lane == 0) lg64[e] = -INFINITY;
-                continue;
-            }
-            double acc = 0.0;
-            const __nv_bfloat16* row = wr + (int64_t)e * d;
-            for (int i = lane; i < d; i += 32)
-                acc = fma((double)__bfloat162float(row[i]), (double)__bfloat162float(xt[i]), acc);
+        // fp64 logits of the candidates (sums of exact bf16 products), 8 products
+        // per lane per 256-wide chunk, several chunks in flight
+        for (int ci = 0; ci < n_cand; ci += 2) {
+            const bool two = ci + 1 < n_cand;
+            const int e0 = cand[ci], e1 = two ? cand[ci + 1] : e0;
+            const __nv_bfloat16* row0 = wr + (int64_t)e0 * d;
+            const __nv_bfloat16* row1 = wr + (int64_t)e1 * d;
+            double acc0 = 0.0, acc1 = 0.0;
+#pragma unroll 4
+            for (int i = lane * 8; i < d; i += 256) {
+                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xt + i));
+                const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(row0 + i));
+                const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(row1 + i));
+                const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w}, u0[4] = {w0.x, w0.y, w0.z, w0.w},
+                               u1[4] = {w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0) lg64[e] = acc + (bias ? (double)bias[e] : 0.0);
+                for (int q = 0; q < 4; ++q) {
+                    const double xl = (double)__uint_as_float(xu[q] << 16);
+                    const double xh = (double)__uint_as_float(xu[q] & 0xFFFF0000u);
+                    acc0 = fma((double)__uint_as_float(u0[q] << 16), xl, acc0);
+                    acc0 = fma((double)__uint_as_float(u0[q] & 0xFFFF0000u), xh, acc0);
+                    acc1 = fma((double)__uint_as_float(u1[q] << 16), xl, acc1);
+                    acc1 = fma((double)__uint_as_float(u1[q] & 0xFFFF0000u), xh, acc1);
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
+                acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
+            }
+            if (lane == 0) {
+                lg64[ci] = acc0 + (bias ? (double)bias[e0] : 0.0);
+                if (two) lg64[ci + 1] = acc1 + (bias ? (double)bias[e1] : 0.0);
+            }
         }
         __syncwarp();
-        uint32_t tk = 0;
+        // exact ranking among the candidates: k rounds of warp argmax on (fp64 logit, index)
+        uint32_t tk = 0;  // bit j <-> candidate lane + 32 j (n_cand <= E <= 1024, so j < 32)
         for (int r = 0; r < k; ++r) {
             double bv = -INFINITY;
-            int bi = 0x7fffffff;
-            for (int j = 0, e = lane; e < E; ++j, e += 32)
-                if (!((tk >> j) & 1u) && (bi == 0x7fffffff || better64(lg64[e], e, bv, bi))) {
-                    bv = lg64[e];
-                    bi = e;
+            int bi = 0x7fffffff, bc = -1;
+            for (int j = 0, ci = lane; ci < n_cand; ++j, ci += 32) {
+                if (!((tk >> j) & 1u) && (bi == 0x7fffffff || better64(lg64[ci], cand[ci], bv, bi))) {
+                    bv = lg64[ci];
+                    bi = cand[ci];
+                    bc = ci;
                 }
+            }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 double ov = __shfl_xor_sync(0xffffffffu, bv, o);
                 int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                int oc = __shfl_xor_sync(0xffffffffu, bc, o);
                 if (oi != 0x7fffffff && (bi == 0x7fffffff || better64(ov, oi, bv, bi))) {
                     bv = ov;
                     bi = oi;
+                    bc = oc;
                 }
             }
             sel[r] = bi;
             wsel[r] = (float)bv;
-            if ((bi & 31) == lane) tk |= 1u << (bi >> 5);
+            if (bc >= 0 && (bc & 31) == lane) tk |= 1u << (bc >> 5);
         }
         if (lane == 0) atomicAdd(&meta->n_fixup, 1);
     }
