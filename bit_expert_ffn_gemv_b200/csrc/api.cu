@@ -15,7 +15,7 @@
 
 static const char* const kKernelNames[MOE_KERNEL_COUNT] = {
     "router_logits", "topk", "bucket", "gemv_gateup", "gemv_down", "combine", "gemm_gateup", "gemm_down",
-    "router_gemm", "decode_fused", "to_f16", "tile_list"};
+    "router_gemm", "decode_fused", "gather_f16", "tile_list"};
 
 struct moe_layer_state {
     const uint8_t* codes = nullptr;
@@ -23,6 +23,8 @@ struct moe_layer_state {
     const void* router_w = nullptr;
     const float* bias = nullptr;
     float* wnorm = nullptr;  // owned
+    moe::GemmMaps w_gu{};    // codes/scales TMA maps, gate/up geometry
+    moe::GemmMaps w_dn{};    // codes/scales TMA maps, down geometry
     bool loaded = false;
 };
 
@@ -48,7 +50,9 @@ struct moe_handle {
     int* sync = nullptr;
     void* x_stage = nullptr;
     void* y_stage = nullptr;
-    void* xh = nullptr;          // fp16 copy of x for the tensor-core path
+    void* xg = nullptr;          // fp16 x rows in group order (tensor-core path)
+    moe::GemmMaps gu_maps{};     // TMA maps of xg (gate/up B) and h (down B); the
+    moe::GemmMaps dn_maps{};     // codes/scales maps come from the layer
     int4* desc_gu = nullptr;     // gate/up tile descriptors
     int4* desc_dn = nullptr;     // down tile descriptors
     int32_t* n_tiles = nullptr;  // [2] descriptor counts
@@ -179,11 +183,6 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
         return do_decode(h, layer, x, T, y, flags, s);
     const bool tc = use_tensor_cores(T, flags);
     cudaError_t e;
-    if (tc) {
-        e = run(h, MOE_K_TO_F16, s,
-                [&] { return moe::launch_to_f16(x, h->xh, (int64_t)T * c.d, h->status, s); });
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
-    }
     moe_status st = do_route(h, layer, x, T, h->ids, h->w, tc, s);
     if (st != MOE_OK) return st;
     moe::BucketArgs ba;
@@ -224,15 +223,30 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     ea.obuf = h->obuf;
     ea.status = h->status;
     if (tc) {
+        e = run(h, MOE_K_GATHER_F16, s, [&] {
+            return moe::launch_gather_f16(x, T, c.d, c.top_k, c.n_shared, h->pairs, h->offsets + c.n_experts, h->xg,
+                                          h->status, s);
+        });
+        if (e != cudaSuccess) return MOE_ERR_CUDA;
         e = run(h, MOE_K_TILE_LIST, s,
                 [&] { return moe::launch_build_tiles(ea, h->desc_gu, h->desc_dn, h->n_tiles, s); });
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         e = run(h, MOE_K_GEMM_GATEUP, s,
-                [&] { return moe::launch_gemm_gateup(ea, h->xh, h->desc_gu, h->n_tiles, s); });
+                [&] {
+                    moe::GemmMaps m = h->gu_maps;
+                    m.codes = L.w_gu.codes;
+                    m.scales = L.w_gu.scales;
+                    return moe::launch_gemm_gateup(ea, m, h->desc_gu, h->n_tiles, s);
+                });
         if (e != cudaSuccess) return MOE_ERR_CUDA;
         // the fp16 partial outputs reuse the fp32 partial-output buffer
         e = run(h, MOE_K_GEMM_DOWN, s,
-                [&] { return moe::launch_gemm_down(ea, h->wsorted, h->obuf, h->desc_dn, h->n_tiles, s); });
+                [&] {
+                    moe::GemmMaps m = h->dn_maps;
+                    m.codes = L.w_dn.codes;
+                    m.scales = L.w_dn.scales;
+                    return moe::launch_gemm_down(ea, m, h->wsorted, h->obuf, h->desc_dn, h->n_tiles, s);
+                });
         if (e != cudaSuccess) return MOE_ERR_CUDA;
     } else {
         e = run(h, MOE_K_GEMV_GATEUP, s, [&] { return moe::launch_gemv_gateup(ea, s); });
@@ -312,7 +326,7 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     const size_t o_ys = take(sizeof(float) * T * (size_t)c.d);
     const size_t o_norms = take(sizeof(float) * E * (size_t)c.n_layers);
     const size_t o_l64 = take(sizeof(double) * std::min<size_t>(T, moe::kDecodeMaxTokens) * E);
-    const size_t o_xh = take(sizeof(uint16_t) * T * (size_t)c.d);
+    const size_t o_xg = take(sizeof(uint16_t) * rows * (size_t)c.d);
     const size_t o_dgu = take(sizeof(int4) * moe::tile_desc_count(c.max_tokens, c.top_k, c.n_experts, c.n_shared,
                                                                    c.f / 128));
     const size_t o_ddn = take(sizeof(int4) * moe::tile_desc_count(c.max_tokens, c.top_k, c.n_experts, c.n_shared,
@@ -344,13 +358,15 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     h->sync = reinterpret_cast<int*>(base + o_sync);
     h->x_stage = base + o_xs;
     h->y_stage = base + o_ys;
-    h->xh = base + o_xh;
+    h->xg = base + o_xg;
     h->desc_gu = reinterpret_cast<int4*>(base + o_dgu);
     h->desc_dn = reinterpret_cast<int4*>(base + o_ddn);
     h->n_tiles = reinterpret_cast<int32_t*>(base + o_ntiles);
     h->wsorted = reinterpret_cast<float*>(base + o_wsorted);
     for (int l = 0; l < c.n_layers; ++l) h->layers[l].wnorm = reinterpret_cast<float*>(base + o_norms) + E * l;
-    if (cudaMemset(h->arena, 0, h->arena_bytes) != cudaSuccess) {
+    if (cudaMemset(h->arena, 0, h->arena_bytes) != cudaSuccess ||
+        moe::make_row_maps(&h->gu_maps, h->xg, (int64_t)rows, c.d) != cudaSuccess ||
+        moe::make_row_maps(&h->dn_maps, h->h, (int64_t)rows, c.f) != cudaSuccess) {
         cudaFree(h->arena);
         delete h;
         return MOE_ERR_CUDA;
@@ -371,6 +387,10 @@ moe_status moe_load_layer(moe_handle* h, int32_t layer, const moe_layer_weights*
     L.scales = static_cast<const uint16_t*>(w->scales);
     L.router_w = w->router_w;
     L.bias = w->router_bias;
+    const int ne = h->cfg.n_experts + h->cfg.n_shared;
+    if (moe::make_weight_maps(&L.w_gu, L.codes, L.scales, ne, h->cfg.f, h->cfg.d, h->cfg.bits) != cudaSuccess ||
+        moe::make_weight_maps(&L.w_dn, L.codes, L.scales, ne, h->cfg.d, h->cfg.f, h->cfg.bits) != cudaSuccess)
+        return MOE_ERR_CUDA;
     cudaError_t e = moe::launch_router_norms(L.router_w, h->cfg.n_experts, h->cfg.d, L.wnorm, 0);
     if (e == cudaSuccess) e = cudaStreamSynchronize(0);
     if (e != cudaSuccess) return MOE_ERR_CUDA;

@@ -11,12 +11,13 @@
 // Each CTA owns one tile at a time: 128 weight rows (the MMA's M, "swap AB")
 // by up to 256 tokens (the MMA's N, rounded up to a multiple of 16 for small
 // expert groups), accumulated in tensor memory (TMEM) over K in steps of 64.
-// A 3- or 4-stage cp.async pipeline brings in the tokens' activation rows and
-// the packed weight codes; the CTA's threads turn codes into fp16(q * s) and
-// write them straight into the 128-byte-swizzled K-major layout the MMA reads;
-// one thread issues tcgen05.mma (kind::f16, fp32 accumulate) and commits each
-// step to an mbarrier, so dequantising step s overlaps the MMAs of step s - 1.
-// The epilogue reads TMEM with tcgen05.ld.  Every wait is bounded.
+// The tokens' activation rows (h, or x gathered into group order) arrive by
+// 2-D TMA straight into the 128-byte-swizzled K-major layout the MMA reads;
+// the packed codes and scales arrive by 1-D bulk copies; the CTA's threads
+// turn codes into fp16(q * s) in the same swizzled layout; one thread issues
+// tcgen05.mma (kind::f16, fp32 accumulate); the epilogue reads TMEM with
+// tcgen05.ld.  Every wait is bounded.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -25,7 +26,7 @@
 namespace moe {
 namespace tc {
 
-constexpr uint32_t kSpin = 1u << 20;
+constexpr uint32_t kSpin = 1u << 24;  // polls of a non-blocking test (about 0.5 s)
 
 MOE_DEV uint64_t sdesc(uint32_t addr) {
     // K-major, 128-byte swizzle: 8-row atoms of 1024 B, 16-B LBO, SM100 version 1
@@ -66,13 +67,18 @@ MOE_DEV void commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
                  : "memory");
 }
-MOE_DEV void ld16(uint32_t taddr, uint32_t (&r)[16]) {
+// 16 consecutive 32-bit columns of the warp's 32 TMEM lanes (no wait)
+MOE_DEV void ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
           "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+MOE_DEV void ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+MOE_DEV void ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    ld16_nowait(taddr, r);
+    ld_wait();
 }
 
 MOE_DEV void cp16(void* dst, const void* src) {
@@ -90,10 +96,22 @@ MOE_DEV void cp_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// bounded wait on an mbarrier phase; false if it gave up
+MOE_DEV bool test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// bounded wait on an mbarrier phase; false if it gave up.  A non-blocking
+// test in a loop: the waiting thread sees the phase flip at once (a blocking
+// try_wait can leave it suspended for a while after the flip).
 MOE_DEV bool bar_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
     for (uint32_t it = 0; it < kSpin; ++it)
-        if (mbar_try_wait(bar, parity)) return true;
+        if (test_wait(bar, parity)) return true;
     flag_status(status, kStatusTimeout);
     return false;
 }
@@ -205,7 +223,6 @@ __global__ void __launch_bounds__(kTileListThreads)
 
 struct GemmArgs {
     ExpertArgs e;
-    const uint16_t* xh;      // fp16 activations [T x d]
     const float* wsorted;    // routing weight of each pair, in group order [T*k]
     __half* o;               // fp16 weighted expert outputs [rows x d]
     const int4* desc;        // tile descriptors
@@ -214,39 +231,47 @@ struct GemmArgs {
 
 // ---------------------------------------------------------------- grouped expert GEMM
 // GATEUP: A0 = W_g rows, A1 = W_u rows (row-tile jt of f), B = x rows of the
-// slot's tokens; epilogue h = silu(g) * u -> fp16.  Otherwise: A0 = W_d rows
-// (row-tile jt of d), B = h rows; epilogue o = w_p * acc -> fp16.
+// slot's tokens (gathered, fp16); epilogue h = silu(g) * u -> fp16.
+// Otherwise: A0 = W_d rows (row-tile jt of d), B = h rows; epilogue
+// o = w_p * acc -> fp16.
 //
 // Warp roles (persistent; every role walks the same tile sequence
 // blockIdx.x, blockIdx.x + gridDim.x, ...):
-//   warps 0-7   producers: cp.async of codes, scales and B rows S-1 steps
-//               ahead; dequantise the codes of the current step into the A
-//               tiles; signal full[stage]
+//   warp 13     loader (one thread): for each K = 64 step, once the MMAs that
+//               last read the stage are done, TMA loads of the B rows and bulk
+//               copies of the 8 row-tiles' code super-tiles and scales (into the
+//               stage's A area), all completing on load[stage]
+//   warps 0-7   dequant: copy their codes and scales to registers, then write
+//               fp16(q * s) over the same area in the swizzled A layout;
+//               signal full[stage]
+//   warp 12     MMA issuer (one thread): wait full[stage], issue the step's
+//               MMAs, commit to empty[stage]; at the end of a tile commit to
+//               acc_full[buffer]
 //   warps 8-11  epilogue: wait for a finished accumulator, tcgen05.ld, SwiGLU
 //               or weighting, fp16 stores; signal acc_empty[buffer]
-//   warp 12     MMA issuer (one thread): wait full[stage], issue the K = 64
-//               step's MMAs, commit to empty[stage]; at the end of a tile
-//               commit to acc_full[buffer]
 template <int BITS, bool GATEUP>
 struct GemmCfg {
     static constexpr int kN = kExpertTileN;
     static constexpr int kStages = GATEUP ? 3 : 4;
     static constexpr int kMats = GATEUP ? 2 : 1;
-    static constexpr int kCodeBytes = 4096;  // [8 row-tiles][32 lanes][16 B]
-    static constexpr int kScaleBytes = 512;  // [8 row-tiles][8 g][8 B]
     static constexpr int kA = kTileM * 128, kB = kN * 128;
-    static constexpr int kStageRaw = kMats * kA + kB + kMats * (kCodeBytes + kScaleBytes);
-    static constexpr int kStageBytes = (kStageRaw + 1023) & ~1023;
+    static constexpr int kCodeBytes = 8 * 256 * BITS;  // 8 row-tiles x one super-tile, in the A area
+    static constexpr int kScaleBytes = 8 * 128;
+    static_assert(kCodeBytes + kScaleBytes <= kA, "codes fit in the A area");
+    static constexpr int kStageBytes = kMats * kA + kB;
     static constexpr int kSmem = kStages * kStageBytes + 1024;  // + alignment slack
     static constexpr int kAccCols = kMats * kN;                 // one accumulator set
     static constexpr int kAccBufs = 512 / kAccCols;             // 1 (gate/up) or 2 (down)
+    static constexpr uint32_t kStageTxFixed = kMats * (kCodeBytes + kScaleBytes);
     static_assert(kSmem <= 227 * 1024, "shared memory");
     static_assert(kAccBufs >= 1, "tensor memory");
 };
-constexpr int kProducerThreads = 256;
+constexpr int kBRowsSmall = 32;   // rows of the small B TMA box (groups of <= 64 tokens)
+constexpr int kBRowsBig = 256;    // rows of the large B TMA box
 constexpr int kEpilogueWarp0 = 8;
 constexpr int kMmaWarp = 12;
-constexpr int kExpertThreads = 13 * 32;
+constexpr int kLoaderWarp = 13;
+constexpr int kExpertThreads = 14 * 32;
 
 MOE_DEV void producer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
@@ -257,12 +282,25 @@ MOE_DEV bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
     return __shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0;
 }
 
+// 2-D TMA tile load (no multicast) completing on `bar`
+MOE_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
 MOE_DEV int4 load_desc(const GemmArgs& g, int tile) { return __ldg(&g.desc[tile]); }
 
 template <int BITS, bool GATEUP>
-__global__ void __launch_bounds__(kExpertThreads, 1) expert_gemm_kernel(const GemmArgs g) {
+__global__ void __launch_bounds__(kExpertThreads, 1)
+    expert_gemm_kernel(const GemmArgs g, const __grid_constant__ CUtensorMap bmap_s,
+                       const __grid_constant__ CUtensorMap bmap_b, const __grid_constant__ CUtensorMap cmap,
+                       const __grid_constant__ CUtensorMap smap) {
     using C = GemmCfg<BITS, GATEUP>;
     extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t load_bar[C::kStages];
     __shared__ __align__(8) uint64_t full_bar[C::kStages];
     __shared__ __align__(8) uint64_t empty_bar[C::kStages];
     __shared__ __align__(8) uint64_t accf_bar[C::kAccBufs];
@@ -274,11 +312,10 @@ __global__ void __launch_bounds__(kExpertThreads, 1) expert_gemm_kernel(const Ge
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     const int K = GATEUP ? a.d : a.f;  // contraction length
     const int KS = K / kStepK;         // pipeline steps per tile
-    const int KT = K / 128;            // super-tiles along K
-    const int64_t mc = (int64_t)a.f * a.d * BITS / 8, ms = (int64_t)a.f * a.d / 32;
 
     if (tid == 0) {
         for (int i = 0; i < C::kStages; ++i) {
+            mbar_init(&load_bar[i], 1);
             mbar_init(&full_bar[i], 1);
             mbar_init(&empty_bar[i], 1);
         }
@@ -297,95 +334,50 @@ __global__ void __launch_bounds__(kExpertThreads, 1) expert_gemm_kernel(const Ge
     const int total_tiles = *g.n_tiles;
     const int bid = (int)blockIdx.x, grid = (int)gridDim.x;
     const int my_tiles = total_tiles > bid ? (total_tiles - 1 - bid) / grid + 1 : 0;
+    const int total = my_tiles * KS;  // K steps of this CTA
 
     if (warp < kEpilogueWarp0) {
-        // ======================= producers
-        const int total = my_tiles * KS;
-        constexpr int L = C::kStages - 1;  // steps loaded ahead
+        // ======================= dequant
         bool ok = true;
-        // load cursor: its tile's descriptor, the next one (prefetched), and this
-        // thread's 8 B-row sources (rows rb + 32 i, 16-byte chunk cb)
-        const int cb = tid & 7, rb = tid >> 3;
-        int lt_idx = -1;
-        int4 ld = make_int4(0, 0, 0, 0), nd = my_tiles > 0 ? load_desc(g, bid) : make_int4(0, 0, 0, 0);
-        const uint16_t* rowp[8];
-        int lt_nmma = 0;
-        auto load_step = [&](int j) {
-            const int ti_local = j / KS, s = j - ti_local * KS, st = j % C::kStages;
-            if (ti_local != lt_idx) {
-                lt_idx = ti_local;
-                ld = nd;
-                if (ti_local + 1 < my_tiles) nd = load_desc(g, bid + (ti_local + 1) * grid);
-                const int n = ld.z & 0xFFFF;
-                lt_nmma = (n + 15) & ~15;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int rr = min(rb + 32 * i, n - 1);  // rows past the group repeat its last row
-                    if (GATEUP) {
-                        const int tok = ld.w >= 0 ? ld.w + rr : __ldg(&a.pairs[ld.y + rr]) / a.k;
-                        rowp[i] = g.xh + (int64_t)tok * a.d;
-                    } else {
-                        rowp[i] = reinterpret_cast<const uint16_t*>(a.h) + (int64_t)(ld.y + rr) * a.f;
-                    }
-                }
-            }
+        const int rt = tid >> 5, ln = tid & 31, gg = ln >> 2, c = ln & 3;
+        for (int gs = 0; gs < total; ++gs) {
+            const int st = gs % C::kStages, hs = (gs % KS) & 1;
+            if (tid == 0 && ok) ok = tc::bar_wait(&load_bar[st], (gs / C::kStages) & 1, a.status);
+            producer_sync();  // codes, scales and B rows of step gs have landed
             uint8_t* sb = smem + st * C::kStageBytes;
-            uint8_t* Bs = sb + C::kMats * C::kA;
-            uint8_t* Cs = Bs + C::kB;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int r = rb + 32 * i;
-                if (r < lt_nmma) tc::cp16(Bs + tc::sw128_chunk(r, cb), rowp[i] + s * kStepK + cb * 8);
-            }
-            // codes and scales: thread = (row-tile, lane); step s is half hs of super-tile kt
-            const int expert = ld.x, jt = ld.z >> 16;
-            const uint8_t* cbase = a.codes + ((int64_t)expert * 3 + (GATEUP ? 0 : 2)) * mc;
-            const uint8_t* sbase =
-                reinterpret_cast<const uint8_t*>(a.scales) + ((int64_t)expert * 3 + (GATEUP ? 0 : 2)) * ms * 2;
-            const int kt = s >> 1, hs = s & 1;
-            const int rt = tid >> 5, ln = tid & 31;
+            uint32_t lo[C::kMats][2], hi[C::kMats][2], sc[C::kMats][2];
 #pragma unroll
             for (int m = 0; m < C::kMats; ++m) {
-                uint8_t* cs = Cs + m * (C::kCodeBytes + C::kScaleBytes);
-                uint8_t* ss = cs + C::kCodeBytes;
-                const int64_t st_idx = (int64_t)(jt * 8 + rt) * KT + kt;
-                const uint8_t* stile = cbase + m * mc + st_idx * (256 * BITS);
-                uint8_t* dst = cs + (rt * 32 + ln) * 16;
-                tc::cp8(dst, stile + ln * 16 + hs * 8);
-                if (BITS == 3) tc::cp4(dst + 8, stile + 512 + ln * 8 + hs * 4);
-                if (BITS == 4) tc::cp8(dst + 8, stile + 512 + ln * 16 + hs * 8);
-                if (ln < 8) tc::cp8(ss + rt * 64 + ln * 8, sbase + m * ms * 2 + st_idx * 128 + ln * 16 + hs * 8);
+                const uint8_t* cs = sb + m * C::kA + rt * (256 * BITS);
+                const uint2 w = *reinterpret_cast<const uint2*>(cs + 16 * ln + 8 * hs);
+                lo[m][0] = w.x;
+                lo[m][1] = w.y;
+                if (BITS == 3) {
+                    const uint32_t hv = *reinterpret_cast<const uint32_t*>(cs + 512 + 8 * ln + 4 * hs);
+                    hi[m][0] = hv & 0xFFFFu;
+                    hi[m][1] = hv >> 16;
+                } else if (BITS == 4) {
+                    const uint2 hv = *reinterpret_cast<const uint2*>(cs + 512 + 16 * ln + 8 * hs);
+                    hi[m][0] = hv.x;
+                    hi[m][1] = hv.y;
+                } else {
+                    hi[m][0] = hi[m][1] = 0;
+                }
+                const uint2 sv = *reinterpret_cast<const uint2*>(sb + m * C::kA + C::kCodeBytes + rt * 128 +
+                                                                 16 * gg + 8 * hs);
+                sc[m][0] = sv.x;
+                sc[m][1] = sv.y;
             }
-        };
-        // codes of stage st -> fp16(q * s) in the SW128 A tiles of that stage
-        auto dequant_step = [&](int st) {
-            uint8_t* sb = smem + st * C::kStageBytes;
-            uint8_t* Cs = sb + C::kMats * C::kA + C::kB;
-            const int rt = tid >> 5, ln = tid & 31, gg = ln >> 2, c = ln & 3;
+            producer_sync();  // every read of the staged codes is done before A overwrites them
 #pragma unroll
             for (int m = 0; m < C::kMats; ++m) {
                 uint8_t* A = sb + m * C::kA;
-                const uint8_t* cs = Cs + m * (C::kCodeBytes + C::kScaleBytes);
-                const uint8_t* src = cs + (rt * 32 + ln) * 16;
-                const uint2 lo = *reinterpret_cast<const uint2*>(src);
-                uint32_t hi0 = 0, hi1 = 0;
-                if (BITS == 3) {
-                    const uint32_t hv = *reinterpret_cast<const uint32_t*>(src + 8);
-                    hi0 = hv & 0xFFFFu;
-                    hi1 = hv >> 16;
-                } else if (BITS == 4) {
-                    const uint2 hv = *reinterpret_cast<const uint2*>(src + 8);
-                    hi0 = hv.x;
-                    hi1 = hv.y;
-                }
-                const uint2 sc = *reinterpret_cast<const uint2*>(cs + C::kCodeBytes + rt * 64 + gg * 8);
-                const uint32_t words[2] = {lo.x, lo.y}, his[2] = {hi0, hi1}, scs[2] = {sc.x, sc.y};
 #pragma unroll
                 for (int kbl = 0; kbl < 2; ++kbl) {
                     uint32_t q[8];
-                    decode_block<true, BITS>(words[kbl], his[kbl], q);
-                    const __half2 s_lo = __half2half2(__ushort_as_half((unsigned short)(scs[kbl] & 0xFFFFu)));
-                    const __half2 s_hi = __half2half2(__ushort_as_half((unsigned short)(scs[kbl] >> 16)));
+                    decode_block<true, BITS>(lo[m][kbl], hi[m][kbl], q);
+                    const __half2 s_lo = __half2half2(__ushort_as_half((unsigned short)(sc[m][kbl] & 0xFFFFu)));
+                    const __half2 s_hi = __half2half2(__ushort_as_half((unsigned short)(sc[m][kbl] >> 16)));
 #pragma unroll
                     for (int p = 0; p < 8; ++p) {
                         // pair p = 4 ks + 2 (m / 8) + r / 8 of the A-fragment layout
@@ -397,29 +389,10 @@ __global__ void __launch_bounds__(kExpertThreads, 1) expert_gemm_kernel(const Ge
                     }
                 }
             }
-        };
-        // the first S steps find their stages free
-        for (int j = 0; j < L; ++j) {
-            if (j < total) load_step(j);
-            tc::cp_commit();
-        }
-        for (int gs = 0; gs < total; ++gs) {
-            const int st = gs % C::kStages;
-            tc::cp_wait<L - 1>();  // this thread's copies of step gs have landed
-            producer_sync();       // ... and every producer's
-            dequant_step(st);
-            fence_proxy_async_smem();  // A and B tiles visible to the tensor core
+            fence_proxy_async_smem();  // A tiles visible to the tensor core
             producer_sync();
             if (tid == 0) mbar_arrive(&full_bar[st]);
-            const int j = gs + L;
-            if (j < total) {
-                if (j >= C::kStages && ok)  // the MMAs of step j - S have read the stage
-                    ok = tc::bar_wait(&empty_bar[j % C::kStages], ((j / C::kStages) - 1) & 1, a.status);
-                load_step(j);
-            }
-            tc::cp_commit();
         }
-        tc::cp_wait<0>();
     } else if (warp < kMmaWarp) {
         // ======================= epilogue
         const int q = warp & 3;  // TMEM lanes 32 q .. 32 q + 31 = weight rows
@@ -441,23 +414,26 @@ __global__ void __launch_bounds__(kExpertThreads, 1) expert_gemm_kernel(const Ge
             const uint32_t tb = tmem + ((uint32_t)(32 * q) << 16) + b * C::kAccCols;
             for (int c0 = 0; c0 < nmma && ok; c0 += 16) {
                 uint32_t r0[16];
-                tc::ld16(tb + c0, r0);
                 if (GATEUP) {
                     uint32_t r1[16];
-                    tc::ld16(tb + C::kN + c0, r1);
+                    tc::ld16_nowait(tb + c0, r0);
+                    tc::ld16_nowait(tb + C::kN + c0, r1);
+                    tc::ld_wait();
                     bool finite = true;
                     __half* hrow = static_cast<__half*>(a.h) + (int64_t)ds.y * a.f + jt * kTileM + row;
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int tok = c0 + i;
                         if (tok < n) {
-                            const float hv = silu(__uint_as_float(r0[i])) * __uint_as_float(r1[i]);
+                            const float gv = __uint_as_float(r0[i]);
+                            const float hv = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(r1[i]);
                             finite = finite && fabsf(hv) <= 65504.0f;
                             hrow[(int64_t)tok * a.f] = __float2half_rn(hv);
                         }
                     }
                     if (!finite) flag_status(a.status, kStatusRange);
                 } else {
+                    tc::ld16(tb + c0, r0);
                     __half* orow = g.o + (int64_t)ds.y * a.d + jt * kTileM + row;
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
@@ -470,36 +446,81 @@ __global__ void __launch_bounds__(kExpertThreads, 1) expert_gemm_kernel(const Ge
             mbar_arrive(&acce_bar[b]);
             if (!GATEUP) asm volatile("bar.sync 2, 128;" ::: "memory");  // w_s reads done
         }
-    } else if (lane == 0) {
-        // ======================= MMA issuer
-        bool ok = true;
-        int gs = 0;
-        int4 nd = my_tiles > 0 ? load_desc(g, bid) : make_int4(0, 0, 0, 0);
-        for (int it = 0; it < my_tiles; ++it) {
-            const int4 ds = nd;
-            if (it + 1 < my_tiles) nd = load_desc(g, bid + (it + 1) * grid);
-            const int nmma = ((ds.z & 0xFFFF) + 15) & ~15;
-            const uint32_t idesc = tc::idesc_f16(kTileM, nmma, false);
-            const int b = it % C::kAccBufs, use = it / C::kAccBufs;
-            if (use > 0 && ok) ok = tc::bar_wait(&acce_bar[b], (use - 1) & 1, a.status);
-            tc::fence_after();
-            const uint32_t acc_addr = tmem + b * C::kAccCols;
-            for (int s = 0; s < KS; ++s, ++gs) {
-                const int st = gs % C::kStages;
-                if (ok) ok = tc::bar_wait(&full_bar[st], (gs / C::kStages) & 1, a.status);
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            // ======================= MMA issuer
+            bool ok = true;
+            int gs = 0;
+            int4 nd = my_tiles > 0 ? load_desc(g, bid) : make_int4(0, 0, 0, 0);
+            for (int it = 0; it < my_tiles; ++it) {
+                const int4 ds = nd;
+                if (it + 1 < my_tiles) nd = load_desc(g, bid + (it + 1) * grid);
+                const int nmma = ((ds.z & 0xFFFF) + 15) & ~15;
+                const uint32_t idesc = tc::idesc_f16(kTileM, nmma, false);
+                const int b = it % C::kAccBufs, use = it / C::kAccBufs;
+                if (use > 0 && ok) ok = tc::bar_wait(&acce_bar[b], (use - 1) & 1, a.status);
                 tc::fence_after();
-                uint8_t* sb = smem + st * C::kStageBytes;
-                const uint32_t a_addr = smem_addr(sb), b_addr = smem_addr(sb + C::kMats * C::kA);
+                const uint32_t acc_addr = tmem + b * C::kAccCols;
+                for (int s = 0; s < KS; ++s, ++gs) {
+                    const int st = gs % C::kStages;
+                    if (ok) ok = tc::bar_wait(&full_bar[st], (gs / C::kStages) & 1, a.status);
+                    tc::fence_after();
+                    uint8_t* sb = smem + st * C::kStageBytes;
+                    const uint32_t a_addr = smem_addr(sb), b_addr = smem_addr(sb + C::kMats * C::kA);
 #pragma unroll
-                for (int kk = 0; kk < kStepK / 16; ++kk) {
-                    const uint64_t bd = tc::sdesc(b_addr + kk * 32);
-                    const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-                    tc::mma(acc_addr, tc::sdesc(a_addr + kk * 32), bd, idesc, acc);
-                    if (GATEUP) tc::mma(acc_addr + C::kN, tc::sdesc(a_addr + C::kA + kk * 32), bd, idesc, acc);
+                    for (int kk = 0; kk < kStepK / 16; ++kk) {
+                        const uint64_t bd = tc::sdesc(b_addr + kk * 32);
+                        const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                        tc::mma(acc_addr, tc::sdesc(a_addr + kk * 32), bd, idesc, acc);
+                        if (GATEUP) tc::mma(acc_addr + C::kN, tc::sdesc(a_addr + C::kA + kk * 32), bd, idesc, acc);
+                    }
+                    tc::commit(&empty_bar[st]);
                 }
-                tc::commit(&empty_bar[st]);
+                tc::commit(&accf_bar[b]);
             }
-            tc::commit(&accf_bar[b]);
+        }
+    } else if (warp == kLoaderWarp && lane == 0) {
+        // ======================= loader
+        // Per step: the B rows (one 256-row box, or 32-row boxes for small
+        // groups) and, per matrix, one box of 8 row-tiles x one super-tile of
+        // codes and one of scales (the codes and scales tensor maps view a
+        // matrix as rows of 16-row tiles, columns of 128-wide super-tiles).
+        bool ok = true;
+        const int mrows = (GATEUP ? a.f : a.d) / 16;  // map rows per matrix
+        int4 ds = make_int4(0, 0, 0, 0);
+        int4 nd = my_tiles > 0 ? load_desc(g, bid) : make_int4(0, 0, 0, 0);
+        int cur = -1, nmma = 0;
+        for (int j = 0; j < total; ++j) {
+            const int ti_local = j / KS, s = j - ti_local * KS, st = j % C::kStages;
+            if (ti_local != cur) {
+                cur = ti_local;
+                ds = nd;
+                if (ti_local + 1 < my_tiles) nd = load_desc(g, bid + (ti_local + 1) * grid);
+                nmma = ((ds.z & 0xFFFF) + 15) & ~15;
+            }
+            if (j >= C::kStages && ok)  // the MMAs of step j - S have read the stage
+                ok = tc::bar_wait(&empty_bar[st], ((j / C::kStages) - 1) & 1, a.status);
+            uint8_t* sb = smem + st * C::kStageBytes;
+            uint8_t* Bs = sb + C::kMats * C::kA;
+            const bool big = nmma > 2 * kBRowsSmall;
+            const int nsmall = (nmma + kBRowsSmall - 1) / kBRowsSmall;
+            mbar_arrive_expect_tx(&load_bar[st],
+                                  C::kStageTxFixed + (uint32_t)(big ? kBRowsBig : nsmall * kBRowsSmall) * 128);
+            if (big) {
+                tma_load_2d(Bs, &bmap_b, s * kStepK, ds.y, &load_bar[st]);
+            } else {
+                for (int i = 0; i < nsmall; ++i)
+                    tma_load_2d(Bs + i * kBRowsSmall * 128, &bmap_s, s * kStepK, ds.y + i * kBRowsSmall,
+                                &load_bar[st]);
+            }
+            const int expert = ds.x, jt = ds.z >> 16, kt = s >> 1;
+#pragma unroll
+            for (int m = 0; m < C::kMats; ++m) {
+                uint8_t* A = sb + m * C::kA;
+                const int row = (expert * 3 + (GATEUP ? m : 2)) * mrows + jt * 8;
+                tma_load_2d(A, &cmap, kt * 64 * BITS, row, &load_bar[st]);
+                tma_load_2d(A + C::kCodeBytes, &smap, kt * 64, row, &load_bar[st]);
+            }
         }
     }
     tc::fence_before();
@@ -608,23 +629,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 0) tc::tmem_dealloc(tmem, kRouterTileN);
 }
 
-// ---------------------------------------------------------------- activations to fp16, combine
-__global__ void to_f16_kernel(const __nv_bfloat16* __restrict__ x, __half* __restrict__ xh, int64_t n,
-                              uint32_t* status) {
-    const int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
-    if (i >= n) return;
-    const uint4 v = *reinterpret_cast<const uint4*>(x + i);
-    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-    uint32_t out[4];
-    bool finite = true;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float lo = __uint_as_float(in[j] << 16), hi = __uint_as_float(in[j] & 0xFFFF0000u);
-        finite = finite && fabsf(lo) <= 65504.0f && fabsf(hi) <= 65504.0f;
-        const __half2 hv = __floats2half2_rn(lo, hi);
-        out[j] = *reinterpret_cast<const uint32_t*>(&hv);
+// ---------------------------------------------------------------- activation gather, combine
+// xg[row] = fp16(x[token of row]) in group order: rows [0, offsets[E]) are
+// the routed pairs (token pairs[row] / k), rows T*k + t the shared expert's.
+__global__ void gather_f16_kernel(const __nv_bfloat16* __restrict__ x, int T, int d, int k, int n_shared,
+                                  const int32_t* __restrict__ pairs, const int32_t* __restrict__ n_pairs,
+                                  __half* __restrict__ xg, uint32_t* status) {
+    const int row = blockIdx.x;
+    int tok;
+    if (row < T * k) {
+        if (row >= *n_pairs) return;
+        tok = pairs[row] / k;
+    } else {
+        tok = row - T * k;
     }
-    *reinterpret_cast<uint4*>(xh + i) = make_uint4(out[0], out[1], out[2], out[3]);
+    bool finite = true;
+    for (int i = threadIdx.x * 8; i < d; i += blockDim.x * 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(x + (int64_t)tok * d + i);
+        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+        uint32_t out[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float lo = __uint_as_float(in[j] << 16), hi = __uint_as_float(in[j] & 0xFFFF0000u);
+            finite = finite && fabsf(lo) <= 65504.0f && fabsf(hi) <= 65504.0f;
+            const __half2 hv = __floats2half2_rn(lo, hi);
+            out[j] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        *reinterpret_cast<uint4*>(xg + (int64_t)row * d + i) = make_uint4(out[0], out[1], out[2], out[3]);
+    }
     if (!finite) flag_status(status, kStatusRange);
 }
 
@@ -679,12 +711,12 @@ static int num_sms() {
 }
 
 template <int BITS, bool GATEUP>
-static cudaError_t gemm_bits(const GemmArgs& g, cudaStream_t s) {
+static cudaError_t gemm_bits(const GemmArgs& g, const GemmMaps& m, cudaStream_t s) {
     using C = GemmCfg<BITS, GATEUP>;
     auto kern = expert_gemm_kernel<BITS, GATEUP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     if (e != cudaSuccess) return e;
-    kern<<<num_sms(), kExpertThreads, C::kSmem, s>>>(g);
+    kern<<<num_sms(), kExpertThreads, C::kSmem, s>>>(g, m.b_small, m.b_big, m.codes, m.scales);
     return cudaGetLastError();
 }
 
@@ -698,38 +730,91 @@ cudaError_t launch_build_tiles(const ExpertArgs& a, int4* desc_gu, int4* desc_dn
     return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_gateup(const ExpertArgs& a, const void* xh, const int4* desc, const int32_t* counts,
+cudaError_t launch_gemm_gateup(const ExpertArgs& a, const GemmMaps& maps, const int4* desc, const int32_t* counts,
                                cudaStream_t s) {
     GemmArgs g;
     g.e = a;
-    g.xh = static_cast<const uint16_t*>(xh);
     g.wsorted = nullptr;
     g.o = nullptr;
     g.desc = desc;
     g.n_tiles = counts;
     switch (a.bits) {
-        case 2: return gemm_bits<2, true>(g, s);
-        case 3: return gemm_bits<3, true>(g, s);
-        case 4: return gemm_bits<4, true>(g, s);
+        case 2: return gemm_bits<2, true>(g, maps, s);
+        case 3: return gemm_bits<3, true>(g, maps, s);
+        case 4: return gemm_bits<4, true>(g, maps, s);
         default: return cudaErrorInvalidValue;
     }
 }
 
-cudaError_t launch_gemm_down(const ExpertArgs& a, const float* wsorted, void* o, const int4* desc,
-                             const int32_t* counts, cudaStream_t s) {
+cudaError_t launch_gemm_down(const ExpertArgs& a, const GemmMaps& maps, const float* wsorted, void* o,
+                             const int4* desc, const int32_t* counts, cudaStream_t s) {
     GemmArgs g;
     g.e = a;
-    g.xh = nullptr;
     g.wsorted = wsorted;
     g.o = static_cast<__half*>(o);
     g.desc = desc;
     g.n_tiles = counts + 1;
     switch (a.bits) {
-        case 2: return gemm_bits<2, false>(g, s);
-        case 3: return gemm_bits<3, false>(g, s);
-        case 4: return gemm_bits<4, false>(g, s);
+        case 2: return gemm_bits<2, false>(g, maps, s);
+        case 3: return gemm_bits<3, false>(g, maps, s);
+        case 4: return gemm_bits<4, false>(g, maps, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+using Encode = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                            const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                            CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+static Encode encoder() {
+    static Encode encode = nullptr;
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return nullptr;
+        encode = reinterpret_cast<Encode>(fn);
+    }
+    return encode;
+}
+
+static cudaError_t encode_2d(CUtensorMap* map, CUtensorMapDataType type, int elem_bytes, const void* base,
+                             int64_t rows, int64_t row_elems, int box_inner, int box_rows, CUtensorMapSwizzle swz) {
+    Encode encode = encoder();
+    if (!encode) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {(cuuint64_t)row_elems, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)row_elems * elem_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Maps of a row-major fp16 activation matrix [rows x cols] (xg or h) for
+// boxes of 64 columns (128 B) x 32 or 256 rows, 128-byte swizzle (the MMA's
+// K-major layout); rows past the end read as zeros.
+cudaError_t make_row_maps(GemmMaps* m, const void* base, int64_t rows, int cols) {
+    cudaError_t e = encode_2d(&m->b_small, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, rows, cols, 64, kBRowsSmall,
+                              CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    return encode_2d(&m->b_big, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, rows, cols, 64, kBRowsBig,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Maps of a layer's packed codes and scales for matrices [N x K] (gate/up:
+// N = f, K = d; down: N = d, K = f): every matrix is N/16 rows of K/128
+// super-tiles, and all E + n_shared experts' three matrices are stacked, so
+// row (expert * 3 + mat) * N/16 + tile is 16-row tile `tile` of that matrix.
+// One box = 8 row-tiles x one super-tile (256 b bytes of codes as 32-bit
+// words; 64 fp16 scales).
+cudaError_t make_weight_maps(GemmMaps* m, const void* codes, const void* scales, int n_experts_total, int N, int K,
+                             int bits) {
+    const int64_t rows = (int64_t)n_experts_total * 3 * (N / 16);
+    cudaError_t e = encode_2d(&m->codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, codes, rows, (int64_t)(K / 128) * 64 * bits,
+                              64 * bits, 8, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e != cudaSuccess) return e;
+    return encode_2d(&m->scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, scales, rows, (int64_t)(K / 128) * 64, 64, 8,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 cudaError_t launch_router_gemm(const RouteArgs& a, uint32_t* status, cudaStream_t s) {
@@ -753,10 +838,11 @@ cudaError_t launch_router_gemm(const RouteArgs& a, uint32_t* status, cudaStream_
 // plus the fp32 bias add: depth = 34 * (d / 16) + 2.
 float router_gemm_depth(int d) { return 34.0f * (float)(d / 16) + 2.0f; }
 
-cudaError_t launch_to_f16(const void* x, void* xh, int64_t n, uint32_t* status, cudaStream_t s) {
-    const int64_t threads = n / 8;
-    to_f16_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x),
-                                                                    static_cast<__half*>(xh), n, status);
+cudaError_t launch_gather_f16(const void* x, int T, int d, int k, int n_shared, const int32_t* pairs,
+                              const int32_t* n_pairs, void* xg, uint32_t* status, cudaStream_t s) {
+    const int rows = T * k + n_shared * T;
+    gather_f16_kernel<<<rows, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, d, k, n_shared, pairs, n_pairs,
+                                          static_cast<__half*>(xg), status);
     return cudaGetLastError();
 }
 

@@ -1,5 +1,6 @@
 // kernels.h -- host-side launchers of the routed-MoE kernels (internal).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -95,15 +96,24 @@ cudaError_t launch_gemv_gateup(const ExpertArgs& a, cudaStream_t s);
 cudaError_t launch_gemv_down(const ExpertArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 // tcgen05 path (T > kDecodeMaxTokens)
-cudaError_t launch_to_f16(const void* x, void* xh, int64_t n, uint32_t* status, cudaStream_t s);
 cudaError_t launch_router_gemm(const RouteArgs& a, uint32_t* status, cudaStream_t s);
 float router_gemm_depth(int d);
 size_t tile_desc_count(int T, int k, int E, int n_shared, int jt);
 cudaError_t launch_build_tiles(const ExpertArgs& a, int4* desc_gu, int4* desc_dn, int32_t* counts, cudaStream_t s);
-cudaError_t launch_gemm_gateup(const ExpertArgs& a, const void* xh, const int4* desc, const int32_t* counts,
+// TMA descriptors of one expert GEMM: its activation rows (two box heights)
+// and the layer's packed codes and scales.
+struct GemmMaps {
+    CUtensorMap b_small, b_big, codes, scales;
+};
+cudaError_t make_row_maps(GemmMaps* m, const void* base, int64_t rows, int cols);
+cudaError_t make_weight_maps(GemmMaps* m, const void* codes, const void* scales, int n_experts_total, int N, int K,
+                             int bits);
+cudaError_t launch_gather_f16(const void* x, int T, int d, int k, int n_shared, const int32_t* pairs,
+                              const int32_t* n_pairs, void* xg, uint32_t* status, cudaStream_t s);
+cudaError_t launch_gemm_gateup(const ExpertArgs& a, const GemmMaps& maps, const int4* desc, const int32_t* counts,
                                cudaStream_t s);
-cudaError_t launch_gemm_down(const ExpertArgs& a, const float* wsorted, void* o, const int4* desc,
-                             const int32_t* counts, cudaStream_t s);
+cudaError_t launch_gemm_down(const ExpertArgs& a, const GemmMaps& maps, const float* wsorted, void* o,
+                             const int4* desc, const int32_t* counts, cudaStream_t s);
 cudaError_t launch_combine_f16(const CombineArgs& a, const void* o, cudaStream_t s);
 cudaError_t launch_dequant(const uint8_t* codes, const uint16_t* scales, int N, int K, int bits, float* out,
                            cudaStream_t s);

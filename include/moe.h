@@ -240,7 +240,7 @@ enum {
     MOE_K_GEMM_DOWN = 7,
     MOE_K_ROUTER_GEMM = 8,
     MOE_K_DECODE = 9,
-    MOE_K_TO_F16 = 10,
+    MOE_K_GATHER_F16 = 10,
     MOE_K_TILE_LIST = 11,
     MOE_KERNEL_COUNT = 12
 };
