@@ -307,6 +307,7 @@ __global__ void __launch_bounds__(kExpertThreads, 1)
     __shared__ __align__(8) uint64_t acce_bar[C::kAccBufs];
     __shared__ uint32_t tmem_slot;
     __shared__ float w_s[GATEUP ? 1 : kExpertTileN];  // routing weights of the epilogue's tile
+    __shared__ __align__(16) __half ep_stage[4][16][32];  // epilogue transpose, one [token][row] block per warp
     const ExpertArgs& a = g.e;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
@@ -395,9 +396,14 @@ __global__ void __launch_bounds__(kExpertThreads, 1)
         }
     } else if (warp < kMmaWarp) {
         // ======================= epilogue
+        // Thread = weight row (TMEM lane); per 16-token chunk the next chunk's
+        // TMEM loads are in flight while this one is converted, staged as
+        // [token][32 rows] fp16 in shared memory and written out as 16-byte
+        // vectors (4 lanes cover the warp's 64 contiguous bytes of a token row).
         const int q = warp & 3;  // TMEM lanes 32 q .. 32 q + 31 = weight rows
-        const int row = 32 * q + lane;
         const int et = tid - 32 * kEpilogueWarp0;  // 0 .. 127
+        __half* stg = &ep_stage[q][0][0];
+        const int vt = lane >> 2, seg = lane & 3;  // vector store: token vt (+8), 16-byte segment seg
         bool ok = true;
         int4 nd = my_tiles > 0 ? load_desc(g, bid) : make_int4(0, 0, 0, 0);
         for (int it = 0; it < my_tiles; ++it) {
@@ -412,36 +418,48 @@ __global__ void __launch_bounds__(kExpertThreads, 1)
             if (ok) ok = warp_wait(&accf_bar[b], use & 1, a.status);
             tc::fence_after();
             const uint32_t tb = tmem + ((uint32_t)(32 * q) << 16) + b * C::kAccCols;
+            const int ld_cols = GATEUP ? a.f : a.d;  // row length of h / o
+            __half* dst = (GATEUP ? static_cast<__half*>(a.h) : g.o) + (int64_t)ds.y * ld_cols + jt * kTileM + 32 * q +
+                          seg * 8;
+            uint32_t r0[16], r1[16];
+            if (ok && nmma > 0) {
+                tc::ld16_nowait(tb, r0);
+                if (GATEUP) tc::ld16_nowait(tb + C::kN, r1);
+                tc::ld_wait();
+            }
+            bool finite = true;
             for (int c0 = 0; c0 < nmma && ok; c0 += 16) {
-                uint32_t r0[16];
-                if (GATEUP) {
-                    uint32_t r1[16];
-                    tc::ld16_nowait(tb + c0, r0);
-                    tc::ld16_nowait(tb + C::kN + c0, r1);
-                    tc::ld_wait();
-                    bool finite = true;
-                    __half* hrow = static_cast<__half*>(a.h) + (int64_t)ds.y * a.f + jt * kTileM + row;
+                float v[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int tok = c0 + i;
-                        if (tok < n) {
-                            const float gv = __uint_as_float(r0[i]);
-                            const float hv = __fdividef(gv, 1.0f + __expf(-gv)) * __uint_as_float(r1[i]);
-                            finite = finite && fabsf(hv) <= 65504.0f;
-                            hrow[(int64_t)tok * a.f] = __float2half_rn(hv);
-                        }
-                    }
-                    if (!finite) flag_status(a.status, kStatusRange);
-                } else {
-                    tc::ld16(tb + c0, r0);
-                    __half* orow = g.o + (int64_t)ds.y * a.d + jt * kTileM + row;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int tok = c0 + i;
-                        if (tok < n) orow[(int64_t)tok * a.d] = __float2half_rn(w_s[tok] * __uint_as_float(r0[i]));
+                for (int i = 0; i < 16; ++i) {
+                    const float acc = __uint_as_float(r0[i]);
+                    if (GATEUP) {
+                        const float hv = __fdividef(acc, 1.0f + __expf(-acc)) * __uint_as_float(r1[i]);
+                        finite = finite && fabsf(hv) <= 65504.0f;
+                        v[i] = hv;
+                    } else {
+                        v[i] = w_s[min(c0 + i, kExpertTileN - 1)] * acc;
                     }
                 }
+                const bool more = c0 + 16 < nmma;
+                if (more) {  // next chunk's accumulators load while this one is stored
+                    tc::ld16_nowait(tb + c0 + 16, r0);
+                    if (GATEUP) tc::ld16_nowait(tb + C::kN + c0 + 16, r1);
+                }
+#pragma unroll
+                for (int i = 0; i < 16; ++i) stg[i * 32 + lane] = __float2half_rn(v[i]);
+                __syncwarp();
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int tl = vt + 8 * hh, tok = c0 + tl;
+                    if (tok < n)
+                        *reinterpret_cast<uint4*>(dst + (int64_t)tok * ld_cols) =
+                            *reinterpret_cast<const uint4*>(stg + tl * 32 + seg * 8);
+                }
+                __syncwarp();
+                if (more) tc::ld_wait();
             }
+            if (GATEUP && !finite) flag_status(a.status, kStatusRange);
             tc::fence_before();
             mbar_arrive(&acce_bar[b]);
             if (!GATEUP) asm volatile("bar.sync 2, 128;" ::: "memory");  // w_s reads done
