@@ -49,6 +49,57 @@ def parse():
     return p.parse_args()
 
 
+# ---------------------------------------------------------------- ncu traffic of the dominant kernel
+_KERNEL_SOURCE = {"gemm_gateup": "gemm_sm100.cu", "gemm_down": "gemm_sm100.cu", "router_gemm": "gemm_sm100.cu",
+                  "decode_fused": "decode.cu", "gemv_gateup": "gemv.cu", "gemv_down": "gemv.cu"}
+
+
+def profile_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary (profiles/*.md lines
+    `traffic: kernel=K source_sha256_16=H dram_bytes_per_launch=B`), or None when no capture exists or
+    the kernel's source changed since it was taken."""
+    import glob
+    import hashlib
+    src = _KERNEL_SOURCE.get(kernel)
+    if not src:
+        return None
+    path = os.path.join(ROOT, "bit_expert_ffn_gemv_b200", "csrc", src)
+    try:
+        cur = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    for f in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for line in open(f):
+            if not line.startswith("traffic:"):
+                continue
+            kv = dict(t.split("=", 1) for t in line.split()[1:] if "=" in t)
+            if kv.get("kernel") == kernel and kv.get("source_sha256_16") == cur:
+                return int(kv["dram_bytes_per_launch"])
+    return None
+
+
+# ---------------------------------------------------------------- replicas (one process per GPU)
+def rank_master(master: int, rank: int) -> int:
+    """Seed of a replica's weights and inputs: every rank draws its own data."""
+    return master + 1000 * rank
+
+
+def max_over_ranks(value: float, world: int, device="cuda") -> float:
+    """The slowest rank's time (all ranks call this at the same point)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(tokens_per_step: int, steps: int, world: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank processes its own batches; time is the slowest rank's."""
+    return tokens_per_step * steps * world / (ms_max / 1000.0)
+
+
 # ---------------------------------------------------------------- workload description
 def workload(args):
     from synth import WORKLOADS, MoeShape
@@ -224,21 +275,23 @@ def ours(args):
     h = moe.MoeLayer(sh.d, sh.f, sh.E, sh.k, sh.n_shared, layers, sh.bits, T)
     weights = []
     for l in range(layers):
-        w = sgpu.layer_device(sh, wl.master + 1000 * rank, l, wl.zipf)
+        w = sgpu.layer_device(sh, rank_master(wl.master, rank), l, wl.zipf)
         h.load_layer(l, *w)
         weights.append(w)
     n_x = 16
-    xs = [sgpu.x_device(sh, wl.master + 1000 * rank, 10000 + i, T) for i in range(n_x)]
+    xs = [sgpu.x_device(sh, rank_master(wl.master, rank), 10000 + i, T) for i in range(n_x)]
     chain = args.workload == "chain48"
     resid = [torch.empty_like(xs[0]) for _ in range(2)]
+    normed = torch.empty_like(xs[0])
 
     def step(i, stream=None):
         if chain:
-            # x_{l+1} = x_l + layer_l(x_l), in place in the residual buffer
+            # residual chain: u_l = rmsnorm(x_l), x_{l+1} = x_l + layer_l(u_l) in place
             r = resid[i & 1]
             r.copy_(xs[i % n_x])
             for l in range(layers):
-                h.forward(l, r, r, flags=flags | moe.MOE_ACCUMULATE, stream=stream)
+                moe.rms_normalize(r, normed, stream=stream)
+                h.forward(l, normed, r, flags=flags | moe.MOE_ACCUMULATE, stream=stream)
             return r
         return h.forward(i % layers, xs[i % n_x], ys[i & 1], flags=flags, stream=stream)
 
@@ -288,13 +341,11 @@ def ours(args):
     launches = h.stats()["launches"] - launches0
     if graph is not None:  # the library counts launches when enqueued (at capture): count n_cap steps
         launches = _graph_launches(h, step, n_cap) * reps
+    ms = max_over_ranks(ms, world)
     if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     tok_per_step = T
-    value = tok_per_step * n_steps * world / (ms / 1000.0)
+    value = replica_throughput(tok_per_step, n_steps, world, ms)
 
     # ---- per-kernel device time (events on the library's launch stream), separate pass.
     # Pass 1 records each step's distinct experts; pass 2 replays the same steps
@@ -327,13 +378,13 @@ def ours(args):
         dom_ms = prof[dom][0] / prof[dom][1]
         ach = flops[dom] / (dom_ms / 1000.0) / 1e12
         roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": tc_burst, "unit": "TFLOP/s",
-                "frac": ach / tc_burst, "traffic": None, "peak_kind": peak_kind + " bf16 dense (burst)",
+                "frac": ach / tc_burst, "traffic": profile_traffic(dom), "peak_kind": peak_kind + " bf16 dense (burst)",
                 "flops_per_launch": flops[dom], "avg_launch_us": 1000.0 * dom_ms}
     elif dom in ("gemv_gateup", "gemv_down", "decode_fused"):
         dom_ms = prof[dom][0]
         ach = alg_bytes[dom] / (dom_ms / 1000.0) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                "traffic": None, "peak_kind": peak_kind,
+                "traffic": profile_traffic(dom), "peak_kind": peak_kind,
                 "bytes_per_launch": alg_bytes[dom] / max(1, prof[dom][1]),
                 "avg_launch_us": 1000.0 * dom_ms / max(1, prof[dom][1])}
     layer_time = sum(v[0] for v in prof.values())
@@ -354,12 +405,8 @@ def ours(args):
             h.forward_host(i % layers, xh[i % n_x], yh, flags=flags)
         e1.record()
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": T * k2 * world / (ems / 1000.0), "unit": "tok/s", "h2d_bytes_per_step": T * sh.d * 2,
+        ems = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e = {"value": replica_throughput(T, k2, world, ems), "unit": "tok/s", "h2d_bytes_per_step": T * sh.d * 2,
                "d2h_bytes_per_step": T * sh.d * 2}
 
     cpu = None

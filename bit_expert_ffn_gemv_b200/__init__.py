@@ -20,7 +20,7 @@ __all__ = ["MoeError", "MoeConfig", "MoeLayerWeights", "MoeLayer", "lib", "libra
            "MOE_ACCUMULATE", "MOE_FORCE_GEMV", "MOE_FORCE_GEMM", "MOE_FORCE_UNFUSED", "STATUS", "moe_layer_init", "moe_load_layer",
            "moe_route", "moe_route_noalloc", "moe_forward", "moe_forward_host", "moe_destroy", "moe_debug_dequant", "moe_debug_last_routing", "moe_check_status",
            "moe_get_stats", "moe_status_string", "moe_profile", "moe_profile_read", "moe_kernel_name", "MoeStats",
-           "moe_debug_router_logits", "moe_router_error_depth"]
+           "moe_debug_router_logits", "moe_router_error_depth", "moe_rms_normalize", "rms_normalize"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libmoe.so")
@@ -105,6 +105,8 @@ def lib() -> ctypes.CDLL:
             L.moe_debug_router_logits.argtypes = [vp, i32, vp, i32, vp, i32, vp]
             L.moe_router_error_depth.restype = ctypes.c_float
             L.moe_router_error_depth.argtypes = [i32, i32]
+            L.moe_rms_normalize.restype = st
+            L.moe_rms_normalize.argtypes = [vp, i32, i32, vp, vp]
             L.moe_status_string.restype = ctypes.c_char_p
             L.moe_status_string.argtypes = [st]
             _lib = L
@@ -175,6 +177,10 @@ def moe_router_error_depth(d: int, tensor_cores: bool) -> float:
     return float(lib().moe_router_error_depth(d, 1 if tensor_cores else 0))
 
 
+def moe_rms_normalize(x_ptr: int, T: int, d: int, out_ptr: int, stream: int) -> None:
+    _check(lib().moe_rms_normalize(x_ptr, T, d, out_ptr, stream), "moe_rms_normalize")
+
+
 def moe_check_status(handle: int) -> int:
     return int(lib().moe_check_status(handle))
 
@@ -210,6 +216,15 @@ def _stream_ptr(stream) -> int:
     import torch
     s = stream if stream is not None else torch.cuda.current_stream()
     return int(s.cuda_stream)
+
+
+def rms_normalize(x, out=None, stream=None):
+    """bf16 [T, d] -> bf16 x / rms(x) per row (the residual-stream pre-norm of a layer chain)."""
+    import torch
+    if out is None:
+        out = torch.empty_like(x)
+    moe_rms_normalize(x.data_ptr(), x.shape[0], x.shape[1], out.data_ptr(), _stream_ptr(stream))
+    return out
 
 
 class MoeLayer:

@@ -468,6 +468,13 @@ moe_status moe_forward_host(moe_handle* h, int32_t layer, const void* x_host, in
     return cuda_status(cudaStreamSynchronize(s));
 }
 
+moe_status moe_rms_normalize(const void* x, int32_t T, int32_t d, void* out, void* stream) {
+    if (T < 0 || d <= 0 || d % 8) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !out || !aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    return cuda_status(moe::launch_rms_normalize(x, T, d, out, 1e-6f, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_destroy(moe_handle* h) {
     if (!h) return MOE_OK;
     cudaError_t e = cudaSuccess;

@@ -1124,12 +1124,40 @@ static cudaError_t decode_bits_nt(const DecodeLaunch& L, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+static int max_smem_optin() {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 227 * 1024;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 227 * 1024;
+    return v;
+}
+
+static bool fits(int BITS, int NT, const DecodeLaunch& L) {
+    int r, b, w;
+    return decode_smem(BITS, NT, L.d, L.f, L.E, L.T, L.k, &r, &b, &w) <= (size_t)max_smem_optin();
+}
+
+// Tokens per task: the smallest of 1, 2, 4, 8 that covers T in 8 slots and
+// whose shared memory fits; a batch that fits no variant runs as 32-token
+// slices (each slice a full layer pass over its own tokens).
 template <int BITS>
 static cudaError_t decode_bits(const DecodeLaunch& L, cudaStream_t s) {
-    if (L.T <= 8) return decode_bits_nt<BITS, 1>(L, s);
-    if (L.T <= 16) return decode_bits_nt<BITS, 2>(L, s);
-    if (L.T <= 32) return decode_bits_nt<BITS, 4>(L, s);
-    return decode_bits_nt<BITS, 8>(L, s);
+    if (L.T <= 8 && fits(BITS, 1, L)) return decode_bits_nt<BITS, 1>(L, s);
+    if (L.T <= 16 && fits(BITS, 2, L)) return decode_bits_nt<BITS, 2>(L, s);
+    if (L.T <= 32 && fits(BITS, 4, L)) return decode_bits_nt<BITS, 4>(L, s);
+    if (fits(BITS, 8, L)) return decode_bits_nt<BITS, 8>(L, s);
+    const size_t ysz = L.out_fp32 ? 4 : 2;
+    for (int t0 = 0; t0 < L.T; t0 += 32) {
+        DecodeLaunch S = L;
+        S.T = std::min(32, L.T - t0);
+        S.x = static_cast<const uint16_t*>(L.x) + (size_t)t0 * L.d;
+        S.y = static_cast<char*>(L.y) + (size_t)t0 * L.d * ysz;
+        S.ids = L.ids + (size_t)t0 * L.k;
+        S.w = L.w + (size_t)t0 * L.k;
+        if (!fits(BITS, 4, S)) return cudaErrorInvalidConfiguration;
+        cudaError_t e = decode_bits_nt<BITS, 4>(S, s);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t s) {

@@ -115,6 +115,7 @@ cudaError_t launch_gemm_gateup(const ExpertArgs& a, const GemmMaps& maps, const 
 cudaError_t launch_gemm_down(const ExpertArgs& a, const GemmMaps& maps, const float* wsorted, void* o,
                              const int4* desc, const int32_t* counts, cudaStream_t s);
 cudaError_t launch_combine_f16(const CombineArgs& a, const void* o, cudaStream_t s);
+cudaError_t launch_rms_normalize(const void* x, int T, int d, void* out, float eps, cudaStream_t s);
 cudaError_t launch_dequant(const uint8_t* codes, const uint16_t* scales, int N, int K, int bits, float* out,
                            cudaStream_t s);
 

@@ -176,6 +176,16 @@ moe_status moe_route_noalloc(const void* x, int32_t T, int32_t d, int32_t n_expe
                              const void* router_w, const float* router_bias, int32_t* ids, float* w,
                              void* stream);
 
+/*
+ * Helper for callers that chain layers (not a step of the routed-MoE layer):
+ * out[t] = bf16(x[t] / sqrt(mean_i x[t,i]^2 + 1e-6)) for bf16 x, out [T x d]
+ * (device, 16-byte aligned, d % 8 == 0; out may equal x).  The model family
+ * the pages describe normalises the residual stream before each MoE layer;
+ * without it, x_{l+1} = x_l + layer(x_l) diverges, the SwiGLU output being
+ * quadratic in its input.  Errors: INVALID_ARG, CUDA.
+ */
+moe_status moe_rms_normalize(const void* x, int32_t T, int32_t d, void* out, void* stream);
+
 /* Free the handle's own memory (never the borrowed weights).  NULL is a no-op. */
 moe_status moe_destroy(moe_handle* h);
 
