@@ -374,7 +374,11 @@ MOE_DEV void topk_token(const DecodeArgs& a, int t, int lane, double* v, int* id
                 }
         }
         // candidates: key prefix >= the k-th key's prefix (a sorted prefix of kk)
-        const uint32_t pk = kk[k - 1] & 0xFFFFFC00u;
+        uint32_t kth = 0xFFFFFFFFu;
+#pragma unroll
+        for (int j = 0; j < kTopkLane; ++j)
+            if (j < k) kth = min(kth, kk[j]);
+        const uint32_t pk = kth & 0xFFFFFC00u;
         if ((kk[kTopkLane - 1] & 0xFFFFFC00u) < pk) {
             int m = 0;
             uint32_t mine = 0;

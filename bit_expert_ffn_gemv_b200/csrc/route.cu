@@ -144,11 +144,11 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
     }
     __syncwarp();
 
-    // top-(k+1) by repeated warp argmax; `taken` bit j <-> element lane + 32 j
+    // top-k by repeated warp argmax; `taken` bit j <-> element lane + 32 j.
+    // Rank r lives in lane r (k <= 32), so nothing is indexed by the runtime k.
     uint32_t taken = 0;
-    int sel[kMaxK + 1];
-    const int kk = min(k + 1, E);
-    for (int r = 0; r < kk; ++r) {
+    int my_sel = -1;  // lane r < k: expert of rank r
+    for (int r = 0; r < k; ++r) {
         float bv = -INFINITY;
         int bi = 0x7fffffff;
         for (int j = 0, e = lane; e < E; ++j, e += 32)
@@ -165,17 +165,16 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
                 bi = oi;
             }
         }
-        sel[r] = bi;
+        if (lane == r) my_sel = bi;
         if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
     }
 
-    // certification of the fp32 order
-    bool ok = true;
-    for (int r = 0; r + 1 < k; ++r) {
-        int a = sel[r], b = sel[r + 1];
-        if (!(lv[a] - dv[a] > lv[b] + dv[b])) ok = false;
-    }
-    const float lower_k = lv[sel[k - 1]] - dv[sel[k - 1]];
+    // certification of the fp32 order: rank r's interval lies strictly above rank r+1's
+    const int next_sel = __shfl_down_sync(0xffffffffu, my_sel, 1);
+    const bool pair_ok = lane + 1 >= k || (lv[my_sel] - dv[my_sel] > lv[next_sel] + dv[next_sel]);
+    bool ok = __all_sync(0xffffffffu, pair_ok);
+    const int sel_k = __shfl_sync(0xffffffffu, my_sel, k - 1);
+    const float lower_k = lv[sel_k] - dv[sel_k];
     // candidates: every expert whose interval reaches the k-th one's lower end,
     // listed in ascending index order (reusing the bound array, no longer needed)
     int* cand = reinterpret_cast<int*>(dv);
@@ -192,12 +191,12 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
     if (n_cand != k) ok = false;
     if (isnan(lower_k)) ok = false;
 
-    float wsel[kMaxK];
+    float my_w = 0.f;  // lane r < k: logit of rank r
     if (ok) {
-        for (int r = 0; r < k; ++r) wsel[r] = lv[sel[r]];
+        if (lane < k) my_w = lv[my_sel];
     } else {
         // fp64 logits of the candidates (sums of exact bf16 products), 8 products
-        // per lane per 256-wide chunk, several chunks in flight
+        // per lane per 256-wide chunk, two candidates per pass
         for (int ci = 0; ci < n_cand; ci += 2) {
             const bool two = ci + 1 < n_cand;
             const int e0 = cand[ci], e1 = two ? cand[ci + 1] : e0;
@@ -255,27 +254,24 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
                     bc = oc;
                 }
             }
-            sel[r] = bi;
-            wsel[r] = (float)bv;
+            if (lane == r) {
+                my_sel = bi;
+                my_w = (float)bv;
+            }
             if (bc >= 0 && (bc & 31) == lane) tk |= 1u << (bc >> 5);
         }
         if (lane == 0) atomicAdd(&meta->n_fixup, 1);
     }
 
-    // renormalised weights = softmax over the k selected logits
-    if (lane == 0) {
-        float m = wsel[0];
-        float z = 0.f;
-        float ex[kMaxK];
-        for (int r = 0; r < k; ++r) {
-            ex[r] = expf(wsel[r] - m);
-            z += ex[r];
-        }
-        const float inv = 1.0f / z;
-        for (int r = 0; r < k; ++r) {
-            ids_out[(int64_t)t * k + r] = sel[r];
-            w_out[(int64_t)t * k + r] = ex[r] * inv;
-        }
+    // renormalised weights = softmax over the k selected logits (lane r: rank r)
+    const float m = __shfl_sync(0xffffffffu, my_w, 0);
+    const float ex = lane < k ? expf(my_w - m) : 0.0f;
+    float z = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane < k) {
+        ids_out[(int64_t)t * k + lane] = my_sel;
+        w_out[(int64_t)t * k + lane] = ex * (1.0f / z);
     }
 }
 
