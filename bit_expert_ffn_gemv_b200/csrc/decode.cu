@@ -879,7 +879,7 @@ template <int BITS, int NT>
 __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     __shared__ __align__(8) uint64_t bars[2];
-    __shared__ int s_claim, s_flag, s_issued[2];
+    __shared__ int s_claim, s_flag, s_issued[2], s_nact;
     constexpr bool STAGE = NT <= 2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const TaskMap m = task_map(a);
@@ -896,11 +896,37 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecodeArgs a)
         mbar_init(&bars[0], 1);
         mbar_init(&bars[1], 1);
         fence_proxy_async_smem();
+        s_nact = -1;
     }
     __syncthreads();
 
+    // Claim the next task.  Routed tasks exist for min(T*k, E) expert slots,
+    // but only n_active of them have an expert: once the bucketing is
+    // published, a claim that lands past the last active slot moves the head
+    // to the next phase (or the end), so empty tasks are never run.
     auto claim = [&]() {
-        if (threadIdx.x == 0) s_claim = ld_relaxed(sync + SY_ABORT) ? m.total : atomicAdd(sync + SY_HEAD, 1);
+        if (threadIdx.x == 0) {
+            int v;
+            for (;;) {
+                v = ld_relaxed(sync + SY_ABORT) ? m.total : atomicAdd(sync + SY_HEAD, 1);
+                if (v < m.b4 || v >= m.total) break;
+                if (s_nact < 0) {
+                    if (ld_relaxed(sync + SY_BUCKET) < 1) break;  // not known yet: run it (it checks)
+                    fence_acq_rel_gpu();
+                    s_nact = a.meta->n_active;
+                }
+                if (v < m.b5) {
+                    if ((v - m.b4) / m.FT < s_nact) break;
+                    atomicMax(sync + SY_HEAD, m.b5);  // no gate/up work left: go to the down tasks
+                    continue;
+                }
+                if ((v - m.b5) / m.nRTG < s_nact) break;
+                atomicMax(sync + SY_HEAD, m.total);  // no down work left
+                v = m.total;
+                break;
+            }
+            s_claim = v;
+        }
         __syncthreads();
         const int v = s_claim;
         __syncthreads();

@@ -99,7 +99,6 @@ MOE_DEV bool better64(double va, int ia, double vb, int ib) {
 }
 
 constexpr int kTopkWarps = 4;
-constexpr int kMaxK = 32;
 
 // One warp per token.  Shared memory per warp: E floats (fp32 logits),
 // E floats (bounds), E doubles (fp64 logits of candidates).
