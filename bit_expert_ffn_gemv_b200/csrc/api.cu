@@ -57,6 +57,7 @@ struct moe_handle {
     int4* desc_dn = nullptr;     // down tile descriptors
     int32_t* n_tiles = nullptr;  // [2] descriptor counts
     float* wsorted = nullptr;    // routing weights in group order
+    int32_t* bucket_cnt = nullptr;  // per-chunk expert counts (multi-CTA bucketing)
     // launch accounting and optional per-kernel event timing
     int64_t launches = 0;
     bool prof_on = false;
@@ -200,7 +201,9 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
         ba.w = h->w;
         ba.wsorted = h->wsorted;
     }
+    ba.cnt = h->bucket_cnt;
     e = run(h, MOE_K_BUCKET, s, [&] { return moe::launch_bucket(ba, s); });
+    h->launches += moe::bucket_kernel_count(ba) - 1;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
 
     const moe_layer_state& L = h->layers[layer];
@@ -333,6 +336,7 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
                                                                    c.d / 128));
     const size_t o_ntiles = take(sizeof(int32_t) * 2);
     const size_t o_wsorted = take(sizeof(float) * T * k);
+    const size_t o_bcnt = take(sizeof(int32_t) * moe::bucket_scratch_words(c.n_experts));
     const size_t o_sync =
         take(sizeof(int) * moe::decode_sync_words(std::min(c.max_tokens, moe::kDecodeMaxTokens), c.n_experts, c.d));
     h->arena_bytes = off;
@@ -363,6 +367,7 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     h->desc_dn = reinterpret_cast<int4*>(base + o_ddn);
     h->n_tiles = reinterpret_cast<int32_t*>(base + o_ntiles);
     h->wsorted = reinterpret_cast<float*>(base + o_wsorted);
+    h->bucket_cnt = reinterpret_cast<int32_t*>(base + o_bcnt);
     for (int l = 0; l < c.n_layers; ++l) h->layers[l].wnorm = reinterpret_cast<float*>(base + o_norms) + E * l;
     if (cudaMemset(h->arena, 0, h->arena_bytes) != cudaSuccess ||
         moe::make_row_maps(&h->gu_maps, h->xg, (int64_t)rows, c.d) != cudaSuccess ||

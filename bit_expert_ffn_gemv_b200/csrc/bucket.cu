@@ -13,6 +13,7 @@
 namespace moe {
 
 constexpr int kBucketWarps = 32;
+int bucket_kernel_count(const BucketArgs& a);
 
 // Warp w owns the contiguous range of pair indices p = t*k + r in
 // [w*ppw, (w+1)*ppw); ascending p means ascending t, so per-warp counts and
@@ -135,7 +136,154 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
     }
 }
 
+// ---------------------------------------------------------------- multi-CTA variant (large T)
+// The single-CTA kernel issues every scattered store of `pairs` (and of the
+// sorted weights) from one SM, which bounds it at large T.  Three kernels
+// spread the work over kChunks CTAs while keeping the same stable order:
+//   count:   CTA c counts the experts of its contiguous pair range -> cnt[c][e]
+//   scan:    one CTA turns cnt into per-(chunk, expert) bases, the expert
+//            offsets, the active list and the meta block
+//   scatter: CTA c ranks its pairs (per-warp counts in shared memory, lanes by
+//            match-any, as in the single-CTA kernel) and writes them at
+//            base[c][e] + rank.
+constexpr int kChunks = 128;
+constexpr int kChunkWarps = 8;
+
+__global__ void __launch_bounds__(kChunkWarps * 32)
+    bucket_count_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int chunk, int32_t* __restrict__ cnt,
+                        uint32_t* __restrict__ status) {
+    extern __shared__ int32_t h[];  // [E]
+    const int c = blockIdx.x;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+    __syncthreads();
+    const int p0 = c * chunk, p1 = min(n_pairs, p0 + chunk);
+    for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
+        const int e = __ldg(&ids[p]);
+        if (e >= 0 && e < E) atomicAdd(&h[e], 1);
+        else flag_status(status, kStatusBounds);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[(int64_t)c * E + e] = h[e];
+}
+
+__global__ void __launch_bounds__(1024) bucket_scan_kernel(int32_t* __restrict__ cnt, int nchunks, int E,
+                                                           int32_t* __restrict__ offsets,
+                                                           int32_t* __restrict__ active, Meta* __restrict__ meta) {
+    extern __shared__ int32_t tot[];  // [E]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // per expert: exclusive prefix over the chunks (in place), total
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = 0;
+#pragma unroll 8
+        for (int c = 0; c < nchunks; ++c) {
+            const int v = cnt[(int64_t)c * E + e];
+            cnt[(int64_t)c * E + e] = run;
+            run += v;
+        }
+        tot[e] = run;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int base = 0, nact = 0, mx = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int cv = e < E ? tot[e] : 0;
+            int inc = cv;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += v;
+            }
+            if (e < E) offsets[e] = base + inc - cv;
+            const unsigned b = __ballot_sync(0xffffffffu, cv > 0);
+            if (cv > 0) active[nact + __popc(b & ((1u << lane) - 1u))] = e;
+            nact += __popc(b);
+            int m = cv;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+            mx = max(mx, m);
+            base += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        if (lane == 0) {
+            offsets[E] = base;
+            meta->n_active = nact;
+            meta->max_count = mx;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kChunkWarps * 32)
+    bucket_scatter_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int chunk,
+                          const int32_t* __restrict__ cbase, const int32_t* __restrict__ offsets,
+                          int32_t* __restrict__ pairs, int32_t* __restrict__ inv, const float* __restrict__ w,
+                          float* __restrict__ wsorted) {
+    extern __shared__ int32_t wc[];  // [kChunkWarps][E] per-warp running position
+    const int c = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t lt = (1u << lane) - 1u;
+    const int p0 = c * chunk, p1 = min(n_pairs, p0 + chunk);
+    const int wchunk = ((chunk + kChunkWarps - 1) / kChunkWarps + 31) & ~31;
+    const int q0 = min(p1, p0 + warp * wchunk), q1 = min(p1, q0 + wchunk);
+    for (int i = threadIdx.x; i < kChunkWarps * E; i += blockDim.x) wc[i] = 0;
+    __syncthreads();
+    // per-warp counts of this warp's sub-range
+    for (int p = q0; p < q1; p += 32) {
+        const int e = p + lane < q1 ? __ldg(&ids[p + lane]) : -1;
+        const bool valid = e >= 0 && e < E;
+        const uint32_t same = __match_any_sync(0xffffffffu, valid ? e : -1);
+        if (valid && (same & lt) == 0) wc[warp * E + e] += __popc(same);
+    }
+    __syncthreads();
+    // exclusive prefix over the warps, plus this chunk's base and the expert offset
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = offsets[e] + cbase[(int64_t)c * E + e];
+#pragma unroll
+        for (int wv = 0; wv < kChunkWarps; ++wv) {
+            const int v = wc[wv * E + e];
+            wc[wv * E + e] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    for (int p = q0; p < q1; p += 32) {
+        const bool live = p + lane < q1;
+        const int e = live ? __ldg(&ids[p + lane]) : -1;
+        const bool valid = e >= 0 && e < E;
+        const uint32_t same = __match_any_sync(0xffffffffu, valid ? e : -1);
+        const int leader = __ffs(same) - 1;
+        int base = 0;
+        if (valid && lane == leader) {
+            base = wc[warp * E + e];
+            wc[warp * E + e] += __popc(same);
+        }
+        base = __shfl_sync(0xffffffffu, base, leader);
+        if (valid) {
+            const int pos = base + __popc(same & lt);
+            pairs[pos] = p + lane;
+            inv[p + lane] = pos;
+            if (wsorted) wsorted[pos] = __ldg(&w[p + lane]);
+        } else if (live) {
+            inv[p + lane] = -1;
+        }
+    }
+}
+
 cudaError_t launch_bucket(const BucketArgs& a, cudaStream_t s) {
+    const int n_pairs = a.T * a.k;
+    if (bucket_kernel_count(a) == 3) {
+        const int chunk = (n_pairs + kChunks - 1) / kChunks;
+        bucket_count_kernel<<<kChunks, kChunkWarps * 32, sizeof(int32_t) * a.E, s>>>(a.ids, n_pairs, a.E, chunk, a.cnt,
+                                                                                     a.status);
+        bucket_scan_kernel<<<1, 1024, sizeof(int32_t) * a.E, s>>>(a.cnt, kChunks, a.E, a.offsets, a.active, a.meta);
+        const size_t smem = sizeof(int32_t) * (size_t)kChunkWarps * a.E;
+        if (smem > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(bucket_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        bucket_scatter_kernel<<<kChunks, kChunkWarps * 32, smem, s>>>(a.ids, n_pairs, a.E, chunk, a.cnt, a.offsets,
+                                                                      a.pairs, a.inv, a.w, a.wsorted);
+        return cudaGetLastError();
+    }
     const size_t smem = sizeof(int32_t) * ((size_t)kBucketWarps * a.E + 2 * (size_t)a.E + 1);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(bucket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -146,4 +294,9 @@ cudaError_t launch_bucket(const BucketArgs& a, cudaStream_t s) {
     return cudaGetLastError();
 }
 
+}  // namespace moe
+
+namespace moe {
+size_t bucket_scratch_words(int E) { return (size_t)kChunks * E; }
+int bucket_kernel_count(const BucketArgs& a) { return (a.cnt && a.T * a.k >= 8192) ? 3 : 1; }
 }  // namespace moe

@@ -33,7 +33,10 @@ struct BucketArgs {
     uint32_t* status;
     const float* w = nullptr;  // [T x k] routing weights; with wsorted:
     float* wsorted = nullptr;  // [T*k] w of pairs[pos] at pos (or null: not written)
+    int32_t* cnt = nullptr;    // scratch [128 x E] for the multi-CTA variant (large T), or null
 };
+size_t bucket_scratch_words(int E);
+int bucket_kernel_count(const BucketArgs& a);  // kernels launch_bucket enqueues: 1, or 3 at large T
 
 // Grouped GEMV/GEMM problem description shared by the expert kernels.
 struct ExpertArgs {
