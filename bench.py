@@ -373,8 +373,7 @@ def ours(args):
     roof = None
     rows = T * sh.k + T * sh.n_shared
     flops = {"gemm_gateup": 2.0 * rows * 2 * sh.f * sh.d, "gemm_down": 2.0 * rows * sh.d * sh.f}
-    flops["gemv_gateup"], flops["gemv_down"] = flops["gemm_gateup"], flops["gemm_down"]
-    if T > 64 and dom in flops:
+    if dom in ("gemm_gateup", "gemm_down"):
         dom_ms = prof[dom][0] / prof[dom][1]
         ach = flops[dom] / (dom_ms / 1000.0) / 1e12
         roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": tc_burst, "unit": "TFLOP/s",

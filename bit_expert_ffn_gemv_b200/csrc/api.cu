@@ -105,10 +105,11 @@ moe_status check_layer(moe_handle* h, int32_t layer) {
     return MOE_OK;
 }
 
-// Large token counts take the tensor-core router (bf16 tcgen05 GEMM).
+// moe_forward takes the tensor-core path (bf16 tcgen05 router, grouped
+// dequant GEMMs) above kFusedMaxTokens tokens, or when forced.
 bool use_tensor_cores(int32_t T, uint32_t flags) {
     if (flags & (MOE_FORCE_GEMV | MOE_FORCE_UNFUSED)) return false;
-    return T > moe::kDecodeMaxTokens || (flags & MOE_FORCE_GEMM);
+    return T > moe::kFusedMaxTokens || (flags & MOE_FORCE_GEMM);
 }
 
 // router -> certified top-k; writes ids / w (device)
@@ -180,7 +181,7 @@ moe_status do_decode(moe_handle* h, int32_t layer, const void* x, int32_t T, voi
 moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, void* y, uint32_t flags,
                       cudaStream_t s) {
     const moe_config& c = h->cfg;
-    if (T <= moe::kDecodeMaxTokens && !(flags & (MOE_FORCE_GEMM | MOE_FORCE_UNFUSED)))
+    if (T <= moe::kDecodeMaxTokens && !use_tensor_cores(T, flags) && !(flags & MOE_FORCE_UNFUSED))
         return do_decode(h, layer, x, T, y, flags, s);
     const bool tc = use_tensor_cores(T, flags);
     cudaError_t e;
@@ -410,7 +411,8 @@ moe_status moe_route(moe_handle* h, int32_t layer, const void* x, int32_t T, int
     if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x || !ids || !w || !aligned16(x) || !aligned16(ids) || !aligned16(w)) return MOE_ERR_INVALID_ARG;
-    return do_route(h, layer, x, T, ids, w, use_tensor_cores(T, 0), static_cast<cudaStream_t>(stream));
+    // routing alone: the CUDA-core router up to 64 tokens, the tensor-core router above
+    return do_route(h, layer, x, T, ids, w, T > moe::kDecodeMaxTokens, static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_debug_router_logits(moe_handle* h, int32_t layer, const void* x, int32_t T, float* logits,

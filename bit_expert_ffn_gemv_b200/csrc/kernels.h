@@ -64,6 +64,10 @@ struct CombineArgs {
 
 // Whole layer for up to kDecodeMaxTokens tokens in one persistent kernel.
 constexpr int kDecodeMaxTokens = 64;
+// Automatic dispatch of moe_forward: the fused kernel up to this many tokens,
+// the tensor-core path above (measured crossover on the full-shape layer:
+// equal at 16 tokens, the tensor-core path 2.6x faster at 64).
+constexpr int kFusedMaxTokens = 16;
 struct DecodeLaunch {
     int T, d, f, E, k, n_shared, bits;
     const void* x;

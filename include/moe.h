@@ -96,9 +96,11 @@ typedef struct {
 /* forward flags */
 #define MOE_OUT_FP32 0x1u   /* y is fp32 [T x d] (default: bf16) */
 #define MOE_ACCUMULATE 0x2u /* y += layer output (default: y = layer output) */
-#define MOE_FORCE_GEMV 0x4u /* use the grouped-GEMV path whatever T is */
-#define MOE_FORCE_GEMM 0x8u /* use the grouped-GEMM path whatever T is */
-#define MOE_FORCE_UNFUSED 0x10u /* small T: one kernel per step instead of the fused persistent kernel */
+/* Path selection (default: the fused persistent kernel for T <= 16, the
+ * tensor-core grouped-GEMM path above -- the measured crossover). */
+#define MOE_FORCE_GEMV 0x4u /* CUDA-core paths: the fused kernel up to 64 tokens, grouped GEMV above */
+#define MOE_FORCE_GEMM 0x8u /* the tensor-core grouped-GEMM path whatever T is */
+#define MOE_FORCE_UNFUSED 0x10u /* one kernel per step (grouped GEMV) instead of the fused persistent kernel */
 
 /*
  * Create a handle on the current CUDA device.  Checks the configuration and

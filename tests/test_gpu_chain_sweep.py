@@ -137,7 +137,7 @@ def wide(torch_cuda, request):
 
 @pytest.mark.parametrize("T", [1, 4, 64, 512])
 def test_wide_full_layer(torch_cuda, wide, T):
-    """3/4-bit full shape: fused decode path up to 64 tokens, tensor-core path at 512 (sampled rows)."""
+    """3/4-bit full shape: fused decode path up to 16 tokens, tensor-core path above (sampled rows at 512)."""
     import bit_expert_ffn_gemv_b200 as moe
     wl, sh, h, w = wide
     xb = synth.x_host(sh, wl.master, 300 + T, T)
@@ -152,4 +152,4 @@ def test_wide_full_layer(torch_cuda, wide, T):
     ids_ref, _ = oracle.route(sh, xb, L["router_w"], L["bias"])
     assert np.array_equal(ids.cpu().numpy(), ids_ref), f"b{sh.bits} T={T}: expert selection differs"
     _compare(sh, L, xb, y32, y16, label=f"b{sh.bits} T={T}", rows=rows,
-             fp32_tol=REL_L2_FP32 if T <= 64 else REL_L2_FP32_TC)
+             fp32_tol=REL_L2_FP32 if T <= 16 else REL_L2_FP32_TC)

@@ -191,7 +191,7 @@ def test_router_gemm_error_bound(torch_cuda, full):
     assert (err <= bound).all()
 
 
-@pytest.mark.parametrize("T", [65, 1000, 8192])
+@pytest.mark.parametrize("T", [17, 33, 65, 1000, 8192])
 def test_full_layer_gemm(torch_cuda, full, T):
     """Full shape (E = 512, k = 10, d = 2048, f = 768); outputs checked on a sample of tokens."""
     wl, L, h, dev = full

@@ -38,14 +38,17 @@ def _check_layer(torch, h, shape, L, x_bits, layer=0, flags_extra=0, label=""):
     y32 = h.forward(layer, x, flags=moe.MOE_OUT_FP32 | flags_extra)
     ids_f, w_f = h.last_routing(T)
     torch.cuda.synchronize()
+    # above 16 tokens (unless forced onto the CUDA-core paths) moe_forward takes the
+    # tensor-core path: fp32 tensor-core logits (1e-4 on the weights) and fp16 operands
+    tc = T > 16 and not (flags_extra & (moe.MOE_FORCE_GEMV | moe.MOE_FORCE_UNFUSED))
     assert np.array_equal(ids_f.cpu().numpy(), ids_ref), f"{label}: forward's expert selection differs"
-    assert np.allclose(w_f.cpu().numpy(), w_ref, rtol=2e-6, atol=1e-7), label
+    assert np.allclose(w_f.cpu().numpy(), w_ref, rtol=1e-4 if tc else 2e-6, atol=1e-7), label
     assert h.check_status() == 0
     g16, g32 = y_to_f64(y16), y_to_f64(y32)
     r16, m16, r32 = rel_l2(g16, y_ref), max_abs(g16, y_ref), rel_l2(g32, y_ref)
     print(f"{label} T={T}: rel_l2 bf16 {r16:.3e} max_abs {m16:.3e} fp32 {r32:.3e} stats {h.stats()}")
     assert r16 <= REL_L2 and m16 <= MAX_ABS, label
-    assert r32 <= REL_L2_FP32, label
+    assert r32 <= (8e-4 if tc else REL_L2_FP32), label
     return y16, y32
 
 
@@ -161,9 +164,11 @@ def decode_layer(torch_cuda):
 
 @pytest.mark.parametrize("T", [1, 4, 16, 64, 7, 33])
 def test_decode_layer(torch_cuda, decode_layer, T):
+    """The fused persistent kernel (the default up to 16 tokens, MOE_FORCE_GEMV up to 64)."""
+    import bit_expert_ffn_gemv_b200 as moe
     wl, L, h = decode_layer
     x = synth.x_host(wl.shape, wl.master, 200 + T, T)
-    _check_layer(torch_cuda, h, wl.shape, L, x, label="decode")
+    _check_layer(torch_cuda, h, wl.shape, L, x, flags_extra=moe.MOE_FORCE_GEMV if T > 16 else 0, label="decode")
 
 
 @pytest.mark.parametrize("T", [1, 4, 64])
@@ -174,7 +179,7 @@ def test_decode_layer_unfused(torch_cuda, decode_layer, T):
     xb = synth.x_host(wl.shape, wl.master, 400 + T, T)
     _check_layer(torch_cuda, h, wl.shape, L, xb, flags_extra=moe.MOE_FORCE_UNFUSED, label="decode-unfused")
     x = x_to_device(xb)
-    a = h.forward(0, x, flags=moe.MOE_OUT_FP32)
+    a = h.forward(0, x, flags=moe.MOE_OUT_FP32 | moe.MOE_FORCE_GEMV)  # the fused kernel up to 64 tokens
     b = h.forward(0, x, flags=moe.MOE_OUT_FP32 | moe.MOE_FORCE_UNFUSED)
     torch_cuda.cuda.synchronize()
     assert rel_l2(y_to_f64(a), y_to_f64(b)) < 1e-5
