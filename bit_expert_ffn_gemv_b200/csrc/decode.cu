@@ -148,16 +148,31 @@ MOE_DEV TaskMap task_map(const DecodeArgs& a) {
 struct Slot {
     int expert, count, hbase, pair0;
     bool shared;
+    const int* tok;  // routed slot with the CTA's slot table: token of each of its pairs (shared memory)
 };
 
-MOE_DEV Slot make_slot(const DecodeArgs& a, int slot) {
+// The CTA's copy of the bucketing, loaded once after it is published:
+// tbl[0] = n_active, tbl[1] = pairs, then expert[maxR], pair0[maxR],
+// count[maxR], token[T*k] (token of each pair position).
+__host__ __device__ inline size_t slot_table_words(int maxR, int npairs) { return 2 + 3 * (size_t)maxR + (size_t)npairs; }
+
+MOE_DEV Slot make_slot(const DecodeArgs& a, int slot, const int* tbl, int maxR) {
     Slot s;
+    s.tok = nullptr;
     if (slot < a.n_shared) {
         s.expert = a.E;
         s.count = a.T;
         s.hbase = a.T * a.k;
         s.pair0 = 0;
         s.shared = true;
+    } else if (tbl) {
+        const int i = slot - a.n_shared;
+        s.expert = tbl[2 + i];
+        s.pair0 = tbl[2 + maxR + i];
+        s.count = tbl[2 + 2 * maxR + i];
+        s.hbase = s.pair0;
+        s.shared = false;
+        s.tok = tbl + 2 + 3 * maxR + s.pair0;
     } else {
         const int e = a.active[slot - a.n_shared];
         s.expert = e;
@@ -168,8 +183,11 @@ MOE_DEV Slot make_slot(const DecodeArgs& a, int slot) {
     }
     return s;
 }
+MOE_DEV Slot make_slot(const DecodeArgs& a, int slot) { return make_slot(a, slot, nullptr, 0); }
 
-MOE_DEV int slot_tok(const DecodeArgs& a, const Slot& s, int i) { return s.shared ? i : a.pairs[s.pair0 + i] / a.k; }
+MOE_DEV int slot_tok(const DecodeArgs& a, const Slot& s, int i) {
+    return s.shared ? i : (s.tok ? s.tok[i] : a.pairs[s.pair0 + i] / a.k);
+}
 
 MOE_DEV float h_lo(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v & 0xFFFFu))); }
 MOE_DEV float h_hi(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v >> 16))); }
@@ -841,7 +859,7 @@ struct Pipe {
 // Thread 0: issue the copies a task can start now (routed tasks need the
 // bucketing, which the caller has checked).  Returns 1 if copies were issued.
 template <int BITS, bool STAGE>
-MOE_DEV int issue_task(const DecodeArgs& a, const TaskMap& m, const Task& t, Pipe& p, int buf) {
+MOE_DEV int issue_task(const DecodeArgs& a, const TaskMap& m, const Task& t, Pipe& p, int buf, const int* tbl) {
     uint8_t* W = p.R[buf];
     uint16_t* A = reinterpret_cast<uint16_t*>(p.R[buf] + p.w_bytes);
     uint64_t* bar = p.bar + buf;
@@ -862,13 +880,13 @@ MOE_DEV int issue_task(const DecodeArgs& a, const TaskMap& m, const Task& t, Pip
             down_issue_weights<BITS>(a, make_slot(a, 0), t.idx, m.RT16, W, bar);
             return 1;
         case K_RGU:
-            if (t.sidx >= a.meta->n_active) return 0;
-            gateup_issue<BITS, STAGE>(a, make_slot(a, a.n_shared + t.sidx), t.idx, W, A, bar);
+            if (!tbl || t.sidx >= tbl[0]) return 0;
+            gateup_issue<BITS, STAGE>(a, make_slot(a, a.n_shared + t.sidx, tbl, m.maxR), t.idx, W, A, bar);
             return 1;
         case K_RDN:
-            if (t.sidx >= a.meta->n_active) return 0;
+            if (!tbl || t.sidx >= tbl[0]) return 0;
             mbar_arrive_expect_tx(bar, down_weight_bytes<BITS>(a, t.idx, m.RT16));
-            down_issue_weights<BITS>(a, make_slot(a, a.n_shared + t.sidx), t.idx, m.RT16, W, bar);
+            down_issue_weights<BITS>(a, make_slot(a, a.n_shared + t.sidx, tbl, m.maxR), t.idx, m.RT16, W, bar);
             return 1;
         default:
             return 0;
@@ -932,25 +950,47 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecodeArgs a)
         __syncthreads();
         return v;
     };
-    // Stage a task's operands into buffer `buf`.  blocking: wait for the
-    // bucketing if the task needs it; otherwise give up (return false) when it
-    // is not published yet.
+    // Stage a task's operands into buffer `buf`.  Routed tasks need the
+    // bucketing: the first one a CTA meets waits for it (blocking) or gives up
+    // (returns false) when it is not published yet; then all threads copy the
+    // slot table into shared memory once, and every later routed task reads it
+    // there instead of chasing active -> offsets -> pairs in global memory.
+    int* tbl = reinterpret_cast<int*>(p.R[1] + a.buf_bytes);
+    bool tbl_ready = false;
     auto prepare = [&](int task, int buf, bool blocking) {
         const Task t = decode_task(m, task);
-        if (threadIdx.x == 0) {
-            int ok = 1;
-            if (t.kind == K_RGU || t.kind == K_RDN) {
+        if ((t.kind == K_RGU || t.kind == K_RDN) && !tbl_ready) {
+            if (threadIdx.x == 0) {
+                int ok = 1;
                 if (blocking) ok = wait_geq(sync + SY_BUCKET, 1, sync, a.status) ? 1 : 0;
                 else if (ld_relaxed(sync + SY_BUCKET) >= 1) fence_acq_rel_gpu();
                 else ok = -1;
+                s_flag = ok;
             }
-            s_flag = ok;
-            s_issued[buf] = ok == 1 ? issue_task<BITS, STAGE>(a, m, t, p, buf) : 0;
+            __syncthreads();
+            const int f = s_flag;
+            __syncthreads();
+            if (f == -1) return false;
+            if (f == 1) {
+                const int nact = a.meta->n_active, npairs = a.offsets[a.E];
+                for (int i = threadIdx.x; i < nact; i += kDecThreads) {
+                    const int e = a.active[i], p0 = a.offsets[e];
+                    tbl[2 + i] = e;
+                    tbl[2 + m.maxR + i] = p0;
+                    tbl[2 + 2 * m.maxR + i] = a.offsets[e + 1] - p0;
+                }
+                for (int q = threadIdx.x; q < npairs; q += kDecThreads) tbl[2 + 3 * m.maxR + q] = a.pairs[q] / a.k;
+                if (threadIdx.x == 0) {
+                    tbl[0] = nact;
+                    tbl[1] = npairs;
+                }
+                __syncthreads();
+                tbl_ready = true;
+            }
         }
+        if (threadIdx.x == 0) s_issued[buf] = issue_task<BITS, STAGE>(a, m, t, p, buf, tbl_ready ? tbl : nullptr);
         __syncthreads();
-        const bool done = s_flag != -1;
-        __syncthreads();
-        return done;
+        return true;
     };
     auto run = [&](int task, int buf) {
         const Task t = decode_task(m, task);
@@ -988,7 +1028,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecodeArgs a)
             case K_RGU: {
                 if (!staged) break;  // an expert slot beyond the active ones
                 const int slot = t.kind == K_SGU ? 0 : a.n_shared + t.sidx;
-                const Slot sl = make_slot(a, slot);
+                const Slot sl = make_slot(a, slot, tbl_ready ? tbl : nullptr, m.maxR);
                 if (ok) gateup_compute<BITS, NT, STAGE>(a, sl, t.idx, red, W, A, warp, lane);
                 __threadfence();
                 __syncthreads();
@@ -1025,7 +1065,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecodeArgs a)
                     if (s_flag && t.kind == K_SDN) s_flag = wait_geq(sync + SY_BUCKET, 1, sync, a.status) ? 1 : 0;
                 }
                 __syncthreads();
-                const Slot sl = make_slot(a, slot);
+                const Slot sl = make_slot(a, slot, (t.kind == K_RDN && tbl_ready) ? tbl : nullptr, m.maxR);
                 if (STAGE && s_flag) {
                     stage_h_rows(a, sl, A);
                     __syncthreads();
@@ -1063,9 +1103,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecodeArgs a)
 }
 
 // ---------------------------------------------------------------- launcher
-// Shared memory: [gate/up reduction] [staged weights: max of router rows,
-// gate/up tile, down task] [activations: max of router x chunk, gate/up x rows,
-// down h rows, top-k buffers (8 warps x 2E floats), bucket (2E + 1 + T*k ints)].
+// Shared memory: [gate/up reduction] 2 x [staged weights: max of router rows,
+// gate/up tile, down task | activations: max of router x chunk, gate/up x rows,
+// down h rows, top-k buffers (8 warps x 2E floats), bucket (2E + 1 + T*k ints)]
+// [slot table].
 static size_t round128(size_t n) { return (n + 127) & ~size_t(127); }
 
 static size_t decode_smem(int BITS, int NT, int d, int f, int E, int T, int k, int* red_b, int* buf_b, int* w_b) {
@@ -1089,7 +1130,8 @@ static size_t decode_smem(int BITS, int NT, int d, int f, int E, int T, int k, i
     *red_b = (int)red;
     *buf_b = (int)buf;
     *w_b = (int)w;
-    return red + 2 * buf;
+    const size_t tbl = round128(4 * slot_table_words(std::min(T * k, E), T * k));  // the CTA's slot table
+    return red + 2 * buf + tbl;
 }
 
 template <int BITS, int NT>
