@@ -650,30 +650,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // ---------------------------------------------------------------- activation gather, combine
 // xg[row] = fp16(x[token of row]) in group order: rows [0, offsets[E]) are
 // the routed pairs (token pairs[row] / k), rows T*k + t the shared expert's.
-__global__ void gather_f16_kernel(const __nv_bfloat16* __restrict__ x, int T, int d, int k, int n_shared,
-                                  const int32_t* __restrict__ pairs, const int32_t* __restrict__ n_pairs,
-                                  __half* __restrict__ xg, uint32_t* status) {
-    const int row = blockIdx.x;
-    int tok;
-    if (row < T * k) {
-        if (row >= *n_pairs) return;
-        tok = pairs[row] / k;
-    } else {
-        tok = row - T * k;
+// One warp per row (32 lanes x 16 bytes per step), kGatherRowsPerCta rows per
+// CTA, so the grid is a few thousand CTAs that each stream whole rows.
+constexpr int kGatherWarps = 8;
+constexpr int kGatherRowsPerWarp = 4;
+constexpr int kGatherRowsPerCta = kGatherWarps * kGatherRowsPerWarp;
+
+__global__ void __launch_bounds__(kGatherWarps * 32)
+    gather_f16_kernel(const __nv_bfloat16* __restrict__ x, int T, int d, int k, int n_shared,
+                      const int32_t* __restrict__ pairs, const int32_t* __restrict__ n_pairs,
+                      __half* __restrict__ xg, uint32_t* status) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rows = T * k + n_shared * T, np = *n_pairs;
+    const int r0 = (blockIdx.x * kGatherWarps + warp) * kGatherRowsPerWarp;
+    int tok[kGatherRowsPerWarp];
+#pragma unroll
+    for (int i = 0; i < kGatherRowsPerWarp; ++i) {
+        const int row = r0 + i;
+        tok[i] = -1;
+        if (row < T * k) {
+            if (row < np) tok[i] = __ldg(&pairs[row]) / k;
+        } else if (row < rows) {
+            tok[i] = row - T * k;
+        }
     }
     bool finite = true;
-    for (int i = threadIdx.x * 8; i < d; i += blockDim.x * 8) {
-        const uint4 v = *reinterpret_cast<const uint4*>(x + (int64_t)tok * d + i);
-        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-        uint32_t out[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float lo = __uint_as_float(in[j] << 16), hi = __uint_as_float(in[j] & 0xFFFF0000u);
-            finite = finite && fabsf(lo) <= 65504.0f && fabsf(hi) <= 65504.0f;
-            const __half2 hv = __floats2half2_rn(lo, hi);
-            out[j] = *reinterpret_cast<const uint32_t*>(&hv);
+    for (int i = 0; i < kGatherRowsPerWarp; ++i) {
+        if (tok[i] < 0) continue;
+        const __nv_bfloat16* src = x + (int64_t)tok[i] * d;
+        __half* dst = xg + (int64_t)(r0 + i) * d;
+        for (int c = lane * 8; c < d; c += 256) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + c));
+            const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+            uint32_t out[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float lo = __uint_as_float(in[j] << 16), hi = __uint_as_float(in[j] & 0xFFFF0000u);
+                finite = finite && fabsf(lo) <= 65504.0f && fabsf(hi) <= 65504.0f;
+                const __half2 hv = __floats2half2_rn(lo, hi);
+                out[j] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
+            *reinterpret_cast<uint4*>(dst + c) = make_uint4(out[0], out[1], out[2], out[3]);
         }
-        *reinterpret_cast<uint4*>(xg + (int64_t)row * d + i) = make_uint4(out[0], out[1], out[2], out[3]);
     }
     if (!finite) flag_status(status, kStatusRange);
 }
@@ -859,7 +878,7 @@ float router_gemm_depth(int d) { return 34.0f * (float)(d / 16) + 2.0f; }
 cudaError_t launch_gather_f16(const void* x, int T, int d, int k, int n_shared, const int32_t* pairs,
                               const int32_t* n_pairs, void* xg, uint32_t* status, cudaStream_t s) {
     const int rows = T * k + n_shared * T;
-    gather_f16_kernel<<<rows, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, d, k, n_shared, pairs, n_pairs,
+    gather_f16_kernel<<<(rows + kGatherRowsPerCta - 1) / kGatherRowsPerCta, kGatherWarps * 32, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, d, k, n_shared, pairs, n_pairs,
                                           static_cast<__half*>(xg), status);
     return cudaGetLastError();
 }
