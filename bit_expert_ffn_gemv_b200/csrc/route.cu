@@ -195,38 +195,39 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
         if (lane < k) my_w = lv[my_sel];
     } else {
         // fp64 logits of the candidates (sums of exact bf16 products), 8 products
-        // per lane per 256-wide chunk, two candidates per pass
-        for (int ci = 0; ci < n_cand; ci += 2) {
-            const bool two = ci + 1 < n_cand;
-            const int e0 = cand[ci], e1 = two ? cand[ci + 1] : e0;
-            const __nv_bfloat16* row0 = wr + (int64_t)e0 * d;
-            const __nv_bfloat16* row1 = wr + (int64_t)e1 * d;
-            double acc0 = 0.0, acc1 = 0.0;
-#pragma unroll 4
+        // per lane per 256-wide chunk, four candidates per pass (more loads in flight)
+        for (int ci = 0; ci < n_cand; ci += 4) {
+            int ec[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) ec[u] = cand[min(ci + u, n_cand - 1)];
+            double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 2
             for (int i = lane * 8; i < d; i += 256) {
                 const uint4 xv = __ldg(reinterpret_cast<const uint4*>(xt + i));
-                const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(row0 + i));
-                const uint4 w1 = __ldg(reinterpret_cast<const uint4*>(row1 + i));
-                const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w}, u0[4] = {w0.x, w0.y, w0.z, w0.w},
-                               u1[4] = {w1.x, w1.y, w1.z, w1.w};
+                uint4 wv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) wv[u] = __ldg(reinterpret_cast<const uint4*>(wr + (int64_t)ec[u] * d + i));
+                const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const double xl = (double)__uint_as_float(xu[q] << 16);
                     const double xh = (double)__uint_as_float(xu[q] & 0xFFFF0000u);
-                    acc0 = fma((double)__uint_as_float(u0[q] << 16), xl, acc0);
-                    acc0 = fma((double)__uint_as_float(u0[q] & 0xFFFF0000u), xh, acc0);
-                    acc1 = fma((double)__uint_as_float(u1[q] << 16), xl, acc1);
-                    acc1 = fma((double)__uint_as_float(u1[q] & 0xFFFF0000u), xh, acc1);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const uint32_t wq = q == 0 ? wv[u].x : q == 1 ? wv[u].y : q == 2 ? wv[u].z : wv[u].w;
+                        acc[u] = fma((double)__uint_as_float(wq << 16), xl, acc[u]);
+                        acc[u] = fma((double)__uint_as_float(wq & 0xFFFF0000u), xh, acc[u]);
+                    }
                 }
             }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
-                acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
-            }
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
             if (lane == 0) {
-                lg64[ci] = acc0 + (bias ? (double)bias[e0] : 0.0);
-                if (two) lg64[ci + 1] = acc1 + (bias ? (double)bias[e1] : 0.0);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (ci + u < n_cand) lg64[ci + u] = acc[u] + (bias ? (double)bias[ec[u]] : 0.0);
             }
         }
         __syncwarp();
