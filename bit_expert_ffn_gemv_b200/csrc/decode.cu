@@ -339,12 +339,9 @@ MOE_DEV void topk_exact_scan(const double* v, int E, int k, int lane, int& sel, 
     }
 }
 
+// v: the token's E fp64 logits, already copied to this warp's shared buffer.
 MOE_DEV void topk_token(const DecodeArgs& a, int t, int lane, double* v, int* ids_s) {
     const int E = a.E, k = a.k;
-    const double* lg = a.logits64 + (int64_t)t * E;
-#pragma unroll 8
-    for (int e = lane; e < E; e += 32) v[e] = lg[e];
-    __syncwarp();
     int sel = -1;     // lane r < k keeps ids[r]
     double lsel = 0;  //   and its logit
     double top = 0;
@@ -1040,8 +1037,17 @@ __global__ void __launch_bounds__(kDecThreads) decode_kernel(const DecodeArgs a)
                 __syncthreads();
                 const int tk = t.idx * kDecWarps + warp;
                 int* ids_s = reinterpret_cast<int*>(red);  // [8 x k] ids of this CTA's tokens
-                if (s_flag && tk < a.T)
-                    topk_token(a, tk, lane, reinterpret_cast<double*>(p.R[buf]) + warp * a.E, ids_s + warp * a.k);
+                // all warps copy the logits of the CTA's tokens (one load round trip),
+                // then warp w ranks token t.idx * 8 + w
+                const int ntk = min(kDecWarps, a.T - t.idx * kDecWarps);
+                double* vb = reinterpret_cast<double*>(p.R[buf]);
+                if (s_flag) {
+                    const double* lg = a.logits64 + (int64_t)t.idx * kDecWarps * a.E;
+#pragma unroll 4
+                    for (int i = threadIdx.x; i < ntk * a.E; i += kDecThreads) vb[i] = lg[i];
+                }
+                __syncthreads();
+                if (s_flag && tk < a.T) topk_token(a, tk, lane, vb + warp * a.E, ids_s + warp * a.k);
                 __threadfence();
                 __syncthreads();
                 if (threadIdx.x == 0) {
