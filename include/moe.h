@@ -209,8 +209,8 @@ moe_status moe_debug_last_routing(moe_handle* h, int32_t T, int32_t* ids, float*
 /*
  * Debug: the fp32 router logits l = W_r x + bias [T x n_experts] (device,
  * row-major) of a loaded layer as one of the two router kernels computes
- * them: tensor_cores != 0 the bf16 tcgen05 GEMM used for T > 64 tokens, else
- * the CUDA-core kernel.  Each logit is within
+ * them: tensor_cores != 0 the bf16 tcgen05 GEMM (a forward uses it above 16
+ * tokens, moe_route above 64), else the CUDA-core kernel.  Each logit is within
  *   delta_e = 2 * depth * 2^-24 * (||W_r,e||_2 ||x||_2 + |bias_e|)
  * of the exact value, depth = moe_router_error_depth(d, tensor_cores); the
  * top-k re-ranks every token whose order these intervals leave open.

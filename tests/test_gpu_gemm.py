@@ -1,6 +1,6 @@
 """Parity of the tensor-core (tcgen05) path with the fp64 oracle.
 
-The path runs for T > 64 tokens, or for any T with MOE_FORCE_GEMM: router
+The path runs for T > 16 tokens, or for any T with MOE_FORCE_GEMM: router
 logits from a bf16 GEMM (certified against their error bound, then re-ranked
 in fp64 where the order is open), grouped gate/up and down GEMMs over expert
 groups with weights dequantised to fp16 in shared memory, and a fixed-order
