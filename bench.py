@@ -41,7 +41,8 @@ def parse():
     p.add_argument("--tokens", type=int, default=None)
     p.add_argument("--bits", type=int, default=2)
     p.add_argument("--rotate", type=int, default=8, help="distinct layers cycled through (decode/sweep)")
-    p.add_argument("--flags", default="", help="extra forward flags: gemv|gemm")
+    p.add_argument("--flags", default="", help="extra forward flags, '+'-separated: gemv, gemm, tailskip "
+                   "(the route-tail skip approximation)")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU-baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -269,7 +270,10 @@ def ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
     build.build()
     wl, sh, T, layers = workload(args)
-    flags = {"": 0, "gemv": moe.MOE_FORCE_GEMV, "gemm": moe.MOE_FORCE_GEMM}[args.flags]
+    names = {"gemv": moe.MOE_FORCE_GEMV, "gemm": moe.MOE_FORCE_GEMM, "tailskip": moe.MOE_ROUTE_TAIL_SKIP}
+    flags = 0
+    for f in filter(None, args.flags.split("+")):
+        flags |= names[f]
 
     # ---- setup: layers generated on the device, one handle holding all of them
     h = moe.MoeLayer(sh.d, sh.f, sh.E, sh.k, sh.n_shared, layers, sh.bits, T)
@@ -423,7 +427,8 @@ def ours(args):
                            "top_k": sh.k, "shared": sh.n_shared, "bits": sh.bits, "layers": layers,
                            "l2": ("inputs larger than L2: 48 layers x 756 MB per step" if chain else
                                   f"inputs larger than L2: {layers} distinct layers cycled, {n_x} fresh inputs"),
-                           "parallelism": f"replicas x{world}", "timing": "CUDA graph replay" if graph is not None else "eager"},
+                           "parallelism": f"replicas x{world}", "timing": "CUDA graph replay" if graph is not None else "eager",
+                           **({"flags": args.flags} if args.flags else {})},
                 "roofline": roof, "layer_hbm_gbs": layer_gbs,
                 "kernels_ms_per_step": {k: v[0] / nprof for k, v in prof.items()},
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary()}

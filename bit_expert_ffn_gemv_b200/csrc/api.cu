@@ -70,7 +70,13 @@ struct moe_handle {
 namespace {
 
 
-constexpr uint32_t kAllFlags = MOE_OUT_FP32 | MOE_ACCUMULATE | MOE_FORCE_GEMV | MOE_FORCE_GEMM | MOE_FORCE_UNFUSED;
+constexpr uint32_t kAllFlags =
+    MOE_OUT_FP32 | MOE_ACCUMULATE | MOE_FORCE_GEMV | MOE_FORCE_GEMM | MOE_FORCE_UNFUSED | MOE_ROUTE_TAIL_SKIP;
+
+// Rank from which the route-tail skip drops an expert (0: off, or no rank of k reaches it).
+int skip_rank(const moe_config& c, uint32_t flags) {
+    return (flags & MOE_ROUTE_TAIL_SKIP) && MOE_TAIL_SKIP_RANK < c.top_k ? MOE_TAIL_SKIP_RANK : 0;
+}
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -175,6 +181,7 @@ moe_status do_decode(moe_handle* h, int32_t layer, const void* x, int32_t T, voi
     d.h = h->h;
     d.obuf = h->obuf;
     d.sync = h->sync;
+    d.skip_rank = skip_rank(c, flags);
     return cuda_status(run(h, MOE_K_DECODE, s, [&] { return moe::launch_decode(d, s); }));
 }
 
@@ -203,6 +210,7 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
         ba.wsorted = h->wsorted;
     }
     ba.cnt = h->bucket_cnt;
+    ba.skip_rank = skip_rank(c, flags);
     e = run(h, MOE_K_BUCKET, s, [&] { return moe::launch_bucket(ba, s); });
     h->launches += moe::bucket_kernel_count(ba) - 1;
     if (e != cudaSuccess) return MOE_ERR_CUDA;

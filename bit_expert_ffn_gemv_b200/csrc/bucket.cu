@@ -22,11 +22,12 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
     bucket_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int32_t* __restrict__ offsets,
                   int32_t* __restrict__ pairs, int32_t* __restrict__ inv, int32_t* __restrict__ active,
                   Meta* __restrict__ meta, uint32_t* __restrict__ status, const float* __restrict__ w,
-                  float* __restrict__ wsorted) {
+                  float* __restrict__ wsorted, int R) {
     extern __shared__ int32_t sm[];
     int32_t* cnt = sm;                          // [kBucketWarps][E]
     int32_t* total = sm + kBucketWarps * E;     // [E]
     int32_t* off_s = total + E;                 // [E + 1]
+    int32_t* best = off_s + E + 1;              // [E] lowest rank of each expert (route-tail skip, R > 0)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_pairs = T * k;
     const int ppw = ((n_pairs + kBucketWarps - 1) / kBucketWarps + 31) & ~31;
@@ -34,6 +35,7 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
     const uint32_t lt = (1u << lane) - 1u;
 
     for (int i = threadIdx.x; i < kBucketWarps * E; i += blockDim.x) cnt[i] = 0;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) best[e] = k;
     __syncthreads();
 
     // phase 1: per-warp counts (one smem update per distinct expert per 32
@@ -53,11 +55,13 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
             if (live && !valid) flag_status(status, kStatusBounds);
             const uint32_t same = __match_any_sync(0xffffffffu, valid ? e : -1);
             if (valid && (same & lt) == 0) cnt[warp * E + e] += __popc(same);
+            if (R > 0 && valid) atomicMin(&best[e], (p0 + 32 * u + lane) % k);
         }
     }
     __syncthreads();
 
-    // phase 2: per-expert prefix over warps, totals
+    // phase 2: per-expert prefix over warps, totals; an expert that no token
+    // ranks before R (route-tail skip) gets no group
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int run = 0;
         for (int w = 0; w < kBucketWarps; ++w) {
@@ -65,7 +69,7 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
             cnt[w * E + e] = run;
             run += c;
         }
-        total[e] = run;
+        total[e] = (R > 0 && best[e] >= R) ? 0 : run;
     }
     __syncthreads();
 
@@ -115,7 +119,7 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
             const int e = ev[u];
             const int p = p0 + 32 * u + lane;
             const bool live = p < p_end;
-            const bool valid = live && e >= 0 && e < E;
+            const bool valid = live && e >= 0 && e < E && !(R > 0 && best[e] >= R);
             const uint32_t same = __match_any_sync(0xffffffffu, valid ? e : -1);
             const int leader = __ffs(same) - 1;
             int base = 0;
@@ -150,28 +154,41 @@ constexpr int kChunks = 128;
 constexpr int kChunkWarps = 8;
 
 __global__ void __launch_bounds__(kChunkWarps * 32)
-    bucket_count_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int chunk, int32_t* __restrict__ cnt,
-                        uint32_t* __restrict__ status) {
-    extern __shared__ int32_t h[];  // [E]
+    bucket_count_kernel(const int32_t* __restrict__ ids, int n_pairs, int k, int E, int chunk,
+                        int32_t* __restrict__ cnt, int32_t* __restrict__ best, int R, uint32_t* __restrict__ status) {
+    extern __shared__ int32_t h[];  // [E] counts | [E] lowest rank (R > 0)
+    int32_t* hb = h + E;
     const int c = blockIdx.x;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        h[e] = 0;
+        if (R > 0) hb[e] = k;
+    }
     __syncthreads();
     const int p0 = c * chunk, p1 = min(n_pairs, p0 + chunk);
     for (int p = p0 + threadIdx.x; p < p1; p += blockDim.x) {
         const int e = __ldg(&ids[p]);
-        if (e >= 0 && e < E) atomicAdd(&h[e], 1);
-        else flag_status(status, kStatusBounds);
+        if (e >= 0 && e < E) {
+            atomicAdd(&h[e], 1);
+            if (R > 0) atomicMin(&hb[e], p % k);
+        } else {
+            flag_status(status, kStatusBounds);
+        }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[(int64_t)c * E + e] = h[e];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        cnt[(int64_t)c * E + e] = h[e];
+        if (R > 0) best[(int64_t)c * E + e] = hb[e];
+    }
 }
 
-__global__ void __launch_bounds__(1024) bucket_scan_kernel(int32_t* __restrict__ cnt, int nchunks, int E,
-                                                           int32_t* __restrict__ offsets,
+__global__ void __launch_bounds__(1024) bucket_scan_kernel(int32_t* __restrict__ cnt, int32_t* __restrict__ best,
+                                                           int R, int nchunks, int E, int32_t* __restrict__ offsets,
                                                            int32_t* __restrict__ active, Meta* __restrict__ meta) {
     extern __shared__ int32_t tot[];  // [E]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // per expert: exclusive prefix over the chunks (in place), total
+    // per expert: exclusive prefix over the chunks (in place), total; with
+    // R > 0, the lowest rank over the chunks goes to best[e] (row 0) and an
+    // expert with none below R gets no group
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int run = 0;
 #pragma unroll 8
@@ -179,6 +196,12 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(int32_t* __restrict__
             const int v = cnt[(int64_t)c * E + e];
             cnt[(int64_t)c * E + e] = run;
             run += v;
+        }
+        if (R > 0) {
+            int b = best[e];
+            for (int c = 1; c < nchunks; ++c) b = min(b, best[(int64_t)c * E + e]);
+            best[e] = b;
+            if (b >= R) run = 0;
         }
         tot[e] = run;
     }
@@ -216,7 +239,7 @@ __global__ void __launch_bounds__(kChunkWarps * 32)
     bucket_scatter_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int chunk,
                           const int32_t* __restrict__ cbase, const int32_t* __restrict__ offsets,
                           int32_t* __restrict__ pairs, int32_t* __restrict__ inv, const float* __restrict__ w,
-                          float* __restrict__ wsorted) {
+                          float* __restrict__ wsorted, const int32_t* __restrict__ best, int R) {
     extern __shared__ int32_t wc[];  // [kChunkWarps][E] per-warp running position
     const int c = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t lt = (1u << lane) - 1u;
@@ -228,7 +251,7 @@ __global__ void __launch_bounds__(kChunkWarps * 32)
     // per-warp counts of this warp's sub-range
     for (int p = q0; p < q1; p += 32) {
         const int e = p + lane < q1 ? __ldg(&ids[p + lane]) : -1;
-        const bool valid = e >= 0 && e < E;
+        const bool valid = e >= 0 && e < E && !(R > 0 && best[e] >= R);
         const uint32_t same = __match_any_sync(0xffffffffu, valid ? e : -1);
         if (valid && (same & lt) == 0) wc[warp * E + e] += __popc(same);
     }
@@ -247,7 +270,7 @@ __global__ void __launch_bounds__(kChunkWarps * 32)
     for (int p = q0; p < q1; p += 32) {
         const bool live = p + lane < q1;
         const int e = live ? __ldg(&ids[p + lane]) : -1;
-        const bool valid = e >= 0 && e < E;
+        const bool valid = e >= 0 && e < E && !(R > 0 && best[e] >= R);
         const uint32_t same = __match_any_sync(0xffffffffu, valid ? e : -1);
         const int leader = __ffs(same) - 1;
         int base = 0;
@@ -269,11 +292,15 @@ __global__ void __launch_bounds__(kChunkWarps * 32)
 
 cudaError_t launch_bucket(const BucketArgs& a, cudaStream_t s) {
     const int n_pairs = a.T * a.k;
+    const int R = a.skip_rank > 0 && a.skip_rank < a.k ? a.skip_rank : 0;
     if (bucket_kernel_count(a) == 3) {
         const int chunk = (n_pairs + kChunks - 1) / kChunks;
-        bucket_count_kernel<<<kChunks, kChunkWarps * 32, sizeof(int32_t) * a.E, s>>>(a.ids, n_pairs, a.E, chunk, a.cnt,
-                                                                                     a.status);
-        bucket_scan_kernel<<<1, 1024, sizeof(int32_t) * a.E, s>>>(a.cnt, kChunks, a.E, a.offsets, a.active, a.meta);
+        int32_t* best = a.cnt + (size_t)kChunks * a.E;
+        bucket_count_kernel<<<kChunks, kChunkWarps * 32, 2 * sizeof(int32_t) * a.E, s>>>(a.ids, n_pairs, a.k, a.E,
+                                                                                         chunk, a.cnt, best, R,
+                                                                                         a.status);
+        bucket_scan_kernel<<<1, 1024, sizeof(int32_t) * a.E, s>>>(a.cnt, best, R, kChunks, a.E, a.offsets, a.active,
+                                                                   a.meta);
         const size_t smem = sizeof(int32_t) * (size_t)kChunkWarps * a.E;
         if (smem > 48 * 1024) {
             cudaError_t e = cudaFuncSetAttribute(bucket_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -281,22 +308,22 @@ cudaError_t launch_bucket(const BucketArgs& a, cudaStream_t s) {
             if (e != cudaSuccess) return e;
         }
         bucket_scatter_kernel<<<kChunks, kChunkWarps * 32, smem, s>>>(a.ids, n_pairs, a.E, chunk, a.cnt, a.offsets,
-                                                                      a.pairs, a.inv, a.w, a.wsorted);
+                                                                      a.pairs, a.inv, a.w, a.wsorted, best, R);
         return cudaGetLastError();
     }
-    const size_t smem = sizeof(int32_t) * ((size_t)kBucketWarps * a.E + 2 * (size_t)a.E + 1);
+    const size_t smem = sizeof(int32_t) * ((size_t)kBucketWarps * a.E + 3 * (size_t)a.E + 1);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(bucket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
     bucket_kernel<<<1, kBucketWarps * 32, smem, s>>>(a.ids, a.T, a.k, a.E, a.offsets, a.pairs, a.inv, a.active,
-                                                     a.meta, a.status, a.w, a.wsorted);
+                                                     a.meta, a.status, a.w, a.wsorted, R);
     return cudaGetLastError();
 }
 
 }  // namespace moe
 
 namespace moe {
-size_t bucket_scratch_words(int E) { return (size_t)kChunks * E; }
+size_t bucket_scratch_words(int E) { return 2 * (size_t)kChunks * E; }
 int bucket_kernel_count(const BucketArgs& a) { return (a.cnt && a.T * a.k >= 8192) ? 3 : 1; }
 }  // namespace moe

@@ -113,6 +113,7 @@ struct DecodeArgs {
     __half* h;
     float* obuf;
     int* sync;
+    int skip_rank;  // route-tail skip: drop experts whose best rank is >= this (0: off)
     int red_bytes;  // shared memory: [red_bytes] reductions | 2 x [buf_bytes] staging buffers
     int buf_bytes;  //   each buffer: [w_bytes] weights | activations
     int w_bytes;
@@ -448,15 +449,46 @@ MOE_DEV void bucket_cta(const DecodeArgs& a, int* sm, const int* ids_local) {
     int* off = sm + E;
     int* ids = off + E + 1;
     int* wtot = ids + n;
-    for (int e = threadIdx.x; e < E; e += kDecThreads) cnt[e] = 0;
+    const int R = a.skip_rank;  // > 0: route-tail skip from this rank on
+    for (int e = threadIdx.x; e < E; e += kDecThreads) {
+        cnt[e] = 0;
+        off[e] = k;  // best (lowest) rank of expert e in the batch, until the scan
+    }
     for (int i = threadIdx.x; i < n; i += kDecThreads) ids[i] = ids_local ? ids_local[i] : a.ids[i];
     __syncthreads();
     for (int i = threadIdx.x; i < n; i += kDecThreads) {
         const int e = ids[i];
-        if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);
-        else flag_status(a.status, kStatusBounds);
+        if (e >= 0 && e < E) {
+            atomicAdd(&cnt[e], 1);
+            if (R > 0) atomicMin(&off[e], i % k);
+        } else {
+            flag_status(a.status, kStatusBounds);
+        }
     }
     __syncthreads();
+    if (R > 0) {
+        // experts no token ranks before R drop out: no count, their pairs get inv = -1
+        for (int e = threadIdx.x; e < E; e += kDecThreads)
+            if (off[e] >= R) cnt[e] = 0;
+        for (int i = threadIdx.x; i < n; i += kDecThreads) {
+            const int e = ids[i];
+            if (e >= 0 && e < E && off[e] >= R) ids[i] = -1;
+        }
+        __syncthreads();
+        // A dropped pair never reports to its token's combine counters (one per
+        // 16-row output tile, complete at k + n_shared): count it in advance.
+        // Nothing touches these counters before the bucketing is published.
+        const int RT = a.d / 16;
+        for (int j = threadIdx.x; j < a.T * RT; j += kDecThreads) {
+            const int t = j / RT;
+            int nd = 0;
+            for (int r = 0; r < k; ++r) {
+                const int e = ids[t * k + r];
+                nd += (e < 0 || e >= E) ? 1 : 0;
+            }
+            if (nd) atomicAdd(a.sync + SY_SLOTS + (1 + E) + j, nd);
+        }
+    }
     // block-wide exclusive scan of cnt and of the active flags: warp w owns a
     // contiguous chunk of experts, 32 per step
     const int chunk = ((E + kDecWarps - 1) / kDecWarps + 31) & ~31;
@@ -1194,6 +1226,7 @@ static cudaError_t decode_bits_nt(const DecodeLaunch& L, cudaStream_t st) {
     a.h = static_cast<__half*>(L.h);
     a.obuf = L.obuf;
     a.sync = L.sync;
+    a.skip_rank = L.skip_rank;
     a.red_bytes = red_b;
     a.buf_bytes = buf_b;
     a.w_bytes = w_b;

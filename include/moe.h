@@ -101,6 +101,20 @@ typedef struct {
 #define MOE_FORCE_GEMV 0x4u /* CUDA-core paths: the fused kernel up to 64 tokens, grouped GEMV above */
 #define MOE_FORCE_GEMM 0x8u /* the tensor-core grouped-GEMM path whatever T is */
 #define MOE_FORCE_UNFUSED 0x10u /* one kernel per step (grouped GEMV) instead of the fused persistent kernel */
+/*
+ * Route-tail skip (an approximation, off by default): a routed expert is not
+ * computed when every token of the call that selected it ranked it at
+ * position MOE_TAIL_SKIP_RANK or later (0-based, i.e. 7th to 10th of a
+ * top-10).  Its (token, rank) pairs drop out of the sum; the remaining
+ * weights keep their values (no second renormalisation), and the routing
+ * that moe_debug_last_routing reports is unchanged.  The rule is the one the
+ * discuss.pytorch.kr post describes in "Strata's operating principle /
+ * experts split across VRAM, RAM and SSD" for experts outside the GPU cache;
+ * here it applies to every routed expert, since all of them are resident.
+ * The decision is per call: it depends on which tokens share the batch.
+ */
+#define MOE_ROUTE_TAIL_SKIP 0x20u
+#define MOE_TAIL_SKIP_RANK 6
 
 /*
  * Create a handle on the current CUDA device.  Checks the configuration and

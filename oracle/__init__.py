@@ -56,7 +56,7 @@ def lib():
             L.oracle_route.restype = i32
             L.oracle_route.argtypes = [ctypes.POINTER(Shape), vp, i32, vp, vp, vp, vp, vp]
             L.oracle_layer.restype = i32
-            L.oracle_layer.argtypes = [ctypes.POINTER(Shape), vp, i32, vp, vp, vp, vp, vp, vp, vp]
+            L.oracle_layer.argtypes = [ctypes.POINTER(Shape), vp, i32, vp, vp, vp, vp, vp, vp, vp, vp]
             L.oracle_threads.restype = i32
             L.oracle_threads.argtypes = [i32]
             _lib = L
@@ -108,11 +108,37 @@ def route(shape, x: np.ndarray, router_w: np.ndarray, bias, with_logits: bool = 
     return (ids, w, lg) if with_logits else (ids, w)
 
 
-def layer(shape, x: np.ndarray, router_w: np.ndarray, bias, codes: list, scales: list):
+def tail_skip(ids: np.ndarray, E: int, rank: int) -> np.ndarray:
+    """Route-tail skip of one batch: drop[e] = 1 for every expert that some
+    token of the batch selects and that every token selecting it ranks at
+    position `rank` or later (0-based; 6 = "7th or lower" of a top-10).
+
+    The rule of the discuss.pytorch.kr post, section "Strata's operating
+    principle / experts split across VRAM, RAM and SSD": an expert that all
+    the tokens processed together picked only at ranks 7 to 10 is skipped.
+    Written as its definition: the best (lowest) rank of each expert over the
+    batch, then the comparison.
+    """
+    T, k = ids.shape
+    best = {}
+    for t in range(T):
+        for r in range(k):
+            e = int(ids[t, r])
+            best[e] = min(best.get(e, k), r)
+    drop = np.zeros(E, np.uint8)
+    for e, b in best.items():
+        if b >= rank:
+            drop[e] = 1
+    return drop
+
+
+def layer(shape, x: np.ndarray, router_w: np.ndarray, bias, codes: list, scales: list, drop=None):
     """Full layer: (y [T,d] f64, ids [T,k], w [T,k]).
 
     codes/scales: per-expert packed arrays (index E = shared expert); None for
-    experts that no token selects.
+    experts that no token selects.  drop: optional uint8 [E] mask (see
+    tail_skip); the terms of dropped experts leave the routed sum and the
+    other weights keep their values.
     """
     x = np.ascontiguousarray(x, np.uint16)
     T = x.shape[0]
@@ -124,9 +150,11 @@ def layer(shape, x: np.ndarray, router_w: np.ndarray, bias, codes: list, scales:
     ids = np.empty((T, shape.k), np.int32)
     w = np.empty((T, shape.k), np.float64)
     b = None if bias is None else np.ascontiguousarray(bias, np.float32)
+    dm = None if drop is None else np.ascontiguousarray(drop, np.uint8)
+    assert dm is None or dm.shape == (shape.E,)
     rc = lib().oracle_layer(ctypes.byref(_shape(shape)), _p(x), T, _p(np.ascontiguousarray(router_w, np.uint16)),
-                            _p(b), ctypes.cast(cptr, ctypes.c_void_p), ctypes.cast(sptr, ctypes.c_void_p), _p(y),
-                            _p(ids), _p(w))
+                            _p(b), ctypes.cast(cptr, ctypes.c_void_p), ctypes.cast(sptr, ctypes.c_void_p), _p(dm),
+                            _p(y), _p(ids), _p(w))
     if rc == -2:
         raise KeyError("oracle_layer: a selected expert was not materialised")
     if rc != 0:

@@ -23,6 +23,9 @@
  *        What[n,k] = q[n,k] * double(s[n, k/32])
  *        g = What_g x, u = What_u x, h = g / (1 + exp(-g)) * u, o = What_d h
  *   6. y = o_shared + sum_r w_r o_r
+ *      (with the route-tail skip, the caller passes drop[e] = 1 for the
+ *      experts the batch-level rule removes, and their terms leave the sum;
+ *      see tail_skip in __init__.py)
  * Everything is in fp64; nothing intermediate is rounded.  Step 3 is a
  * selection scan: repeatedly take the largest remaining l, the lowest index
  * among equals (NaN ranks as -inf).
@@ -216,8 +219,8 @@ static void expert_eval(const oracle_shape* s, const uint8_t* codes, const uint1
  * Returns 0, -1 on bad arguments, -2 when a needed expert is NULL.
  */
 int oracle_layer(const oracle_shape* s, const uint16_t* x, int T, const uint16_t* wr, const float* bias,
-                 const uint8_t* const* codes, const uint16_t* const* scales, double* y, int32_t* ids_out,
-                 double* w_out) {
+                 const uint8_t* const* codes, const uint16_t* const* scales, const unsigned char* drop, double* y,
+                 int32_t* ids_out, double* w_out) {
     if (!shape_ok(s) || T < 0 || (T > 0 && (!x || !wr || !codes || !scales || !y))) return -1;
     int d = s->d, E = s->E, k = s->k;
     int bad = 0;
@@ -250,6 +253,7 @@ int oracle_layer(const oracle_shape* s, const uint16_t* x, int T, const uint16_t
             }
             for (int r = 0; r < k; ++r) {
                 int e = ids[r];
+                if (drop && drop[e]) continue; /* route-tail skip: the pair leaves the sum, w keeps its value */
                 if (!codes[e] || !scales[e]) {
 #pragma omp atomic write
                     bad = 1;

@@ -69,3 +69,12 @@ def test_null_arguments(L):
     assert L.moe_profile(None, 1) == 1
     assert L.moe_profile_read(None, None, None) == 1
     assert moe.moe_kernel_name(0) == "router_logits" and moe.moe_kernel_name(99) == "unknown"
+
+
+def test_flag_constants_match_the_header():
+    """Every #define MOE_* value of the header equals the binding's constant of the same name."""
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    defs = dict(re.findall(r"#define\s+(MOE_[A-Z0-9_]+)\s+(0x[0-9a-fA-F]+|\d+)u?\b", src))
+    assert {"MOE_OUT_FP32", "MOE_ROUTE_TAIL_SKIP", "MOE_TAIL_SKIP_RANK"} <= set(defs)
+    for name, v in defs.items():
+        assert getattr(moe, name) == int(v, 0), name

@@ -329,3 +329,57 @@ def test_bad_arguments():
     shape = MoeShape(d=128, f=128, E=8, k=9, n_shared=1, bits=2)
     with pytest.raises(ValueError):
         oracle.route(shape, np.zeros((1, 128), np.uint16), np.zeros((8, 128), np.uint16), None)
+
+
+# ------------------------------------------------------------------ route-tail skip
+def test_tail_skip_hand_worked_batch():
+    """Two tokens of a top-10 over 16 experts, worked by hand: best ranks 5:0 9:0 2:2 6:2 7:3 12:3 11:4
+    3:5 10:5 4:6 13:6 0:7 8:7 1:8 14:8 15:9, so rank 6 drops {0, 1, 4, 8, 13, 14, 15} -- expert 0 is
+    7th for one token and 10th for the other, expert 2 stays because token 0 ranks it 3rd."""
+    ids = np.array([[5, 9, 2, 7, 11, 3, 4, 8, 1, 0],
+                    [9, 5, 6, 12, 2, 10, 13, 0, 14, 15]], np.int32)
+    drop = oracle.tail_skip(ids, 16, 6)
+    assert sorted(np.flatnonzero(drop).tolist()) == [0, 1, 4, 8, 13, 14, 15]
+    # each token alone: its own ranks 6..9
+    assert sorted(np.flatnonzero(oracle.tail_skip(ids[:1], 16, 6)).tolist()) == sorted([4, 8, 1, 0])
+    assert sorted(np.flatnonzero(oracle.tail_skip(ids[1:], 16, 6)).tolist()) == sorted([13, 0, 14, 15])
+
+
+def test_tail_skip_limits(tiny):
+    """rank >= k drops nothing (the layer is unchanged bit for bit); rank 0 drops every selected expert
+    (only the shared expert is left)."""
+    shape, L = tiny
+    x = _x(shape, 8, 11)
+    ids, _ = oracle.route(shape, x, L["router_w"], L["bias"])
+    assert not oracle.tail_skip(ids, shape.E, shape.k).any()
+    y, _, _ = oracle.layer(shape, x, L["router_w"], L["bias"], L["codes"], L["scales"])
+    y0, _, _ = oracle.layer(shape, x, L["router_w"], L["bias"], L["codes"], L["scales"],
+                            drop=oracle.tail_skip(ids, shape.E, shape.k))
+    assert np.array_equal(y, y0)
+    all_drop = oracle.tail_skip(ids, shape.E, 0)
+    assert np.array_equal(np.flatnonzero(all_drop), np.unique(ids))
+    ys, _, _ = oracle.layer(shape, x, L["router_w"], L["bias"], L["codes"], L["scales"], drop=all_drop)
+    g = _bf16(x) @ L["deq"][shape.E][0].T
+    u = _bf16(x) @ L["deq"][shape.E][1].T
+    o = (g / (1 + np.exp(-g)) * u) @ L["deq"][shape.E][2].T
+    assert np.allclose(ys, o, rtol=1e-12, atol=1e-15)
+
+
+def test_tail_skip_equals_zeroed_experts():
+    """Dropping an expert's terms equals giving that expert all-zero scales (its output is then exactly
+    0, and routing depends on the router alone): a different mechanism for the same sum."""
+    shape = MoeShape(d=128, f=128, E=24, k=8, n_shared=1, bits=3)
+    L = _random_layer(shape, seed=91, bias_scale=0.8)
+    x = _x(shape, 6, 12)
+    ids, _ = oracle.route(shape, x, L["router_w"], L["bias"])
+    drop = oracle.tail_skip(ids, shape.E, 6)
+    assert drop.any() and (np.unique(ids).size > drop.sum()), "test needs some dropped and some kept experts"
+    ys, ids_s, w_s = oracle.layer(shape, x, L["router_w"], L["bias"], L["codes"], L["scales"], drop=drop)
+    scales = [np.zeros_like(s) if e < shape.E and drop[e] else s for e, s in enumerate(L["scales"])]
+    yz, ids_z, w_z = oracle.layer(shape, x, L["router_w"], L["bias"], L["codes"], scales)
+    assert np.array_equal(ids_s, ids) and np.array_equal(ids_z, ids) and np.array_equal(w_s, w_z)
+    assert np.array_equal(ys, yz)
+    # and the single-token batch drops exactly that token's ranks 6.. (nothing else can save them)
+    for t in range(x.shape[0]):
+        d1 = oracle.tail_skip(ids[t:t + 1], shape.E, 6)
+        assert sorted(np.flatnonzero(d1).tolist()) == sorted(ids[t, 6:].tolist())
