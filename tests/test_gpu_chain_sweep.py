@@ -153,3 +153,40 @@ def test_wide_full_layer(torch_cuda, wide, T):
     assert np.array_equal(ids.cpu().numpy(), ids_ref), f"b{sh.bits} T={T}: expert selection differs"
     _compare(sh, L, xb, y32, y16, label=f"b{sh.bits} T={T}", rows=rows,
              fp32_tol=REL_L2_FP32 if T <= 16 else REL_L2_FP32_TC)
+
+
+# ------------------------------------------------------------------ Coder shape (256 routed experts)
+@pytest.fixture(scope="module")
+def coder(torch_cuda):
+    from synth import gpu as sgpu
+    import bit_expert_ffn_gemv_b200 as moe
+    wl = WORKLOADS["sweep"]
+    b = wl.shape
+    sh = MoeShape(b.d, b.f, 256, b.k, b.n_shared, 2)
+    w = sgpu.layer_device(sh, wl.master + 256, 0, wl.zipf)
+    h = moe.MoeLayer(sh.d, sh.f, sh.E, sh.k, sh.n_shared, 1, sh.bits, 512)
+    h.load_layer(0, *w)
+    yield wl, sh, h
+    h.close()
+
+
+@pytest.mark.parametrize("T", [1, 4, 16, 64, 512])
+def test_coder_shape_layer(torch_cuda, coder, T):
+    """E = 256 (the Coder variant keeps 256 of the 512 experts), k = 10, d = 2048, f = 768: fused decode
+    path up to 16 tokens, tensor-core path above (sampled rows at 512)."""
+    import bit_expert_ffn_gemv_b200 as moe
+    wl, sh, h = coder
+    master = wl.master + 256
+    xb = synth.x_host(sh, master, 700 + T, T)
+    rows = np.arange(T) if T <= 64 else np.unique(np.r_[0, T - 1, np.random.default_rng(T).choice(T, 30, False)])
+    x = x_to_device(xb)
+    y32 = h.forward(0, x, flags=moe.MOE_OUT_FP32)
+    y16 = h.forward(0, x)
+    ids, _ = h.last_routing(T)
+    torch_cuda.cuda.synchronize()
+    assert h.check_status() == 0
+    L = _host_layer(sh, master, 0, wl.zipf, xb[rows])
+    ids_ref, _ = oracle.route(sh, xb, L["router_w"], L["bias"])
+    assert np.array_equal(ids.cpu().numpy(), ids_ref), f"E=256 T={T}: expert selection differs"
+    _compare(sh, L, xb, y32, y16, label=f"E=256 T={T}", rows=rows,
+             fp32_tol=REL_L2_FP32 if T <= 16 else REL_L2_FP32_TC)
