@@ -21,7 +21,8 @@ __all__ = ["MoeError", "MoeConfig", "MoeLayerWeights", "MoeLayer", "lib", "libra
            "MOE_TAIL_SKIP_RANK", "STATUS", "moe_layer_init", "moe_load_layer",
            "moe_route", "moe_route_noalloc", "moe_forward", "moe_forward_host", "moe_destroy", "moe_debug_dequant", "moe_debug_last_routing", "moe_check_status",
            "moe_get_stats", "moe_status_string", "moe_profile", "moe_profile_read", "moe_kernel_name", "MoeStats",
-           "moe_debug_router_logits", "moe_router_error_depth", "moe_rms_normalize", "rms_normalize"]
+           "moe_debug_router_logits", "moe_router_error_depth", "moe_rms_normalize", "rms_normalize",
+           "moe_set_expert_range"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libmoe.so")
@@ -110,6 +111,8 @@ def lib() -> ctypes.CDLL:
             L.moe_router_error_depth.argtypes = [i32, i32]
             L.moe_rms_normalize.restype = st
             L.moe_rms_normalize.argtypes = [vp, i32, i32, vp, vp]
+            L.moe_set_expert_range.restype = st
+            L.moe_set_expert_range.argtypes = [vp, i32, i32, i32]
             L.moe_status_string.restype = ctypes.c_char_p
             L.moe_status_string.argtypes = [st]
             _lib = L
@@ -156,6 +159,10 @@ def moe_route_noalloc(x_ptr: int, T: int, d: int, n_experts: int, top_k: int, ro
     """Routing for callers that cannot allocate device memory (no handle; fixed in-library scratch)."""
     _check(lib().moe_route_noalloc(x_ptr, T, d, n_experts, top_k, router_w_ptr, bias_ptr, ids_ptr, w_ptr, stream),
            "moe_route_noalloc")
+
+
+def moe_set_expert_range(handle: int, begin: int, end: int, with_shared: int) -> None:
+    _check(lib().moe_set_expert_range(handle, begin, end, with_shared), "moe_set_expert_range")
 
 
 def moe_destroy(handle: int) -> None:
@@ -307,6 +314,10 @@ class MoeLayer:
 
     def profile_read(self):
         return moe_profile_read(self.handle)
+
+    def set_expert_range(self, begin, end, with_shared=True):
+        """Compute only routed experts [begin, end) (and the shared one if with_shared) from now on."""
+        moe_set_expert_range(self.handle, begin, end, 1 if with_shared else 0)
 
     def close(self):
         if self.handle:

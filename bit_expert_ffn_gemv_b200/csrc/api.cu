@@ -58,6 +58,8 @@ struct moe_handle {
     int32_t* n_tiles = nullptr;  // [2] descriptor counts
     float* wsorted = nullptr;    // routing weights in group order
     int32_t* bucket_cnt = nullptr;  // per-chunk expert counts (multi-CTA bucketing)
+    // expert parallelism: the routed experts this handle computes, and whether it adds the shared one
+    int32_t ep_begin = 0, ep_end = 1 << 30, ep_shared = 1;
     // launch accounting and optional per-kernel event timing
     int64_t launches = 0;
     bool prof_on = false;
@@ -72,6 +74,9 @@ namespace {
 
 constexpr uint32_t kAllFlags =
     MOE_OUT_FP32 | MOE_ACCUMULATE | MOE_FORCE_GEMV | MOE_FORCE_GEMM | MOE_FORCE_UNFUSED | MOE_ROUTE_TAIL_SKIP;
+
+// Shared experts this handle computes (0 when another rank owns the shared expert).
+int eff_shared(const moe_handle* h) { return h->ep_shared ? h->cfg.n_shared : 0; }
 
 // Rank from which the route-tail skip drops an expert (0: off, or no rank of k reaches it).
 int skip_rank(const moe_config& c, uint32_t flags) {
@@ -157,7 +162,7 @@ moe_status do_decode(moe_handle* h, int32_t layer, const void* x, int32_t T, voi
     d.f = c.f;
     d.E = c.n_experts;
     d.k = c.top_k;
-    d.n_shared = c.n_shared;
+    d.n_shared = eff_shared(h);
     d.bits = c.bits;
     d.x = x;
     d.y = y;
@@ -182,6 +187,8 @@ moe_status do_decode(moe_handle* h, int32_t layer, const void* x, int32_t T, voi
     d.obuf = h->obuf;
     d.sync = h->sync;
     d.skip_rank = skip_rank(c, flags);
+    d.e_begin = h->ep_begin;
+    d.e_end = h->ep_end;
     return cuda_status(run(h, MOE_K_DECODE, s, [&] { return moe::launch_decode(d, s); }));
 }
 
@@ -211,6 +218,8 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     }
     ba.cnt = h->bucket_cnt;
     ba.skip_rank = skip_rank(c, flags);
+    ba.e_begin = h->ep_begin;
+    ba.e_end = h->ep_end;
     e = run(h, MOE_K_BUCKET, s, [&] { return moe::launch_bucket(ba, s); });
     h->launches += moe::bucket_kernel_count(ba) - 1;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -222,7 +231,7 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     ea.f = c.f;
     ea.E = c.n_experts;
     ea.k = c.top_k;
-    ea.n_shared = c.n_shared;
+    ea.n_shared = eff_shared(h);
     ea.bits = c.bits;
     ea.codes = L.codes;
     ea.scales = L.scales;
@@ -236,7 +245,7 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     ea.status = h->status;
     if (tc) {
         e = run(h, MOE_K_GATHER_F16, s, [&] {
-            return moe::launch_gather_f16(x, T, c.d, c.top_k, c.n_shared, h->pairs, h->offsets + c.n_experts, h->xg,
+            return moe::launch_gather_f16(x, T, c.d, c.top_k, ea.n_shared, h->pairs, h->offsets + c.n_experts, h->xg,
                                           h->status, s);
         });
         if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -271,7 +280,7 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     ca.T = T;
     ca.d = c.d;
     ca.k = c.top_k;
-    ca.n_shared = c.n_shared;
+    ca.n_shared = eff_shared(h);
     ca.obuf = h->obuf;
     ca.inv = h->inv;
     ca.w = h->w;
@@ -488,6 +497,15 @@ moe_status moe_rms_normalize(const void* x, int32_t T, int32_t d, void* out, voi
     if (T == 0) return MOE_OK;
     if (!x || !out || !aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
     return cuda_status(moe::launch_rms_normalize(x, T, d, out, 1e-6f, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_set_expert_range(moe_handle* h, int32_t begin, int32_t end, int32_t with_shared) {
+    if (!h || begin < 0 || end < begin || end > h->cfg.n_experts || (with_shared != 0 && with_shared != 1))
+        return MOE_ERR_INVALID_ARG;
+    h->ep_begin = begin;
+    h->ep_end = end;
+    h->ep_shared = with_shared;
+    return MOE_OK;
 }
 
 moe_status moe_destroy(moe_handle* h) {

@@ -22,7 +22,7 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
     bucket_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int32_t* __restrict__ offsets,
                   int32_t* __restrict__ pairs, int32_t* __restrict__ inv, int32_t* __restrict__ active,
                   Meta* __restrict__ meta, uint32_t* __restrict__ status, const float* __restrict__ w,
-                  float* __restrict__ wsorted, int R) {
+                  float* __restrict__ wsorted, int R, int e0, int e1) {
     extern __shared__ int32_t sm[];
     int32_t* cnt = sm;                          // [kBucketWarps][E]
     int32_t* total = sm + kBucketWarps * E;     // [E]
@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
             cnt[w * E + e] = run;
             run += c;
         }
-        total[e] = (R > 0 && best[e] >= R) ? 0 : run;
+        total[e] = ((R > 0 && best[e] >= R) || e < e0 || e >= e1) ? 0 : run;
     }
     __syncthreads();
 
@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
             const int e = ev[u];
             const int p = p0 + 32 * u + lane;
             const bool live = p < p_end;
-            const bool valid = live && e >= 0 && e < E && !(R > 0 && best[e] >= R);
+            const bool valid = live && e >= 0 && e < E && !(R > 0 && best[e] >= R) && e >= e0 && e < e1;
             const uint32_t same = __match_any_sync(0xffffffffu, valid ? e : -1);
             const int leader = __ffs(same) - 1;
             int base = 0;
@@ -182,7 +182,8 @@ __global__ void __launch_bounds__(kChunkWarps * 32)
 }
 
 __global__ void __launch_bounds__(1024) bucket_scan_kernel(int32_t* __restrict__ cnt, int32_t* __restrict__ best,
-                                                           int R, int nchunks, int E, int32_t* __restrict__ offsets,
+                                                           int R, int e0, int e1, int nchunks, int E,
+                                                           int32_t* __restrict__ offsets,
                                                            int32_t* __restrict__ active, Meta* __restrict__ meta) {
     extern __shared__ int32_t tot[];  // [E]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -203,6 +204,7 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(int32_t* __restrict__
             best[e] = b;
             if (b >= R) run = 0;
         }
+        if (e < e0 || e >= e1) run = 0;
         tot[e] = run;
     }
     __syncthreads();
@@ -239,7 +241,7 @@ __global__ void __launch_bounds__(kChunkWarps * 32)
     bucket_scatter_kernel(const int32_t* __restrict__ ids, int n_pairs, int E, int chunk,
                           const int32_t* __restrict__ cbase, const int32_t* __restrict__ offsets,
                           int32_t* __restrict__ pairs, int32_t* __restrict__ inv, const float* __restrict__ w,
-                          float* __restrict__ wsorted, const int32_t* __restrict__ best, int R) {
+                          float* __restrict__ wsorted, const int32_t* __restrict__ best, int R, int e0, int e1) {
     extern __shared__ int32_t wc[];  // [kChunkWarps][E] per-warp running position
     const int c = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t lt = (1u << lane) - 1u;
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(kChunkWarps * 32)
     // per-warp counts of this warp's sub-range
     for (int p = q0; p < q1; p += 32) {
         const int e = p + lane < q1 ? __ldg(&ids[p + lane]) : -1;
-        const bool valid = e >= 0 && e < E && !(R > 0 && best[e] >= R);
+        const bool valid = e >= e0 && e < e1 && e < E && !(R > 0 && best[e] >= R);
         const uint32_t same = __match_any_sync(0xffffffffu, valid ? e : -1);
         if (valid && (same & lt) == 0) wc[warp * E + e] += __popc(same);
     }
@@ -270,7 +272,7 @@ __global__ void __launch_bounds__(kChunkWarps * 32)
     for (int p = q0; p < q1; p += 32) {
         const bool live = p + lane < q1;
         const int e = live ? __ldg(&ids[p + lane]) : -1;
-        const bool valid = e >= 0 && e < E && !(R > 0 && best[e] >= R);
+        const bool valid = e >= e0 && e < e1 && e < E && !(R > 0 && best[e] >= R);
         const uint32_t same = __match_any_sync(0xffffffffu, valid ? e : -1);
         const int leader = __ffs(same) - 1;
         int base = 0;
@@ -293,14 +295,15 @@ __global__ void __launch_bounds__(kChunkWarps * 32)
 cudaError_t launch_bucket(const BucketArgs& a, cudaStream_t s) {
     const int n_pairs = a.T * a.k;
     const int R = a.skip_rank > 0 && a.skip_rank < a.k ? a.skip_rank : 0;
+    const int e0 = max(0, a.e_begin), e1 = min(a.E, a.e_end);
     if (bucket_kernel_count(a) == 3) {
         const int chunk = (n_pairs + kChunks - 1) / kChunks;
         int32_t* best = a.cnt + (size_t)kChunks * a.E;
         bucket_count_kernel<<<kChunks, kChunkWarps * 32, 2 * sizeof(int32_t) * a.E, s>>>(a.ids, n_pairs, a.k, a.E,
                                                                                          chunk, a.cnt, best, R,
                                                                                          a.status);
-        bucket_scan_kernel<<<1, 1024, sizeof(int32_t) * a.E, s>>>(a.cnt, best, R, kChunks, a.E, a.offsets, a.active,
-                                                                   a.meta);
+        bucket_scan_kernel<<<1, 1024, sizeof(int32_t) * a.E, s>>>(a.cnt, best, R, e0, e1, kChunks, a.E, a.offsets,
+                                                                   a.active, a.meta);
         const size_t smem = sizeof(int32_t) * (size_t)kChunkWarps * a.E;
         if (smem > 48 * 1024) {
             cudaError_t e = cudaFuncSetAttribute(bucket_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -308,7 +311,7 @@ cudaError_t launch_bucket(const BucketArgs& a, cudaStream_t s) {
             if (e != cudaSuccess) return e;
         }
         bucket_scatter_kernel<<<kChunks, kChunkWarps * 32, smem, s>>>(a.ids, n_pairs, a.E, chunk, a.cnt, a.offsets,
-                                                                      a.pairs, a.inv, a.w, a.wsorted, best, R);
+                                                                      a.pairs, a.inv, a.w, a.wsorted, best, R, e0, e1);
         return cudaGetLastError();
     }
     const size_t smem = sizeof(int32_t) * ((size_t)kBucketWarps * a.E + 3 * (size_t)a.E + 1);
@@ -317,7 +320,7 @@ cudaError_t launch_bucket(const BucketArgs& a, cudaStream_t s) {
         if (e != cudaSuccess) return e;
     }
     bucket_kernel<<<1, kBucketWarps * 32, smem, s>>>(a.ids, a.T, a.k, a.E, a.offsets, a.pairs, a.inv, a.active,
-                                                     a.meta, a.status, a.w, a.wsorted, R);
+                                                     a.meta, a.status, a.w, a.wsorted, R, e0, e1);
     return cudaGetLastError();
 }
 

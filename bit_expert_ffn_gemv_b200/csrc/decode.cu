@@ -114,6 +114,7 @@ struct DecodeArgs {
     float* obuf;
     int* sync;
     int skip_rank;  // route-tail skip: drop experts whose best rank is >= this (0: off)
+    int e_begin, e_end;  // experts outside [e_begin, e_end) are dropped (expert parallelism)
     int red_bytes;  // shared memory: [red_bytes] reductions | 2 x [buf_bytes] staging buffers
     int buf_bytes;  //   each buffer: [w_bytes] weights | activations
     int w_bytes;
@@ -450,6 +451,7 @@ MOE_DEV void bucket_cta(const DecodeArgs& a, int* sm, const int* ids_local) {
     int* ids = off + E + 1;
     int* wtot = ids + n;
     const int R = a.skip_rank;  // > 0: route-tail skip from this rank on
+    const int e0 = a.e_begin, e1 = a.e_end;  // kept expert range
     for (int e = threadIdx.x; e < E; e += kDecThreads) {
         cnt[e] = 0;
         off[e] = k;  // best (lowest) rank of expert e in the batch, until the scan
@@ -466,13 +468,16 @@ MOE_DEV void bucket_cta(const DecodeArgs& a, int* sm, const int* ids_local) {
         }
     }
     __syncthreads();
-    if (R > 0) {
-        // experts no token ranks before R drop out: no count, their pairs get inv = -1
+    if (R > 0 || e0 > 0 || e1 < E) {
+        // dropped experts (no rank below R in the batch, or outside the kept
+        // range): no count, their pairs get inv = -1
+        auto dropped = [&](int e) { return (R > 0 && off[e] >= R) || e < e0 || e >= e1; };
         for (int e = threadIdx.x; e < E; e += kDecThreads)
-            if (off[e] >= R) cnt[e] = 0;
+            if (dropped(e)) cnt[e] = 0;
+        __syncthreads();
         for (int i = threadIdx.x; i < n; i += kDecThreads) {
             const int e = ids[i];
-            if (e >= 0 && e < E && off[e] >= R) ids[i] = -1;
+            if (e >= 0 && e < E && dropped(e)) ids[i] = -1;
         }
         __syncthreads();
         // A dropped pair never reports to its token's combine counters (one per
@@ -486,7 +491,20 @@ MOE_DEV void bucket_cta(const DecodeArgs& a, int* sm, const int* ids_local) {
                 const int e = ids[t * k + r];
                 nd += (e < 0 || e >= E) ? 1 : 0;
             }
-            if (nd) atomicAdd(a.sync + SY_SLOTS + (1 + E) + j, nd);
+            if (nd == k && a.n_shared == 0) {
+                // nothing reaches this token's combine: its output is 0 here
+                const int n0 = (j - t * RT) * 16;
+                if (a.out_fp32) {
+                    float* y = static_cast<float*>(a.y) + (int64_t)t * a.d + n0;
+                    if (!a.accumulate)
+                        for (int q = 0; q < 16; ++q) y[q] = 0.0f;
+                } else if (!a.accumulate) {
+                    __nv_bfloat16* y = static_cast<__nv_bfloat16*>(a.y) + (int64_t)t * a.d + n0;
+                    for (int q = 0; q < 16; ++q) y[q] = __float2bfloat16_rn(0.0f);
+                }
+            } else if (nd) {
+                atomicAdd(a.sync + SY_SLOTS + (1 + E) + j, nd);
+            }
         }
     }
     // block-wide exclusive scan of cnt and of the active flags: warp w owns a
@@ -1227,6 +1245,8 @@ static cudaError_t decode_bits_nt(const DecodeLaunch& L, cudaStream_t st) {
     a.obuf = L.obuf;
     a.sync = L.sync;
     a.skip_rank = L.skip_rank;
+    a.e_begin = max(0, L.e_begin);
+    a.e_end = min(L.E, L.e_end);
     a.red_bytes = red_b;
     a.buf_bytes = buf_b;
     a.w_bytes = w_b;

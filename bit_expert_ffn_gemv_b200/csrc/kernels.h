@@ -35,6 +35,7 @@ struct BucketArgs {
     float* wsorted = nullptr;  // [T*k] w of pairs[pos] at pos (or null: not written)
     int32_t* cnt = nullptr;    // scratch [2 x 128 x E] for the multi-CTA variant (large T), or null
     int skip_rank = 0;         // route-tail skip: drop experts whose best rank in the batch is >= this (0: off)
+    int e_begin = 0, e_end = 1 << 30;  // experts outside [e_begin, e_end) are dropped (expert parallelism)
 };
 size_t bucket_scratch_words(int E);
 int bucket_kernel_count(const BucketArgs& a);  // kernels launch_bucket enqueues: 1, or 3 at large T
@@ -93,6 +94,7 @@ struct DecodeLaunch {
     float* obuf;
     int* sync;  // zeroed once; the kernel leaves it zeroed
     int skip_rank = 0;  // route-tail skip: drop experts whose best rank in the batch is >= this (0: off)
+    int e_begin = 0, e_end = 1 << 30;  // experts outside [e_begin, e_end) are dropped (expert parallelism)
 };
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t s);
 size_t decode_sync_words(int max_tokens, int E, int d);

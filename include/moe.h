@@ -243,6 +243,22 @@ float moe_router_error_depth(int32_t d, int32_t tensor_cores);
  */
 moe_status moe_check_status(moe_handle* h);
 
+/*
+ * Expert parallelism: from now on, moe_forward on this handle computes only
+ * the routed experts e with begin <= e < end, plus the shared expert when
+ * with_shared is 1; the terms of the other experts leave the sum, which makes
+ * y this handle's partial output.  Every rank routes all tokens over all E
+ * experts (the router is replicated), so the ranks agree on the selection and
+ * weights; summing the ranks' fp32 partial outputs over disjoint ranges that
+ * cover [0, E), with the shared expert on exactly one rank, gives the layer
+ * (an all-reduce; the expert weights outside the range are never read, so a
+ * rank needs only its own experts' bytes at their usual offsets).  Default:
+ * [0, E) with the shared expert.  Combines with MOE_ROUTE_TAIL_SKIP.
+ * Errors: INVALID_ARG (NULL handle, begin < 0, end < begin, end > E,
+ * with_shared not 0 or 1).
+ */
+moe_status moe_set_expert_range(moe_handle* h, int32_t begin, int32_t end, int32_t with_shared);
+
 /* Counters (moe_get_stats). */
 typedef struct {
     int64_t fixup_tokens;   /* tokens of the last routing re-ranked from fp64 logits */

@@ -57,6 +57,7 @@ def test_init_rejects_bad_config_before_touching_the_gpu(L, bad):
 
 def test_null_arguments(L):
     assert L.moe_layer_init(None, None) == 1
+    assert L.moe_set_expert_range(None, 0, 1, 1) == 1
     assert L.moe_destroy(None) == 0
     assert L.moe_route(None, 0, None, 1, None, None, None) == 1
     assert L.moe_forward(None, 0, None, 1, None, 0, None) == 1
