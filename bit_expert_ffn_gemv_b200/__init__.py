@@ -47,7 +47,7 @@ class MoeError(RuntimeError):
 class MoeConfig(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("f", ctypes.c_int32), ("n_experts", ctypes.c_int32),
                 ("top_k", ctypes.c_int32), ("n_shared", ctypes.c_int32), ("n_layers", ctypes.c_int32),
-                ("bits", ctypes.c_int32), ("max_tokens", ctypes.c_int32)]
+                ("bits", ctypes.c_int32), ("max_tokens", ctypes.c_int32), ("bits_down", ctypes.c_int32)]
 
 
 class MoeStats(ctypes.Structure):
@@ -240,8 +240,8 @@ def rms_normalize(x, out=None, stream=None):
 class MoeLayer:
     """A handle holding up to n_layers routed-MoE layers (weights borrowed from torch tensors)."""
 
-    def __init__(self, d, f, n_experts, top_k, n_shared=1, n_layers=1, bits=2, max_tokens=64):
-        self.cfg = MoeConfig(d, f, n_experts, top_k, n_shared, n_layers, bits, max_tokens)
+    def __init__(self, d, f, n_experts, top_k, n_shared=1, n_layers=1, bits=2, max_tokens=64, bits_down=0):
+        self.cfg = MoeConfig(d, f, n_experts, top_k, n_shared, n_layers, bits, max_tokens, bits_down)
         self.handle = moe_layer_init(self.cfg)
         self._keep = {}
 

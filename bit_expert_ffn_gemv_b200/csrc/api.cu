@@ -116,9 +116,15 @@ moe_status check_layer(moe_handle* h, int32_t layer) {
     return MOE_OK;
 }
 
+// Code width of the down matrices, and whether it differs from gate/up's.
+int bits_down(const moe_config& c) { return c.bits_down ? c.bits_down : c.bits; }
+bool mixed_widths(const moe_config& c) { return bits_down(c) != c.bits; }
+
 // moe_forward takes the tensor-core path (bf16 tcgen05 router, grouped
-// dequant GEMMs) above kFusedMaxTokens tokens, or when forced.
-bool use_tensor_cores(int32_t T, uint32_t flags) {
+// dequant GEMMs) above kFusedMaxTokens tokens, or when forced.  Layers with
+// mixed code widths run on the grouped-GEMV path at every T.
+bool use_tensor_cores(const moe_config& c, int32_t T, uint32_t flags) {
+    if (mixed_widths(c)) return false;
     if (flags & (MOE_FORCE_GEMV | MOE_FORCE_UNFUSED)) return false;
     return T > moe::kFusedMaxTokens || (flags & MOE_FORCE_GEMM);
 }
@@ -195,9 +201,10 @@ moe_status do_decode(moe_handle* h, int32_t layer, const void* x, int32_t T, voi
 moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, void* y, uint32_t flags,
                       cudaStream_t s) {
     const moe_config& c = h->cfg;
-    if (T <= moe::kDecodeMaxTokens && !use_tensor_cores(T, flags) && !(flags & MOE_FORCE_UNFUSED))
+    if (T <= moe::kDecodeMaxTokens && !use_tensor_cores(c, T, flags) && !(flags & MOE_FORCE_UNFUSED) &&
+        !mixed_widths(c))
         return do_decode(h, layer, x, T, y, flags, s);
-    const bool tc = use_tensor_cores(T, flags);
+    const bool tc = use_tensor_cores(c, T, flags);
     cudaError_t e;
     moe_status st = do_route(h, layer, x, T, h->ids, h->w, tc, s);
     if (st != MOE_OK) return st;
@@ -233,6 +240,8 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     ea.k = c.top_k;
     ea.n_shared = eff_shared(h);
     ea.bits = c.bits;
+    ea.bits_down = bits_down(c);
+    ea.code_stride = (int64_t)c.f * c.d * (2 * c.bits + bits_down(c)) / 8;
     ea.codes = L.codes;
     ea.scales = L.scales;
     ea.x = x;
@@ -298,6 +307,7 @@ moe_status check_forward_args(moe_handle* h, int32_t layer, const void* x, int32
     if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
     if (flags & ~kAllFlags) return MOE_ERR_INVALID_ARG;
     if ((flags & MOE_FORCE_GEMV) && (flags & MOE_FORCE_GEMM)) return MOE_ERR_INVALID_ARG;
+    if ((flags & MOE_FORCE_GEMM) && mixed_widths(h->cfg)) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!x || !y || !aligned16(x) || !aligned16(y))) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
@@ -313,7 +323,8 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     const moe_config c = *cfg;
     if (c.d <= 0 || c.f <= 0 || c.d % 128 || c.f % 128 || c.n_experts < 1 || c.n_experts > 1024 || c.top_k < 1 ||
         c.top_k > c.n_experts || c.top_k > 32 || (c.n_shared != 0 && c.n_shared != 1) || c.n_layers < 1 ||
-        c.n_layers > 4096 || c.bits < 2 || c.bits > 4 || c.max_tokens < 1 || c.max_tokens > (1 << 20))
+        c.n_layers > 4096 || c.bits < 2 || c.bits > 4 || c.max_tokens < 1 || c.max_tokens > (1 << 20) ||
+        (c.bits_down != 0 && (c.bits_down < 2 || c.bits_down > 4)))
         return MOE_ERR_INVALID_ARG;
     moe_handle* h = new (std::nothrow) moe_handle();
     if (!h) return MOE_ERR_OOM;
@@ -411,8 +422,10 @@ moe_status moe_load_layer(moe_handle* h, int32_t layer, const moe_layer_weights*
     L.router_w = w->router_w;
     L.bias = w->router_bias;
     const int ne = h->cfg.n_experts + h->cfg.n_shared;
-    if (moe::make_weight_maps(&L.w_gu, L.codes, L.scales, ne, h->cfg.f, h->cfg.d, h->cfg.bits) != cudaSuccess ||
-        moe::make_weight_maps(&L.w_dn, L.codes, L.scales, ne, h->cfg.d, h->cfg.f, h->cfg.bits) != cudaSuccess)
+    // the tensor-core path's maps assume one code width for all three matrices
+    if (!mixed_widths(h->cfg) &&
+        (moe::make_weight_maps(&L.w_gu, L.codes, L.scales, ne, h->cfg.f, h->cfg.d, h->cfg.bits) != cudaSuccess ||
+         moe::make_weight_maps(&L.w_dn, L.codes, L.scales, ne, h->cfg.d, h->cfg.f, h->cfg.bits) != cudaSuccess))
         return MOE_ERR_CUDA;
     cudaError_t e = moe::launch_router_norms(L.router_w, h->cfg.n_experts, h->cfg.d, L.wnorm, 0);
     if (e == cudaSuccess) e = cudaStreamSynchronize(0);
@@ -525,9 +538,11 @@ moe_status moe_debug_dequant(moe_handle* h, int32_t layer, int32_t expert, int32
         return MOE_ERR_INVALID_ARG;
     const moe_layer_state& L = h->layers[layer];
     const int64_t mc = (int64_t)c.f * c.d * c.bits / 8, ms = (int64_t)c.f * c.d / 32;
+    const int64_t stride = (int64_t)c.f * c.d * (2 * c.bits + bits_down(c)) / 8;
     const int N = mat < 2 ? c.f : c.d, K = mat < 2 ? c.d : c.f;
-    return cuda_status(moe::launch_dequant(L.codes + (expert * 3 + mat) * mc, L.scales + (expert * 3 + mat) * ms, N,
-                                           K, c.bits, out, static_cast<cudaStream_t>(stream)));
+    return cuda_status(moe::launch_dequant(L.codes + expert * stride + mat * mc, L.scales + (expert * 3 + mat) * ms,
+                                           N, K, mat < 2 ? c.bits : bits_down(c), out,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_debug_last_routing(moe_handle* h, int32_t T, int32_t* ids, float* w, void* stream) {

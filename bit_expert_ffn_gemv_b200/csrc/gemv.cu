@@ -75,7 +75,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_gateup_kernel(const Expe
     const int g = lane >> 2, c = lane & 3;
     const int KT = a.d / 128;
     const int64_t mat_codes = (int64_t)a.f * a.d * BITS / 8, mat_scales = (int64_t)a.f * a.d / 32;
-    const uint8_t* cg = a.codes + (int64_t)s.expert * 3 * mat_codes;
+    const int64_t stride = a.code_stride ? a.code_stride : 3 * mat_codes;
+    const uint8_t* cg = a.codes + (int64_t)s.expert * stride;
     const uint8_t* cu = cg + mat_codes;
     const __half* sg = reinterpret_cast<const __half*>(a.scales) + (int64_t)s.expert * 3 * mat_scales;
     const __half* su = sg + mat_scales;
@@ -166,8 +167,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_down_kernel(const Expert
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
     const int KT = a.f / 128;
+    // BITS is the down matrices' width; gate and up (at a.bits) come first in each expert's block
     const int64_t mat_codes = (int64_t)a.f * a.d * BITS / 8, mat_scales = (int64_t)a.f * a.d / 32;
-    const uint8_t* cd = a.codes + (int64_t)s.expert * 3 * mat_codes + 2 * mat_codes;
+    const int64_t gu_codes = (int64_t)a.f * a.d * a.bits / 8;
+    const int64_t stride = a.code_stride ? a.code_stride : 2 * gu_codes + mat_codes;
+    const uint8_t* cd = a.codes + (int64_t)s.expert * stride + 2 * gu_codes;
     const __half* sd = reinterpret_cast<const __half*>(a.scales) + (int64_t)s.expert * 3 * mat_scales + 2 * mat_scales;
     const uint16_t* h = static_cast<const uint16_t*>(a.h);
 
@@ -277,7 +281,7 @@ cudaError_t launch_gemv_gateup(const ExpertArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_gemv_down(const ExpertArgs& a, cudaStream_t s) {
-    switch (a.bits) {
+    switch (a.bits_down ? a.bits_down : a.bits) {
         case 2: return down_bits<2>(a, s);
         case 3: return down_bits<3>(a, s);
         case 4: return down_bits<4>(a, s);

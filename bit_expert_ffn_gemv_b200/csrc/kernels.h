@@ -43,6 +43,8 @@ int bucket_kernel_count(const BucketArgs& a);  // kernels launch_bucket enqueues
 // Grouped GEMV/GEMM problem description shared by the expert kernels.
 struct ExpertArgs {
     int T, d, f, E, k, n_shared, bits;
+    int bits_down = 0;        // code width of the down matrices (0: bits)
+    int64_t code_stride = 0;  // code bytes per expert: f*d*(2*bits + bits_down)/8 (0: 3*f*d*bits/8)
     const uint8_t* codes;   // layer codes, expert-major (gate, up, down)
     const uint16_t* scales; // layer scales, same order
     const void* x;          // bf16 [T x d]

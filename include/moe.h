@@ -36,6 +36,7 @@
  * Packed weight layout of one layer (memory owned by the caller, borrowed):
  *   codes : expert-major; expert e (the shared expert is e = E) holds
  *           gate [f x d], up [f x d], down [d x f], each f*d*b/8 bytes
+ *           (down: f*d*bits_down/8 when bits_down is set)
  *   scales: same order, each matrix f*d/32 fp16 values
  * Each matrix W[N x K] is tiled into 16 x 128 super-tiles stored at
  * (n/16)*(K/128) + k/128, 256*b code bytes and 64 fp16 scales each.  Inside
@@ -84,6 +85,12 @@ typedef struct {
     int32_t n_layers;   /* layers this handle can hold, >= 1 */
     int32_t bits;       /* code width b: 2, 3 or 4 */
     int32_t max_tokens; /* largest T a call may pass, >= 1 */
+    int32_t bits_down;  /* code width of the down matrices: 0 (= bits) or 2..4.
+                           A width other than `bits` gives per-tensor mixed
+                           precision (GSQ-RCO's per-tensor bit allocation, as the
+                           tech.okbari.net guide describes it in its GSQ-RCO
+                           section); such layers run on the grouped-GEMV kernels
+                           at every T (MOE_FORCE_GEMM is then an INVALID_ARG). */
 } moe_config;
 
 typedef struct {

@@ -25,7 +25,7 @@ _lib = None
 
 class Shape(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int32), ("f", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
-                ("n_shared", ctypes.c_int32), ("bits", ctypes.c_int32)]
+                ("n_shared", ctypes.c_int32), ("bits", ctypes.c_int32), ("bits_down", ctypes.c_int32)]
 
 
 def build(force: bool = False) -> str:
@@ -71,7 +71,7 @@ def _p(a):
 
 
 def _shape(shape) -> Shape:
-    return Shape(shape.d, shape.f, shape.E, shape.k, shape.n_shared, shape.bits)
+    return Shape(shape.d, shape.f, shape.E, shape.k, shape.n_shared, shape.bits, getattr(shape, "bits_down", 0))
 
 
 def threads(n: int = 0) -> int:

@@ -53,6 +53,7 @@
 
 typedef struct {
     int32_t d, f, E, k, n_shared, bits;
+    int32_t bits_down; /* code width of the down matrices; 0: bits (gate, up and down alike) */
 } oracle_shape;
 
 /* ---- scalar decoders ---- */
@@ -125,7 +126,8 @@ int oracle_dequant(int N, int K, int bits, const uint8_t* codes, const uint16_t*
 
 static int shape_ok(const oracle_shape* s) {
     return s && s->d > 0 && s->f > 0 && s->d % 128 == 0 && s->f % 128 == 0 && s->E > 0 && s->k >= 1 &&
-           s->k <= s->E && (s->n_shared == 0 || s->n_shared == 1) && s->bits >= 2 && s->bits <= 4;
+           s->k <= s->E && (s->n_shared == 0 || s->n_shared == 1) && s->bits >= 2 && s->bits <= 4 &&
+           (s->bits_down == 0 || (s->bits_down >= 2 && s->bits_down <= 4));
 }
 
 /* ---- routing of one token ---- */
@@ -190,7 +192,8 @@ int oracle_route(const oracle_shape* s, const uint16_t* x, int T, const uint16_t
 /* o = What_d (silu(What_g x) * What_u x) for one expert; row scratch of max(d, f) */
 static void expert_eval(const oracle_shape* s, const uint8_t* codes, const uint16_t* scales, const double* x,
                         double* h, double* row, double* o) {
-    int d = s->d, f = s->f, b = s->bits;
+    /* per-tensor widths: gate and up at b, down at bd (the mixed precision of GSQ-RCO) */
+    int d = s->d, f = s->f, b = s->bits, bd = s->bits_down ? s->bits_down : s->bits;
     int64_t mc = (int64_t)f * d * b / 8, ms = (int64_t)f * d / 32;
     const uint8_t *cg = codes, *cu = codes + mc, *cd = codes + 2 * mc;
     const uint16_t *sg = scales, *su = scales + ms, *sd = scales + 2 * ms;
@@ -204,7 +207,7 @@ static void expert_eval(const oracle_shape* s, const uint8_t* codes, const uint1
     }
     for (int n = 0; n < d; ++n) {
         double acc = 0.0;
-        dequant_row(cd, sd, d, f, b, n, row);
+        dequant_row(cd, sd, d, f, bd, n, row);
         for (int j = 0; j < f; ++j) acc += row[j] * h[j];
         o[n] = acc;
     }

@@ -56,6 +56,9 @@ def _stream():
 
 def experts_into(codes, scales, shape: MoeShape, master: int, layer: int, expert0: int, n: int):
     """Generate experts expert0..expert0+n-1 of a layer into CUDA tensors (uint8 / int16)."""
+    if shape.bd != shape.bits:
+        raise ValueError("the device generator draws one code width per layer; generate mixed-width layers "
+                         "on the host (synth.layer_host)")
     cb, sb = expert_bytes(shape)
     assert codes.numel() >= n * cb and scales.numel() * 2 >= n * sb
     rc = lib().synth_gpu_experts(master, layer, shape.d, shape.f, expert0, n, shape.bits, codes.data_ptr(),

@@ -13,7 +13,7 @@ import numpy as np
 from . import (MASTER_BASE, MAT_TENSOR, T_PERM, T_WR, T_X, codes_bytes, expert_matrix, key, normal_bf16,
                scales_bytes, zipf_bias)
 
-__all__ = ["MoeShape", "Workload", "WORKLOADS", "mat_dims", "expert_bytes", "router_host", "expert_host",
+__all__ = ["MoeShape", "Workload", "WORKLOADS", "mat_dims", "mat_bits", "expert_bytes", "router_host", "expert_host",
            "layer_host", "x_host"]
 
 
@@ -25,10 +25,15 @@ class MoeShape:
     k: int
     n_shared: int = 1
     bits: int = 2
+    bits_down: int = 0  # code width of the down matrices; 0: bits (per-tensor mixed precision otherwise)
 
     @property
     def n_experts_total(self) -> int:
         return self.E + self.n_shared
+
+    @property
+    def bd(self) -> int:
+        return self.bits_down or self.bits
 
 
 @dataclass(frozen=True)
@@ -64,10 +69,15 @@ def mat_dims(shape: MoeShape, mat: int):
     return (shape.f, shape.d) if mat < 2 else (shape.d, shape.f)
 
 
+def mat_bits(shape: MoeShape, mat: int) -> int:
+    """Code width of matrix mat: gate and up at `bits`, down at `bits_down` (when set)."""
+    return shape.bd if mat == 2 else shape.bits
+
+
 def expert_bytes(shape: MoeShape):
     """(codes bytes, scale bytes) of one expert's three matrices."""
     n = shape.f * shape.d
-    return 3 * n * shape.bits // 8, 3 * (n // 32) * 2
+    return n * (2 * shape.bits + shape.bd) // 8, 3 * (n // 32) * 2
 
 
 def router_host(shape: MoeShape, master: int, layer: int, zipf: bool):
@@ -85,12 +95,12 @@ def expert_host(shape: MoeShape, master: int, layer: int, expert: int):
     co = so = 0
     for mat in range(3):
         N, K = mat_dims(shape, mat)
-        c, s = expert_matrix(key(master, layer, MAT_TENSOR[mat], expert), N, K, shape.bits)
+        c, s = expert_matrix(key(master, layer, MAT_TENSOR[mat], expert), N, K, mat_bits(shape, mat))
         codes[co:co + c.size] = c
         scales[so:so + s.size] = s
         co += c.size
         so += s.size
-    assert co == codes_bytes(shape.f, shape.d, shape.bits) * 3 and so * 2 == 3 * scales_bytes(shape.f, shape.d)
+    assert co == cb and so * 2 == 3 * scales_bytes(shape.f, shape.d)
     return codes, scales
 
 

@@ -48,7 +48,8 @@ def _cfg(**kw):
 
 @pytest.mark.parametrize("bad", [dict(d=200), dict(f=100), dict(n_experts=0), dict(n_experts=2000),
                                  dict(top_k=0), dict(top_k=17), dict(n_shared=2), dict(bits=1), dict(bits=5),
-                                 dict(max_tokens=0), dict(n_layers=0), dict(top_k=33, n_experts=64)])
+                                 dict(max_tokens=0), dict(n_layers=0), dict(top_k=33, n_experts=64),
+                                 dict(bits_down=1), dict(bits_down=5)])
 def test_init_rejects_bad_config_before_touching_the_gpu(L, bad):
     h = ctypes.c_void_p(1234)
     s = L.moe_layer_init(ctypes.byref(_cfg(**bad)), ctypes.byref(h))

@@ -114,7 +114,7 @@ def _layer_from_q(shape, qs, ss, wr, bias):
     for e in range(shape.E + shape.n_shared):
         cs, ssc = [], []
         for m in range(3):
-            c, sc = synth.pack(qs[e][m], ss[e][m], shape.bits)
+            c, sc = synth.pack(qs[e][m], ss[e][m], synth.mat_bits(shape, m))
             cs.append(c)
             ssc.append(sc)
         codes.append(np.concatenate(cs))
@@ -130,7 +130,7 @@ def _random_layer(shape, seed, wr_scale=0.02, bias_scale=0.0):
         for m in range(3):
             N, K = synth.mat_dims(shape, m)
             w = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
-            _, _, q, s = synth.quantize(w, shape.bits)
+            _, _, q, s = synth.quantize(w, synth.mat_bits(shape, m))
             qe.append(q)
             se.append(s)
             de.append(q.astype(np.float64) * np.repeat(_f16(s), 32, axis=1))
@@ -383,3 +383,31 @@ def test_tail_skip_equals_zeroed_experts():
     for t in range(x.shape[0]):
         d1 = oracle.tail_skip(ids[t:t + 1], shape.E, 6)
         assert sorted(np.flatnonzero(d1).tolist()) == sorted(ids[t, 6:].tolist())
+
+
+# ------------------------------------------------------------------ per-tensor mixed precision
+@pytest.mark.parametrize("bits,bits_down", [(2, 3), (2, 4), (3, 2), (4, 2)])
+def test_mixed_widths_match_dense_formulation(bits, bits_down):
+    """Gate/up at one code width and down at another: the oracle equals the dense formulation built from
+    numpy-quantised matrices of those widths (k-subset enumeration for the selection)."""
+    shape = MoeShape(d=128, f=128, E=6, k=2, n_shared=1, bits=bits, bits_down=bits_down)
+    L = _random_layer(shape, seed=400 + 10 * bits + bits_down, bias_scale=0.3)
+    x = _x(shape, 5, 41)
+    y, ids, w = oracle.layer(shape, x, L["router_w"], L["bias"], L["codes"], L["scales"])
+    yd, idsd = _dense(shape, L, x)[:2]
+    assert np.array_equal(ids, idsd)
+    assert np.allclose(y, yd, rtol=1e-11, atol=1e-14)
+    # each expert's block really holds three matrices of those widths
+    assert L["codes"][0].size == 128 * 128 * (2 * bits + bits_down) // 8
+
+
+def test_mixed_widths_differ_from_uniform_reading():
+    """Reading a mixed layer as uniform width gives a different output: the down width is used."""
+    mixed = MoeShape(d=128, f=128, E=6, k=2, n_shared=1, bits=2, bits_down=4)
+    L = _random_layer(mixed, seed=77)
+    x = _x(mixed, 3, 5)
+    y, _, _ = oracle.layer(mixed, x, L["router_w"], L["bias"], L["codes"], L["scales"])
+    same = MoeShape(d=128, f=128, E=6, k=2, n_shared=1, bits=2, bits_down=2)
+    short = [c[:128 * 128 * 6 // 8] for c in L["codes"]]
+    y2, _, _ = oracle.layer(same, x, L["router_w"], L["bias"], short, L["scales"])
+    assert not np.allclose(y, y2)
