@@ -269,7 +269,9 @@ moe_status moe_set_expert_range(moe_handle* h, int32_t begin, int32_t end, int32
 /* Counters (moe_get_stats). */
 typedef struct {
     int64_t fixup_tokens;   /* tokens of the last routing re-ranked from fp64 logits */
-    int64_t active_experts; /* distinct routed experts of the last moe_forward */
+    int64_t active_experts; /* routed experts the last moe_forward computed (distinct
+                               selected experts, less those the route-tail skip or
+                               the expert range dropped) */
     int64_t max_group;      /* largest expert group of the last moe_forward */
     int64_t launches;       /* kernels this handle has launched since moe_layer_init */
 } moe_stats;
