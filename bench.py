@@ -186,58 +186,84 @@ def measured_peaks():
 
 
 # ---------------------------------------------------------------- oracle CPU baseline
-def oracle_sample(sh, wl, T, seconds, steps=None, warmup=0, layer_of=lambda i: 0):
-    """Time the fp64 oracle on batches of T tokens of the workload; returns (tok/s, tokens, secs, threads)."""
-    import numpy as np
+def oracle_sample(sh, wl, T, seconds, steps=None, warmup=0, layer_of=lambda i: 0, tokens_after_warmup=None):
+    """Time the fp64 oracle on batches of T tokens of the workload; returns (tok/s, tokens, secs, threads).
 
+    Runs `warmup` untimed batches, then either `steps` timed batches or timed batches until `seconds` of
+    oracle time.  tokens_after_warmup(sec_per_token) may shrink the timed batches (>= 1 token) so that a
+    fixed step count stays within a time budget.
+    """
     import oracle
     import synth
     threads = oracle.threads()
-    routers = {}
+    routers, experts = {}, {}
     done_tok, spent, i = 0, 0.0, 0
+    warm_tok, warm_s = 0, 0.0
+    Tb = T
     while True:
         if steps is not None and i >= steps + warmup:
             break
         if steps is None and spent >= seconds:
             break
+        if i == warmup and tokens_after_warmup is not None and warm_tok:
+            Tb = max(1, min(T, tokens_after_warmup(warm_s / warm_tok)))
         layer = layer_of(i)
         if layer not in routers:
             routers[layer] = synth.router_host(sh, wl.master, layer, wl.zipf)
         wr, bias = routers[layer]
-        x = synth.x_host(sh, wl.master, 50000 + i, T)
+        x = synth.x_host(sh, wl.master, 50000 + i, Tb)
         ids, _ = oracle.route(sh, x, wr, bias)
         need = sorted(set(ids.ravel().tolist()) | ({sh.E} if sh.n_shared else set()))
         codes = [None] * sh.n_experts_total
         scales = [None] * sh.n_experts_total
         for e in need:
-            codes[e], scales[e] = synth.expert_host(sh, wl.master, layer, e)
+            key = (layer, e)
+            if key not in experts:
+                pair = synth.expert_host(sh, wl.master, layer, e)
+                if len(experts) >= 1024:  # bounded host cache (~1.5 GB at the full shape)
+                    codes[e], scales[e] = pair
+                    continue
+                experts[key] = pair
+            codes[e], scales[e] = experts[key]
         t0 = time.perf_counter()
         oracle.layer(sh, x, wr, bias, codes, scales)
         dt = time.perf_counter() - t0
         if i >= warmup:
             spent += dt
-            done_tok += T
+            done_tok += Tb
+        else:
+            warm_s += dt
+            warm_tok += Tb
         i += 1
     return done_tok / spent, done_tok, spent, threads
 
 
 def reference_arm(args):
-    """The oracle as the reference arm: rank 0 alone, on the host cores."""
+    """The oracle as the reference arm: rank 0 alone, on the host cores.
+
+    Exactly `--warmup` untimed and `--steps` timed batches.  Each timed batch is a bounded sample of the
+    workload: up to 16 of its tokens, fewer when the step count would otherwise take more than about
+    150 s of oracle time (the warm-up batches give the time per token).
+    """
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     wl, sh, T, layers = workload(args)
-    Tref = min(T, 16)  # oracle batches: each is a bounded sample of the workload
-    steps = max(1, args.steps if args.steps <= 20 else 20)
-    tps, ntok, secs, threads = oracle_sample(sh, wl, Tref, None, steps=steps, warmup=min(args.warmup, 1),
-                                             layer_of=lambda i: i % layers)
-    line = {"metric": METRIC, "value": tps, "unit": "tok/s", "n_gpus": 0, "steps": steps, "warmup": min(args.warmup, 1),
+    Tref = min(T, 16)
+    steps, warmup = max(1, args.steps), max(0, args.warmup)
+    budget_s = 150.0
+    tps, ntok, secs, threads = oracle_sample(
+        sh, wl, Tref, None, steps=steps, warmup=warmup, layer_of=lambda i: i % layers,
+        tokens_after_warmup=lambda s_tok: int(budget_s / (steps * s_tok)))
+    per_step = ntok // steps
+    line = {"metric": METRIC, "value": tps, "unit": "tok/s", "n_gpus": 0, "steps": steps, "warmup": warmup,
             "ms_per_step": 1000.0 * secs / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": args.workload, "tokens_per_step": Tref, "bits": sh.bits, "d": sh.d, "f": sh.f,
-                       "experts": sh.E, "top_k": sh.k, "shared": sh.n_shared},
+            "config": {"workload": args.workload, "tokens_per_step": T, "bits": sh.bits, "d": sh.d, "f": sh.f,
+                       "experts": sh.E, "top_k": sh.k, "shared": sh.n_shared, "layers": layers},
             "cpu_baseline": {"value": tps, "unit": "tok/s", "cores": threads, "kind": "oracle",
-                             "sample": f"{ntok} tokens in {steps} batches of {Tref} (fp64 C oracle)"},
+                             "sample": f"{ntok} tokens in {steps} timed batches of {per_step} "
+                                       f"(workload batches hold {T}; fp64 C oracle)"},
             "e2e": {"value": tps, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
