@@ -43,6 +43,8 @@ def parse():
     p.add_argument("--rotate", type=int, default=8, help="distinct layers cycled through (decode/sweep)")
     p.add_argument("--flags", default="", help="extra forward flags, '+'-separated: gemv, gemm, tailskip "
                    "(the route-tail skip approximation)")
+    p.add_argument("--expert-shard", default="", help="r/w: time one rank's partial layer of a w-way expert "
+                   "split (the routed experts of range r, plus the shared one on rank 0)")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU-baseline sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
@@ -308,6 +310,10 @@ def ours(args):
         w = sgpu.layer_device(sh, rank_master(wl.master, rank), l, wl.zipf)
         h.load_layer(l, *w)
         weights.append(w)
+    if args.expert_shard:
+        from bit_expert_ffn_gemv_b200.expert_parallel import expert_shard
+        r, w = (int(v) for v in args.expert_shard.split("/"))
+        h.set_expert_range(*expert_shard(sh.E, r, w))
     n_x = 16
     xs = [sgpu.x_device(sh, rank_master(wl.master, rank), 10000 + i, T) for i in range(n_x)]
     chain = args.workload == "chain48"
@@ -454,7 +460,8 @@ def ours(args):
                            "l2": ("inputs larger than L2: 48 layers x 756 MB per step" if chain else
                                   f"inputs larger than L2: {layers} distinct layers cycled, {n_x} fresh inputs"),
                            "parallelism": f"replicas x{world}", "timing": "CUDA graph replay" if graph is not None else "eager",
-                           **({"flags": args.flags} if args.flags else {})},
+                           **({"flags": args.flags} if args.flags else {}),
+                           **({"expert_shard": args.expert_shard} if args.expert_shard else {})},
                 "roofline": roof, "layer_hbm_gbs": layer_gbs,
                 "kernels_ms_per_step": {k: v[0] / nprof for k, v in prof.items()},
                 "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary()}
