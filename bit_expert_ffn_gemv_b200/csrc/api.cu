@@ -300,14 +300,21 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     return cuda_status(run(h, MOE_K_COMBINE, s, [&] { return moe::launch_combine(ca, s); }));
 }
 
-moe_status check_forward_args(moe_handle* h, int32_t layer, const void* x, int32_t T, const void* y,
-                              uint32_t flags) {
+// Layer, token count and flags of a forward call (both entry points).
+moe_status check_forward_call(moe_handle* h, int32_t layer, int32_t T, uint32_t flags) {
     moe_status st = check_layer(h, layer);
     if (st != MOE_OK) return st;
     if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
     if (flags & ~kAllFlags) return MOE_ERR_INVALID_ARG;
     if ((flags & MOE_FORCE_GEMV) && (flags & MOE_FORCE_GEMM)) return MOE_ERR_INVALID_ARG;
     if ((flags & MOE_FORCE_GEMM) && mixed_widths(h->cfg)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+moe_status check_forward_args(moe_handle* h, int32_t layer, const void* x, int32_t T, const void* y,
+                              uint32_t flags) {
+    moe_status st = check_forward_call(h, layer, T, flags);
+    if (st != MOE_OK) return st;
     if (T > 0 && (!x || !y || !aligned16(x) || !aligned16(y))) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
@@ -485,13 +492,10 @@ moe_status moe_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, v
 
 moe_status moe_forward_host(moe_handle* h, int32_t layer, const void* x_host, int32_t T, void* y_host,
                             uint32_t flags, void* stream) {
-    moe_status st = check_layer(h, layer);
+    moe_status st = check_forward_call(h, layer, T, flags);
     if (st != MOE_OK) return st;
-    if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x_host || !y_host) return MOE_ERR_INVALID_ARG;
-    if (flags & ~kAllFlags) return MOE_ERR_INVALID_ARG;
-    if ((flags & MOE_FORCE_GEMV) && (flags & MOE_FORCE_GEMM)) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t xb = sizeof(uint16_t) * (size_t)T * h->cfg.d;
     const size_t yb = ((flags & MOE_OUT_FP32) ? sizeof(float) : sizeof(uint16_t)) * (size_t)T * h->cfg.d;
