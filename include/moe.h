@@ -158,7 +158,11 @@ moe_status moe_route(moe_handle* h, int32_t layer, const void* x, int32_t T, int
  * must not overlap, except y == x (bf16) with MOE_ACCUMULATE, which updates a
  * residual stream in place (x += layer(x)): every read of x is enqueued
  * before the final write of y.  T = 0 is a no-op.
- * Errors: INVALID_ARG, NOT_LOADED, CUDA.
+ * Errors: INVALID_ARG (layer out of range, T < 0 or > max_tokens, NULL or
+ * misaligned x / y, an unknown flag, MOE_FORCE_GEMV with MOE_FORCE_GEMM,
+ * MOE_FORCE_GEMM on a mixed-width layer), NOT_LOADED, CUDA; nothing is
+ * enqueued on an argument error.  Device-side errors (MOE_ERR_TIMEOUT,
+ * MOE_ERR_BOUNDS, MOE_ERR_RANGE) surface through moe_check_status.
  */
 moe_status moe_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, void* y, uint32_t flags,
                        void* stream);
@@ -215,7 +219,10 @@ moe_status moe_destroy(moe_handle* h);
 /*
  * Debug: the fp32 values q * s of matrix `mat` (0 gate [f x d], 1 up [f x d],
  * 2 down [d x f]) of expert `expert` (E = shared) of a loaded layer, written
- * row-major to out (device).  Exact: |q| <= 8 and s is fp16.
+ * row-major to out (device), each matrix decoded at its own code width.
+ * Exact: |q| <= 8 and s is fp16.
+ * Errors: INVALID_ARG (expert or mat out of range, NULL or misaligned out),
+ * NOT_LOADED, CUDA.
  */
 moe_status moe_debug_dequant(moe_handle* h, int32_t layer, int32_t expert, int32_t mat, float* out,
                              void* stream);
