@@ -301,6 +301,8 @@ def ours(args):
     names = {"gemv": moe.MOE_FORCE_GEMV, "gemm": moe.MOE_FORCE_GEMM, "tailskip": moe.MOE_ROUTE_TAIL_SKIP}
     flags = 0
     for f in filter(None, args.flags.split("+")):
+        if f not in names:
+            raise SystemExit(f"--flags: unknown flag {f!r} (known: {', '.join(names)})")
         flags |= names[f]
 
     # ---- setup: layers generated on the device, one handle holding all of them

@@ -83,3 +83,17 @@ def test_single_process_reduce_is_identity():
     from bit_expert_ffn_gemv_b200.expert_parallel import reduce_partial
     y = torch.arange(6.0).reshape(2, 3)
     assert torch.equal(reduce_partial(y.clone()), y)
+
+
+def test_forward_refuses_accumulate():
+    """Every rank would add the residual once: the expert-parallel forward refuses MOE_ACCUMULATE before
+    touching the handle."""
+    import bit_expert_ffn_gemv_b200 as moe
+    from bit_expert_ffn_gemv_b200.expert_parallel import forward
+
+    class NoHandle:
+        def forward(self, *a, **k):
+            raise AssertionError("must not be reached")
+
+    with pytest.raises(ValueError):
+        forward(NoHandle(), 0, None, flags=moe.MOE_ACCUMULATE)
