@@ -411,3 +411,31 @@ def test_mixed_widths_differ_from_uniform_reading():
     short = [c[:128 * 128 * 6 // 8] for c in L["codes"]]
     y2, _, _ = oracle.layer(same, x, L["router_w"], L["bias"], short, L["scales"])
     assert not np.allclose(y, y2)
+
+
+def test_tail_skip_depends_on_the_batch():
+    """An expert that one token ranks 7th or lower is dropped when that token is alone, and kept when a
+    token that ranks it among its first six shares the batch; the first token's output then gains that
+    expert's term."""
+    shape = MoeShape(d=128, f=128, E=24, k=8, n_shared=1, bits=2)
+    L = _random_layer(shape, seed=515, bias_scale=0.3)
+    xs = _x(shape, 40, 77)
+    ids, _ = oracle.route(shape, xs, L["router_w"], L["bias"])
+    found = None
+    for a in range(40):
+        for r in range(6, shape.k):
+            e = int(ids[a, r])
+            b = next((b for b in range(40) if e in ids[b, :6].tolist()), None)
+            if b is not None:
+                found = (a, b, e)
+                break
+        if found:
+            break
+    assert found is not None, "test needs such a pair of tokens"
+    a, b, e = found
+    alone = oracle.tail_skip(ids[[a]], shape.E, 6)
+    both = oracle.tail_skip(ids[[a, b]], shape.E, 6)
+    assert alone[e] == 1 and both[e] == 0
+    ya, _, _ = oracle.layer(shape, xs[[a]], L["router_w"], L["bias"], L["codes"], L["scales"], drop=alone)
+    yab, _, _ = oracle.layer(shape, xs[[a, b]], L["router_w"], L["bias"], L["codes"], L["scales"], drop=both)
+    assert not np.allclose(ya[0], yab[0])
