@@ -32,11 +32,20 @@ def shard_handle(h, rank: int, world: int) -> None:
     h.set_expert_range(*expert_shard(h.cfg.n_experts, rank, world))
 
 
-def reduce_partial(y, group=None):
-    """Sum the ranks' fp32 partial outputs in place: afterwards y holds the layer on every rank."""
+def reduce_partial(y, group=None, stream=None):
+    """Sum the ranks' fp32 partial outputs in place: afterwards y holds the layer on every rank.
+
+    With a CUDA stream, the all-reduce is ordered on that stream (the one the partial output was computed
+    on); without one, on the current stream.
+    """
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
-        dist.all_reduce(y, op=dist.ReduceOp.SUM, group=group)
+        if stream is None:
+            dist.all_reduce(y, op=dist.ReduceOp.SUM, group=group)
+        else:
+            import torch
+            with torch.cuda.stream(stream):
+                dist.all_reduce(y, op=dist.ReduceOp.SUM, group=group)
     return y
 
 
@@ -49,4 +58,4 @@ def forward(h, layer: int, x, y=None, flags: int = 0, group=None, stream=None):
     if flags & MOE_ACCUMULATE:
         raise ValueError("expert-parallel forward sums partial outputs: add the residual after the call")
     y = h.forward(layer, x, y, flags=flags | MOE_OUT_FP32, stream=stream)
-    return reduce_partial(y, group)
+    return reduce_partial(y, group, stream)
