@@ -22,7 +22,7 @@ __all__ = ["MoeError", "MoeConfig", "MoeLayerWeights", "MoeLayer", "lib", "libra
            "moe_route", "moe_route_noalloc", "moe_forward", "moe_forward_host", "moe_destroy", "moe_debug_dequant", "moe_debug_last_routing", "moe_check_status",
            "moe_get_stats", "moe_status_string", "moe_profile", "moe_profile_read", "moe_kernel_name", "MoeStats",
            "moe_debug_router_logits", "moe_router_error_depth", "moe_rms_normalize", "rms_normalize",
-           "moe_set_expert_range"]
+           "moe_set_expert_range", "moe_debug_wait_limit"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libmoe.so")
@@ -113,6 +113,8 @@ def lib() -> ctypes.CDLL:
             L.moe_rms_normalize.argtypes = [vp, i32, i32, vp, vp]
             L.moe_set_expert_range.restype = st
             L.moe_set_expert_range.argtypes = [vp, i32, i32, i32]
+            L.moe_debug_wait_limit.restype = st
+            L.moe_debug_wait_limit.argtypes = [vp, u32, i32]
             L.moe_status_string.restype = ctypes.c_char_p
             L.moe_status_string.argtypes = [st]
             _lib = L
@@ -163,6 +165,11 @@ def moe_route_noalloc(x_ptr: int, T: int, d: int, n_experts: int, top_k: int, ro
 
 def moe_set_expert_range(handle: int, begin: int, end: int, with_shared: int) -> None:
     _check(lib().moe_set_expert_range(handle, begin, end, with_shared), "moe_set_expert_range")
+
+
+def moe_debug_wait_limit(handle: int, spins: int, withhold_cta: int = -1) -> None:
+    """Test hook: device-side waits give up after `spins` polls; CTA withhold_cta withholds its router rows."""
+    _check(lib().moe_debug_wait_limit(handle, spins, withhold_cta), "moe_debug_wait_limit")
 
 
 def moe_destroy(handle: int) -> None:
@@ -318,6 +325,10 @@ class MoeLayer:
     def set_expert_range(self, begin, end, with_shared=True):
         """Compute only routed experts [begin, end) (and the shared one if with_shared) from now on."""
         moe_set_expert_range(self.handle, begin, end, 1 if with_shared else 0)
+
+    def debug_wait_limit(self, spins: int, withhold_cta: int = -1):
+        """Test hook of the device watchdog (see moe_debug_wait_limit in include/moe.h)."""
+        moe_debug_wait_limit(self.handle, spins, withhold_cta)
 
     def close(self):
         if self.handle:

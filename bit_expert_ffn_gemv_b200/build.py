@@ -1,6 +1,11 @@
-"""Build libmoe.so (the C-ABI library) in-tree with nvcc for sm_100a."""
+"""Build libmoe.so (the C-ABI library) in-tree with nvcc for sm_100a.
+
+Each .cu file compiles to its own object in _build/ (in parallel, and only when
+it or a header changed), then one link step writes libmoe.so next to this file.
+"""
 from __future__ import annotations
 
+import concurrent.futures as cf
 import glob
 import os
 import subprocess
@@ -10,18 +15,25 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
+OBJ = os.path.join(ROOT, "_build", "moe")
 LIB = os.path.join(PKG, "libmoe.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC,
+         "--expt-relaxed-constexpr", "-Xcompiler", "-Wall"]
 
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _inputs():
-    return sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
+def _headers():
+    return glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
         glob.glob(os.path.join(INCLUDE, "*.h"))
+
+
+def _inputs():
+    return sources() + _headers()
 
 
 def stale() -> bool:
@@ -31,14 +43,35 @@ def stale() -> bool:
     return any(os.path.getmtime(p) > t for p in _inputs())
 
 
+def _obj(src: str) -> str:
+    return os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+
+
+def _compile(src: str, force: bool, ptxas_v: bool, verbose: bool) -> str:
+    out = _obj(src)
+    newest = max([os.path.getmtime(src)] + [os.path.getmtime(h) for h in _headers()])
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= newest:
+        return out
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", tmp]
+    if ptxas_v:
+        cmd.insert(1, "-Xptxas=-v")
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    subprocess.check_call(cmd)
+    os.replace(tmp, out)
+    return out
+
+
 def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False) -> str:
     if not force and not stale():
         return LIB
+    os.makedirs(OBJ, exist_ok=True)
+    srcs = sources()
+    with cf.ThreadPoolExecutor(max_workers=min(len(srcs), os.cpu_count() or 4)) as ex:
+        objs = list(ex.map(lambda s: _compile(s, force, ptxas_v, verbose), srcs))
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-I", CSRC,
-           "--expt-relaxed-constexpr", "-Xcompiler", "-Wall", "-o", tmp, *sources()]
-    if ptxas_v:
-        cmd.insert(1, "-Xptxas=-v")
+    cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
@@ -47,5 +80,5 @@ def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False) -> 
 
 
 if __name__ == "__main__":
-    build(force=True, verbose=True, ptxas_v="-v" in sys.argv)
+    build(force="-f" in sys.argv, verbose=True, ptxas_v="-v" in sys.argv)
     print(LIB)

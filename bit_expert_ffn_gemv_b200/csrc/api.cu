@@ -25,6 +25,8 @@ struct moe_layer_state {
     float* wnorm = nullptr;  // owned
     moe::GemmMaps w_gu{};    // codes/scales TMA maps, gate/up geometry
     moe::GemmMaps w_dn{};    // codes/scales TMA maps, down geometry
+    CUtensorMap pair_dc{};   // down codes / scales maps of the clustered decode kernel
+    CUtensorMap pair_ds{};
     bool loaded = false;
 };
 
@@ -48,6 +50,10 @@ struct moe_handle {
     float* obuf = nullptr;
     double* logits64 = nullptr;
     int* sync = nullptr;
+    float* part = nullptr;               // partial sums of the clustered decode kernel
+    unsigned long long* ctr = nullptr;   // its monotonic counters
+    uint32_t spin_limit = 1u << 21;      // polls before a device-side wait gives up
+    int withhold = -1;                   // test hook: a CTA that never announces its router rows
     void* x_stage = nullptr;
     void* y_stage = nullptr;
     void* xg = nullptr;          // fp16 x rows in group order (tensor-core path)
@@ -158,9 +164,14 @@ moe_status do_route(moe_handle* h, int32_t layer, const void* x, int32_t T, int3
     return cuda_status(run(h, MOE_K_TOPK, s, [&] { return moe::launch_topk(ra, s); }));
 }
 
-moe_status do_decode(moe_handle* h, int32_t layer, const void* x, int32_t T, void* y, uint32_t flags,
-                     cudaStream_t s) {
+// The fused decode kernels: the clustered kernel (any code widths) up to
+// kPairMaxTokens tokens when its shared-memory layout fits, else the older
+// persistent kernel (one code width) up to kDecodeMaxTokens.  Returns false,
+// enqueueing nothing, when neither applies.
+bool try_decode(moe_handle* h, int32_t layer, const void* x, int32_t T, void* y, uint32_t flags, cudaStream_t s,
+                moe_status* st) {
     const moe_config& c = h->cfg;
+    if (use_tensor_cores(c, T, flags) || (flags & MOE_FORCE_UNFUSED)) return false;
     const moe_layer_state& L = h->layers[layer];
     moe::DecodeLaunch d;
     d.T = T;
@@ -195,15 +206,29 @@ moe_status do_decode(moe_handle* h, int32_t layer, const void* x, int32_t T, voi
     d.skip_rank = skip_rank(c, flags);
     d.e_begin = h->ep_begin;
     d.e_end = h->ep_end;
-    return cuda_status(run(h, MOE_K_DECODE, s, [&] { return moe::launch_decode(d, s); }));
+    d.bits_down = bits_down(c);
+    d.part = h->part;
+    d.ctr = h->ctr;
+    d.spin_limit = h->spin_limit;
+    d.withhold = h->withhold;
+    d.down_codes_map = &L.pair_dc;
+    d.down_scales_map = &L.pair_ds;
+    if (T <= moe::kPairMaxTokens && moe::pair_decode_supported(d)) {
+        *st = cuda_status(run(h, MOE_K_DECODE, s, [&] { return moe::launch_decode_pair(d, s); }));
+        return true;
+    }
+    if (T <= moe::kDecodeMaxTokens && !mixed_widths(c)) {
+        *st = cuda_status(run(h, MOE_K_DECODE, s, [&] { return moe::launch_decode(d, s); }));
+        return true;
+    }
+    return false;
 }
 
 moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, void* y, uint32_t flags,
                       cudaStream_t s) {
     const moe_config& c = h->cfg;
-    if (T <= moe::kDecodeMaxTokens && !use_tensor_cores(c, T, flags) && !(flags & MOE_FORCE_UNFUSED) &&
-        !mixed_widths(c))
-        return do_decode(h, layer, x, T, y, flags, s);
+    moe_status dst = MOE_OK;
+    if (try_decode(h, layer, x, T, y, flags, s, &dst)) return dst;
     const bool tc = use_tensor_cores(c, T, flags);
     cudaError_t e;
     moe_status st = do_route(h, layer, x, T, h->ids, h->w, tc, s);
@@ -375,6 +400,8 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     const size_t o_bcnt = take(sizeof(int32_t) * moe::bucket_scratch_words(c.n_experts));
     const size_t o_sync =
         take(sizeof(int) * moe::decode_sync_words(std::min(c.max_tokens, moe::kDecodeMaxTokens), c.n_experts, c.d));
+    const size_t o_part = take(sizeof(float) * moe::pair_part_floats(c.max_tokens, c.top_k, c.n_shared, c.d, c.f));
+    const size_t o_ctr = take(sizeof(unsigned long long) * moe::kPairCounters);
     h->arena_bytes = off;
     cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
     if (e != cudaSuccess) {
@@ -396,6 +423,8 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     h->obuf = reinterpret_cast<float*>(base + o_obuf);
     h->logits64 = reinterpret_cast<double*>(base + o_l64);
     h->sync = reinterpret_cast<int*>(base + o_sync);
+    h->part = reinterpret_cast<float*>(base + o_part);
+    h->ctr = reinterpret_cast<unsigned long long*>(base + o_ctr);
     h->x_stage = base + o_xs;
     h->y_stage = base + o_ys;
     h->xg = base + o_xg;
@@ -433,6 +462,9 @@ moe_status moe_load_layer(moe_handle* h, int32_t layer, const moe_layer_weights*
     if (!mixed_widths(h->cfg) &&
         (moe::make_weight_maps(&L.w_gu, L.codes, L.scales, ne, h->cfg.f, h->cfg.d, h->cfg.bits) != cudaSuccess ||
          moe::make_weight_maps(&L.w_dn, L.codes, L.scales, ne, h->cfg.d, h->cfg.f, h->cfg.bits) != cudaSuccess))
+        return MOE_ERR_CUDA;
+    if (moe::make_pair_down_maps(&L.pair_dc, &L.pair_ds, L.codes, L.scales, ne, h->cfg.d, h->cfg.f, h->cfg.bits,
+                                 bits_down(h->cfg)) != cudaSuccess)
         return MOE_ERR_CUDA;
     cudaError_t e = moe::launch_router_norms(L.router_w, h->cfg.n_experts, h->cfg.d, L.wnorm, 0);
     if (e == cudaSuccess) e = cudaStreamSynchronize(0);
@@ -565,9 +597,26 @@ moe_status moe_check_status(moe_handle* h) {
     uint32_t v = 0;
     if (cudaMemcpy(&v, h->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
     if (cudaMemset(h->status, 0, sizeof(uint32_t)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (v) {
+        // A launch that hit an anomaly may have left the fused kernels' counters
+        // out of step: start them afresh (nothing is in flight).
+        const size_t sync_bytes = sizeof(int) * moe::decode_sync_words(
+                                                   std::min(h->cfg.max_tokens, moe::kDecodeMaxTokens),
+                                                   h->cfg.n_experts, h->cfg.d);
+        if (cudaMemset(h->sync, 0, sync_bytes) != cudaSuccess ||
+            cudaMemset(h->ctr, 0, sizeof(unsigned long long) * moe::kPairCounters) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
     if (v & moe::kStatusTimeout) return MOE_ERR_TIMEOUT;
     if (v & moe::kStatusBounds) return MOE_ERR_BOUNDS;
     if (v & moe::kStatusRange) return MOE_ERR_RANGE;
+    return MOE_OK;
+}
+
+moe_status moe_debug_wait_limit(moe_handle* h, uint32_t spins, int32_t withhold_cta) {
+    if (!h || spins == 0 || withhold_cta < -1) return MOE_ERR_INVALID_ARG;
+    h->spin_limit = spins;
+    h->withhold = withhold_cta;
     return MOE_OK;
 }
 

@@ -1,0 +1,1245 @@
+// decode_pair.cu -- the whole routed-MoE layer for up to 16 tokens in ONE launch
+// of 148 CTAs (74 clusters of two, one CTA per SM).
+//
+// A decode or draft-verify batch (one token plus up to three drafts; the layer
+// the Strata pages run per generated token: the router picks the experts, the
+// GPU combines their results, then moves to the next layer -- discuss.pytorch.kr
+// post, section "Strata's operating principle") touches ~18 MB of packed
+// expert weights per token, a few microseconds of HBM time.  The launch is
+// shaped so that those bytes stream at full bandwidth behind a short chain of
+// hand-offs:
+//
+//   1. Router.  CTA b computes the exact logits of experts [bE/G, (b+1)E/G)
+//      for all T tokens (bf16 x bf16 products are exact in fp64, summed by
+//      fp64 FMAs), writes them to global memory and announces them on a
+//      64-bit arrival counter.  Clusters whose first work unit belongs to the
+//      shared expert run that unit meanwhile (it needs no routing).
+//   2. Top-k and schedule, redundantly in every CTA, once all CTAs arrived:
+//      each warp ranks one token's E logits (ties to the lower index, exact
+//      rank order), then the CTA lists the active experts ("slots": the shared
+//      expert, then the selected routed experts in ascending order) and the
+//      work units.  No second grid-wide hand-off is needed before the experts.
+//   3. Work units.  Unit u = (slot u / (f/128), chunk j = u % (f/128)) covers
+//      the 128 intermediate rows [128j, 128j + 128) of one expert: its gate/up
+//      rows and the matching 128 input columns of its down matrix.  Cluster c
+//      takes units c, c + 74, c + 148, ...  Inside the cluster, CTA r computes
+//      gate/up rows [64r, 64r + 64) of the chunk (warp w: 16-row tile w/2 of
+//      gate (w even) or up (w odd) over the whole input dimension), writes the
+//      h rows into both CTAs' shared memory, and multiplies the chunk's 128 h
+//      values by down rows [r d/2, (r+1) d/2).  Every expert byte is read
+//      once and h never leaves the cluster.  The down partial sums, times the
+//      routing weight, are stored (no atomics) per (token, slot, chunk).
+//   4. Combine.  After a second arrival count, every CTA sums a slice of the
+//      partial sums in a fixed order (slot, then chunk) and writes y, so the
+//      result does not depend on timing.
+//
+// Warp 8 is the producer: it moves the weights by bulk copies (TMA) into two
+// rings of shared-memory slots (gate/up items: one 16-row tile of gate and of
+// up; down items: d/64 row tiles x one 128-column super-tile, fetched through
+// a 3-D tensor map), as far ahead as the rings allow.  Warps 0-7 compute:
+// warp MMAs on exact 16-bit integer codes (bf16 for gate/up against bf16 x,
+// fp16 for down against fp16 h) with the fp16 block scale applied in fp32 per
+// 32-block.  Slots, h buffers and the pair's h exchange are tracked by
+// mbarriers (the peer's h rows arrive by st.async stores that complete
+// bytes on this CTA's barrier), so no wait involves the producer and the
+// consumers together.
+//
+// Every wait is bounded: an mbarrier or counter wait gives up after a limit,
+// sets the status word and carries on (a copy wait then waits once more,
+// bounded, for its bytes).  The only hardware cluster barriers are one at the
+// start and one at the end, run by every thread.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace pair {
+
+constexpr int kCWarps = 8;                 // compute (consumer) warps
+constexpr int kConsumers = kCWarps * 32;
+constexpr int kProducer = kCWarps;         // warp index of the producer
+constexpr int kThreads = kConsumers + 32;
+constexpr int kCS = 2;                     // CTAs per cluster
+constexpr int kMaxSlots = 16;              // ring slots of each kind (upper bound)
+constexpr int kXPad = 32;                  // 16-bit elements of padding per staged row
+constexpr int kHRow = 128 + kXPad;
+constexpr int kCandBytes = 64 * 16;        // per-warp top-k candidate buffer
+
+// Optional phase trace (build with -DMOE_PAIR_TRACE): thread 0 of every CTA
+// records the global timer at phase boundaries and adds clock64() differences
+// per phase; moe_debug_pair_trace() / moe_debug_pair_cycles() copy them out.
+#ifdef MOE_PAIR_TRACE
+constexpr int kTraceSlots = 48;
+__device__ unsigned long long g_trace[1024 * kTraceSlots];
+__device__ unsigned long long g_cyc[1024 * 32];
+MOE_DEV void trace(int slot) {
+    if (threadIdx.x == 0 && slot < kTraceSlots) {
+        unsigned long long t;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        g_trace[blockIdx.x * kTraceSlots + slot] = t;
+    }
+}
+MOE_DEV unsigned long long cyc() { return (unsigned long long)clock64(); }
+MOE_DEV void cyc_add(int slot, unsigned long long t0) {
+    if (threadIdx.x == 0) g_cyc[blockIdx.x * 32 + slot] += cyc() - t0;
+}
+MOE_DEV void cyc_reset() {
+    if (threadIdx.x == 0)
+        for (int i = 0; i < 32; ++i) g_cyc[blockIdx.x * 32 + i] = 0;
+}
+#else
+MOE_DEV void trace(int) {}
+MOE_DEV unsigned long long cyc() { return 0; }
+MOE_DEV void cyc_add(int, unsigned long long) {}
+MOE_DEV void cyc_reset() {}
+#endif
+
+struct Args {
+    int T, d, f, E, k, n_shared;
+    const uint16_t* x;  // bf16 [T x d]
+    void* y;
+    int out_fp32, accumulate;
+    const uint8_t* codes;
+    const uint16_t* scales;
+    int64_t code_stride;   // code bytes per expert (gate, up, down)
+    int64_t scale_stride;  // fp16 scales per expert
+    const uint16_t* wr;    // bf16 [E x d]
+    const float* bias;
+    double* logits64;      // [T x E]
+    int32_t* ids;          // [T x k] (written by CTA 0)
+    float* w;
+    Meta* meta;
+    uint32_t* status;
+    float* part;           // [T x (k + n_shared) x f/128 x d] partial sums
+    unsigned long long* ctr;  // [0] router arrivals, [1] partial sums written
+    int skip_rank;
+    int e_begin, e_end;
+    int nc;                // clusters in the grid
+    uint32_t spin_limit;   // polls before a wait gives up
+    int withhold;          // test only: this CTA never announces its router rows (-1: off)
+    // shared memory layout (bytes from the dynamic base)
+    int ng, nd;            // ring slots
+    int g_bytes, d_bytes;  // item sizes
+    int off_x, off_h, off_gus, off_cand, off_route, off_emask, off_slots, off_pos, off_g, off_d;
+};
+
+// ---------------------------------------------------------------- cluster, mbarrier and memory-order helpers
+MOE_DEV uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+MOE_DEV uint32_t cluster_idx() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+MOE_DEV void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+MOE_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+MOE_DEV void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory"); }
+// address of the same shared-memory location in CTA `rank` of the cluster
+MOE_DEV uint32_t peer_addr(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+    return r;
+}
+MOE_DEV void fence_mbar_init_cluster() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+// store 4 bytes into the peer's shared memory; the store completes 4 bytes
+// of transactions on the peer's mbarrier (no fence needed before the peer reads)
+MOE_DEV void st_async_remote(uint32_t addr, uint32_t v, uint32_t bar_addr) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(addr), "r"(v),
+                 "r"(bar_addr)
+                 : "memory");
+}
+MOE_DEV void mbar_arrive_relaxed_remote(uint32_t addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+MOE_DEV bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, "
+        "p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+MOE_DEV unsigned long long ld_acquire_u64(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+MOE_DEV unsigned long long atom_add_acqrel_u64(unsigned long long* p, unsigned long long v) {
+    unsigned long long old;
+    asm volatile("atom.add.acq_rel.gpu.global.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+    return old;
+}
+MOE_DEV void fence_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+MOE_DEV void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// Bounded waits.  A copy wait that gives up waits once more (bounded) so that
+// no copy is still landing when the caller moves on.
+MOE_DEV void copy_wait(uint64_t* bar, uint32_t parity, const Args& a) {
+    for (uint32_t it = 0; it <= a.spin_limit; ++it)
+        if (mbar_try_wait(bar, parity)) return;
+    if ((threadIdx.x & 31) == 0) flag_status(a.status, kStatusTimeout);
+    for (uint32_t it = 0; it <= a.spin_limit; ++it)
+        if (mbar_try_wait(bar, parity)) return;
+}
+MOE_DEV void slot_wait(uint64_t* bar, uint32_t parity, const Args& a) {
+    for (uint32_t it = 0; it <= a.spin_limit; ++it)
+        if (mbar_try_wait(bar, parity)) return;
+    if ((threadIdx.x & 31) == 0) flag_status(a.status, kStatusTimeout);
+}
+MOE_DEV void pair_wait(uint64_t* bar, uint32_t parity, const Args& a) {
+    for (uint32_t it = 0; it <= a.spin_limit; ++it)
+        if (mbar_try_wait_cluster(bar, parity)) return;
+    if ((threadIdx.x & 31) == 0) flag_status(a.status, kStatusTimeout);
+}
+// One thread per CTA: add this CTA's arrival (unless withheld) to a counter
+// that only grows; the launch's full count is the next multiple of the grid
+// size above the value found at arrival.
+MOE_DEV unsigned long long grid_arrive(unsigned long long* ctr, bool arrive) {
+    const unsigned long long G = gridDim.x;
+    fence_gpu();
+    const unsigned long long old = arrive ? atom_add_acqrel_u64(ctr, 1ull) : ld_acquire_u64(ctr);
+    return (old / G + 1ull) * G;
+}
+MOE_DEV void grid_wait(const unsigned long long* ctr, unsigned long long target, const Args& a) {
+    uint32_t ns = 32;
+    for (uint32_t it = 0; it <= a.spin_limit; ++it) {
+        if (ld_acquire_u64(ctr) >= target) return;
+        __nanosleep(ns);
+        if (ns < 128) ns <<= 1;
+    }
+    flag_status(a.status, kStatusTimeout);
+}
+
+// ---------------------------------------------------------------- code decoding (faster form, 2-bit)
+// Each A-fragment register holds two codes u at bits [2p, 2p+1] and
+// [16+2p, 17+2p] of the lane's 32-bit code word.  Instead of shifting every
+// pair down to bit 0, the word is masked in place and OR-ed into a 16-bit
+// float whose exponent makes bit 2p the unit: 2^E + u exactly; subtracting
+// 2^E + 2 leaves q = u - 2 exactly.  Pairs whose bits reach the exponent
+// field are first shifted down once.
+//   bf16 (7 mantissa bits): bits 0-1, 2-3, 4-5 with 2^E = 128, 32, 8
+//   fp16 (10 mantissa bits): bits 0-1 .. 8-9 with 2^E = 1024, 256, 64, 16, 4
+template <bool F16>
+MOE_DEV uint32_t sub2(uint32_t v, uint32_t c) {
+    uint32_t r;
+    if (F16)
+        asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(c));
+    else
+        asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(c));
+    return r;
+}
+MOE_DEV uint32_t dup16(uint32_t h) { return h | (h << 16); }
+
+template <bool F16>
+MOE_DEV void decode2_fast(uint32_t lo, uint32_t (&q)[8]) {
+    if (F16) {
+        const uint32_t s10 = lo >> 10;
+        q[0] = sub2<true>((lo & 0x00030003u) | dup16(0x6400u), dup16(0x6402u));
+        q[1] = sub2<true>((lo & 0x000C000Cu) | dup16(0x5C00u), dup16(0x5C08u));
+        q[2] = sub2<true>((lo & 0x00300030u) | dup16(0x5400u), dup16(0x5420u));
+        q[3] = sub2<true>((lo & 0x00C000C0u) | dup16(0x4C00u), dup16(0x4C80u));
+        q[4] = sub2<true>((lo & 0x03000300u) | dup16(0x4400u), dup16(0x4600u));
+        q[5] = sub2<true>((s10 & 0x00030003u) | dup16(0x6400u), dup16(0x6402u));
+        q[6] = sub2<true>((s10 & 0x000C000Cu) | dup16(0x5C00u), dup16(0x5C08u));
+        q[7] = sub2<true>((s10 & 0x00300030u) | dup16(0x5400u), dup16(0x5420u));
+    } else {
+        const uint32_t s6 = lo >> 6, s12 = lo >> 12;
+        q[0] = sub2<false>((lo & 0x00030003u) | dup16(0x4300u), dup16(0x4302u));
+        q[1] = sub2<false>((lo & 0x000C000Cu) | dup16(0x4200u), dup16(0x4208u));
+        q[2] = sub2<false>((lo & 0x00300030u) | dup16(0x4100u), dup16(0x4120u));
+        q[3] = sub2<false>((s6 & 0x00030003u) | dup16(0x4300u), dup16(0x4302u));
+        q[4] = sub2<false>((s6 & 0x000C000Cu) | dup16(0x4200u), dup16(0x4208u));
+        q[5] = sub2<false>((s6 & 0x00300030u) | dup16(0x4100u), dup16(0x4120u));
+        q[6] = sub2<false>((s12 & 0x00030003u) | dup16(0x4300u), dup16(0x4302u));
+        q[7] = sub2<false>((s12 & 0x000C000Cu) | dup16(0x4200u), dup16(0x4208u));
+    }
+}
+
+template <bool F16, int BITS>
+MOE_DEV void decode_any(uint32_t lo, uint32_t hi, uint32_t (&q)[8]) {
+    if (BITS == 2)
+        decode2_fast<F16>(lo, q);
+    else
+        decode_block<F16, BITS>(lo, hi, q);
+}
+
+MOE_DEV void scale_acc(float (&acc)[4], const float (&t)[4], uint32_t sc) {
+    const float slo = __half2float(__ushort_as_half((unsigned short)(sc & 0xFFFFu)));
+    const float shi = __half2float(__ushort_as_half((unsigned short)(sc >> 16)));
+    acc[0] = fmaf(slo, t[0], acc[0]);
+    acc[1] = fmaf(slo, t[1], acc[1]);
+    acc[2] = fmaf(shi, t[2], acc[2]);
+    acc[3] = fmaf(shi, t[3], acc[3]);
+}
+
+// position of element k (0..31) of a 32-element block in the staged row layout:
+// the four pairs a lane's B fragment needs (k = 2c + 8j + e, j = 0..3) sit
+// together at 8c + 2j + e, so one 16-byte load fetches them.
+MOE_DEV int perm32(int k) { return ((k & 7) >> 1) * 8 + (k >> 3) * 2 + (k & 1); }
+
+// ---------------------------------------------------------------- top-k of one token (warp)
+MOE_DEV uint64_t order_key64(double v) {
+    if (isnan(v)) v = -INFINITY;
+    v = v + 0.0;  // -0 -> +0
+    const uint64_t b = (uint64_t)__double_as_longlong(v);
+    return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+MOE_DEV bool better64(uint64_t ka, int ia, uint64_t kb, int ib) { return ka > kb || (ka == kb && ia < ib); }
+// 32-bit key: order-preserving image of fp32(l) with the low 10 bits replaced
+// by 1023 - e.  A strictly larger prefix (the upper 22 bits) means a strictly
+// larger logit; keys are unique.
+MOE_DEV uint32_t key32(double v, int e) {
+    float f = (float)(isnan(v) ? -INFINITY : v);
+    f = f + 0.0f;
+    const uint32_t b = __float_as_uint(f);
+    const uint32_t o = (b >> 31) ? ~b : (b | 0x80000000u);
+    return (o & 0xFFFFFC00u) | (uint32_t)(1023 - e);
+}
+
+struct Cand {
+    double v;
+    int e;
+    int pad;
+};
+
+// Slow exact selection (when more than 32 logits share the candidate prefix).
+MOE_DEV void topk_scan(const double* lg, int E, int k, int lane, int& sel, double& lsel, double& top) {
+    int prev_e = -1;
+    uint64_t prev_k = 0;
+    for (int r = 0; r < k; ++r) {
+        uint64_t bk = 0;
+        int bi = 0x7fffffff;
+        for (int e = lane; e < E; e += 32) {
+            const uint64_t ke = order_key64(__ldcg(lg + e));
+            if (prev_e >= 0 && !better64(prev_k, prev_e, ke, e)) continue;  // not strictly worse than the last pick
+            if (bi == 0x7fffffff || better64(ke, e, bk, bi)) {
+                bk = ke;
+                bi = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const uint64_t ok = __shfl_xor_sync(0xffffffffu, bk, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (oi != 0x7fffffff && (bi == 0x7fffffff || better64(ok, oi, bk, bi))) {
+                bk = ok;
+                bi = oi;
+            }
+        }
+        const double lv = __ldcg(lg + bi);
+        if (lane == r) {
+            sel = bi;
+            lsel = lv;
+        }
+        if (r == 0) top = lv;
+        prev_e = bi;
+        prev_k = bk;
+    }
+}
+
+// Exact top-k of one token's E fp64 logits (global memory, read through L2).
+// tau = the k-th largest of the 32 lanes' largest keys: at least k logits have
+// a key >= tau, so every logit of the exact top k has a key prefix >= tau's
+// (a smaller prefix means a smaller logit than all of those k).  Those
+// candidates (usually a few more than k) are compacted into shared memory
+// and ranked by (fp64 logit desc, index asc).  Lane r < k returns id r and
+// its weight w_r = softmax over the k selected logits.
+template <int KPL>
+MOE_DEV void topk_token(const double* lg, int E, int k, int lane, Cand* cand, int& id_out, float& w_out) {
+    double v[KPL];
+    uint32_t key[KPL];
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) v[j] = __ldcg(lg + min(lane + 32 * j, E - 1));
+    uint32_t lmax = 0u;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+        const int e = lane + 32 * j;
+        key[j] = e < E ? key32(v[j], e) : 0u;
+        lmax = max(lmax, key[j]);
+    }
+    int rk = 0;  // lanes whose largest key beats mine
+#pragma unroll
+    for (int o = 1; o < 32; ++o) rk += __shfl_sync(0xffffffffu, lmax, (lane + o) & 31) > lmax ? 1 : 0;
+    const int src = __ffs(__ballot_sync(0xffffffffu, rk == k - 1 && lmax != 0u)) - 1;
+    const uint32_t P = __shfl_sync(0xffffffffu, lmax, max(src, 0)) & 0xFFFFFC00u;
+    int cnt = 0;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) cnt += (key[j] != 0u && (key[j] & 0xFFFFFC00u) >= P) ? 1 : 0;
+    const int C = (int)__reduce_add_sync(0xffffffffu, (unsigned)cnt);
+    int sel = -1;
+    double lsel = 0.0, top = 0.0;
+    if (src >= 0 && C >= k && C <= 32) {
+        int off = 0;
+#pragma unroll
+        for (int j = 0; j < KPL; ++j) {
+            const bool in = key[j] != 0u && (key[j] & 0xFFFFFC00u) >= P;
+            const unsigned bal = __ballot_sync(0xffffffffu, in);
+            if (in) {
+                Cand& cd = cand[off + __popc(bal & ((1u << lane) - 1u))];
+                cd.v = v[j];
+                cd.e = lane + 32 * j;
+            }
+            off += __popc(bal);
+        }
+        __syncwarp();
+        int rank = 0, my_e = 0;
+        double my_v = 0.0;
+        if (lane < C) {
+            my_v = cand[lane].v;
+            my_e = cand[lane].e;
+            const uint64_t my_k = order_key64(my_v);
+            for (int j = 0; j < C; ++j) {
+                const Cand o = cand[j];
+                if (j != lane && better64(order_key64(o.v), o.e, my_k, my_e)) ++rank;
+            }
+        }
+        __syncwarp();
+        if (lane < C && rank < k) {
+            cand[32 + rank].v = my_v;
+            cand[32 + rank].e = my_e;
+        }
+        __syncwarp();
+        top = cand[32].v;
+        if (lane < k) {
+            sel = cand[32 + lane].e;
+            lsel = cand[32 + lane].v;
+        }
+        __syncwarp();
+    } else {
+        topk_scan(lg, E, k, lane, sel, lsel, top);
+    }
+    const float ex = lane < k ? expf((float)(lsel - top)) : 0.0f;
+    float z = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    id_out = sel;
+    w_out = lane < k ? ex / z : 0.0f;
+}
+
+MOE_DEV double bf16_to_f64(uint32_t bits16) { return (double)__uint_as_float(bits16 << 16); }
+
+// ---------------------------------------------------------------- the kernel
+template <int BG, int BD, int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_pair_kernel(const __grid_constant__ Args a, const __grid_constant__ CUtensorMap dmap_c,
+                       const __grid_constant__ CUtensorMap dmap_s) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t fullG[kMaxSlots], emptyG[kMaxSlots], fullD[kMaxSlots], emptyD[kMaxSlots];
+    __shared__ __align__(8) uint64_t hfull[3], hempty[3], barX, sched;
+    __shared__ int s_nslots, s_nunits, s_wcnt[kCWarps];
+    __shared__ float s_w[2][16];
+    __shared__ uint32_t s_mask[2];
+    __shared__ int s_slot[2];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, c = lane & 3;
+    trace(0);
+    cyc_reset();
+    const uint32_t rank = cluster_ctarank();
+    const int q = (int)cluster_idx();
+    const int nc = a.nc, G = (int)gridDim.x, b = (int)blockIdx.x;
+    const int T = a.T, d = a.d, f = a.f, E = a.E, k = a.k, ns = a.n_shared;
+    const int KT = d / 128, FC = f / 128, RT = d / 16, RTI = RT / 4, KS = k + ns;
+    constexpr int GCB = 256 * BG, DCB = 256 * BD;  // code bytes of one super-tile
+    const int64_t mg = (int64_t)f * d * BG / 8;    // code bytes of one gate/up matrix
+    const int64_t msc = (int64_t)f * d / 32;       // scales of one matrix
+    const int xstride = d + kXPad;
+
+    uint16_t* xs = reinterpret_cast<uint16_t*>(smem + a.off_x);     // [T][d + pad] bf16
+    uint16_t* hb = reinterpret_cast<uint16_t*>(smem + a.off_h);     // [3][T][128 + pad] fp16, permuted
+    float* gus = reinterpret_cast<float*>(smem + a.off_gus);        // gate/up outputs / router partials
+    Cand* cand = reinterpret_cast<Cand*>(smem + a.off_cand);        // [8 warps][64]
+    int* sids = reinterpret_cast<int*>(smem + a.off_route);         // [T * k]
+    float* sw = reinterpret_cast<float*>(sids + T * k);             // [T * k]
+    uint32_t* emask = reinterpret_cast<uint32_t*>(smem + a.off_emask);  // [E] tokens selecting e
+    int* ebest = reinterpret_cast<int*>(emask + E);                 // [E] best rank of e in the batch
+    int* slot_e = reinterpret_cast<int*>(smem + a.off_slots);       // [n_slots] expert of each slot
+    int* tn = reinterpret_cast<int*>(smem + a.off_pos);             // [16] slots of token t
+    unsigned char* pos = smem + a.off_pos + 64;                     // [n_slots][T] place of slot s in t's list
+    uint8_t* gring = smem + a.off_g;
+    uint8_t* dring = smem + a.off_d;
+
+    if (tid == 0) {
+        for (int i = 0; i < a.ng; ++i) {
+            mbar_init(&fullG[i], 1);
+            mbar_init(&emptyG[i], 2);  // the gate warp and the up warp of its row tile
+        }
+        for (int i = 0; i < a.nd; ++i) {
+            mbar_init(&fullD[i], 1);
+            mbar_init(&emptyD[i], kCWarps);
+        }
+        for (int i = 0; i < 3; ++i) {
+            mbar_init(&hfull[i], 1);   // armed here with the bytes the peer's h stores bring
+            mbar_init(&hempty[i], 1);  // the peer has read its copy of the buffer
+        }
+        mbar_init(&barX, 1);
+        mbar_init(&sched, 1);
+        fence_mbar_init_cluster();
+        fence_proxy_async_smem();
+    }
+    for (int e = tid; e < E; e += kThreads) {
+        emask[e] = 0u;
+        ebest[e] = k;
+    }
+    __syncthreads();
+    cluster_arrive();  // the peer's barriers are initialised once this completes (waited below)
+
+    // ---- work units of this cluster: u = q + i * nc -> (slot u / FC, chunk u % FC)
+    const int n_pre = (q < FC * ns) ? (FC * ns - 1 - q) / nc + 1 : 0;  // shared-expert units
+    auto unit_expert = [&](int i, int& e, int& j, int& s) {
+        const int u = q + i * nc;
+        s = u / FC;
+        j = u - s * FC;
+        e = s < ns ? E : slot_e[s];
+    };
+
+    if (warp == kProducer) {
+        // ================================================================ producer
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&barX, (uint32_t)T * d * 2);
+            for (int t = 0; t < T; ++t) bulk_g2s(xs + t * xstride, a.x + (int64_t)t * d, d * 2, &barX);
+        }
+        int item = 0;
+        auto issue_until = [&](int n_units) {
+            for (; item < 6 * n_units; ++item) {
+                const int i = item / 6, r6 = item - 6 * i;
+                int e, j, s;
+                unit_expert(i, e, j, s);
+                const uint8_t* ce = a.codes + (int64_t)e * a.code_stride;
+                const uint8_t* se = reinterpret_cast<const uint8_t*>(a.scales + (int64_t)e * a.scale_stride);
+                if (r6 < 4) {
+                    const int gi = 4 * i + r6, sl = gi % a.ng, use = gi / a.ng;
+                    if (use > 0) slot_wait(&emptyG[sl], (uint32_t)(use - 1) & 1u, a);
+                    if (lane == 0) {
+                        uint8_t* dst = gring + (size_t)sl * a.g_bytes;
+                        const int rtg = 8 * j + 4 * (int)rank + r6;  // 16-row tile of the gate/up matrices
+                        const uint32_t cb = KT * GCB, sb = KT * 128;
+                        mbar_arrive_expect_tx(&fullG[sl], 2 * (cb + sb));
+                        bulk_g2s(dst, ce + (int64_t)rtg * cb, cb, &fullG[sl]);
+                        bulk_g2s(dst + cb, se + (int64_t)rtg * sb, sb, &fullG[sl]);
+                        bulk_g2s(dst + cb + sb, ce + mg + (int64_t)rtg * cb, cb, &fullG[sl]);
+                        bulk_g2s(dst + 2 * cb + sb, se + 2 * msc + (int64_t)rtg * sb, sb, &fullG[sl]);
+                    }
+                } else {
+                    const int di = 2 * i + (r6 - 4), sl = di % a.nd, use = di / a.nd;
+                    if (use > 0) slot_wait(&emptyD[sl], (uint32_t)(use - 1) & 1u, a);
+                    if (lane == 0) {
+                        // RTI row tiles x super-tile column j of expert e's down matrix
+                        uint8_t* dst = dring + (size_t)sl * a.d_bytes;
+                        const int rt0 = (int)rank * (RT / 2) + (r6 - 4) * RTI;
+                        mbar_arrive_expect_tx(&fullD[sl], (uint32_t)RTI * (DCB + 128));
+                        tma_load_3d(dst, &dmap_c, j * 64 * BD, rt0, e, &fullD[sl]);
+                        tma_load_3d(dst + (size_t)RTI * DCB, &dmap_s, j * 64, rt0, e, &fullD[sl]);
+                    }
+                }
+                __syncwarp();
+            }
+        };
+        issue_until(n_pre);
+        slot_wait(&sched, 0u, a);  // the consumers published the schedule
+        issue_until(s_nunits);
+        cluster_wait();  // the producer's half of the first cluster barrier
+    } else {
+        // ================================================================ consumers
+        const unsigned long long c_start = cyc();
+        // ---- 1. router rows [r0, r1): exact logits, 4 rows x 4 tokens per pass
+        {
+            const int r0 = (int)((int64_t)b * E / G), r1 = (int)((int64_t)(b + 1) * E / G), R = r1 - r0;
+            double* part = reinterpret_cast<double*>(gus);  // [kCWarps][4 rows][4 tokens]
+            bool x_ready = false;
+            for (int rp = 0; rp < R; rp += 4) {
+                const int nr = min(4, R - rp);
+                for (int t0 = 0; t0 < T; t0 += 4) {
+                    const int nt4 = min(4, T - t0);
+                    double acc[4][4];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) acc[r][t] = 0.0;
+                    for (int cg = tid; cg < d / 4; cg += kConsumers) {
+                        uint2 wv[4];
+#pragma unroll
+                        for (int r = 0; r < 4; ++r)
+                            wv[r] = r < nr ? __ldg(reinterpret_cast<const uint2*>(a.wr + (int64_t)(r0 + rp + r) * d) + cg)
+                                           : make_uint2(0, 0);
+                        if (!x_ready) {
+                            copy_wait(&barX, 0u, a);
+                            x_ready = true;
+                        }
+                        double xd[4][4];
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const uint2 xv = t < nt4 ? *reinterpret_cast<const uint2*>(xs + (t0 + t) * xstride + 4 * cg)
+                                                     : make_uint2(0, 0);
+                            xd[t][0] = bf16_to_f64(xv.x & 0xFFFFu);
+                            xd[t][1] = bf16_to_f64(xv.x >> 16);
+                            xd[t][2] = bf16_to_f64(xv.y & 0xFFFFu);
+                            xd[t][3] = bf16_to_f64(xv.y >> 16);
+                        }
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            const double w0 = bf16_to_f64(wv[r].x & 0xFFFFu), w1 = bf16_to_f64(wv[r].x >> 16);
+                            const double w2 = bf16_to_f64(wv[r].y & 0xFFFFu), w3 = bf16_to_f64(wv[r].y >> 16);
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                acc[r][t] = fma(w0, xd[t][0], acc[r][t]);
+                                acc[r][t] = fma(w1, xd[t][1], acc[r][t]);
+                                acc[r][t] = fma(w2, xd[t][2], acc[r][t]);
+                                acc[r][t] = fma(w3, xd[t][3], acc[r][t]);
+                            }
+                        }
+                    }
+                    if (!x_ready) {
+                        copy_wait(&barX, 0u, a);
+                        x_ready = true;
+                    }
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            double v = acc[r][t];
+#pragma unroll
+                            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                            if (lane == 0) part[(warp * 4 + r) * 4 + t] = v;
+                        }
+                    consumer_sync();
+                    if (tid < nr * nt4) {
+                        const int r = tid / nt4, t = tid - r * nt4, e = r0 + rp + r;
+                        const double bb = a.bias ? (double)a.bias[e] : 0.0;
+                        double sum = 0.0;
+                        for (int w = 0; w < kCWarps; ++w) sum += part[(w * 4 + r) * 4 + t];
+                        a.logits64[(int64_t)(t0 + t) * E + e] = sum + bb;
+                    }
+                    consumer_sync();
+                }
+            }
+            if (!x_ready) copy_wait(&barX, 0u, a);  // a CTA without router rows
+        }
+        cyc_add(27, c_start);
+        trace(1);
+        // announce the logits (release), unless this CTA is the test's withheld one
+        unsigned long long router_target = 0;
+        if (tid == 0) router_target = grid_arrive(a.ctr, b != a.withhold);
+        // x in place: permute every 32-element block so that a lane's B fragment
+        // (pairs 2c + 8j, j = 0..3) is one 16-byte load (u32 pair 4j + c -> 4c + j)
+        for (int blk = tid; blk < T * (d / 32); blk += kConsumers) {
+            const int t = blk / (d / 32), kb = blk - t * (d / 32);
+            uint4* p4 = reinterpret_cast<uint4*>(xs + t * xstride + kb * 32);
+            const uint4 v0 = p4[0], v1 = p4[1], v2 = p4[2], v3 = p4[3];  // one thread per block
+            p4[0] = make_uint4(v0.x, v1.x, v2.x, v3.x);
+            p4[1] = make_uint4(v0.y, v1.y, v2.y, v3.y);
+            p4[2] = make_uint4(v0.z, v1.z, v2.z, v3.z);
+            p4[3] = make_uint4(v0.w, v1.w, v2.w, v3.w);
+        }
+        consumer_sync();
+        cluster_wait();  // the peer is running and its barriers are initialised
+
+        // routing weight and token mask of unit i's expert (kept for its down step)
+        auto unit_weights = [&](int i) {
+            if (warp != 0) return;
+            int e, j, s;
+            unit_expert(i, e, j, s);
+            uint32_t bit = 0u;
+            float wt = 0.f;
+            if (lane < T) {
+                if (e == E) {
+                    wt = 1.f;
+                    bit = 1u;
+                } else {
+                    for (int r = 0; r < k; ++r)
+                        if (sids[lane * k + r] == e) {
+                            wt = sw[lane * k + r];
+                            bit = 1u;
+                        }
+                }
+                s_w[i & 1][lane] = wt;
+            }
+            const uint32_t m = __ballot_sync(0xffffffffu, bit != 0u);
+            if (lane == 0) {
+                s_mask[i & 1] = m;
+                s_slot[i & 1] = s;
+            }
+        };
+
+        // ---- gate/up of unit i: warp w computes 16-row tile w/2 of gate (w even) or up (w odd)
+        auto gate_up = [&](int i) {
+            const int qt = warp >> 1, mat = warp & 1;
+            const int gi = 4 * i + qt, sl = gi % a.ng, use = gi / a.ng;
+            unsigned long long c0 = cyc();
+            // With fewer than 4 gate/up slots the previous use of this slot may
+            // belong to other warps of the same unit: wait for its release first,
+            // so that the parity wait below cannot match a phase two behind.
+            if (use > 0) slot_wait(&emptyG[sl], (uint32_t)(use - 1) & 1u, a);
+            copy_wait(&fullG[sl], (uint32_t)use & 1u, a);
+            cyc_add(1, c0);
+            c0 = cyc();
+            const uint8_t* base = gring + (size_t)sl * a.g_bytes + (size_t)mat * KT * (GCB + 128);
+            float acc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) acc[nt][r] = 0.f;
+#pragma unroll 2
+            for (int st = 0; st < KT; ++st) {
+                TileRegs<BG> tr;
+                load_tile_smem<BG>(base + st * GCB, base + KT * GCB + st * 128, lane, tr);
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb) {
+                    const int k0 = st * 128 + kb * 32 + 8 * c;
+                    uint4 bx[NT];
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const int tok = nt * 8 + g;
+                        bx[nt] = tok < T ? *reinterpret_cast<const uint4*>(xs + tok * xstride + k0)
+                                         : make_uint4(0, 0, 0, 0);
+                    }
+                    uint32_t qq[8];
+                    decode_any<false, BG>(tr.lo[kb], tr.hi[kb], qq);
+                    const uint32_t q0[4] = {qq[0], qq[1], qq[2], qq[3]}, q1[4] = {qq[4], qq[5], qq[6], qq[7]};
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        float t4[4] = {0.f, 0.f, 0.f, 0.f};
+                        mma_bf16(t4, q0, bx[nt].x, bx[nt].y, t4);
+                        mma_bf16(t4, q1, bx[nt].z, bx[nt].w, t4);
+                        scale_acc(acc[nt], t4, tr.sc[kb]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&emptyG[sl]);  // this warp is done with the slot
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) gus[((warp * NT + nt) * 4 + r) * 32 + lane] = acc[nt][r];
+            unit_weights(i);
+            const int hb3 = i % 3;
+            // before writing the peer's copy of buffer hb3: the peer is done with unit i - 3
+            if (tid == 0 && i >= 3) pair_wait(&hempty[hb3], (uint32_t)((i - 3) / 3) & 1u, a);
+            cyc_add(2, c0);
+            c0 = cyc();
+            consumer_sync();
+            // h rows (2mp, 2mp + 1) of this CTA's 64 and token n -> both CTAs' h buffer
+            const uint32_t peer_full = peer_addr(&hfull[hb3], rank ^ 1u);
+            for (int id = tid; id < 32 * T; id += kConsumers) {
+                const int mp = id & 31, n = id >> 5;
+                const int qt2 = mp >> 3, nt = n >> 3;
+                float hv[2];
+#pragma unroll
+                for (int e2 = 0; e2 < 2; ++e2) {
+                    const int m = 2 * (mp & 7) + e2;  // row within the 16-row tile
+                    const int rr = 2 * (m >> 3) + (n & 1), ln = 4 * (m & 7) + ((n & 7) >> 1);
+                    const float gv = gus[(((2 * qt2 + 0) * NT + nt) * 4 + rr) * 32 + ln];
+                    const float uv = gus[(((2 * qt2 + 1) * NT + nt) * 4 + rr) * 32 + ln];
+                    hv[e2] = silu(gv) * uv;
+                }
+                const __half2 h2 = __floats2half2_rn(hv[0], hv[1]);
+                const uint32_t hw = *reinterpret_cast<const uint32_t*>(&h2);
+                const int rl = 64 * (int)rank + 2 * mp;  // chunk-local row (even)
+                uint16_t* dst = hb + (hb3 * T + n) * kHRow + (rl & ~31) + perm32(rl & 31);
+                *reinterpret_cast<uint32_t*>(dst) = hw;
+                st_async_remote(peer_addr(dst, rank ^ 1u), hw, peer_full);
+            }
+            // arm this CTA's barrier for the peer's 32 * T stores (their completion may come first)
+            if (tid == 0) mbar_arrive_expect_tx(&hfull[hb3], 128u * (uint32_t)T);
+            consumer_sync();  // this CTA's own h rows are in place for its down step
+            cyc_add(3, c0);
+        };
+
+        // ---- down of unit i: the chunk's 128 h values times this CTA's d/2 down rows
+        auto down = [&](int i) {
+            const int hb3 = i % 3;
+            unsigned long long c0 = cyc();
+            pair_wait(&hfull[hb3], (uint32_t)(i / 3) & 1u, a);
+            int e, j, s;
+            unit_expert(i, e, j, s);
+            const uint32_t mask = s_mask[i & 1];
+            const int slot = s_slot[i & 1];
+            const uint16_t* hbuf = hb + hb3 * T * kHRow;
+            const int di0 = 2 * i;
+            copy_wait(&fullD[di0 % a.nd], (uint32_t)(di0 / a.nd) & 1u, a);
+            copy_wait(&fullD[(di0 + 1) % a.nd], (uint32_t)((di0 + 1) / a.nd) & 1u, a);
+            cyc_add(4, c0);
+            c0 = cyc();
+            for (int qi = 0; qi < 2; ++qi) {
+                const int di = di0 + qi;
+                const uint8_t* dc = dring + (size_t)(di % a.nd) * a.d_bytes;
+                const uint8_t* ds = dc + (size_t)RTI * DCB;
+                const int rt0 = (int)rank * (RT / 2) + qi * RTI;
+#pragma unroll 2
+                for (int lt = warp; lt < RTI; lt += kCWarps) {
+                    TileRegs<BD> td;
+                    load_tile_smem<BD>(dc + lt * DCB, ds + lt * 128, lane, td);
+                    float acc[NT][4];
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) acc[nt][r] = 0.f;
+#pragma unroll
+                    for (int kb = 0; kb < 4; ++kb) {
+                        uint4 bh[NT];
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            const int tok = nt * 8 + g;
+                            bh[nt] = tok < T ? *reinterpret_cast<const uint4*>(hbuf + tok * kHRow + kb * 32 + 8 * c)
+                                             : make_uint4(0, 0, 0, 0);
+                        }
+                        uint32_t qq[8];
+                        decode_any<true, BD>(td.lo[kb], td.hi[kb], qq);
+                        const uint32_t q0[4] = {qq[0], qq[1], qq[2], qq[3]}, q1[4] = {qq[4], qq[5], qq[6], qq[7]};
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            float t4[4] = {0.f, 0.f, 0.f, 0.f};
+                            mma_f16(t4, q0, bh[nt].x, bh[nt].y, t4);
+                            mma_f16(t4, q1, bh[nt].z, bh[nt].w, t4);
+                            scale_acc(acc[nt], t4, td.sc[kb]);
+                        }
+                    }
+                    // partial sums of (token t, slot, chunk j) for output rows n, n + 8
+                    const int n = (rt0 + lt) * 16 + g;
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            const int t = nt * 8 + 2 * c + (r & 1);
+                            if (t < T && ((mask >> t) & 1u)) {
+                                // the shared expert comes first in every token's list; the
+                                // routed slots' places exist once the schedule is built
+                                const int pl = slot < ns ? 0 : pos[slot * T + t];
+                                if (pl < KS) {
+                                    const int64_t row = ((int64_t)t * KS + pl) * FC + j;
+                                    a.part[row * d + n + 8 * (r >> 1)] = s_w[i & 1][t] * acc[nt][r];
+                                } else {
+                                    flag_status(a.status, kStatusBounds);
+                                }
+                            }
+                        }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&emptyD[di0 % a.nd]);
+                mbar_arrive(&emptyD[(di0 + 1) % a.nd]);
+            }
+            cyc_add(5, c0);
+            consumer_sync();  // every warp is done with h buffer hb3: the peer may refill it
+            if (tid == 0) mbar_arrive_relaxed_remote(peer_addr(&hempty[hb3], rank ^ 1u));
+        };
+
+        // ---- shared-expert units, overlapping the router hand-off
+        for (int i = 0; i < n_pre; ++i) {
+            gate_up(i);
+            down(i);
+        }
+        trace(2);
+
+        // ---- 2. every CTA's router rows, then top-k and the schedule
+        if (tid == 0) grid_wait(a.ctr, router_target, a);
+        consumer_sync();
+        trace(3);
+        const unsigned long long ctk = cyc();
+        for (int t = warp; t < T; t += kCWarps) {
+            const double* lg = a.logits64 + (int64_t)t * E;
+            int id;
+            float wt;
+            if (E <= 512)
+                topk_token<16>(lg, E, k, lane, cand + warp * 64, id, wt);
+            else
+                topk_token<32>(lg, E, k, lane, cand + warp * 64, id, wt);
+            if (lane < k) {
+                sids[t * k + lane] = id;
+                sw[t * k + lane] = wt;
+                if (b == 0) {
+                    a.ids[(int64_t)t * k + lane] = id;
+                    a.w[(int64_t)t * k + lane] = wt;
+                }
+            }
+        }
+        cyc_add(6, ctk);
+        consumer_sync();
+        trace(4);
+        for (int p = tid; p < T * k; p += kConsumers) {
+            const int e = sids[p], t = p / k, r = p - t * k;
+            if (e >= 0 && e < E) {
+                atomicOr(&emask[e], 1u << t);
+                atomicMin(&ebest[e], r);
+            } else {
+                flag_status(a.status, kStatusBounds);
+            }
+        }
+        consumer_sync();
+        {
+            // kept experts in ascending order: warp w owns a contiguous chunk
+            const int chunk = ((E + kCWarps - 1) / kCWarps + 31) & ~31;
+            const int e0 = warp * chunk, e1 = min(E, e0 + chunk);
+            auto keep = [&](int e) {
+                return e < e1 && emask[e] != 0u && !(a.skip_rank > 0 && ebest[e] >= a.skip_rank) &&
+                       e >= a.e_begin && e < a.e_end;
+            };
+            int cnt = 0;
+            for (int base = e0; base < e1; base += 32) cnt += __popc(__ballot_sync(0xffffffffu, keep(base + lane)));
+            if (lane == 0) s_wcnt[warp] = cnt;
+            consumer_sync();
+            int p0 = ns;
+            for (int w = 0; w < warp; ++w) p0 += s_wcnt[w];
+            for (int base = e0; base < e1; base += 32) {
+                const bool kp = keep(base + lane);
+                const unsigned bal = __ballot_sync(0xffffffffu, kp);
+                if (kp) slot_e[p0 + __popc(bal & ((1u << lane) - 1u))] = base + lane;
+                p0 += __popc(bal);
+            }
+            if (tid == 0) {
+                int tot = ns;
+                for (int w = 0; w < kCWarps; ++w) tot += s_wcnt[w];
+                s_nslots = tot;
+            }
+            consumer_sync();
+        }
+        const int n_slots = s_nslots;
+        // place of each slot in its tokens' lists (slot order): the partial sums' row index
+        if (tid < T) {
+            int r = 0;
+            for (int s = 0; s < n_slots; ++s) {
+                const uint32_t m = s < ns ? 0xFFFFFFFFu : emask[slot_e[s]];
+                if ((m >> tid) & 1u) pos[s * T + tid] = (unsigned char)r++;
+            }
+            tn[tid] = r;
+        }
+        if (tid == 0) {
+            const int U = n_slots * FC;
+            const int nu = U > q ? (U - 1 - q) / nc + 1 : 0;
+            s_nunits = max(nu, n_pre);
+            if (b == 0) {
+                int big = 0;
+                for (int s2 = ns; s2 < n_slots; ++s2) big = max(big, __popc(emask[slot_e[s2]]));
+                a.meta->n_active = n_slots - ns;
+                a.meta->max_count = big;
+                a.meta->n_fixup = 0;  // the fp64 logits are ranked exactly
+            }
+        }
+        consumer_sync();
+        if (tid == 0) mbar_arrive(&sched);  // the producer may issue the routed units
+        const int n_units = s_nunits;
+        cyc_add(7, ctk);
+        trace(5);
+
+        // ---- 3. routed units, pipelined: gate/up of unit i, then the down of unit i - 1
+        for (int i = n_pre; i < n_units; ++i) {
+            gate_up(i);
+            trace(6 + 2 * min(i - n_pre, 15));
+            if (i > n_pre) down(i - 1);
+        }
+        if (n_units > n_pre) down(n_units - 1);
+        trace(38);
+
+        // ---- 4. every CTA's partial sums, then this CTA's slice of y
+        consumer_sync();
+        if (tid == 0) grid_wait(a.ctr + 1, grid_arrive(a.ctr + 1, true), a);
+        consumer_sync();
+        trace(39);
+        {
+            // output quads (t, n..n+3); a half-warp per quad, lane `sub` summing
+            // contributions sub, sub + 16, ... in order, then a fixed-order tree
+            const int NG4 = T * (d / 4);
+            const int g0 = (int)((int64_t)b * NG4 / G), g1 = (int)((int64_t)(b + 1) * NG4 / G);
+            const int sub = lane & 15;
+            for (int base = g0 + 2 * warp; base < g1; base += 2 * kCWarps) {  // warp-uniform trip count
+                const int gq = base + (lane >> 4);
+                const bool valid = gq < g1;
+                const int t = valid ? gq / (d / 4) : 0, n = valid ? 4 * (gq - t * (d / 4)) : 0;
+                const int ncon = valid ? tn[t] * FC : 0;
+                const float* pr = a.part + (int64_t)t * KS * FC * d + n;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int cc = sub; cc < ncon; cc += 16) {
+                    const float4 v = __ldcg(reinterpret_cast<const float4*>(pr + (int64_t)cc * d));
+                    acc.x += v.x;
+                    acc.y += v.y;
+                    acc.z += v.z;
+                    acc.w += v.w;
+                }
+#pragma unroll
+                for (int o = 8; o > 0; o >>= 1) {
+                    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+                    acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+                    acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+                    acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+                }
+                if (valid && sub == 0) {
+                    if (a.out_fp32) {
+                        float4* y4 = reinterpret_cast<float4*>(static_cast<float*>(a.y) + (int64_t)t * d + n);
+                        if (a.accumulate) {
+                            const float4 yi = *y4;
+                            acc.x += yi.x;
+                            acc.y += yi.y;
+                            acc.z += yi.z;
+                            acc.w += yi.w;
+                        }
+                        *y4 = acc;
+                    } else {
+                        uint2* y2 = reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.y) + (int64_t)t * d + n);
+                        if (a.accumulate) {
+                            const uint2 yi = *y2;
+                            acc.x += __uint_as_float(yi.x << 16);
+                            acc.y += __uint_as_float(yi.x & 0xFFFF0000u);
+                            acc.z += __uint_as_float(yi.y << 16);
+                            acc.w += __uint_as_float(yi.y & 0xFFFF0000u);
+                        }
+                        const __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x, acc.y);
+                        const __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z, acc.w);
+                        uint2 out;
+                        out.x = *reinterpret_cast<const uint32_t*>(&lo2);
+                        out.y = *reinterpret_cast<const uint32_t*>(&hi2);
+                        *y2 = out;
+                    }
+                }
+            }
+        }
+        trace(40);
+    }
+    // every thread of both CTAs: no remote access is still in flight when a CTA exits
+    cluster_arrive();
+    cluster_wait();
+}
+
+// ---------------------------------------------------------------- launcher
+static size_t round128(size_t n) { return (n + 127) & ~size_t(127); }
+
+struct Layout {
+    int ng, nd, g_bytes, d_bytes;
+    int off_x, off_h, off_gus, off_cand, off_route, off_emask, off_slots, off_pos, off_g, off_d;
+    size_t total;
+};
+
+// Shared memory: staged x | h buffers | gate/up outputs | top-k candidates |
+// routing | expert masks | slot list | slot places | gate/up ring | down ring.
+// The rings take what is left of the per-CTA limit, two thirds of it for
+// gate/up items.  Items are issued in order (G0..G3, D0, D1 of each unit) and
+// the down of unit i runs after the gate/up of unit i + 1, so the down ring
+// needs two slots for the gate/up items of unit i + 1 to be issued in time.
+static bool make_layout(int BG, int BD, int NT, int T, int d, int f, int E, int k, int smem_max, Layout* L) {
+    const int KT = d / 128, RTI = d / 64;
+    const int maxS = std::min(T * k, E) + 1;
+    (void)f;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += round128(bytes);
+        return (int)o;
+    };
+    L->off_x = take((size_t)T * (d + kXPad) * 2);
+    L->off_h = take((size_t)3 * T * kHRow * 2);
+    L->off_gus = take(std::max((size_t)kCWarps * NT * 4 * 32 * 4, (size_t)kCWarps * 16 * 8));
+    L->off_cand = take((size_t)kCWarps * kCandBytes);
+    L->off_route = take((size_t)T * k * 8);
+    L->off_emask = take((size_t)E * 8);
+    L->off_slots = take((size_t)maxS * 4);
+    L->off_pos = take(64 + (size_t)maxS * T);  // token counts [16], then the places
+    L->g_bytes = 2 * KT * (256 * BG + 128);
+    L->d_bytes = RTI * (256 * BD + 128);
+    const long avail = (long)smem_max - (long)off;
+    if (avail < (long)(L->g_bytes + 2 * L->d_bytes)) return false;
+    int ng = std::max(1, (int)((avail * 2 / 3) / L->g_bytes));
+    ng = std::min(ng, kMaxSlots);
+    int nd = (int)((avail - (long)ng * L->g_bytes) / L->d_bytes);
+    if (nd < 2) {
+        ng = (int)((avail - 2L * L->d_bytes) / L->g_bytes);
+        nd = 2;
+    }
+    nd = std::min(nd, kMaxSlots);
+    if (ng < 1) return false;
+    L->ng = ng;
+    L->nd = nd;
+    L->off_g = take((size_t)ng * L->g_bytes);
+    L->off_d = take((size_t)nd * L->d_bytes);
+    L->total = off;
+    return true;
+}
+
+struct Occ {
+    int dev;
+    const void* fn;
+    size_t smem;
+    int clusters;
+};
+
+template <int BG, int BD, int NT>
+static cudaError_t launch_t(const DecodeLaunch& L, cudaStream_t st) {
+    auto kern = decode_pair_kernel<BG, BD, NT>;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int smem_max = 0;
+    e = cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    // static shared memory of the kernel (barriers and a few words) comes off the limit
+    Layout lay;
+    if (!make_layout(BG, BD, NT, L.T, L.d, L.f, L.E, L.k, smem_max - 1024, &lay)) return cudaErrorInvalidConfiguration;
+
+    static std::mutex mu;
+    static std::vector<Occ> cache;
+    int clusters = 0;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        for (const Occ& o : cache)
+            if (o.dev == dev && o.fn == (const void*)kern && o.smem == lay.total) clusters = o.clusters;
+        if (clusters == 0) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total);
+            if (e != cudaSuccess) return e;
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = kCS;
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.gridDim = dim3(kCS);
+            cfg.blockDim = dim3(kThreads);
+            cfg.dynamicSmemBytes = lay.total;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+            if (e != cudaSuccess) return e;
+            if (clusters < 1) return cudaErrorInvalidConfiguration;
+            cache.push_back({dev, (const void*)kern, lay.total, clusters});
+        }
+    }
+
+    Args a;
+    a.T = L.T;
+    a.d = L.d;
+    a.f = L.f;
+    a.E = L.E;
+    a.k = L.k;
+    a.n_shared = L.n_shared;
+    a.x = static_cast<const uint16_t*>(L.x);
+    a.y = L.y;
+    a.out_fp32 = L.out_fp32;
+    a.accumulate = L.accumulate;
+    a.codes = L.codes;
+    a.scales = L.scales;
+    a.code_stride = (int64_t)L.f * L.d * (2 * BG + BD) / 8;
+    a.scale_stride = (int64_t)3 * L.f * L.d / 32;
+    a.wr = static_cast<const uint16_t*>(L.wr);
+    a.bias = L.bias;
+    a.logits64 = L.logits64;
+    a.ids = L.ids;
+    a.w = L.w;
+    a.meta = L.meta;
+    a.status = L.status;
+    a.part = L.part;
+    a.ctr = L.ctr;
+    a.skip_rank = L.skip_rank;
+    a.e_begin = std::max(0, L.e_begin);
+    a.e_end = std::min(L.E, L.e_end);
+    a.nc = clusters;
+    a.spin_limit = L.spin_limit;
+    a.withhold = L.withhold;
+    a.ng = lay.ng;
+    a.nd = lay.nd;
+    a.g_bytes = lay.g_bytes;
+    a.d_bytes = lay.d_bytes;
+    a.off_x = lay.off_x;
+    a.off_h = lay.off_h;
+    a.off_gus = lay.off_gus;
+    a.off_cand = lay.off_cand;
+    a.off_route = lay.off_route;
+    a.off_emask = lay.off_emask;
+    a.off_slots = lay.off_slots;
+    a.off_pos = lay.off_pos;
+    a.off_g = lay.off_g;
+    a.off_d = lay.off_d;
+
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = kCS;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeCooperative;
+    at[1].val.cooperative = 1;
+    cfg.gridDim = dim3(kCS * clusters);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = lay.total;
+    cfg.stream = st;
+    cfg.attrs = at;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, kern, a, *L.down_codes_map, *L.down_scales_map);
+    if (e == cudaSuccess) return e;
+    // A cooperative launch can be refused where the grid is still co-resident in
+    // practice (a profiler replaying the kernel): launch the same clusters
+    // without the guarantee.  Should they not all be resident, the bounded
+    // waits report MOE_ERR_TIMEOUT instead of hanging.
+    (void)cudaGetLastError();
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a, *L.down_codes_map, *L.down_scales_map);
+}
+
+template <int BG, int BD>
+static cudaError_t launch_bits(const DecodeLaunch& L, cudaStream_t s) {
+    return L.T <= 8 ? launch_t<BG, BD, 1>(L, s) : launch_t<BG, BD, 2>(L, s);
+}
+
+template <int BG>
+static cudaError_t launch_gu(const DecodeLaunch& L, cudaStream_t s) {
+    switch (L.bits_down) {
+        case 2: return launch_bits<BG, 2>(L, s);
+        case 3: return launch_bits<BG, 3>(L, s);
+        case 4: return launch_bits<BG, 4>(L, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace pair
+
+#ifdef MOE_PAIR_TRACE
+extern "C" int moe_debug_pair_trace(unsigned long long* host, int n) {
+    return cudaMemcpyFromSymbol(host, pair::g_trace, sizeof(unsigned long long) * (size_t)n) == cudaSuccess ? 0 : 2;
+}
+extern "C" int moe_debug_pair_cycles(unsigned long long* host, int n) {  // [1024][32]
+    return cudaMemcpyFromSymbol(host, pair::g_cyc, sizeof(unsigned long long) * (size_t)n) == cudaSuccess ? 0 : 2;
+}
+#endif
+
+size_t pair_part_floats(int max_tokens, int k, int n_shared, int d, int f) {
+    return (size_t)std::min(max_tokens, kPairMaxTokens) * (size_t)(k + n_shared) * (size_t)(f / 128) * (size_t)d;
+}
+
+bool pair_decode_supported(const DecodeLaunch& L) {
+    if (!L.down_codes_map || !L.down_scales_map || !L.part) return false;
+    int smem_max = 232448;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        (void)cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    pair::Layout lay;
+    const int bd = L.bits_down ? L.bits_down : L.bits;
+    return L.T >= 1 && L.T <= kPairMaxTokens && L.E <= 1024 && L.k <= 32 && L.d % 128 == 0 && L.f % 128 == 0 &&
+           pair::make_layout(L.bits, bd, L.T <= 8 ? 1 : 2, L.T, L.d, L.f, L.E, L.k, smem_max - 1024, &lay);
+}
+
+cudaError_t launch_decode_pair(const DecodeLaunch& L, cudaStream_t s) {
+    if (!pair_decode_supported(L)) return cudaErrorInvalidValue;
+    DecodeLaunch M = L;
+    if (!M.bits_down) M.bits_down = M.bits;
+    switch (M.bits) {
+        case 2: return pair::launch_gu<2>(M, s);
+        case 3: return pair::launch_gu<3>(M, s);
+        case 4: return pair::launch_gu<4>(M, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace moe

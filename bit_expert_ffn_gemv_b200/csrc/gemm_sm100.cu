@@ -854,6 +854,42 @@ cudaError_t make_weight_maps(GemmMaps* m, const void* codes, const void* scales,
                      CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+// Maps of the down matrices for the clustered decode kernel: a 3-D view
+// (super-tile words, 16-row tile, expert) of every expert's down codes and
+// scales, any code widths.  One box = RTI row tiles x one super-tile column,
+// so a kernel fetches the 128 input columns [128j, 128j + 128) of RTI
+// consecutive row tiles with one instruction per map.
+static cudaError_t encode_3d(CUtensorMap* map, CUtensorMapDataType type, int elem_bytes, const void* base,
+                             const cuuint64_t (&dims)[3], const cuuint64_t (&strides_bytes)[2], const cuuint32_t (&box)[3]) {
+    Encode encode = encoder();
+    if (!encode) return cudaErrorNotSupported;
+    (void)elem_bytes;
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = encode(map, type, 3, const_cast<void*>(base), dims, strides_bytes, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_pair_down_maps(CUtensorMap* codes_map, CUtensorMap* scales_map, const void* codes,
+                                const void* scales, int n_experts_total, int d, int f, int bits, int bits_down) {
+    const int FC = f / 128, RT = d / 16, RTI = d / 64;
+    if (RTI < 1 || RTI > 256) return cudaErrorInvalidValue;
+    const int64_t mg = (int64_t)f * d * bits / 8, msc = (int64_t)f * d / 32;
+    const int64_t code_stride = (int64_t)f * d * (2 * bits + bits_down) / 8;
+    const cuuint64_t cdims[3] = {(cuuint64_t)FC * 64 * bits_down, (cuuint64_t)RT, (cuuint64_t)n_experts_total};
+    const cuuint64_t cstr[2] = {(cuuint64_t)FC * 256 * bits_down, (cuuint64_t)code_stride};
+    const cuuint32_t cbox[3] = {(cuuint32_t)(64 * bits_down), (cuuint32_t)RTI, 1};
+    cudaError_t e = encode_3d(codes_map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4,
+                              static_cast<const uint8_t*>(codes) + 2 * mg, cdims, cstr, cbox);
+    if (e != cudaSuccess) return e;
+    const cuuint64_t sdims[3] = {(cuuint64_t)FC * 64, (cuuint64_t)RT, (cuuint64_t)n_experts_total};
+    const cuuint64_t sstr[2] = {(cuuint64_t)FC * 128, (cuuint64_t)(3 * msc * 2)};
+    const cuuint32_t sbox[3] = {64, (cuuint32_t)RTI, 1};
+    return encode_3d(scales_map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, static_cast<const uint16_t*>(scales) + 2 * msc,
+                     sdims, sstr, sbox);
+}
+
 cudaError_t launch_router_gemm(const RouteArgs& a, uint32_t* status, cudaStream_t s) {
     const int smem = kRouterStages * kRouterStage + 1024;
     cudaError_t e = cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -97,9 +97,26 @@ struct DecodeLaunch {
     int* sync;  // zeroed once; the kernel leaves it zeroed
     int skip_rank = 0;  // route-tail skip: drop experts whose best rank in the batch is >= this (0: off)
     int e_begin = 0, e_end = 1 << 30;  // experts outside [e_begin, e_end) are dropped (expert parallelism)
+    // the clustered kernel (launch_decode_pair)
+    int bits_down = 0;                // code width of the down matrices (0: bits)
+    float* part = nullptr;            // [T x (k + n_shared) x f/128 x d] partial sums (pair_part_floats)
+    unsigned long long* ctr = nullptr;  // [kPairCounters] monotonic counters, zero once
+    uint32_t spin_limit = 1u << 21;   // polls before a bounded wait gives up
+    int withhold = -1;                // test only: this CTA never announces its router rows
+    const CUtensorMap* down_codes_map = nullptr;   // make_pair_down_maps of the layer
+    const CUtensorMap* down_scales_map = nullptr;
 };
 cudaError_t launch_decode(const DecodeLaunch& L, cudaStream_t s);
 size_t decode_sync_words(int max_tokens, int E, int d);
+// Whole layer for up to kPairMaxTokens tokens: 74 clusters of two CTAs, one
+// grid-wide hand-off (decode_pair.cu).  Any code widths.
+constexpr int kPairMaxTokens = 16;
+constexpr int kPairCounters = 8;
+bool pair_decode_supported(const DecodeLaunch& L);
+size_t pair_part_floats(int max_tokens, int k, int n_shared, int d, int f);
+cudaError_t make_pair_down_maps(CUtensorMap* codes_map, CUtensorMap* scales_map, const void* codes,
+                                const void* scales, int n_experts_total, int d, int f, int bits, int bits_down);
+cudaError_t launch_decode_pair(const DecodeLaunch& L, cudaStream_t s);
 
 cudaError_t launch_router_norms(const void* wr, int E, int d, float* out, cudaStream_t s);
 cudaError_t launch_router_logits(const RouteArgs& a, cudaStream_t s);

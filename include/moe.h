@@ -103,9 +103,9 @@ typedef struct {
 /* forward flags */
 #define MOE_OUT_FP32 0x1u   /* y is fp32 [T x d] (default: bf16) */
 #define MOE_ACCUMULATE 0x2u /* y += layer output (default: y = layer output) */
-/* Path selection (default: the fused persistent kernel for T <= 16, the
+/* Path selection (default: the fused decode kernel for T <= 16, the
  * tensor-core grouped-GEMM path above -- the measured crossover). */
-#define MOE_FORCE_GEMV 0x4u /* CUDA-core paths: the fused kernel up to 64 tokens, grouped GEMV above */
+#define MOE_FORCE_GEMV 0x4u /* CUDA-core paths: a fused kernel up to 64 tokens, grouped GEMV above */
 #define MOE_FORCE_GEMM 0x8u /* the tensor-core grouped-GEMM path whatever T is */
 #define MOE_FORCE_UNFUSED 0x10u /* one kernel per step (grouped GEMV) instead of the fused persistent kernel */
 /*
@@ -272,6 +272,19 @@ moe_status moe_check_status(moe_handle* h);
  * with_shared not 0 or 1).
  */
 moe_status moe_set_expert_range(moe_handle* h, int32_t begin, int32_t end, int32_t with_shared);
+
+/*
+ * Test hook for the device watchdog (no counterpart in the pages): from now
+ * on the fused decode kernels give up a device-side wait after `spins` polls
+ * (default 2^21, about half a second) instead of waiting on, and, when
+ * withhold_cta >= 0, that CTA of the clustered decode kernel never announces
+ * its router rows, so that every other CTA's wait for them runs out.  The
+ * forward then reports MOE_ERR_TIMEOUT through moe_check_status, which also
+ * resets the kernels' counters so that the handle computes correctly again
+ * once the hook is off (withhold_cta = -1).  Nothing traps or hangs.
+ * Errors: INVALID_ARG (NULL handle, spins = 0, withhold_cta < -1).
+ */
+moe_status moe_debug_wait_limit(moe_handle* h, uint32_t spins, int32_t withhold_cta);
 
 /* Counters (moe_get_stats). */
 typedef struct {
