@@ -52,7 +52,7 @@ class MoeConfig(ctypes.Structure):
 
 class MoeStats(ctypes.Structure):
     _fields_ = [("fixup_tokens", ctypes.c_int64), ("active_experts", ctypes.c_int64), ("max_group", ctypes.c_int64),
-                ("launches", ctypes.c_int64)]
+                ("launches", ctypes.c_int64), ("cuda_error", ctypes.c_int64)]
 
 
 MOE_KERNEL_COUNT = 12

@@ -68,6 +68,7 @@ struct moe_handle {
     int32_t ep_begin = 0, ep_end = 1 << 30, ep_shared = 1;
     // launch accounting and optional per-kernel event timing
     int64_t launches = 0;
+    int last_cuda_error = 0;  // cudaError_t of the last failed CUDA call (moe_stats.cuda_error)
     bool prof_on = false;
     std::vector<cudaEvent_t> ev;    // pairs (start, stop)
     std::vector<int> ev_kernel;     // kernel id of each recorded pair
@@ -100,7 +101,11 @@ moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_E
 template <class F>
 cudaError_t run(moe_handle* h, int kernel, cudaStream_t s, F&& f) {
     h->launches++;
-    if (!h->prof_on) return f();
+    if (!h->prof_on) {
+        const cudaError_t e = f();
+        if (e != cudaSuccess) h->last_cuda_error = (int)e;
+        return e;
+    }
     const size_t i = 2 * h->ev_kernel.size();
     while (h->ev.size() < i + 2) {
         cudaEvent_t e;
@@ -110,7 +115,10 @@ cudaError_t run(moe_handle* h, int kernel, cudaStream_t s, F&& f) {
     cudaError_t e = cudaEventRecord(h->ev[i], s);
     if (e != cudaSuccess) return e;
     e = f();
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+        h->last_cuda_error = (int)e;
+        return e;
+    }
     e = cudaEventRecord(h->ev[i + 1], s);
     h->ev_kernel.push_back(kernel);
     return e;
@@ -629,6 +637,7 @@ moe_status moe_get_stats(moe_handle* h, moe_stats* out) {
     out->active_experts = m.n_active;
     out->max_group = m.max_count;
     out->launches = h->launches;
+    out->cuda_error = h->last_cuda_error;
     return MOE_OK;
 }
 

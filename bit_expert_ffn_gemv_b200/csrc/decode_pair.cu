@@ -1076,6 +1076,13 @@ struct Occ {
     size_t smem;
     int clusters;
 };
+// The dynamic shared-memory limit is one setting per kernel and device: it is
+// raised to the largest size any launch needed and never lowered.
+struct SmemAttr {
+    int dev;
+    const void* fn;
+    size_t smem;
+};
 
 template <int BG, int BD, int NT>
 static cudaError_t launch_t(const DecodeLaunch& L, cudaStream_t st) {
@@ -1092,14 +1099,24 @@ static cudaError_t launch_t(const DecodeLaunch& L, cudaStream_t st) {
 
     static std::mutex mu;
     static std::vector<Occ> cache;
+    static std::vector<SmemAttr> attrs;
     int clusters = 0;
     {
         std::lock_guard<std::mutex> lk(mu);
+        SmemAttr* at_set = nullptr;
+        for (SmemAttr& s2 : attrs)
+            if (s2.dev == dev && s2.fn == (const void*)kern) at_set = &s2;
+        if (!at_set || at_set->smem < lay.total) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total);
+            if (e != cudaSuccess) return e;
+            if (at_set)
+                at_set->smem = lay.total;
+            else
+                attrs.push_back({dev, (const void*)kern, lay.total});
+        }
         for (const Occ& o : cache)
             if (o.dev == dev && o.fn == (const void*)kern && o.smem == lay.total) clusters = o.clusters;
         if (clusters == 0) {
-            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)lay.total);
-            if (e != cudaSuccess) return e;
             cudaLaunchConfig_t cfg = {};
             cudaLaunchAttribute at[1];
             at[0].id = cudaLaunchAttributeClusterDimension;

@@ -294,6 +294,8 @@ typedef struct {
                                the expert range dropped) */
     int64_t max_group;      /* largest expert group of the last moe_forward */
     int64_t launches;       /* kernels this handle has launched since moe_layer_init */
+    int64_t cuda_error;     /* the cudaError_t of the last CUDA call of this handle that failed
+                               (0 if none): the detail behind a MOE_ERR_CUDA */
 } moe_stats;
 
 /* Synchronise the device and read the counters. */
