@@ -69,6 +69,7 @@ constexpr int kMaxSlots = 16;              // ring slots of each kind (upper bou
 constexpr int kXPad = 32;                  // 16-bit elements of padding per staged row
 constexpr int kHRow = 128 + kXPad;
 constexpr int kCandBytes = 64 * 16;        // per-warp top-k candidate buffer
+constexpr int kMaxKS = 2;                  // input super-tiles per warp of a gate/up tile (d <= 2048)
 
 // Optional phase trace (build with -DMOE_PAIR_TRACE): thread 0 of every CTA
 // records the global timer at phase boundaries and adds clock64() differences
@@ -362,6 +363,7 @@ MOE_DEV void topk_scan(const double* lg, int E, int k, int lane, int& sel, doubl
 // its weight w_r = softmax over the k selected logits.
 template <int KPL>
 MOE_DEV void topk_token(const double* lg, int E, int k, int lane, Cand* cand, int& id_out, float& w_out) {
+    unsigned long long tc = cyc();
     double v[KPL];
     uint32_t key[KPL];
 #pragma unroll
@@ -373,6 +375,8 @@ MOE_DEV void topk_token(const double* lg, int E, int k, int lane, Cand* cand, in
         key[j] = e < E ? key32(v[j], e) : 0u;
         lmax = max(lmax, key[j]);
     }
+    cyc_add(10, tc);  // loads + keys
+    tc = cyc();
     int rk = 0;  // lanes whose largest key beats mine
 #pragma unroll
     for (int o = 1; o < 32; ++o) rk += __shfl_sync(0xffffffffu, lmax, (lane + o) & 31) > lmax ? 1 : 0;
@@ -384,6 +388,8 @@ MOE_DEV void topk_token(const double* lg, int E, int k, int lane, Cand* cand, in
     const int C = (int)__reduce_add_sync(0xffffffffu, (unsigned)cnt);
     int sel = -1;
     double lsel = 0.0, top = 0.0;
+    cyc_add(11, tc);  // threshold + count
+    tc = cyc();
     if (src >= 0 && C >= k && C <= 32) {
         int off = 0;
 #pragma unroll
@@ -398,6 +404,8 @@ MOE_DEV void topk_token(const double* lg, int E, int k, int lane, Cand* cand, in
             off += __popc(bal);
         }
         __syncwarp();
+        cyc_add(12, tc);  // compaction
+        tc = cyc();
         int rank = 0, my_e = 0;
         double my_v = 0.0;
         if (lane < C) {
@@ -423,13 +431,17 @@ MOE_DEV void topk_token(const double* lg, int E, int k, int lane, Cand* cand, in
         __syncwarp();
     } else {
         topk_scan(lg, E, k, lane, sel, lsel, top);
+        cyc_add(15, tc);  // slow path taken
     }
+    cyc_add(13, tc);  // ranking
+    tc = cyc();
     const float ex = lane < k ? expf((float)(lsel - top)) : 0.0f;
     float z = ex;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
     id_out = sel;
     w_out = lane < k ? ex / z : 0.0f;
+    cyc_add(14, tc);  // weights
 }
 
 MOE_DEV double bf16_to_f64(uint32_t bits16) { return (double)__uint_as_float(bits16 << 16); }
@@ -478,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int i = 0; i < a.ng; ++i) {
             mbar_init(&fullG[i], 1);
-            mbar_init(&emptyG[i], 2);  // the gate warp and the up warp of its row tile
+            mbar_init(&emptyG[i], kCWarps);  // every warp reads its slice of every item
         }
         for (int i = 0; i < a.nd; ++i) {
             mbar_init(&fullD[i], 1);
@@ -677,88 +689,119 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         };
 
-        // ---- gate/up of unit i: warp w computes 16-row tile w/2 of gate (w even) or up (w odd)
+        // ---- gate/up of unit i, one 16-row tile at a time: warp w adds its
+        // slice of the input dimension for gate and up, the CTA sums the slices
+        // and writes the tile's h rows into both CTAs' h buffer.
         auto gate_up = [&](int i) {
-            const int qt = warp >> 1, mat = warp & 1;
-            const int gi = 4 * i + qt, sl = gi % a.ng, use = gi / a.ng;
-            unsigned long long c0 = cyc();
-            // With fewer than 4 gate/up slots the previous use of this slot may
-            // belong to other warps of the same unit: wait for its release first,
-            // so that the parity wait below cannot match a phase two behind.
-            if (use > 0) slot_wait(&emptyG[sl], (uint32_t)(use - 1) & 1u, a);
-            copy_wait(&fullG[sl], (uint32_t)use & 1u, a);
-            cyc_add(1, c0);
-            c0 = cyc();
-            const uint8_t* base = gring + (size_t)sl * a.g_bytes + (size_t)mat * KT * (GCB + 128);
-            float acc[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int r = 0; r < 4; ++r) acc[nt][r] = 0.f;
-#pragma unroll 2
-            for (int st = 0; st < KT; ++st) {
-                TileRegs<BG> tr;
-                load_tile_smem<BG>(base + st * GCB, base + KT * GCB + st * 128, lane, tr);
-#pragma unroll
-                for (int kb = 0; kb < 4; ++kb) {
-                    const int k0 = st * 128 + kb * 32 + 8 * c;
-                    uint4 bx[NT];
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const int tok = nt * 8 + g;
-                        bx[nt] = tok < T ? *reinterpret_cast<const uint4*>(xs + tok * xstride + k0)
-                                         : make_uint4(0, 0, 0, 0);
-                    }
-                    uint32_t qq[8];
-                    decode_any<false, BG>(tr.lo[kb], tr.hi[kb], qq);
-                    const uint32_t q0[4] = {qq[0], qq[1], qq[2], qq[3]}, q1[4] = {qq[4], qq[5], qq[6], qq[7]};
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        float t4[4] = {0.f, 0.f, 0.f, 0.f};
-                        mma_bf16(t4, q0, bx[nt].x, bx[nt].y, t4);
-                        mma_bf16(t4, q1, bx[nt].z, bx[nt].w, t4);
-                        scale_acc(acc[nt], t4, tr.sc[kb]);
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&emptyG[sl]);  // this warp is done with the slot
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int r = 0; r < 4; ++r) gus[((warp * NT + nt) * 4 + r) * 32 + lane] = acc[nt][r];
-            unit_weights(i);
             const int hb3 = i % 3;
+            // x fragments of this warp's slice of the input dimension (super-tiles
+            // warp, warp + 8, ...), loaded once and used by all 8 tiles of the unit
+            uint4 xf[kMaxKS][4][NT];
+#pragma unroll
+            for (int js = 0; js < kMaxKS; ++js)
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const int st = warp + kCWarps * js, tok = nt * 8 + g;
+                        xf[js][kb][nt] = (st < KT && tok < T) ? *reinterpret_cast<const uint4*>(
+                                                                    xs + tok * xstride + st * 128 + kb * 32 + 8 * c)
+                                                              : make_uint4(0, 0, 0, 0);
+                    }
+            unit_weights(i);
             // before writing the peer's copy of buffer hb3: the peer is done with unit i - 3
             if (tid == 0 && i >= 3) pair_wait(&hempty[hb3], (uint32_t)((i - 3) / 3) & 1u, a);
-            cyc_add(2, c0);
-            c0 = cyc();
-            consumer_sync();
-            // h rows (2mp, 2mp + 1) of this CTA's 64 and token n -> both CTAs' h buffer
             const uint32_t peer_full = peer_addr(&hfull[hb3], rank ^ 1u);
-            for (int id = tid; id < 32 * T; id += kConsumers) {
-                const int mp = id & 31, n = id >> 5;
-                const int qt2 = mp >> 3, nt = n >> 3;
-                float hv[2];
+            for (int qt = 0; qt < 4; ++qt) {
+                const int gi = 4 * i + qt, sl = gi % a.ng, use = gi / a.ng;
+                unsigned long long c0 = cyc();
+                copy_wait(&fullG[sl], (uint32_t)use & 1u, a);
+                cyc_add(1, c0);
+                c0 = cyc();
+                const uint8_t* gb = gring + (size_t)sl * a.g_bytes;
+                const uint8_t* ub = gb + (size_t)KT * (GCB + 128);
+                float accg[NT][4], accu[NT][4];
 #pragma unroll
-                for (int e2 = 0; e2 < 2; ++e2) {
-                    const int m = 2 * (mp & 7) + e2;  // row within the 16-row tile
-                    const int rr = 2 * (m >> 3) + (n & 1), ln = 4 * (m & 7) + ((n & 7) >> 1);
-                    const float gv = gus[(((2 * qt2 + 0) * NT + nt) * 4 + rr) * 32 + ln];
-                    const float uv = gus[(((2 * qt2 + 1) * NT + nt) * 4 + rr) * 32 + ln];
-                    hv[e2] = silu(gv) * uv;
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) accg[nt][r] = accu[nt][r] = 0.f;
+#pragma unroll
+                for (int js = 0; js < kMaxKS; ++js) {
+                    const int st = warp + kCWarps * js;
+                    if (st < KT) {
+                        TileRegs<BG> tg, tu;
+                        load_tile_smem<BG>(gb + st * GCB, gb + KT * GCB + st * 128, lane, tg);
+                        load_tile_smem<BG>(ub + st * GCB, ub + KT * GCB + st * 128, lane, tu);
+#pragma unroll
+                        for (int kb = 0; kb < 4; ++kb) {
+                            uint32_t qq[8];
+                            decode_any<false, BG>(tg.lo[kb], tg.hi[kb], qq);
+                            {
+                                const uint32_t q0[4] = {qq[0], qq[1], qq[2], qq[3]};
+                                const uint32_t q1[4] = {qq[4], qq[5], qq[6], qq[7]};
+#pragma unroll
+                                for (int nt = 0; nt < NT; ++nt) {
+                                    float t4[4] = {0.f, 0.f, 0.f, 0.f};
+                                    mma_bf16(t4, q0, xf[js][kb][nt].x, xf[js][kb][nt].y, t4);
+                                    mma_bf16(t4, q1, xf[js][kb][nt].z, xf[js][kb][nt].w, t4);
+                                    scale_acc(accg[nt], t4, tg.sc[kb]);
+                                }
+                            }
+                            decode_any<false, BG>(tu.lo[kb], tu.hi[kb], qq);
+                            {
+                                const uint32_t q0[4] = {qq[0], qq[1], qq[2], qq[3]};
+                                const uint32_t q1[4] = {qq[4], qq[5], qq[6], qq[7]};
+#pragma unroll
+                                for (int nt = 0; nt < NT; ++nt) {
+                                    float t4[4] = {0.f, 0.f, 0.f, 0.f};
+                                    mma_bf16(t4, q0, xf[js][kb][nt].x, xf[js][kb][nt].y, t4);
+                                    mma_bf16(t4, q1, xf[js][kb][nt].z, xf[js][kb][nt].w, t4);
+                                    scale_acc(accu[nt], t4, tu.sc[kb]);
+                                }
+                            }
+                        }
+                    }
                 }
-                const __half2 h2 = __floats2half2_rn(hv[0], hv[1]);
-                const uint32_t hw = *reinterpret_cast<const uint32_t*>(&h2);
-                const int rl = 64 * (int)rank + 2 * mp;  // chunk-local row (even)
-                uint16_t* dst = hb + (hb3 * T + n) * kHRow + (rl & ~31) + perm32(rl & 31);
-                *reinterpret_cast<uint32_t*>(dst) = hw;
-                st_async_remote(peer_addr(dst, rank ^ 1u), hw, peer_full);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&emptyG[sl]);  // this warp is done with the slot
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        gus[(((warp * 2 + 0) * NT + nt) * 4 + r) * 32 + lane] = accg[nt][r];
+                        gus[(((warp * 2 + 1) * NT + nt) * 4 + r) * 32 + lane] = accu[nt][r];
+                    }
+                cyc_add(2, c0);
+                c0 = cyc();
+                consumer_sync();
+                // h rows (2m2, 2m2 + 1) of tile qt and token n -> both CTAs' h buffer
+                for (int id = tid; id < 8 * T; id += kConsumers) {
+                    const int m2 = id & 7, n = id >> 3, nt = n >> 3;
+                    float hv[2];
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const int m = 2 * m2 + e2;  // row within the 16-row tile
+                        const int rr = 2 * (m >> 3) + (n & 1), ln = 4 * (m & 7) + ((n & 7) >> 1);
+                        float gsum = 0.f, usum = 0.f;
+#pragma unroll
+                        for (int w = 0; w < kCWarps; ++w) {
+                            gsum += gus[(((w * 2 + 0) * NT + nt) * 4 + rr) * 32 + ln];
+                            usum += gus[(((w * 2 + 1) * NT + nt) * 4 + rr) * 32 + ln];
+                        }
+                        hv[e2] = silu(gsum) * usum;
+                    }
+                    const __half2 h2 = __floats2half2_rn(hv[0], hv[1]);
+                    const uint32_t hw = *reinterpret_cast<const uint32_t*>(&h2);
+                    const int rl = 64 * (int)rank + 16 * qt + 2 * m2;  // chunk-local row (even)
+                    uint16_t* dst = hb + (hb3 * T + n) * kHRow + (rl & ~31) + perm32(rl & 31);
+                    *reinterpret_cast<uint32_t*>(dst) = hw;
+                    st_async_remote(peer_addr(dst, rank ^ 1u), hw, peer_full);
+                }
+                consumer_sync();  // the partial sums may be overwritten by the next tile
+                cyc_add(3, c0);
             }
             // arm this CTA's barrier for the peer's 32 * T stores (their completion may come first)
             if (tid == 0) mbar_arrive_expect_tx(&hfull[hb3], 128u * (uint32_t)T);
-            consumer_sync();  // this CTA's own h rows are in place for its down step
-            cyc_add(3, c0);
         };
 
         // ---- down of unit i: the chunk's 128 h values times this CTA's d/2 down rows
@@ -771,11 +814,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t mask = s_mask[i & 1];
             const int slot = s_slot[i & 1];
             const uint16_t* hbuf = hb + hb3 * T * kHRow;
+            // the h fragments (the same for every down row tile) and, per token of
+            // this lane, the routing weight and the partial-sum row (-1: none)
+            uint4 hf[4][NT];
+            int64_t pbase[NT][2];
+            float wtok[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int tok = nt * 8 + g;
+#pragma unroll
+                for (int kb = 0; kb < 4; ++kb)
+                    hf[kb][nt] = tok < T ? *reinterpret_cast<const uint4*>(hbuf + tok * kHRow + kb * 32 + 8 * c)
+                                         : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int e2 = 0; e2 < 2; ++e2) {
+                    const int t = nt * 8 + 2 * c + e2;
+                    pbase[nt][e2] = -1;
+                    wtok[nt][e2] = 0.f;
+                    if (t < T && ((mask >> t) & 1u)) {
+                        // the shared expert comes first in every token's list; the
+                        // routed slots' places exist once the schedule is built
+                        const int pl = slot < ns ? 0 : pos[slot * T + t];
+                        if (pl < KS) {
+                            pbase[nt][e2] = (((int64_t)t * KS + pl) * FC + j) * d;
+                            wtok[nt][e2] = s_w[i & 1][t];
+                        } else {
+                            flag_status(a.status, kStatusBounds);
+                        }
+                    }
+                }
+            }
             const int di0 = 2 * i;
             copy_wait(&fullD[di0 % a.nd], (uint32_t)(di0 / a.nd) & 1u, a);
             copy_wait(&fullD[(di0 + 1) % a.nd], (uint32_t)((di0 + 1) / a.nd) & 1u, a);
             cyc_add(4, c0);
             c0 = cyc();
+#pragma unroll
             for (int qi = 0; qi < 2; ++qi) {
                 const int di = di0 + qi;
                 const uint8_t* dc = dring + (size_t)(di % a.nd) * a.d_bytes;
@@ -792,42 +866,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int r = 0; r < 4; ++r) acc[nt][r] = 0.f;
 #pragma unroll
                     for (int kb = 0; kb < 4; ++kb) {
-                        uint4 bh[NT];
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            const int tok = nt * 8 + g;
-                            bh[nt] = tok < T ? *reinterpret_cast<const uint4*>(hbuf + tok * kHRow + kb * 32 + 8 * c)
-                                             : make_uint4(0, 0, 0, 0);
-                        }
                         uint32_t qq[8];
                         decode_any<true, BD>(td.lo[kb], td.hi[kb], qq);
                         const uint32_t q0[4] = {qq[0], qq[1], qq[2], qq[3]}, q1[4] = {qq[4], qq[5], qq[6], qq[7]};
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
                             float t4[4] = {0.f, 0.f, 0.f, 0.f};
-                            mma_f16(t4, q0, bh[nt].x, bh[nt].y, t4);
-                            mma_f16(t4, q1, bh[nt].z, bh[nt].w, t4);
+                            mma_f16(t4, q0, hf[kb][nt].x, hf[kb][nt].y, t4);
+                            mma_f16(t4, q1, hf[kb][nt].z, hf[kb][nt].w, t4);
                             scale_acc(acc[nt], t4, td.sc[kb]);
                         }
                     }
-                    // partial sums of (token t, slot, chunk j) for output rows n, n + 8
+                    // partial sums of (token, slot, chunk j) for output rows n, n + 8
                     const int n = (rt0 + lt) * 16 + g;
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                         for (int r = 0; r < 4; ++r) {
-                            const int t = nt * 8 + 2 * c + (r & 1);
-                            if (t < T && ((mask >> t) & 1u)) {
-                                // the shared expert comes first in every token's list; the
-                                // routed slots' places exist once the schedule is built
-                                const int pl = slot < ns ? 0 : pos[slot * T + t];
-                                if (pl < KS) {
-                                    const int64_t row = ((int64_t)t * KS + pl) * FC + j;
-                                    a.part[row * d + n + 8 * (r >> 1)] = s_w[i & 1][t] * acc[nt][r];
-                                } else {
-                                    flag_status(a.status, kStatusBounds);
-                                }
-                            }
+                            const int e2 = r & 1;
+                            if (pbase[nt][e2] >= 0) a.part[pbase[nt][e2] + n + 8 * (r >> 1)] = wtok[nt][e2] * acc[nt][r];
                         }
                 }
             }
@@ -871,7 +928,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         cyc_add(6, ctk);
+        unsigned long long csc = cyc();
         consumer_sync();
+        cyc_add(16, csc);  // wait for the other warps' top-k
+        csc = cyc();
         trace(4);
         for (int p = tid; p < T * k; p += kConsumers) {
             const int e = sids[p], t = p / k, r = p - t * k;
@@ -911,6 +971,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             consumer_sync();
         }
         const int n_slots = s_nslots;
+        cyc_add(17, csc);  // masks + compaction
+        csc = cyc();
         // place of each slot in its tokens' lists (slot order): the partial sums' row index
         if (tid < T) {
             int r = 0;
@@ -932,6 +994,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 a.meta->n_fixup = 0;  // the fp64 logits are ranked exactly
             }
         }
+        cyc_add(18, csc);  // places + meta
         consumer_sync();
         if (tid == 0) mbar_arrive(&sched);  // the producer may issue the routed units
         const int n_units = s_nunits;
@@ -948,9 +1011,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         trace(38);
 
         // ---- 4. every CTA's partial sums, then this CTA's slice of y
+        unsigned long long ctl = cyc();
         consumer_sync();
         if (tid == 0) grid_wait(a.ctr + 1, grid_arrive(a.ctr + 1, true), a);
         consumer_sync();
+        cyc_add(19, ctl);
+        ctl = cyc();
         trace(39);
         {
             // output quads (t, n..n+3); a half-warp per quad, lane `sub` summing
@@ -1009,6 +1075,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
+        cyc_add(20, ctl);
         trace(40);
     }
     // every thread of both CTAs: no remote access is still in flight when a CTA exits
@@ -1043,7 +1110,7 @@ static bool make_layout(int BG, int BD, int NT, int T, int d, int f, int E, int 
     };
     L->off_x = take((size_t)T * (d + kXPad) * 2);
     L->off_h = take((size_t)3 * T * kHRow * 2);
-    L->off_gus = take(std::max((size_t)kCWarps * NT * 4 * 32 * 4, (size_t)kCWarps * 16 * 8));
+    L->off_gus = take(std::max((size_t)kCWarps * 2 * NT * 4 * 32 * 4, (size_t)kCWarps * 16 * 8));
     L->off_cand = take((size_t)kCWarps * kCandBytes);
     L->off_route = take((size_t)T * k * 8);
     L->off_emask = take((size_t)E * 8);
@@ -1194,15 +1261,23 @@ static cudaError_t launch_t(const DecodeLaunch& L, cudaStream_t st) {
     cfg.stream = st;
     cfg.attrs = at;
     cfg.numAttrs = 2;
-    e = cudaLaunchKernelEx(&cfg, kern, a, *L.down_codes_map, *L.down_scales_map);
-    if (e == cudaSuccess) return e;
-    // A cooperative launch can be refused where the grid is still co-resident in
-    // practice (a profiler replaying the kernel): launch the same clusters
-    // without the guarantee.  Should they not all be resident, the bounded
-    // waits report MOE_ERR_TIMEOUT instead of hanging.
-    (void)cudaGetLastError();
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a, *L.down_codes_map, *L.down_scales_map);
+    // The grid barriers need every CTA resident at once, which the cooperative
+    // launch guarantees.  Where fewer clusters fit than the occupancy query
+    // reported (another client holding SMs, a profiler), the launch is refused:
+    // retry with fewer clusters (the work split follows the cluster count) and
+    // remember the count that was accepted.
+    for (int attempt = 0; attempt < 16; ++attempt) {
+        a.nc = clusters;
+        cfg.gridDim = dim3(kCS * clusters);
+        e = cudaLaunchKernelEx(&cfg, kern, a, *L.down_codes_map, *L.down_scales_map);
+        if (e != cudaErrorCooperativeLaunchTooLarge || clusters <= 1) break;
+        (void)cudaGetLastError();
+        clusters = std::max(1, clusters - std::max(1, clusters / 16));
+        std::lock_guard<std::mutex> lk(mu);
+        for (Occ& o : cache)
+            if (o.dev == dev && o.fn == (const void*)kern && o.smem == lay.total) o.clusters = clusters;
+    }
+    return e;
 }
 
 template <int BG, int BD>
@@ -1244,6 +1319,7 @@ bool pair_decode_supported(const DecodeLaunch& L) {
     pair::Layout lay;
     const int bd = L.bits_down ? L.bits_down : L.bits;
     return L.T >= 1 && L.T <= kPairMaxTokens && L.E <= 1024 && L.k <= 32 && L.d % 128 == 0 && L.f % 128 == 0 &&
+           L.d <= 128 * pair::kCWarps * pair::kMaxKS &&
            pair::make_layout(L.bits, bd, L.T <= 8 ? 1 : 2, L.T, L.d, L.f, L.E, L.k, smem_max - 1024, &lay);
 }
 
