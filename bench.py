@@ -49,12 +49,13 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-graph", action="store_true", help="time eager launches instead of a CUDA graph")
+    p.add_argument("--no-sub", action="store_true", help="skip the decode T=1 and prefill sub-measurements")
     return p.parse_args()
 
 
 # ---------------------------------------------------------------- ncu traffic of the dominant kernel
 _KERNEL_SOURCE = {"gemm_gateup": "gemm_sm100.cu", "gemm_down": "gemm_sm100.cu", "router_gemm": "gemm_sm100.cu",
-                  "decode_fused": "decode.cu", "gemv_gateup": "gemv.cu", "gemv_down": "gemv.cu"}
+                  "decode_fused": "decode_pair.cu", "gemv_gateup": "gemv.cu", "gemv_down": "gemv.cu"}
 
 
 def profile_traffic(kernel: str):
@@ -280,6 +281,179 @@ def _graph_launches(h, step, n):
     return h.stats()["launches"] - a
 
 
+def _capture(step, first, n):
+    """A CUDA graph of steps first .. first + n - 1 (each step enqueued once while capturing)."""
+    import torch
+    cap_stream = torch.cuda.Stream()
+    cap_stream.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap_stream):
+        for i in range(n):  # settle any lazy per-kernel setup outside capture
+            step(first + i)
+    torch.cuda.current_stream().wait_stream(cap_stream)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            step(first + i)
+    torch.cuda.synchronize()
+    return g
+
+
+def time_steps(step, steps, warmup, n_cap, use_graph, clock_index=None, world=1):
+    """Device time (ms) of exactly `steps` steps after `warmup` untimed ones.
+
+    With graphs: replays of a graph of n_cap consecutive steps, then one graph of
+    the remaining steps % n_cap, so exactly `steps` steps run.  Returns
+    (ms, clocks summary or None).
+    """
+    import torch
+    import torch.distributed as dist
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    graphs = []
+    if use_graph:
+        n_cap = max(1, min(n_cap, steps))
+        full, rest = divmod(steps, n_cap)
+        g_full = _capture(step, warmup, n_cap)
+        graphs = [g_full] * full
+        if rest:
+            graphs.append(_capture(step, warmup, rest))
+    if world > 1:
+        dist.barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk = ClockSampler(clock_index) if clock_index is not None else None
+    if clk:
+        clk.__enter__()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed")
+    ev0.record()
+    if use_graph:
+        for g in graphs:
+            g.replay()
+    else:
+        for i in range(steps):
+            step(warmup + i)
+    ev1.record()
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    if clk:
+        clk.__exit__()
+    return ev0.elapsed_time(ev1), (clk.summary() if clk else None)
+
+
+def kernel_profile(h, step, first, n):
+    """Per-kernel device time of n steps (events on the library's launch stream), behind a device-side
+    sleep so that the events bracket back-to-back device work: {name: (total ms, launches)}."""
+    import torch
+    torch.cuda.synchronize()
+    h.profile(True)
+    torch.cuda._sleep(int(2e8))
+    for i in range(n):
+        step(first + i)
+    prof = h.profile_read()
+    h.profile(False)
+    return prof
+
+
+def roofline_of(prof, alg_bytes, flops, nprof):
+    """Roofline entry of the dominant kernel of a per-kernel profile."""
+    hbm, tc_burst, tc_sus, peak_kind = measured_peaks()
+    if not prof:
+        return None
+    dom = max(prof.items(), key=lambda kv: kv[1][0])[0]
+    if dom in flops:
+        dom_ms = prof[dom][0] / prof[dom][1]
+        ach = flops[dom] / (dom_ms / 1000.0) / 1e12
+        return {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": tc_burst, "unit": "TFLOP/s",
+                "frac": ach / tc_burst, "traffic": profile_traffic(dom),
+                "peak_kind": peak_kind + " bf16 dense (burst)", "flops_per_launch": flops[dom],
+                "avg_launch_us": 1000.0 * dom_ms}
+    if dom in alg_bytes:
+        dom_ms = prof[dom][0]
+        ach = alg_bytes[dom] / (dom_ms / 1000.0) / 1e9
+        r = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+             "traffic": profile_traffic(dom), "peak_kind": peak_kind,
+             "bytes_per_launch": alg_bytes[dom] / max(1, prof[dom][1]),
+             "avg_launch_us": 1000.0 * dom_ms / max(1, prof[dom][1])}
+        if dom == "decode_fused":
+            r["traffic_note"] = ("the clustered decode kernel needs a cooperative launch, which ncu's replay "
+                                 "cannot reproduce; profiles/decode_pair_T4_phases.md has its device-side trace")
+        return r
+    return None
+
+
+def layer_bytes(sh, D, T):
+    """Algorithmic HBM bytes of one layer step: router, the D distinct routed experts and the shared one,
+    activations in and out."""
+    return sh.E * sh.d * 2 + (D + sh.n_shared) * expert_bytes(sh) + 4 * T * sh.d
+
+
+def measure_decode(moe, h, sh, xs, layers, T, flags, args, steps, warmup, clock_index, world, chain=False):
+    """Throughput and per-kernel breakdown of decode steps of T tokens (layers rotated)."""
+    import torch
+    n_x = len(xs)
+    resid = [torch.empty_like(xs[0]) for _ in range(2)]
+    normed = torch.empty_like(xs[0])
+    ys = [torch.empty(T, sh.d, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+
+    def step(i, stream=None):
+        if chain:
+            # residual chain: u_l = rmsnorm(x_l), x_{l+1} = x_l + layer_l(u_l) in place
+            r = resid[i & 1]
+            r.copy_(xs[i % n_x])
+            for l in range(layers):
+                moe.rms_normalize(r, normed, stream=stream)
+                h.forward(l, normed, r, flags=flags | moe.MOE_ACCUMULATE, stream=stream)
+            return r
+        return h.forward(i % layers, xs[i % n_x], ys[i & 1], flags=flags, stream=stream)
+
+    n_cap = max(layers, n_x) if not chain else 1
+    ms, clocks = time_steps(step, steps, warmup, n_cap, not args.no_graph, clock_index, world)
+    launches = _graph_launches(h, step, steps)
+    # per-kernel device time and the algorithmic bytes of the same steps
+    nl = layers if chain else 1
+    nprof = min(steps, 64)
+    alg = {"gemv_gateup": 0.0, "gemv_down": 0.0, "decode_fused": 0.0, "layer": 0.0}
+    for i in range(nprof):
+        step(warmup + i)
+        D = h.stats()["active_experts"]
+        lb = nl * layer_bytes(sh, D, T)
+        alg["gemv_gateup"] += nl * (D + sh.n_shared) * 2 * mat_bytes(sh)
+        alg["gemv_down"] += nl * (D + sh.n_shared) * mat_bytes(sh)
+        alg["decode_fused"] += lb
+        alg["layer"] += lb
+    prof = kernel_profile(h, step, warmup, nprof)
+    rows = T * sh.k + T * sh.n_shared
+    flops = {"gemm_gateup": 2.0 * rows * 2 * sh.f * sh.d, "gemm_down": 2.0 * rows * sh.d * sh.f}
+    layer_time = sum(v[0] for v in prof.values())
+    return {"ms": ms, "clocks": clocks, "launches": launches, "step": step,
+            "roofline": roofline_of(prof, alg, flops, nprof),
+            "layer_hbm_gbs": alg["layer"] / (layer_time / 1000.0) / 1e9 if layer_time else None,
+            "kernels_ms_per_step": {k: v[0] / nprof for k, v in prof.items()}}
+
+
+def sub_block(moe, sgpu, wl, sh, T, layers, rank, args, steps, warmup):
+    """A separate measured workload (its own handle) reported inside the main line."""
+    import torch
+    h = moe.MoeLayer(sh.d, sh.f, sh.E, sh.k, sh.n_shared, layers, sh.bits, T)
+    keep = []
+    for l in range(layers):
+        w = sgpu.layer_device(sh, rank_master(wl.master, rank), l, wl.zipf)
+        h.load_layer(l, *w)
+        keep.append(w)
+    n_x = 4 if T > 64 else 16
+    xs = [sgpu.x_device(sh, rank_master(wl.master, rank), 20000 + i, T) for i in range(n_x)]
+    torch.cuda.synchronize()
+    r = measure_decode(moe, h, sh, xs, layers, T, 0, args, steps, warmup, None, 1)
+    h.close()
+    del keep
+    torch.cuda.empty_cache()
+    return {"tokens_per_step": T, "layers": layers, "steps": steps, "value": T * steps / (r["ms"] / 1000.0),
+            "unit": "tok/s", "ms_per_step": r["ms"] / steps, "roofline": r["roofline"],
+            "kernels_ms_per_step": r["kernels_ms_per_step"], "gpu_launches": r["launches"]}
+
+
 # ---------------------------------------------------------------- our arm
 def ours(args):
     import torch
@@ -319,113 +493,13 @@ def ours(args):
     n_x = 16
     xs = [sgpu.x_device(sh, rank_master(wl.master, rank), 10000 + i, T) for i in range(n_x)]
     chain = args.workload == "chain48"
-    resid = [torch.empty_like(xs[0]) for _ in range(2)]
-    normed = torch.empty_like(xs[0])
-
-    def step(i, stream=None):
-        if chain:
-            # residual chain: u_l = rmsnorm(x_l), x_{l+1} = x_l + layer_l(u_l) in place
-            r = resid[i & 1]
-            r.copy_(xs[i % n_x])
-            for l in range(layers):
-                moe.rms_normalize(r, normed, stream=stream)
-                h.forward(l, normed, r, flags=flags | moe.MOE_ACCUMULATE, stream=stream)
-            return r
-        return h.forward(i % layers, xs[i % n_x], ys[i & 1], flags=flags, stream=stream)
-
-    ys = [torch.empty(T, sh.d, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
-    torch.cuda.synchronize()
-    for i in range(args.warmup):
-        step(i)
     torch.cuda.synchronize()
 
-    # The timed region replays a CUDA graph of n_cap consecutive steps (host
-    # launch overhead out of the measurement; the device work is unchanged).
-    n_cap = max(layers, n_x) if not chain else 1
-    graph = None
-    if not args.no_graph:
-        cap_stream = torch.cuda.Stream()
-        cap_stream.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(cap_stream):
-            for i in range(n_cap):  # settle any lazy per-kernel setup outside capture
-                step(i)
-        torch.cuda.current_stream().wait_stream(cap_stream)
-        torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            for i in range(n_cap):
-                step(i)
-        torch.cuda.synchronize()
-    reps = max(1, math.ceil(args.steps / n_cap)) if graph is not None else args.steps
-    n_steps = reps * n_cap if graph is not None else args.steps
+    res = measure_decode(moe, h, sh, xs, layers, T, flags, args, args.steps, args.warmup, local, world, chain)
+    ms = max_over_ranks(res["ms"], world)
     if world > 1:
         dist.barrier()
-    launches0 = h.stats()["launches"]
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        torch.cuda.synchronize()
-        torch.cuda.nvtx.range_push("timed")
-        ev0.record()
-        if graph is not None:
-            for _ in range(reps):
-                graph.replay()
-        else:
-            for i in range(n_steps):
-                step(args.warmup + i)
-        ev1.record()
-        torch.cuda.nvtx.range_pop()
-        torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1)
-    launches = h.stats()["launches"] - launches0
-    if graph is not None:  # the library counts launches when enqueued (at capture): count n_cap steps
-        launches = _graph_launches(h, step, n_cap) * reps
-    ms = max_over_ranks(ms, world)
-    if world > 1:
-        dist.barrier()
-    tok_per_step = T
-    value = replica_throughput(tok_per_step, n_steps, world, ms)
-
-    # ---- per-kernel device time (events on the library's launch stream), separate pass.
-    # Pass 1 records each step's distinct experts; pass 2 replays the same steps
-    # behind a device-side sleep so the events bracket back-to-back device work.
-    alg_bytes = {"gemv_gateup": 0.0, "gemv_down": 0.0, "decode_fused": 0.0, "layer": 0.0}
-    nprof = min(n_steps, 64 if T <= 64 else 4)
-    nl = layers if chain else 1
-    for i in range(nprof):
-        step(args.warmup + i)
-        D = h.stats()["active_experts"]
-        lb = nl * (sh.E * sh.d * 2 + (D + sh.n_shared) * expert_bytes(sh) + 4 * T * sh.d)
-        alg_bytes["gemv_gateup"] += nl * (D + sh.n_shared) * 2 * mat_bytes(sh)
-        alg_bytes["gemv_down"] += nl * (D + sh.n_shared) * mat_bytes(sh)
-        alg_bytes["decode_fused"] += lb
-        alg_bytes["layer"] += lb
-    torch.cuda.synchronize()
-    h.profile(True)
-    torch.cuda._sleep(int(2e8))
-    for i in range(nprof):
-        step(args.warmup + i)
-    prof = h.profile_read()
-    h.profile(False)
-    hbm, tc_burst, tc_sus, peak_kind = measured_peaks()
-    dom = max(prof.items(), key=lambda kv: kv[1][0])[0] if prof else None
-    roof = None
-    rows = T * sh.k + T * sh.n_shared
-    flops = {"gemm_gateup": 2.0 * rows * 2 * sh.f * sh.d, "gemm_down": 2.0 * rows * sh.d * sh.f}
-    if dom in ("gemm_gateup", "gemm_down"):
-        dom_ms = prof[dom][0] / prof[dom][1]
-        ach = flops[dom] / (dom_ms / 1000.0) / 1e12
-        roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": tc_burst, "unit": "TFLOP/s",
-                "frac": ach / tc_burst, "traffic": profile_traffic(dom), "peak_kind": peak_kind + " bf16 dense (burst)",
-                "flops_per_launch": flops[dom], "avg_launch_us": 1000.0 * dom_ms}
-    elif dom in ("gemv_gateup", "gemv_down", "decode_fused"):
-        dom_ms = prof[dom][0]
-        ach = alg_bytes[dom] / (dom_ms / 1000.0) / 1e9
-        roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                "traffic": profile_traffic(dom), "peak_kind": peak_kind,
-                "bytes_per_launch": alg_bytes[dom] / max(1, prof[dom][1]),
-                "avg_launch_us": 1000.0 * dom_ms / max(1, prof[dom][1])}
-    layer_time = sum(v[0] for v in prof.values())
-    layer_gbs = alg_bytes["layer"] / (layer_time / 1000.0) / 1e9 if layer_time else None
+    value = replica_throughput(T, args.steps, world, ms)
 
     # ---- end to end through the host-buffer entry point (pinned memory)
     e2e = None
@@ -446,6 +520,18 @@ def ours(args):
         e2e = {"value": replica_throughput(T, k2, world, ems), "unit": "tok/s", "h2d_bytes_per_step": T * sh.d * 2,
                "d2h_bytes_per_step": T * sh.d * 2}
 
+    # ---- the rest of the metric ("decode 1-4 tok, 8K prefill"): decode T = 1 and one 8192-token
+    # prefill chunk, each on its own handle (rank 0 of a single-GPU run only: replicas repeat it)
+    subs = {}
+    if args.workload == "decode" and world == 1 and not args.no_sub and not flags:
+        h.close()
+        del weights
+        torch.cuda.empty_cache()
+        h = None
+        subs["decode_t1"] = sub_block(moe, sgpu, wl, sh, 1, layers, rank, args, max(args.steps, 16), args.warmup)
+        subs["prefill_8192"] = sub_block(moe, sgpu, WORKLOADS_PREFILL(), WORKLOADS_PREFILL().shape, 8192, 1, rank,
+                                         args, 10, 3)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         Tc = min(T, 16)
@@ -454,24 +540,32 @@ def ours(args):
                "sample": f"{ntok} tokens in batches of {Tc}, {secs:.1f} s of fp64 C oracle work"}
 
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": n_steps,
-                "warmup": args.warmup, "ms_per_step": ms / n_steps, "higher_is_better": True, "scaling": "weak",
+        line = {"metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": {"workload": args.workload, "tokens_per_step": T, "d": sh.d, "f": sh.f, "experts": sh.E,
                            "top_k": sh.k, "shared": sh.n_shared, "bits": sh.bits, "layers": layers,
                            "l2": ("inputs larger than L2: 48 layers x 756 MB per step" if chain else
                                   f"inputs larger than L2: {layers} distinct layers cycled, {n_x} fresh inputs"),
-                           "parallelism": f"replicas x{world}", "timing": "CUDA graph replay" if graph is not None else "eager",
+                           "parallelism": f"replicas x{world}",
+                           "timing": "CUDA graph replay" if not args.no_graph else "eager",
                            **({"flags": args.flags} if args.flags else {}),
                            **({"expert_shard": args.expert_shard} if args.expert_shard else {})},
-                "roofline": roof, "layer_hbm_gbs": layer_gbs,
-                "kernels_ms_per_step": {k: v[0] / nprof for k, v in prof.items()},
-                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk.summary()}
+                "roofline": res["roofline"], "layer_hbm_gbs": res["layer_hbm_gbs"],
+                "kernels_ms_per_step": res["kernels_ms_per_step"],
+                **subs,
+                "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": res["launches"], "clocks": res["clocks"]}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
-    h.close()
+    if h is not None:
+        h.close()
+
+
+def WORKLOADS_PREFILL():
+    from synth import WORKLOADS
+    return WORKLOADS["prefill"]
 
 
 def main():
