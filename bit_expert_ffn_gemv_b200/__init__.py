@@ -19,7 +19,7 @@ import threading
 __all__ = ["MoeError", "MoeConfig", "MoeLayerWeights", "MoeLayer", "lib", "library_path", "MOE_OUT_FP32",
            "MOE_ACCUMULATE", "MOE_FORCE_GEMV", "MOE_FORCE_GEMM", "MOE_FORCE_UNFUSED", "MOE_ROUTE_TAIL_SKIP",
            "MOE_TAIL_SKIP_RANK", "STATUS", "moe_layer_init", "moe_load_layer",
-           "moe_route", "moe_route_noalloc", "moe_forward", "moe_forward_host", "moe_destroy", "moe_debug_dequant", "moe_debug_last_routing", "moe_check_status",
+           "moe_route", "moe_route_noalloc", "moe_forward", "moe_forward_host", "moe_destroy", "moe_debug_dequant", "moe_debug_last_routing", "moe_debug_bucket", "moe_check_status",
            "moe_get_stats", "moe_status_string", "moe_profile", "moe_profile_read", "moe_kernel_name", "MoeStats",
            "moe_debug_router_logits", "moe_router_error_depth", "moe_rms_normalize", "rms_normalize",
            "moe_set_expert_range", "moe_debug_wait_limit"]
@@ -93,6 +93,8 @@ def lib() -> ctypes.CDLL:
             L.moe_debug_dequant.argtypes = [vp, i32, i32, i32, vp, vp]
             L.moe_debug_last_routing.restype = st
             L.moe_debug_last_routing.argtypes = [vp, i32, vp, vp, vp]
+            L.moe_debug_bucket.restype = st
+            L.moe_debug_bucket.argtypes = [vp, vp, i32, vp, vp, vp, vp, vp, vp, u32, vp]
             L.moe_check_status.restype = st
             L.moe_check_status.argtypes = [vp]
             L.moe_get_stats.restype = st
@@ -178,6 +180,12 @@ def moe_destroy(handle: int) -> None:
 
 def moe_debug_dequant(handle: int, layer: int, expert: int, mat: int, out_ptr: int, stream: int) -> None:
     _check(lib().moe_debug_dequant(handle, layer, expert, mat, out_ptr, stream), "moe_debug_dequant")
+
+
+def moe_debug_bucket(handle: int, ids_ptr: int, T: int, w_ptr, offsets_ptr: int, pairs_ptr: int, inv_ptr: int,
+                     active_ptr: int, wsorted_ptr, flags: int, stream: int) -> None:
+    _check(lib().moe_debug_bucket(handle, ids_ptr, T, w_ptr, offsets_ptr, pairs_ptr, inv_ptr, active_ptr, wsorted_ptr,
+                                  flags, stream), "moe_debug_bucket")
 
 
 def moe_debug_last_routing(handle: int, T: int, ids_ptr: int, w_ptr: int, stream: int) -> None:
@@ -301,6 +309,21 @@ class MoeLayer:
         w = torch.empty((T, self.cfg.top_k), dtype=torch.float32, device="cuda")
         moe_debug_last_routing(self.handle, T, ids.data_ptr(), w.data_ptr(), _stream_ptr(stream))
         return ids, w
+
+    def bucket(self, ids, w=None, flags=0, stream=None):
+        """The grouping step alone on ids [T x k]: (offsets, pairs, inv, active, wsorted or None)."""
+        import torch
+        T = ids.shape[0]
+        n = T * self.cfg.top_k
+        offsets = torch.full((self.cfg.n_experts + 1,), -7, dtype=torch.int32, device="cuda")
+        pairs = torch.full((max(n, 4),), -7, dtype=torch.int32, device="cuda")
+        inv = torch.full((max(n, 4),), -7, dtype=torch.int32, device="cuda")
+        active = torch.full((self.cfg.n_experts,), -7, dtype=torch.int32, device="cuda")
+        wsorted = torch.full((max(n, 4),), -7.0, dtype=torch.float32, device="cuda") if w is not None else None
+        moe_debug_bucket(self.handle, ids.data_ptr(), T, w.data_ptr() if w is not None else None, offsets.data_ptr(),
+                         pairs.data_ptr(), inv.data_ptr(), active.data_ptr(),
+                         wsorted.data_ptr() if wsorted is not None else None, flags, _stream_ptr(stream))
+        return offsets, pairs[:n], inv[:n], active, (wsorted[:n] if wsorted is not None else None)
 
     def router_logits(self, layer, x, tensor_cores=True, stream=None):
         """fp32 logits [T x E] from one of the two router kernels (for bound checks)."""

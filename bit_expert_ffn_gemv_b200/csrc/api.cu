@@ -589,6 +589,41 @@ moe_status moe_debug_dequant(moe_handle* h, int32_t layer, int32_t expert, int32
                                            static_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_debug_bucket(moe_handle* h, const int32_t* ids, int32_t T, const float* w, int32_t* offsets,
+                            int32_t* pairs, int32_t* inv, int32_t* active, float* wsorted, uint32_t flags,
+                            void* stream) {
+    if (!h || T < 0 || T > h->cfg.max_tokens || (flags & ~kAllFlags)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!ids || !offsets || !pairs || !inv || !active || !aligned16(ids) || !aligned16(offsets) ||
+        !aligned16(pairs) || !aligned16(inv) || !aligned16(active) || (w && !aligned16(w)) ||
+        (wsorted && !aligned16(wsorted)))
+        return MOE_ERR_INVALID_ARG;
+    const moe_config& c = h->cfg;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    moe::BucketArgs ba;
+    ba.ids = ids;
+    ba.T = T;
+    ba.k = c.top_k;
+    ba.E = c.n_experts;
+    ba.offsets = offsets;
+    ba.pairs = pairs;
+    ba.inv = inv;
+    ba.active = active;
+    ba.meta = h->meta;
+    ba.status = h->status;
+    if (w && wsorted) {
+        ba.w = w;
+        ba.wsorted = wsorted;
+    }
+    ba.cnt = h->bucket_cnt;
+    ba.skip_rank = skip_rank(c, flags);
+    ba.e_begin = h->ep_begin;
+    ba.e_end = h->ep_end;
+    const cudaError_t e = run(h, MOE_K_BUCKET, s, [&] { return moe::launch_bucket(ba, s); });
+    h->launches += moe::bucket_kernel_count(ba) - 1;
+    return cuda_status(e);
+}
+
 moe_status moe_debug_last_routing(moe_handle* h, int32_t T, int32_t* ids, float* w, void* stream) {
     if (!h || T < 0 || T > h->cfg.max_tokens || (T > 0 && (!ids || !w))) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;

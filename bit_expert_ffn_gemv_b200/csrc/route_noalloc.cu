@@ -22,26 +22,26 @@ namespace {
 // pairs, norms of up to 1024 experts, and the small counter block.
 constexpr int kMaxLogits = 65536;  // T * E
 constexpr int kMaxExperts = 1024;
+// Largest model width: the logits kernel stages four token rows of d fp32
+// values in shared memory (16 * d bytes), within every sm_100 part's opt-in
+// limit at d = 8192.
+constexpr int kMaxWidth = 8192;
 constexpr size_t kScratchFloats = kMaxLogits + kMaxExperts + 64;
 
 // File-scope device array; the host side only ever sees its symbol, whose
 // device address comes from cudaGetSymbolAddress on the device in use.
 static __device__ __align__(256) float g_route_scratch[kScratchFloats];
 
-constexpr int kMaxDevices = 64;
-float* g_scratch_ptr[kMaxDevices] = {};  // per-device address, looked up once
-
-// Look the array's device address up once per device, with that device
-// current.  Returns nullptr if the lookup fails.
+// The array's device address, looked up on every call with the caller's
+// device current.  The lookup is a host-side table read, cheap next to the
+// three launches; caching it would go stale if the context holding the module
+// were torn down and recreated (the module reloads, and the array may move),
+// and a shared cache would need synchronising between host threads.
+// Returns nullptr if the lookup fails.
 float* scratch_for_current_device() {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) return nullptr;
-        g_scratch_ptr[dev] = static_cast<float*>(p);
-    }
-    return g_scratch_ptr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess) return nullptr;
+    return static_cast<float*>(p);
 }
 
 }  // namespace
@@ -49,7 +49,7 @@ float* scratch_for_current_device() {
 extern "C" moe_status moe_route_noalloc(const void* x, int32_t T, int32_t d, int32_t n_experts, int32_t top_k,
                                         const void* router_w, const float* router_bias, int32_t* ids, float* w,
                                         void* stream) {
-    if (T < 0 || d <= 0 || d % 128 || n_experts < 1 || n_experts > kMaxExperts || top_k < 1 || top_k > 32 ||
+    if (T < 0 || d <= 0 || d % 128 || d > kMaxWidth || n_experts < 1 || n_experts > kMaxExperts || top_k < 1 || top_k > 32 ||
         top_k > n_experts)
         return MOE_ERR_INVALID_ARG;
     if ((int64_t)T * n_experts > kMaxLogits) return MOE_ERR_INVALID_ARG;  // beyond the fixed scratch

@@ -191,10 +191,13 @@ moe_status moe_forward_host(moe_handle* h, int32_t layer, const void* x_host, in
  * Intermediates live in one fixed device array inside the library (about
  * 260 KB, held by every GPU that loads the library until the process exits):
  * T * n_experts must not exceed 65536 and n_experts not 1024, else
- * MOE_ERR_INVALID_ARG and nothing is enqueued.  d must be a multiple of 128,
- * 1 <= top_k <= min(n_experts, 32).  The first call on each device looks the
- * array's address up on the current device; make that first call before any
- * stream capture.  All calls share the array: two calls whose work overlaps
+ * MOE_ERR_INVALID_ARG and nothing is enqueued.  d must be a multiple of 128
+ * and at most 8192 (the logits kernel stages 16 * d bytes of shared memory),
+ * 1 <= top_k <= min(n_experts, 32); outside these limits the call returns
+ * MOE_ERR_INVALID_ARG before enqueuing anything.  Every call looks the
+ * array's address up on the current device (a host-side lookup that follows
+ * a recreated context); the first call on a device may load the library's
+ * module, so make it before any stream capture.  All calls share the array: two calls whose work overlaps
  * on the GPU (different streams, no ordering between them) race and give
  * wrong results -- order them on one stream.
  * Errors: INVALID_ARG, CUDA.
@@ -226,6 +229,35 @@ moe_status moe_destroy(moe_handle* h);
  */
 moe_status moe_debug_dequant(moe_handle* h, int32_t layer, int32_t expert, int32_t mat, float* out,
                              void* stream);
+
+/*
+ * Debug: the grouping step alone, as the unfused and tensor-core paths run it
+ * between routing and the expert kernels (discuss.pytorch.kr post, "how it
+ * works": each token's selected experts are gathered per expert before they
+ * run).  Input: ids [T x k] int32 in moe_route's layout and, optionally, the
+ * routing weights w [T x k] fp32.  Output (device, 16-byte aligned):
+ *   offsets [E + 1]  start of each expert's group in pairs; offsets[E] is the
+ *                    number of kept pairs
+ *   pairs   [T * k]  pair index t * k + r, grouped by expert in ascending
+ *                    expert order, ascending t inside a group (a stable
+ *                    counting sort); entries past offsets[E] are not written
+ *   inv     [T * k]  position of pair t * k + r in pairs, or -1 if dropped
+ *   active  [E]      experts with a non-empty group, ascending; entries past
+ *                    their count are not written
+ *   wsorted [T * k]  w of the pair at each position (only when w and wsorted
+ *                    are both non-NULL)
+ * A pair is dropped when its expert lies outside the handle's expert range
+ * (moe_set_expert_range) or, with MOE_ROUTE_TAIL_SKIP in flags, when no token
+ * ranked its expert before MOE_TAIL_SKIP_RANK.  At T * k >= 8192 the grouping
+ * runs as three kernels over 128 CTAs, below as one CTA; both give the same
+ * result.  Uses the handle's scratch: enqueue it on the stream of the handle's
+ * other calls.  Ids outside [0, E) set the device status (MOE_ERR_BOUNDS).
+ * Errors: INVALID_ARG (T out of range, NULL or misaligned pointer, unknown
+ * flag), CUDA.
+ */
+moe_status moe_debug_bucket(moe_handle* h, const int32_t* ids, int32_t T, const float* w, int32_t* offsets,
+                            int32_t* pairs, int32_t* inv, int32_t* active, float* wsorted, uint32_t flags,
+                            void* stream);
 
 /*
  * Debug: copy the routing the last moe_forward computed internally (rank-order

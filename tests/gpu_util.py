@@ -50,3 +50,34 @@ def y_to_f64(y) -> np.ndarray:
 def make_layer_host(wl, layer=0, experts=None, shape=None):
     shape = shape or wl.shape
     return synth.layer_host(shape, wl.master, layer, wl.zipf, experts)
+
+
+# Tokens per expert tile of the tensor-core path, and rows of its small
+# activation box (groups of at most 64 tokens load 32-row boxes).
+TILE_TOKENS = 256
+SMALL_BOX_ROWS = 32
+SMALL_GROUP = 64
+
+
+def tile_cover_rows(ids: np.ndarray, E: int, n_shared: int = 1) -> np.ndarray:
+    """Tokens to check so that every tile the tensor-core path forms holds at least one of them.
+
+    Each routed expert's group (the tokens that selected it, ascending) is cut
+    into tiles of 256 tokens, and groups of at most 64 tokens are loaded in
+    32-row boxes; the shared expert's group is every token.  Greedily, each
+    tile or box that holds no chosen token adds its last token (the ragged
+    edge); the first and last token of the batch are always in.
+    """
+    T = ids.shape[0]
+    sets = []
+    for e in range(E):
+        g = np.nonzero((ids == e).any(1))[0]
+        step = SMALL_BOX_ROWS if 0 < g.size <= SMALL_GROUP else TILE_TOKENS
+        sets += [g[s:s + step] for s in range(0, g.size, step)]
+    if n_shared:
+        sets += [np.arange(s, min(T, s + TILE_TOKENS)) for s in range(0, T, TILE_TOKENS)]
+    chosen = {0, T - 1}
+    for st in sets:
+        if not chosen.intersection(st.tolist()):
+            chosen.add(int(st[-1]))
+    return np.array(sorted(chosen))

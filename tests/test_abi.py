@@ -80,3 +80,13 @@ def test_flag_constants_match_the_header():
     assert {"MOE_OUT_FP32", "MOE_ROUTE_TAIL_SKIP", "MOE_TAIL_SKIP_RANK"} <= set(defs)
     for name, v in defs.items():
         assert getattr(moe, name) == int(v, 0), name
+
+
+@pytest.mark.parametrize("bad", [dict(d=200), dict(d=8320), dict(T=129), dict(E=1025, T=1), dict(k=0), dict(k=33),
+                                 dict(E=8, k=9), dict(T=-1), dict(x=0), dict(x=8), dict(w=0)])
+def test_noalloc_route_rejects_bad_arguments_before_touching_the_gpu(L, bad):
+    """Every limit moe_route_noalloc states is checked before any CUDA call (so this runs without a GPU)."""
+    a = dict(x=256, T=4, d=256, E=512, k=10, wr=512, bias=None, ids=768, w=1024)
+    a.update(bad)
+    s = L.moe_route_noalloc(a["x"], a["T"], a["d"], a["E"], a["k"], a["wr"], a["bias"], a["ids"], a["w"], None)
+    assert s == 1  # MOE_ERR_INVALID_ARG

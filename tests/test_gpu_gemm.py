@@ -12,7 +12,7 @@ import pytest
 import oracle
 import synth
 from synth import WORKLOADS, MoeShape
-from tests.gpu_util import (MAX_ABS, REL_L2, make_layer_host, max_abs, rel_l2, upload_layer,
+from tests.gpu_util import (MAX_ABS, REL_L2, make_layer_host, max_abs, rel_l2, tile_cover_rows, upload_layer,
                             x_to_device, y_to_f64)
 
 pytestmark = pytest.mark.gpu
@@ -193,12 +193,45 @@ def test_router_gemm_error_bound(torch_cuda, full):
 
 @pytest.mark.parametrize("T", [17, 33, 65, 1000, 8192])
 def test_full_layer_gemm(torch_cuda, full, T):
-    """Full shape (E = 512, k = 10, d = 2048, f = 768); outputs checked on a sample of tokens."""
+    """Full shape (E = 512, k = 10, d = 2048, f = 768); outputs checked on tokens that cover every tile
+    the tensor-core path forms (every expert group, every 256-token tile, every 32-row box of the small
+    groups, the ragged ends), plus a random sample."""
     wl, L, h, dev = full
     x = synth.x_host(wl.shape, wl.master, 600 + T, T)
+    ids, _ = oracle.route(wl.shape, x, L["router_w"], L["bias"])
     rng = np.random.default_rng(T)
-    sample = np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=min(T, 48), replace=False)]))
+    sample = np.unique(np.concatenate([tile_cover_rows(ids, wl.shape.E), rng.choice(T, size=min(T, 16),
+                                                                                        replace=False)]))
     _check(torch_cuda, h, wl.shape, L, x, 0, "full-gemm", sample=sample)
+
+
+def test_prefill_four_chunks(torch_cuda, full):
+    """The 32K-token prompt as four consecutive 8192-token chunks through one handle, enqueued back to
+    back; every chunk's routing checked on all tokens and its outputs on a tile-covering set of rows."""
+    import bit_expert_ffn_gemv_b200 as moe
+    torch = torch_cuda
+    wl, L, h, dev = full
+    sh, T = wl.shape, 8192
+    xs = [synth.x_host(sh, wl.master, 800 + c, T) for c in range(wl.chunks)]
+    xd = [x_to_device(xb) for xb in xs]
+    outs = []
+    for x in xd:  # no synchronisation between the chunks
+        y16 = h.forward(0, x)
+        y32 = h.forward(0, x, flags=moe.MOE_OUT_FP32)
+        outs.append((y16, y32))
+    ids_gpu = [h.route(0, x)[0] for x in xd]
+    torch.cuda.synchronize()
+    assert h.check_status() == 0
+    for c, xb in enumerate(xs):
+        ids_ref, _ = oracle.route(sh, xb, L["router_w"], L["bias"])
+        assert np.array_equal(ids_gpu[c].cpu().numpy(), ids_ref), f"chunk {c}: expert selection differs"
+        rows = tile_cover_rows(ids_ref, sh.E)
+        y_ref, _, _ = oracle.layer(sh, xb[rows], L["router_w"], L["bias"], L["codes"], L["scales"])
+        g16, g32 = y_to_f64(outs[c][0])[rows], y_to_f64(outs[c][1])[rows]
+        r16, m16, r32 = rel_l2(g16, y_ref), max_abs(g16, y_ref), rel_l2(g32, y_ref)
+        print(f"chunk {c} rows={len(rows)}: rel_l2 bf16 {r16:.3e} max_abs {m16:.3e} fp32 {r32:.3e}")
+        assert r16 <= REL_L2 and m16 <= MAX_ABS, c
+        assert r32 <= REL_L2_FP32_TC, c
 
 
 def test_full_layer_forced_small(torch_cuda, full):
