@@ -40,6 +40,7 @@ def parse():
     p.add_argument("--workload", default="decode", choices=["decode", "chain48", "prefill", "sweep", "tiny"])
     p.add_argument("--tokens", type=int, default=None)
     p.add_argument("--bits", type=int, default=2)
+    p.add_argument("--bits-down", type=int, default=0, help="code width of the down matrices (sweep; 0: --bits)")
     p.add_argument("--rotate", type=int, default=8, help="distinct layers cycled through (decode/sweep)")
     p.add_argument("--flags", default="", help="extra forward flags, '+'-separated: gemv, gemm, tailskip "
                    "(the route-tail skip approximation)")
@@ -110,7 +111,7 @@ def workload(args):
     wl = WORKLOADS[args.workload]
     sh = wl.shape
     if args.workload == "sweep":
-        sh = MoeShape(sh.d, sh.f, sh.E, sh.k, sh.n_shared, args.bits)
+        sh = MoeShape(sh.d, sh.f, sh.E, sh.k, sh.n_shared, args.bits, bits_down=args.bits_down)
     T = args.tokens or {"decode": 4, "chain48": 1, "prefill": 8192, "sweep": 4, "tiny": 8}[args.workload]
     layers = 48 if args.workload == "chain48" else (1 if args.workload == "tiny" else max(1, args.rotate))
     return wl, sh, T, layers
@@ -118,12 +119,13 @@ def workload(args):
 
 def expert_bytes(sh):
     n = sh.f * sh.d
-    return 3 * n * sh.bits // 8 + 3 * (n // 32) * 2
+    return n * (2 * sh.bits + sh.bd) // 8 + 3 * (n // 32) * 2
 
 
-def mat_bytes(sh):
+def mat_bytes(sh, mat=0):
+    """Bytes of one matrix (0 gate, 1 up, 2 down) at its own code width."""
     n = sh.f * sh.d
-    return n * sh.bits // 8 + (n // 32) * 2
+    return n * (sh.bd if mat == 2 else sh.bits) // 8 + (n // 32) * 2
 
 
 # ---------------------------------------------------------------- clocks
@@ -419,8 +421,8 @@ def measure_decode(moe, h, sh, xs, layers, T, flags, args, steps, warmup, clock_
         step(warmup + i)
         D = h.stats()["active_experts"]
         lb = nl * layer_bytes(sh, D, T)
-        alg["gemv_gateup"] += nl * (D + sh.n_shared) * 2 * mat_bytes(sh)
-        alg["gemv_down"] += nl * (D + sh.n_shared) * mat_bytes(sh)
+        alg["gemv_gateup"] += nl * (D + sh.n_shared) * 2 * mat_bytes(sh, 0)
+        alg["gemv_down"] += nl * (D + sh.n_shared) * mat_bytes(sh, 2)
         alg["decode_fused"] += lb
         alg["layer"] += lb
     prof = kernel_profile(h, step, warmup, nprof)
@@ -436,7 +438,7 @@ def measure_decode(moe, h, sh, xs, layers, T, flags, args, steps, warmup, clock_
 def sub_block(moe, sgpu, wl, sh, T, layers, rank, args, steps, warmup):
     """A separate measured workload (its own handle) reported inside the main line."""
     import torch
-    h = moe.MoeLayer(sh.d, sh.f, sh.E, sh.k, sh.n_shared, layers, sh.bits, T)
+    h = moe.MoeLayer(sh.d, sh.f, sh.E, sh.k, sh.n_shared, layers, sh.bits, T, bits_down=sh.bits_down)
     keep = []
     for l in range(layers):
         w = sgpu.layer_device(sh, rank_master(wl.master, rank), l, wl.zipf)
@@ -480,7 +482,7 @@ def ours(args):
         flags |= names[f]
 
     # ---- setup: layers generated on the device, one handle holding all of them
-    h = moe.MoeLayer(sh.d, sh.f, sh.E, sh.k, sh.n_shared, layers, sh.bits, T)
+    h = moe.MoeLayer(sh.d, sh.f, sh.E, sh.k, sh.n_shared, layers, sh.bits, T, bits_down=sh.bits_down)
     weights = []
     for l in range(layers):
         w = sgpu.layer_device(sh, rank_master(wl.master, rank), l, wl.zipf)
@@ -544,7 +546,9 @@ def ours(args):
                 "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "config": {"workload": args.workload, "tokens_per_step": T, "d": sh.d, "f": sh.f, "experts": sh.E,
-                           "top_k": sh.k, "shared": sh.n_shared, "bits": sh.bits, "layers": layers,
+                           "top_k": sh.k, "shared": sh.n_shared, "bits": sh.bits,
+                           **({"bits_down": sh.bits_down} if sh.bits_down and sh.bits_down != sh.bits else {}),
+                           "layers": layers,
                            "l2": ("inputs larger than L2: 48 layers x 756 MB per step" if chain else
                                   f"inputs larger than L2: {layers} distinct layers cycled, {n_x} fresh inputs"),
                            "parallelism": f"replicas x{world}",

@@ -1,6 +1,7 @@
 // api.cu -- the C ABI (include/moe.h): handle, scratch, argument checks and the
 // order in which the kernels of one routed-MoE layer are enqueued.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -96,11 +97,30 @@ size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
-// Enqueue one kernel (via `f`), counting it and, when profiling is on,
-// bracketing it with a pair of events on the same stream.
+// An NVTX range named after a kernel (domain "moe") around its launch, so a
+// profiler's timeline shows which library step enqueued it; with no profiler
+// attached the range calls return at once.
+struct NvtxRange {
+    explicit NvtxRange(int kernel) {
+        static nvtxDomainHandle_t dom = nvtxDomainCreateA("moe");
+        nvtxEventAttributes_t at = {};
+        at.version = NVTX_VERSION;
+        at.size = NVTX_EVENT_ATTRIB_STRUCT_SIZE;
+        at.messageType = NVTX_MESSAGE_TYPE_ASCII;
+        at.message.ascii = moe_kernel_name(kernel);
+        nvtxDomainRangePushEx(dom, &at);
+        d = dom;
+    }
+    ~NvtxRange() { nvtxDomainRangePop(d); }
+    nvtxDomainHandle_t d;
+};
+
+// Enqueue one kernel (via `f`) inside its NVTX range, counting it and, when
+// profiling is on, bracketing it with a pair of events on the same stream.
 template <class F>
 cudaError_t run(moe_handle* h, int kernel, cudaStream_t s, F&& f) {
     h->launches++;
+    const NvtxRange range(kernel);
     if (!h->prof_on) {
         const cudaError_t e = f();
         if (e != cudaSuccess) h->last_cuda_error = (int)e;
@@ -135,10 +155,9 @@ int bits_down(const moe_config& c) { return c.bits_down ? c.bits_down : c.bits; 
 bool mixed_widths(const moe_config& c) { return bits_down(c) != c.bits; }
 
 // moe_forward takes the tensor-core path (bf16 tcgen05 router, grouped
-// dequant GEMMs) above kFusedMaxTokens tokens, or when forced.  Layers with
-// mixed code widths run on the grouped-GEMV path at every T.
+// dequant GEMMs) above kFusedMaxTokens tokens, or when forced; any code widths.
 bool use_tensor_cores(const moe_config& c, int32_t T, uint32_t flags) {
-    if (mixed_widths(c)) return false;
+    (void)c;
     if (flags & (MOE_FORCE_GEMV | MOE_FORCE_UNFUSED)) return false;
     return T > moe::kFusedMaxTokens || (flags & MOE_FORCE_GEMM);
 }
@@ -340,7 +359,6 @@ moe_status check_forward_call(moe_handle* h, int32_t layer, int32_t T, uint32_t 
     if (T < 0 || T > h->cfg.max_tokens) return MOE_ERR_INVALID_ARG;
     if (flags & ~kAllFlags) return MOE_ERR_INVALID_ARG;
     if ((flags & MOE_FORCE_GEMV) && (flags & MOE_FORCE_GEMM)) return MOE_ERR_INVALID_ARG;
-    if ((flags & MOE_FORCE_GEMM) && mixed_widths(h->cfg)) return MOE_ERR_INVALID_ARG;
     return MOE_OK;
 }
 
@@ -466,10 +484,10 @@ moe_status moe_load_layer(moe_handle* h, int32_t layer, const moe_layer_weights*
     L.router_w = w->router_w;
     L.bias = w->router_bias;
     const int ne = h->cfg.n_experts + h->cfg.n_shared;
-    // the tensor-core path's maps assume one code width for all three matrices
-    if (!mixed_widths(h->cfg) &&
-        (moe::make_weight_maps(&L.w_gu, L.codes, L.scales, ne, h->cfg.f, h->cfg.d, h->cfg.bits) != cudaSuccess ||
-         moe::make_weight_maps(&L.w_dn, L.codes, L.scales, ne, h->cfg.d, h->cfg.f, h->cfg.bits) != cudaSuccess))
+    if (moe::make_weight_maps(&L.w_gu, L.codes, L.scales, ne, h->cfg.d, h->cfg.f, h->cfg.bits, bits_down(h->cfg),
+                              true) != cudaSuccess ||
+        moe::make_weight_maps(&L.w_dn, L.codes, L.scales, ne, h->cfg.d, h->cfg.f, h->cfg.bits, bits_down(h->cfg),
+                              false) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (moe::make_pair_down_maps(&L.pair_dc, &L.pair_ds, L.codes, L.scales, ne, h->cfg.d, h->cfg.f, h->cfg.bits,
                                  bits_down(h->cfg)) != cudaSuccess)

@@ -70,14 +70,21 @@ constexpr int kXPad = 32;                  // 16-bit elements of padding per sta
 constexpr int kHRow = 128 + kXPad;
 constexpr int kCandBytes = 64 * 16;        // per-warp top-k candidate buffer
 constexpr int kMaxKS = 2;                  // input super-tiles per warp of a gate/up tile (d <= 2048)
+constexpr int kRouterIt = 4;               // 16-byte router loads per lane per half row (d <= 2048)
 
 // Optional phase trace (build with -DMOE_PAIR_TRACE): thread 0 of every CTA
 // records the global timer at phase boundaries and adds clock64() differences
-// per phase; moe_debug_pair_trace() / moe_debug_pair_cycles() copy them out.
+// per phase into shared memory (no global round trip inside a phase), written
+// out once at the end; moe_debug_pair_trace() / moe_debug_pair_cycles() copy
+// them to the host.
 #ifdef MOE_PAIR_TRACE
 constexpr int kTraceSlots = 48;
 __device__ unsigned long long g_trace[1024 * kTraceSlots];
 __device__ unsigned long long g_cyc[1024 * 32];
+MOE_DEV unsigned long long* cyc_acc() {
+    __shared__ unsigned long long acc[32];
+    return acc;
+}
 MOE_DEV void trace(int slot) {
     if (threadIdx.x == 0 && slot < kTraceSlots) {
         unsigned long long t;
@@ -87,17 +94,22 @@ MOE_DEV void trace(int slot) {
 }
 MOE_DEV unsigned long long cyc() { return (unsigned long long)clock64(); }
 MOE_DEV void cyc_add(int slot, unsigned long long t0) {
-    if (threadIdx.x == 0) g_cyc[blockIdx.x * 32 + slot] += cyc() - t0;
+    if (threadIdx.x == 0) cyc_acc()[slot] += cyc() - t0;
 }
 MOE_DEV void cyc_reset() {
     if (threadIdx.x == 0)
-        for (int i = 0; i < 32; ++i) g_cyc[blockIdx.x * 32 + i] = 0;
+        for (int i = 0; i < 32; ++i) cyc_acc()[i] = 0;
+}
+MOE_DEV void cyc_flush() {
+    if (threadIdx.x == 0)
+        for (int i = 0; i < 32; ++i) g_cyc[blockIdx.x * 32 + i] = cyc_acc()[i];
 }
 #else
 MOE_DEV void trace(int) {}
 MOE_DEV unsigned long long cyc() { return 0; }
 MOE_DEV void cyc_add(int, unsigned long long) {}
 MOE_DEV void cyc_reset() {}
+MOE_DEV void cyc_flush() {}
 #endif
 
 struct Args {
@@ -221,8 +233,10 @@ MOE_DEV void grid_wait(const unsigned long long* ctr, unsigned long long target,
     uint32_t ns = 32;
     for (uint32_t it = 0; it <= a.spin_limit; ++it) {
         if (ld_acquire_u64(ctr) >= target) return;
-        __nanosleep(ns);
-        if (ns < 128) ns <<= 1;
+        if (it >= 32) {  // back-to-back polls first (the usual wait is a few of them), then back off
+            __nanosleep(ns);
+            if (ns < 128) ns <<= 1;
+        }
     }
     flag_status(a.status, kStatusTimeout);
 }
@@ -355,12 +369,18 @@ MOE_DEV void topk_scan(const double* lg, int E, int k, int lane, int& sel, doubl
 }
 
 // Exact top-k of one token's E fp64 logits (global memory, read through L2).
-// tau = the k-th largest of the 32 lanes' largest keys: at least k logits have
-// a key >= tau, so every logit of the exact top k has a key prefix >= tau's
-// (a smaller prefix means a smaller logit than all of those k).  Those
-// candidates (usually a few more than k) are compacted into shared memory
-// and ranked by (fp64 logit desc, index asc).  Lane r < k returns id r and
-// its weight w_r = softmax over the k selected logits.
+// Each lane holds KPL logits and their 32-bit keys (fp32 prefix | 1023 - e,
+// unique).  Rounds r = 0 .. k take the warp's largest remaining key with one
+// max-reduction; the index is read back from the key, and the lane that held
+// it parks (logit, index) at cand[r] and drops the key.  The k largest keys
+// are the exact top k when the k-th key's prefix is strictly above the
+// (k+1)-th's: every logit left behind then has a smaller prefix than each
+// selected one, hence a smaller value.  Their order is the keys' order when
+// adjacent prefixes differ; where two selected keys share a prefix the k
+// entries are ranked again by (fp64 logit desc, index asc).  A tie of the
+// k-th and (k+1)-th prefixes (rare: equal fp32 images) takes the exact
+// scan.  Lane r < k returns id r and its weight w_r = softmax over the k
+// selected logits.
 template <int KPL>
 MOE_DEV void topk_token(const double* lg, int E, int k, int lane, Cand* cand, int& id_out, float& w_out) {
     unsigned long long tc = cyc();
@@ -377,63 +397,70 @@ MOE_DEV void topk_token(const double* lg, int E, int k, int lane, Cand* cand, in
     }
     cyc_add(10, tc);  // loads + keys
     tc = cyc();
-    int rk = 0;  // lanes whose largest key beats mine
-#pragma unroll
-    for (int o = 1; o < 32; ++o) rk += __shfl_sync(0xffffffffu, lmax, (lane + o) & 31) > lmax ? 1 : 0;
-    const int src = __ffs(__ballot_sync(0xffffffffu, rk == k - 1 && lmax != 0u)) - 1;
-    const uint32_t P = __shfl_sync(0xffffffffu, lmax, max(src, 0)) & 0xFFFFFC00u;
-    int cnt = 0;
-#pragma unroll
-    for (int j = 0; j < KPL; ++j) cnt += (key[j] != 0u && (key[j] & 0xFFFFFC00u) >= P) ? 1 : 0;
-    const int C = (int)__reduce_add_sync(0xffffffffu, (unsigned)cnt);
-    int sel = -1;
-    double lsel = 0.0, top = 0.0;
-    cyc_add(11, tc);  // threshold + count
-    tc = cyc();
-    if (src >= 0 && C >= k && C <= 32) {
-        int off = 0;
+    const int rounds = min(k + 1, E);
+    uint32_t my_key = 0u;       // lane r < k: the r-th largest key
+    uint32_t pk = 0u, pn = 0u;  // prefixes of the k-th and (k+1)-th largest keys
+    for (int r = 0; r < rounds; ++r) {
+        const uint32_t m = __reduce_max_sync(0xffffffffu, lmax);
+        if (lane == r) my_key = m;
+        if (r == k - 1) pk = m & 0xFFFFFC00u;
+        if (r == k) pn = m & 0xFFFFFC00u;
+        // the holder of key m (keys are unique: one lane, one j) parks it
+        lmax = 0u;
 #pragma unroll
         for (int j = 0; j < KPL; ++j) {
-            const bool in = key[j] != 0u && (key[j] & 0xFFFFFC00u) >= P;
-            const unsigned bal = __ballot_sync(0xffffffffu, in);
-            if (in) {
-                Cand& cd = cand[off + __popc(bal & ((1u << lane) - 1u))];
-                cd.v = v[j];
-                cd.e = lane + 32 * j;
+            if (key[j] == m) {
+                cand[r].v = v[j];
+                cand[r].e = 1023 - (int)(m & 1023u);
+                key[j] = 0u;
             }
-            off += __popc(bal);
+            lmax = max(lmax, key[j]);
         }
-        __syncwarp();
-        cyc_add(12, tc);  // compaction
-        tc = cyc();
-        int rank = 0, my_e = 0;
+    }
+    __syncwarp();
+    cyc_add(11, tc);  // k + 1 extraction rounds
+    tc = cyc();
+    int sel = -1;
+    double lsel = 0.0, top = 0.0;
+    if (rounds == k || pk > pn) {
         double my_v = 0.0;
-        if (lane < C) {
+        int my_e = 0;
+        if (lane < k) {
             my_v = cand[lane].v;
             my_e = cand[lane].e;
-            const uint64_t my_k = order_key64(my_v);
-            for (int j = 0; j < C; ++j) {
-                const Cand o = cand[j];
-                if (j != lane && better64(order_key64(o.v), o.e, my_k, my_e)) ++rank;
+        }
+        // adjacent selected keys with one prefix: rank the k exactly
+        const uint32_t prev = __shfl_up_sync(0xffffffffu, my_key, 1);
+        const bool tie = lane >= 1 && lane < k && (prev & 0xFFFFFC00u) == (my_key & 0xFFFFFC00u);
+        if (__any_sync(0xffffffffu, tie)) {
+            int rank = 0;
+            if (lane < k) {
+                const uint64_t mk = order_key64(my_v);
+                for (int j = 0; j < k; ++j) {
+                    const Cand o = cand[j];
+                    if (j != lane && better64(order_key64(o.v), o.e, mk, my_e)) ++rank;
+                }
+            }
+            __syncwarp();
+            if (lane < k) {
+                cand[32 + rank].v = my_v;
+                cand[32 + rank].e = my_e;
+            }
+            __syncwarp();
+            if (lane < k) {
+                my_v = cand[32 + lane].v;
+                my_e = cand[32 + lane].e;
             }
         }
-        __syncwarp();
-        if (lane < C && rank < k) {
-            cand[32 + rank].v = my_v;
-            cand[32 + rank].e = my_e;
-        }
-        __syncwarp();
-        top = cand[32].v;
-        if (lane < k) {
-            sel = cand[32 + lane].e;
-            lsel = cand[32 + lane].v;
-        }
-        __syncwarp();
+        sel = lane < k ? my_e : -1;
+        lsel = my_v;
+        top = __shfl_sync(0xffffffffu, my_v, 0);
+        cyc_add(13, tc);  // ranking
     } else {
         topk_scan(lg, E, k, lane, sel, lsel, top);
         cyc_add(15, tc);  // slow path taken
     }
-    cyc_add(13, tc);  // ranking
+    __syncwarp();  // cand is reused by the next token of this warp
     tc = cyc();
     const float ex = lane < k ? expf((float)(lsel - top)) : 0.0f;
     float z = ex;
@@ -570,78 +597,74 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ================================================================ consumers
         const unsigned long long c_start = cyc();
-        // ---- 1. router rows [r0, r1): exact logits, 4 rows x 4 tokens per pass
+        // ---- 1. router rows [r0, r1): exact logits.  Warp task = (row, 4
+        // tokens, half of the input dimension): a lane holds 8 of every 256
+        // inputs of its half (all its weight loads issued at once) and sums
+        // exact bf16 products in fp64; the two halves meet in shared memory
+        // and are added in a fixed order.
         {
             const int r0 = (int)((int64_t)b * E / G), r1 = (int)((int64_t)(b + 1) * E / G), R = r1 - r0;
-            double* part = reinterpret_cast<double*>(gus);  // [kCWarps][4 rows][4 tokens]
+            const int TG = (T + 3) / 4, NP = R * TG, hd = d / 2;
+            double* part = reinterpret_cast<double*>(gus);  // [NP][2 halves][4 tokens]
             bool x_ready = false;
-            for (int rp = 0; rp < R; rp += 4) {
-                const int nr = min(4, R - rp);
-                for (int t0 = 0; t0 < T; t0 += 4) {
-                    const int nt4 = min(4, T - t0);
-                    double acc[4][4];
+            for (int task = warp; task < 2 * NP; task += kCWarps) {
+                const int pr = task >> 1, hf = task & 1;
+                const int r = pr / TG, t0 = 4 * (pr - r * TG), nt4 = min(4, T - t0);
+                const uint16_t* wrow = a.wr + (int64_t)(r0 + r) * d + hf * hd;
+                uint4 wv[kRouterIt];
 #pragma unroll
-                    for (int r = 0; r < 4; ++r)
+                for (int it = 0; it < kRouterIt; ++it) {
+                    const int i = lane * 8 + 256 * it;
+                    wv[it] = i < hd ? __ldg(reinterpret_cast<const uint4*>(wrow + i)) : make_uint4(0, 0, 0, 0);
+                }
+                if (!x_ready) {
+                    copy_wait(&barX, 0u, a);
+                    x_ready = true;
+                }
+                double acc[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
-                        for (int t = 0; t < 4; ++t) acc[r][t] = 0.0;
-                    for (int cg = tid; cg < d / 4; cg += kConsumers) {
-                        uint2 wv[4];
-#pragma unroll
-                        for (int r = 0; r < 4; ++r)
-                            wv[r] = r < nr ? __ldg(reinterpret_cast<const uint2*>(a.wr + (int64_t)(r0 + rp + r) * d) + cg)
-                                           : make_uint2(0, 0);
-                        if (!x_ready) {
-                            copy_wait(&barX, 0u, a);
-                            x_ready = true;
-                        }
-                        double xd[4][4];
+                for (int it = 0; it < kRouterIt; ++it) {
+                    const int i = lane * 8 + 256 * it;
+                    if (i < hd) {
+                        const uint32_t wu[4] = {wv[it].x, wv[it].y, wv[it].z, wv[it].w};
 #pragma unroll
                         for (int t = 0; t < 4; ++t) {
-                            const uint2 xv = t < nt4 ? *reinterpret_cast<const uint2*>(xs + (t0 + t) * xstride + 4 * cg)
-                                                     : make_uint2(0, 0);
-                            xd[t][0] = bf16_to_f64(xv.x & 0xFFFFu);
-                            xd[t][1] = bf16_to_f64(xv.x >> 16);
-                            xd[t][2] = bf16_to_f64(xv.y & 0xFFFFu);
-                            xd[t][3] = bf16_to_f64(xv.y >> 16);
-                        }
+                            if (t < nt4) {
+                                const uint4 xv =
+                                    *reinterpret_cast<const uint4*>(xs + (t0 + t) * xstride + hf * hd + i);
+                                const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            const double w0 = bf16_to_f64(wv[r].x & 0xFFFFu), w1 = bf16_to_f64(wv[r].x >> 16);
-                            const double w2 = bf16_to_f64(wv[r].y & 0xFFFFu), w3 = bf16_to_f64(wv[r].y >> 16);
-#pragma unroll
-                            for (int t = 0; t < 4; ++t) {
-                                acc[r][t] = fma(w0, xd[t][0], acc[r][t]);
-                                acc[r][t] = fma(w1, xd[t][1], acc[r][t]);
-                                acc[r][t] = fma(w2, xd[t][2], acc[r][t]);
-                                acc[r][t] = fma(w3, xd[t][3], acc[r][t]);
+                                for (int h2 = 0; h2 < 4; ++h2) {
+                                    acc[t] = fma(bf16_to_f64(wu[h2] & 0xFFFFu), bf16_to_f64(xu[h2] & 0xFFFFu), acc[t]);
+                                    acc[t] = fma(bf16_to_f64(wu[h2] >> 16), bf16_to_f64(xu[h2] >> 16), acc[t]);
+                                }
                             }
                         }
                     }
-                    if (!x_ready) {
-                        copy_wait(&barX, 0u, a);
-                        x_ready = true;
-                    }
+                }
 #pragma unroll
-                    for (int r = 0; r < 4; ++r)
+                for (int t = 0; t < 4; ++t)
 #pragma unroll
-                        for (int t = 0; t < 4; ++t) {
-                            double v = acc[r][t];
+                    for (int o = 16; o > 0; o >>= 1) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+                if (lane < 4) {
+                    double v = acc[0];
 #pragma unroll
-                            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                            if (lane == 0) part[(warp * 4 + r) * 4 + t] = v;
-                        }
-                    consumer_sync();
-                    if (tid < nr * nt4) {
-                        const int r = tid / nt4, t = tid - r * nt4, e = r0 + rp + r;
-                        const double bb = a.bias ? (double)a.bias[e] : 0.0;
-                        double sum = 0.0;
-                        for (int w = 0; w < kCWarps; ++w) sum += part[(w * 4 + r) * 4 + t];
-                        a.logits64[(int64_t)(t0 + t) * E + e] = sum + bb;
-                    }
-                    consumer_sync();
+                    for (int t = 1; t < 4; ++t)
+                        if (lane == t) v = acc[t];
+                    part[(pr * 2 + hf) * 4 + lane] = v;
                 }
             }
-            if (!x_ready) copy_wait(&barX, 0u, a);  // a CTA without router rows
+            if (!x_ready) copy_wait(&barX, 0u, a);  // a warp without router work
+            consumer_sync();
+            for (int idx = tid; idx < NP * 4; idx += kConsumers) {
+                const int pr = idx >> 2, t = idx & 3, r = pr / TG, tt = 4 * (pr - r * TG) + t;
+                if (tt < T) {
+                    const int e = r0 + r;
+                    const double bb = a.bias ? (double)a.bias[e] : 0.0;
+                    a.logits64[(int64_t)tt * E + e] = (part[(pr * 2) * 4 + t] + part[(pr * 2 + 1) * 4 + t]) + bb;
+                }
+            }
+            consumer_sync();  // every logit is written before thread 0 announces them
         }
         cyc_add(27, c_start);
         trace(1);
@@ -898,116 +921,140 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (tid == 0) mbar_arrive_relaxed_remote(peer_addr(&hempty[hb3], rank ^ 1u));
         };
 
-        // ---- shared-expert units, overlapping the router hand-off
-        for (int i = 0; i < n_pre; ++i) {
-            gate_up(i);
-            down(i);
-        }
-        trace(2);
-
-        // ---- 2. every CTA's router rows, then top-k and the schedule
-        if (tid == 0) grid_wait(a.ctr, router_target, a);
-        consumer_sync();
-        trace(3);
-        const unsigned long long ctk = cyc();
-        for (int t = warp; t < T; t += kCWarps) {
-            const double* lg = a.logits64 + (int64_t)t * E;
-            int id;
-            float wt;
-            if (E <= 512)
-                topk_token<16>(lg, E, k, lane, cand + warp * 64, id, wt);
-            else
-                topk_token<32>(lg, E, k, lane, cand + warp * 64, id, wt);
-            if (lane < k) {
-                sids[t * k + lane] = id;
-                sw[t * k + lane] = wt;
-                if (b == 0) {
-                    a.ids[(int64_t)t * k + lane] = id;
-                    a.w[(int64_t)t * k + lane] = wt;
+        // ---- 2. every CTA's router rows, then top-k and the schedule (run once,
+        // between the shared-expert units and the first routed unit); returns
+        // this cluster's unit count
+        auto routing = [&]() -> int {
+            if (tid == 0) grid_wait(a.ctr, router_target, a);
+            consumer_sync();
+            trace(3);
+            const unsigned long long ctk = cyc();
+            for (int t = warp; t < T; t += kCWarps) {
+                const double* lg = a.logits64 + (int64_t)t * E;
+                int id;
+                float wt;
+                if (E <= 512)
+                    topk_token<16>(lg, E, k, lane, cand + warp * 64, id, wt);
+                else
+                    topk_token<32>(lg, E, k, lane, cand + warp * 64, id, wt);
+                if (lane < k) {
+                    sids[t * k + lane] = id;
+                    sw[t * k + lane] = wt;
+                    if (b == 0) {
+                        a.ids[(int64_t)t * k + lane] = id;
+                        a.w[(int64_t)t * k + lane] = wt;
+                    }
                 }
             }
-        }
-        cyc_add(6, ctk);
-        unsigned long long csc = cyc();
-        consumer_sync();
-        cyc_add(16, csc);  // wait for the other warps' top-k
-        csc = cyc();
-        trace(4);
-        for (int p = tid; p < T * k; p += kConsumers) {
-            const int e = sids[p], t = p / k, r = p - t * k;
-            if (e >= 0 && e < E) {
-                atomicOr(&emask[e], 1u << t);
-                atomicMin(&ebest[e], r);
-            } else {
-                flag_status(a.status, kStatusBounds);
-            }
-        }
-        consumer_sync();
-        {
-            // kept experts in ascending order: warp w owns a contiguous chunk
-            const int chunk = ((E + kCWarps - 1) / kCWarps + 31) & ~31;
-            const int e0 = warp * chunk, e1 = min(E, e0 + chunk);
-            auto keep = [&](int e) {
-                return e < e1 && emask[e] != 0u && !(a.skip_rank > 0 && ebest[e] >= a.skip_rank) &&
-                       e >= a.e_begin && e < a.e_end;
-            };
-            int cnt = 0;
-            for (int base = e0; base < e1; base += 32) cnt += __popc(__ballot_sync(0xffffffffu, keep(base + lane)));
-            if (lane == 0) s_wcnt[warp] = cnt;
+            cyc_add(6, ctk);
+            unsigned long long csc = cyc();
             consumer_sync();
-            int p0 = ns;
-            for (int w = 0; w < warp; ++w) p0 += s_wcnt[w];
-            for (int base = e0; base < e1; base += 32) {
-                const bool kp = keep(base + lane);
-                const unsigned bal = __ballot_sync(0xffffffffu, kp);
-                if (kp) slot_e[p0 + __popc(bal & ((1u << lane) - 1u))] = base + lane;
-                p0 += __popc(bal);
-            }
-            if (tid == 0) {
-                int tot = ns;
-                for (int w = 0; w < kCWarps; ++w) tot += s_wcnt[w];
-                s_nslots = tot;
+            cyc_add(16, csc);  // wait for the other warps' top-k
+            csc = cyc();
+            trace(4);
+            for (int p = tid; p < T * k; p += kConsumers) {
+                const int e = sids[p], t = p / k, r = p - t * k;
+                if (e >= 0 && e < E) {
+                    atomicOr(&emask[e], 1u << t);
+                    atomicMin(&ebest[e], r);
+                } else {
+                    flag_status(a.status, kStatusBounds);
+                }
             }
             consumer_sync();
-        }
-        const int n_slots = s_nslots;
-        cyc_add(17, csc);  // masks + compaction
-        csc = cyc();
-        // place of each slot in its tokens' lists (slot order): the partial sums' row index
-        if (tid < T) {
-            int r = 0;
-            for (int s = 0; s < n_slots; ++s) {
-                const uint32_t m = s < ns ? 0xFFFFFFFFu : emask[slot_e[s]];
-                if ((m >> tid) & 1u) pos[s * T + tid] = (unsigned char)r++;
+            {
+                // kept experts in ascending order: warp w owns a contiguous chunk
+                const int chunk = ((E + kCWarps - 1) / kCWarps + 31) & ~31;
+                const int e0 = warp * chunk, e1 = min(E, e0 + chunk);
+                auto keep = [&](int e) {
+                    return e < e1 && emask[e] != 0u && !(a.skip_rank > 0 && ebest[e] >= a.skip_rank) &&
+                           e >= a.e_begin && e < a.e_end;
+                };
+                int cnt = 0;
+                for (int base = e0; base < e1; base += 32) cnt += __popc(__ballot_sync(0xffffffffu, keep(base + lane)));
+                if (lane == 0) s_wcnt[warp] = cnt;
+                consumer_sync();
+                int p0 = ns;
+                for (int w = 0; w < warp; ++w) p0 += s_wcnt[w];
+                for (int base = e0; base < e1; base += 32) {
+                    const bool kp = keep(base + lane);
+                    const unsigned bal = __ballot_sync(0xffffffffu, kp);
+                    if (kp) slot_e[p0 + __popc(bal & ((1u << lane) - 1u))] = base + lane;
+                    p0 += __popc(bal);
+                }
+                if (tid == 0) {
+                    int tot = ns;
+                    for (int w = 0; w < kCWarps; ++w) tot += s_wcnt[w];
+                    s_nslots = tot;
+                }
+                consumer_sync();
             }
-            tn[tid] = r;
-        }
-        if (tid == 0) {
-            const int U = n_slots * FC;
-            const int nu = U > q ? (U - 1 - q) / nc + 1 : 0;
-            s_nunits = max(nu, n_pre);
-            if (b == 0) {
+            const int n_slots = s_nslots;
+            cyc_add(17, csc);  // masks + compaction
+            csc = cyc();
+            // place of each slot in its tokens' lists (slot order): the partial sums'
+            // row index.  Warp 0, lane = slot: per token, a ballot over the slots
+            // that hold it gives each slot's place by a prefix count.
+            if (warp == 0) {
+                int base[kPairMaxTokens];  // places taken so far, per token
+    #pragma unroll
+                for (int t = 0; t < kPairMaxTokens; ++t) base[t] = 0;
                 int big = 0;
-                for (int s2 = ns; s2 < n_slots; ++s2) big = max(big, __popc(emask[slot_e[s2]]));
-                a.meta->n_active = n_slots - ns;
-                a.meta->max_count = big;
-                a.meta->n_fixup = 0;  // the fp64 logits are ranked exactly
+                const uint32_t lt = (1u << lane) - 1u;
+                for (int s0 = 0; s0 < n_slots; s0 += 32) {
+                    const int sl = s0 + lane;
+                    const uint32_t m = sl >= n_slots ? 0u : (sl < ns ? 0xFFFFFFFFu : emask[slot_e[sl]]);
+                    if (sl >= ns && sl < n_slots) big = max(big, __popc(m));
+    #pragma unroll
+                    for (int t = 0; t < kPairMaxTokens; ++t) {
+                        if (t < T) {
+                            const uint32_t bal = __ballot_sync(0xffffffffu, (m >> t) & 1u);
+                            if ((m >> t) & 1u) pos[sl * T + t] = (unsigned char)(base[t] + __popc(bal & lt));
+                            base[t] += __popc(bal);
+                        }
+                    }
+                }
+    #pragma unroll
+                for (int t = 0; t < kPairMaxTokens; ++t)
+                    if (t < T && lane == t) tn[t] = base[t];
+                big = (int)__reduce_max_sync(0xffffffffu, (unsigned)big);
+                if (lane == 0) {
+                    const int U = n_slots * FC;
+                    const int nu = U > q ? (U - 1 - q) / nc + 1 : 0;
+                    s_nunits = max(nu, n_pre);
+                    if (b == 0) {
+                        a.meta->n_active = n_slots - ns;
+                        a.meta->max_count = big;
+                        a.meta->n_fixup = 0;  // the fp64 logits are ranked exactly
+                    }
+                }
             }
-        }
-        cyc_add(18, csc);  // places + meta
-        consumer_sync();
-        if (tid == 0) mbar_arrive(&sched);  // the producer may issue the routed units
-        const int n_units = s_nunits;
-        cyc_add(7, ctk);
-        trace(5);
+            cyc_add(18, csc);  // places + meta
+            consumer_sync();
+            if (tid == 0) mbar_arrive(&sched);  // the producer may issue the routed units
+            cyc_add(7, ctk);
+            trace(5);
+            return s_nunits;
+        };
 
-        // ---- 3. routed units, pipelined: gate/up of unit i, then the down of unit i - 1
-        for (int i = n_pre; i < n_units; ++i) {
+        // ---- 3. units, pipelined: gate/up of unit i, then the down of unit i - 1.
+        // The shared-expert units (i < n_pre) need no routing and overlap the
+        // router hand-off; each unit step is inlined once, which keeps the
+        // kernel's instruction footprint small.
+        int n_units = n_pre;
+        bool routed = false;
+        for (int i = 0;; ++i) {
+            if (i == n_pre && !routed) {
+                trace(2);
+                n_units = routing();
+                routed = true;
+            }
+            if (i >= n_units) break;
             gate_up(i);
-            trace(6 + 2 * min(i - n_pre, 15));
-            if (i > n_pre) down(i - 1);
+            if (i >= n_pre) trace(6 + 2 * min(i - n_pre, 15));
+            if (i > 0) down(i - 1);
         }
-        if (n_units > n_pre) down(n_units - 1);
+        if (n_units > 0) down(n_units - 1);
         trace(38);
 
         // ---- 4. every CTA's partial sums, then this CTA's slice of y
@@ -1077,6 +1124,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         cyc_add(20, ctl);
         trace(40);
+        cyc_flush();
     }
     // every thread of both CTAs: no remote access is still in flight when a CTA exits
     cluster_arrive();

@@ -291,6 +291,15 @@ MOE_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64
         : "memory");
 }
 
+// 3-D TMA tile load (no multicast) completing on `bar`
+MOE_DEV void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar))
+        : "memory");
+}
+
 MOE_DEV int4 load_desc(const GemmArgs& g, int tile) { return __ldg(&g.desc[tile]); }
 
 template <int BITS, bool GATEUP>
@@ -535,9 +544,11 @@ __global__ void __launch_bounds__(kExpertThreads, 1)
 #pragma unroll
             for (int m = 0; m < C::kMats; ++m) {
                 uint8_t* A = sb + m * C::kA;
-                const int row = (expert * 3 + (GATEUP ? m : 2)) * mrows + jt * 8;
-                tma_load_2d(A, &cmap, kt * 64 * BITS, row, &load_bar[st]);
-                tma_load_2d(A + C::kCodeBytes, &smap, kt * 64, row, &load_bar[st]);
+                // codes: (word, row tile of this kernel's matrices, expert); scales: every
+                // expert's three matrices stacked as rows of 16-row tiles
+                tma_load_3d(A, &cmap, kt * 64 * BITS, m * mrows + jt * 8, expert, &load_bar[st]);
+                tma_load_2d(A + C::kCodeBytes, &smap, kt * 64, (expert * 3 + (GATEUP ? m : 2)) * mrows + jt * 8,
+                            &load_bar[st]);
             }
         }
     }
@@ -791,7 +802,7 @@ cudaError_t launch_gemm_down(const ExpertArgs& a, const GemmMaps& maps, const fl
     g.o = static_cast<__half*>(o);
     g.desc = desc;
     g.n_tiles = counts + 1;
-    switch (a.bits) {
+    switch (a.bits_down ? a.bits_down : a.bits) {
         case 2: return gemm_bits<2, false>(g, maps, s);
         case 3: return gemm_bits<3, false>(g, maps, s);
         case 4: return gemm_bits<4, false>(g, maps, s);
@@ -838,18 +849,35 @@ cudaError_t make_row_maps(GemmMaps* m, const void* base, int64_t rows, int cols)
                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// Maps of a layer's packed codes and scales for matrices [N x K] (gate/up:
-// N = f, K = d; down: N = d, K = f): every matrix is N/16 rows of K/128
-// super-tiles, and all E + n_shared experts' three matrices are stacked, so
-// row (expert * 3 + mat) * N/16 + tile is 16-row tile `tile` of that matrix.
-// One box = 8 row-tiles x one super-tile (256 b bytes of codes as 32-bit
-// words; 64 fp16 scales).
-cudaError_t make_weight_maps(GemmMaps* m, const void* codes, const void* scales, int n_experts_total, int N, int K,
-                             int bits) {
-    const int64_t rows = (int64_t)n_experts_total * 3 * (N / 16);
-    cudaError_t e = encode_2d(&m->codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, codes, rows, (int64_t)(K / 128) * 64 * bits,
-                              64 * bits, 8, CU_TENSOR_MAP_SWIZZLE_NONE);
+static cudaError_t encode_3d(CUtensorMap* map, CUtensorMapDataType type, int elem_bytes, const void* base,
+                             const cuuint64_t (&dims)[3], const cuuint64_t (&strides_bytes)[2], const cuuint32_t (&box)[3]);
+
+// Maps of a layer's packed codes and scales for one kernel of the expert
+// GEMM: gate/up (N = f rows per matrix, K = d) or down (N = d, K = f).  Every
+// matrix is N/16 row tiles of K/128 super-tiles (256 b bytes of codes and 64
+// fp16 scales each), at its own code width b.
+//   codes:  a 3-D view (32-bit word, row tile, expert) starting at the
+//           kernel's first matrix -- gate and up are adjacent at the same
+//           width, so their 2N/16 row tiles form one plane -- with the
+//           expert stride f*d*(2*bits + bits_down)/8 bytes, so the two
+//           kernels may read different widths.  One box = 8 row tiles x one
+//           super-tile.
+//   scales: every expert's three matrices stacked as rows of 16-row tiles
+//           (the scales do not depend on the code width), row
+//           (expert * 3 + mat) * N/16 + tile.  One box = 8 row tiles x 64.
+cudaError_t make_weight_maps(GemmMaps* m, const void* codes, const void* scales, int n_experts_total, int d, int f,
+                             int bits, int bits_down, bool gateup) {
+    const int N = gateup ? f : d, K = gateup ? d : f, b = gateup ? bits : bits_down;
+    const int64_t code_stride = (int64_t)f * d * (2 * bits + bits_down) / 8;
+    const uint8_t* base = static_cast<const uint8_t*>(codes) + (gateup ? 0 : 2 * (int64_t)f * d * bits / 8);
+    const int64_t words = (int64_t)(K / 128) * 64 * b;  // per row tile
+    const cuuint64_t cdims[3] = {(cuuint64_t)words, (cuuint64_t)((gateup ? 2 : 1) * (N / 16)),
+                                 (cuuint64_t)n_experts_total};
+    const cuuint64_t cstr[2] = {(cuuint64_t)words * 4, (cuuint64_t)code_stride};
+    const cuuint32_t cbox[3] = {(cuuint32_t)(64 * b), 8, 1};
+    cudaError_t e = encode_3d(&m->codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, base, cdims, cstr, cbox);
     if (e != cudaSuccess) return e;
+    const int64_t rows = (int64_t)n_experts_total * 3 * (N / 16);
     return encode_2d(&m->scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, scales, rows, (int64_t)(K / 128) * 64, 64, 8,
                      CU_TENSOR_MAP_SWIZZLE_NONE);
 }

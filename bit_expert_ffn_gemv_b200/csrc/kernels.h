@@ -136,8 +136,8 @@ struct GemmMaps {
     CUtensorMap b_small, b_big, codes, scales;
 };
 cudaError_t make_row_maps(GemmMaps* m, const void* base, int64_t rows, int cols);
-cudaError_t make_weight_maps(GemmMaps* m, const void* codes, const void* scales, int n_experts_total, int N, int K,
-                             int bits);
+cudaError_t make_weight_maps(GemmMaps* m, const void* codes, const void* scales, int n_experts_total, int d, int f,
+                             int bits, int bits_down, bool gateup);
 cudaError_t launch_gather_f16(const void* x, int T, int d, int k, int n_shared, const int32_t* pairs,
                               const int32_t* n_pairs, void* xg, uint32_t* status, cudaStream_t s);
 cudaError_t launch_gemm_gateup(const ExpertArgs& a, const GemmMaps& maps, const int4* desc, const int32_t* counts,

@@ -89,8 +89,10 @@ typedef struct {
                            A width other than `bits` gives per-tensor mixed
                            precision (GSQ-RCO's per-tensor bit allocation, as the
                            tech.okbari.net guide describes it in its GSQ-RCO
-                           section); such layers run on the grouped-GEMV kernels
-                           at every T (MOE_FORCE_GEMM is then an INVALID_ARG). */
+                           section).  Every path reads each matrix at its own
+                           width: the fused decode kernel (T <= 16; the older
+                           persistent kernel takes one width only), the grouped
+                           GEMV and the tensor-core grouped GEMM. */
 } moe_config;
 
 typedef struct {
@@ -159,8 +161,8 @@ moe_status moe_route(moe_handle* h, int32_t layer, const void* x, int32_t T, int
  * residual stream in place (x += layer(x)): every read of x is enqueued
  * before the final write of y.  T = 0 is a no-op.
  * Errors: INVALID_ARG (layer out of range, T < 0 or > max_tokens, NULL or
- * misaligned x / y, an unknown flag, MOE_FORCE_GEMV with MOE_FORCE_GEMM,
- * MOE_FORCE_GEMM on a mixed-width layer), NOT_LOADED, CUDA; nothing is
+ * misaligned x / y, an unknown flag, MOE_FORCE_GEMV with MOE_FORCE_GEMM),
+ * NOT_LOADED, CUDA; nothing is
  * enqueued on an argument error.  Device-side errors (MOE_ERR_TIMEOUT,
  * MOE_ERR_BOUNDS, MOE_ERR_RANGE) surface through moe_check_status.
  */

@@ -40,7 +40,7 @@ def lib():
             L = ctypes.CDLL(_LIB)
             u64, i32, vp = ctypes.c_uint64, ctypes.c_int, ctypes.c_void_p
             L.synth_gpu_experts.restype = i32
-            L.synth_gpu_experts.argtypes = [u64, ctypes.c_uint32, i32, i32, i32, i32, i32, vp, vp, vp]
+            L.synth_gpu_experts.argtypes = [u64, ctypes.c_uint32, i32, i32, i32, i32, i32, i32, vp, vp, vp]
             L.synth_gpu_normal_bf16.restype = i32
             L.synth_gpu_normal_bf16.argtypes = [u64, ctypes.c_int64, ctypes.c_double, vp, vp]
             L.synth_gpu_key.restype = u64
@@ -56,12 +56,9 @@ def _stream():
 
 def experts_into(codes, scales, shape: MoeShape, master: int, layer: int, expert0: int, n: int):
     """Generate experts expert0..expert0+n-1 of a layer into CUDA tensors (uint8 / int16)."""
-    if shape.bd != shape.bits:
-        raise ValueError("the device generator draws one code width per layer; generate mixed-width layers "
-                         "on the host (synth.layer_host)")
     cb, sb = expert_bytes(shape)
     assert codes.numel() >= n * cb and scales.numel() * 2 >= n * sb
-    rc = lib().synth_gpu_experts(master, layer, shape.d, shape.f, expert0, n, shape.bits, codes.data_ptr(),
+    rc = lib().synth_gpu_experts(master, layer, shape.d, shape.f, expert0, n, shape.bits, shape.bd, codes.data_ptr(),
                                  scales.data_ptr(), _stream())
     if rc != 0:
         raise RuntimeError(f"synth_gpu_experts failed ({rc})")

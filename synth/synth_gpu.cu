@@ -66,12 +66,16 @@ __device__ static void dev_pair(uint64_t key, uint64_t n, double& z0, double& z1
 // One CTA of 64 threads per 16 x 128 super-tile of one matrix.  Thread t
 // generates and quantises the 32-weight block (row t/4, block t%4); lanes
 // 0..31 then pack the super-tile.
+// Matrices mat0 .. mat0 + gridDim.y - 1 of each expert, all at width BITS:
+// expert e's codes start at e * code_stride, matrix mat0's at code_off within
+// them (the next matrices follow at f*d*BITS/8 apart).
 template <int BITS>
 __global__ void __launch_bounds__(64) gen_matrix_kernel(uint64_t master, uint32_t layer, int d, int f, int expert0,
+                                                        int mat0, int64_t code_stride, int64_t code_off,
                                                         uint8_t* __restrict__ codes, uint16_t* __restrict__ scales) {
     __shared__ uint8_t us[16][128];
     __shared__ uint16_t ss[16][4];
-    const int mat = blockIdx.y;                 // 0 gate, 1 up, 2 down
+    const int mat = mat0 + (int)blockIdx.y;     // 0 gate, 1 up, 2 down
     const int expert = expert0 + blockIdx.z;
     const int N = mat < 2 ? f : d, K = mat < 2 ? d : f;
     const int KT = K / 128;
@@ -110,7 +114,8 @@ __global__ void __launch_bounds__(64) gen_matrix_kernel(uint64_t master, uint32_
     if (threadIdx.x >= 32) return;
     const int lane = threadIdx.x, g = lane >> 2, c = lane & 3;
     const int64_t mat_codes = (int64_t)f * d * BITS / 8, mat_scales = (int64_t)f * d / 32;
-    uint8_t* cb = codes + ((int64_t)blockIdx.z * 3 + mat) * mat_codes + (int64_t)st * 256 * BITS;
+    uint8_t* cb = codes + (int64_t)blockIdx.z * code_stride + code_off + (int64_t)(mat - mat0) * mat_codes +
+                  (int64_t)st * 256 * BITS;
     uint16_t* sb = scales + ((int64_t)blockIdx.z * 3 + mat) * mat_scales + (int64_t)st * 64;
     uint32_t lo[4] = {0, 0, 0, 0}, hi[4] = {0, 0, 0, 0};
     for (int kb = 0; kb < 4; ++kb)
@@ -149,24 +154,45 @@ __global__ void gen_bf16_kernel(uint64_t key, int64_t n, double stdv, uint16_t* 
     if (2 * p + 1 < n) out[2 * p + 1] = __bfloat16_as_ushort(__float2bfloat16_rn(b));
 }
 
+template <int B>
+static void launch_gen(uint64_t master, uint32_t layer, int d, int f, int expert0, int n_experts, int mat0, int nmat,
+                       int64_t code_stride, int64_t code_off, uint8_t* c, uint16_t* sc, cudaStream_t s) {
+    const int st_gu = (f / 16) * (d / 128), st_dn = (d / 16) * (f / 128);
+    dim3 grid(st_gu > st_dn ? st_gu : st_dn, nmat, n_experts);
+    gen_matrix_kernel<B><<<grid, 64, 0, s>>>(master, layer, d, f, expert0, mat0, code_stride, code_off, c, sc);
+}
+
+static void gen_mats(int bits, uint64_t master, uint32_t layer, int d, int f, int expert0, int n_experts, int mat0,
+                     int nmat, int64_t code_stride, int64_t code_off, uint8_t* c, uint16_t* sc, cudaStream_t s) {
+    switch (bits) {
+        case 2: launch_gen<2>(master, layer, d, f, expert0, n_experts, mat0, nmat, code_stride, code_off, c, sc, s); break;
+        case 3: launch_gen<3>(master, layer, d, f, expert0, n_experts, mat0, nmat, code_stride, code_off, c, sc, s); break;
+        default: launch_gen<4>(master, layer, d, f, expert0, n_experts, mat0, nmat, code_stride, code_off, c, sc, s);
+    }
+}
+
 extern "C" {
 
 // Experts expert0 .. expert0+n_experts-1 of layer `layer` (gate, up, down
-// each), written back to back into codes/scales (device).  0 on success.
+// each), written back to back into codes/scales (device): gate and up at
+// `bits`, down at `bits_down` (0: bits), so an expert holds
+// f*d*(2*bits + bits_down)/8 code bytes.  0 on success.
 int synth_gpu_experts(uint64_t master, uint32_t layer, int d, int f, int expert0, int n_experts, int bits,
-                      void* codes, void* scales, void* stream) {
-    if (d % 128 || f % 128 || d <= 0 || f <= 0 || n_experts <= 0 || bits < 2 || bits > 4) return -1;
-    const int max_st = (d > f ? d : f) / 16 * ((d > f ? f : d) / 128);
-    const int st_gu = (f / 16) * (d / 128), st_dn = (d / 16) * (f / 128);
-    (void)max_st;
-    dim3 grid(st_gu > st_dn ? st_gu : st_dn, 3, n_experts);
+                      int bits_down, void* codes, void* scales, void* stream) {
+    if (bits_down == 0) bits_down = bits;
+    if (d % 128 || f % 128 || d <= 0 || f <= 0 || n_experts <= 0 || bits < 2 || bits > 4 || bits_down < 2 ||
+        bits_down > 4)
+        return -1;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t* c = static_cast<uint8_t*>(codes);
     uint16_t* sc = static_cast<uint16_t*>(scales);
-    switch (bits) {
-        case 2: gen_matrix_kernel<2><<<grid, 64, 0, s>>>(master, layer, d, f, expert0, c, sc); break;
-        case 3: gen_matrix_kernel<3><<<grid, 64, 0, s>>>(master, layer, d, f, expert0, c, sc); break;
-        default: gen_matrix_kernel<4><<<grid, 64, 0, s>>>(master, layer, d, f, expert0, c, sc); break;
+    const int64_t stride = (int64_t)f * d * (2 * bits + bits_down) / 8;
+    if (bits_down == bits) {
+        gen_mats(bits, master, layer, d, f, expert0, n_experts, 0, 3, stride, 0, c, sc, s);
+    } else {
+        gen_mats(bits, master, layer, d, f, expert0, n_experts, 0, 2, stride, 0, c, sc, s);
+        gen_mats(bits_down, master, layer, d, f, expert0, n_experts, 2, 1, stride, 2 * (int64_t)f * d * bits / 8, c,
+                 sc, s);
     }
     return cudaGetLastError() == cudaSuccess ? 0 : -2;
 }

@@ -8,11 +8,12 @@ from synth import WORKLOADS, MoeShape
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("bits", [2, 3, 4])
-def test_experts_match_host(bits):
+@pytest.mark.parametrize("bits,bits_down", [(2, 0), (3, 0), (4, 0), (2, 3), (2, 4), (3, 2), (4, 2)])
+def test_experts_match_host(bits, bits_down):
+    """Uniform and mixed code widths (gate/up at `bits`, down at `bits_down`)."""
     import torch
     from synth import gpu
-    sh = MoeShape(d=256, f=128, E=16, k=2, n_shared=1, bits=bits)
+    sh = MoeShape(d=256, f=128, E=16, k=2, n_shared=1, bits=bits, bits_down=bits_down)
     cb, sb = synth.expert_bytes(sh)
     codes = torch.empty(17 * cb, dtype=torch.uint8, device="cuda")
     scales = torch.empty(17 * sb // 2, dtype=torch.int16, device="cuda")
