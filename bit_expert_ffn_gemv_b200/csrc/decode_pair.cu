@@ -11,15 +11,21 @@
 //
 //   1. Router.  CTA b computes the exact logits of experts [bE/G, (b+1)E/G)
 //      for all T tokens (bf16 x bf16 products are exact in fp64, summed by
-//      fp64 FMAs), writes them to global memory and announces them on a
-//      64-bit arrival counter.  Clusters whose first work unit belongs to the
-//      shared expert run that unit meanwhile (it needs no routing).
+//      fp64 FMAs; a warp task is one row, four tokens, half the input
+//      dimension), writes them to global memory and announces them on a
+//      64-bit arrival counter.  Clusters whose first work units belong to the
+//      shared expert run those units' gate/up meanwhile (no routing needed).
 //   2. Top-k and schedule, redundantly in every CTA, once all CTAs arrived:
-//      each warp ranks one token's E logits (ties to the lower index, exact
-//      rank order), then the CTA lists the active experts ("slots": the shared
-//      expert, then the selected routed experts in ascending order) and the
-//      work units.  No second grid-wide hand-off is needed before the experts.
-//   3. Work units.  Unit u = (slot u / (f/128), chunk j = u % (f/128)) covers
+//      each warp ranks one token's E logits (k + 1 warp max-reductions over
+//      unique 32-bit keys; fp64 ranking only where keys share a prefix; ties
+//      to the lower index, exact rank order), then the CTA lists the active
+//      experts ("slots": the shared expert, then the selected routed experts
+//      in ascending order) and the work units.  No second grid-wide hand-off
+//      is needed before the experts.  This code runs once per launch, so it is
+//      kept short: cold instructions stream from L2.
+//   3. Work units, pipelined (gate/up of unit i, then down of unit i - 1; one
+//      loop for the shared-expert units, the routing step and the routed
+//      units).  Unit u = (slot u / (f/128), chunk j = u % (f/128)) covers
 //      the 128 intermediate rows [128j, 128j + 128) of one expert: its gate/up
 //      rows and the matching 128 input columns of its down matrix.  Cluster c
 //      takes units c, c + 74, c + 148, ...  Inside the cluster, CTA r computes
@@ -996,27 +1002,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             // row index.  Warp 0, lane = slot: per token, a ballot over the slots
             // that hold it gives each slot's place by a prefix count.
             if (warp == 0) {
-                int base[kPairMaxTokens];  // places taken so far, per token
-    #pragma unroll
-                for (int t = 0; t < kPairMaxTokens; ++t) base[t] = 0;
+                // tn[t] is the running count of token t's places (rolled loops:
+                // this code runs once per launch, so it is kept short)
+                for (int t = lane; t < T; t += 32) tn[t] = 0;
+                __syncwarp();
                 int big = 0;
                 const uint32_t lt = (1u << lane) - 1u;
                 for (int s0 = 0; s0 < n_slots; s0 += 32) {
                     const int sl = s0 + lane;
                     const uint32_t m = sl >= n_slots ? 0u : (sl < ns ? 0xFFFFFFFFu : emask[slot_e[sl]]);
                     if (sl >= ns && sl < n_slots) big = max(big, __popc(m));
-    #pragma unroll
-                    for (int t = 0; t < kPairMaxTokens; ++t) {
-                        if (t < T) {
-                            const uint32_t bal = __ballot_sync(0xffffffffu, (m >> t) & 1u);
-                            if ((m >> t) & 1u) pos[sl * T + t] = (unsigned char)(base[t] + __popc(bal & lt));
-                            base[t] += __popc(bal);
-                        }
+#pragma unroll 1
+                    for (int t = 0; t < T; ++t) {
+                        const uint32_t bit = (m >> t) & 1u;
+                        const uint32_t bal = __ballot_sync(0xffffffffu, bit);
+                        const int base = tn[t];
+                        if (bit) pos[sl * T + t] = (unsigned char)(base + __popc(bal & lt));
+                        __syncwarp();
+                        if (lane == 0) tn[t] = base + __popc(bal);
+                        __syncwarp();
                     }
                 }
-    #pragma unroll
-                for (int t = 0; t < kPairMaxTokens; ++t)
-                    if (t < T && lane == t) tn[t] = base[t];
                 big = (int)__reduce_max_sync(0xffffffffu, (unsigned)big);
                 if (lane == 0) {
                     const int U = n_slots * FC;

@@ -100,8 +100,29 @@ MOE_DEV bool better64(double va, int ia, double vb, int ib) {
 
 constexpr int kTopkWarps = 4;
 
-// One warp per token.  Shared memory per warp: E floats (fp32 logits),
-// E floats (bounds), E doubles (fp64 logits of candidates).
+// order-preserving image of an fp32 logit (NaN as -inf): a larger key is a
+// larger value; 0 is below every key
+MOE_DEV uint32_t fkey(float v) {
+    v = isnan(v) ? -INFINITY : v;
+    v = v + 0.0f;  // -0 -> +0
+    const uint32_t b = __float_as_uint(v);
+    return (b >> 31) ? ~b : (b | 0x80000000u);
+}
+
+// One warp per token.  Shared memory per warp: E doubles (fp64 logits of the
+// candidates), E floats (fp32 logits), E floats (their error bounds, later
+// the candidate list).
+//
+// Every fp32 logit l_e lies within d_e of the exact one.  k rounds of a warp
+// max-reduction over the logits' keys select S, the k largest fp32 logits (in
+// descending order; equal values in any order).  Every expert of S is then
+// at least L = min over S of (l_s - d_s) exactly, so an expert whose interval
+// ends below L has k experts above it: the exact top k lies within the
+// candidates {e : l_e + d_e >= L}.  When the candidates are S itself and the
+// intervals of consecutive ranks are disjoint, S in its fp32 order is the
+// exact selection; otherwise the candidates' logits are recomputed in fp64
+// (sums of exact bf16 products) and ranked exactly by (value desc, index asc).
+template <int KPL>
 __global__ void __launch_bounds__(kTopkWarps * 32)
     topk_kernel(const float* __restrict__ logits, const __nv_bfloat16* __restrict__ x, int T, int d, int E, int k,
                 const __nv_bfloat16* __restrict__ wr, const float* __restrict__ bias,
@@ -134,65 +155,78 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
     const float xn = sqrtf(ss) * (1.0f + 1e-5f);
     const float c = 2.0f * depth * 5.9604645e-8f * (1.0f + 1e-5f);
 
-#pragma unroll 8
-    for (int e = lane; e < E; e += 32) {
-        const float v = __ldg(&logits[(int64_t)t * E + e]);
-        const float wn = __ldg(&wnorm[e]), b = bias ? fabsf(__ldg(&bias[e])) : 0.0f;
-        lv[e] = v;
-        dv[e] = c * (wn * xn + b);
+    // logits, bounds and keys; lane holds experts lane + 32 j
+    uint32_t key[KPL];
+    uint32_t lmax = 0u;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+        const int e = lane + 32 * j;
+        key[j] = 0u;
+        if (e < E) {
+            const float v = __ldg(&logits[(int64_t)t * E + e]);
+            const float wn = __ldg(&wnorm[e]), b = bias ? fabsf(__ldg(&bias[e])) : 0.0f;
+            lv[e] = v;
+            dv[e] = c * (wn * xn + b);
+            key[j] = fkey(v);
+        }
+        lmax = max(lmax, key[j]);
     }
     __syncwarp();
 
-    // top-k by repeated warp argmax; `taken` bit j <-> element lane + 32 j.
-    // Rank r lives in lane r (k <= 32), so nothing is indexed by the runtime k.
-    uint32_t taken = 0;
-    int my_sel = -1;  // lane r < k: expert of rank r
+    // S: k rounds, each taking the largest remaining key (the lowest lane that
+    // holds it, its first copy) -- lane r keeps rank r
+    int my_sel = -1;
+    float my_l = 0.f, my_d = 0.f, lo_min = INFINITY;
+    bool nan_seen = false;
     for (int r = 0; r < k; ++r) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-        for (int j = 0, e = lane; e < E; ++j, e += 32)
-            if (!((taken >> j) & 1u) && (bi == 0x7fffffff || better(lv[e], e, bv, bi))) {
-                bv = lv[e];
-                bi = e;
-            }
+        const uint32_t m = __reduce_max_sync(0xffffffffu, lmax);
+        const int owner = __ffs(__ballot_sync(0xffffffffu, lmax == m)) - 1;
+        int er = 0;
+        if (lane == owner) {
+            bool done = false;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (oi != 0x7fffffff && (bi == 0x7fffffff || better(ov, oi, bv, bi))) {
-                bv = ov;
-                bi = oi;
+            for (int j = 0; j < KPL; ++j) {
+                if (!done && key[j] == m) {
+                    er = lane + 32 * j;
+                    key[j] = 0u;
+                    done = true;
+                }
             }
+            lmax = 0u;
+#pragma unroll
+            for (int j = 0; j < KPL; ++j) lmax = max(lmax, key[j]);
         }
-        if (lane == r) my_sel = bi;
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        er = __shfl_sync(0xffffffffu, er, owner);
+        const float lr = lv[er], dr = dv[er];
+        if (lane == r) {
+            my_sel = er;
+            my_l = lr;
+            my_d = dr;
+        }
+        nan_seen |= isnan(lr);
+        lo_min = fminf(lo_min, lr - dr);
     }
 
-    // certification of the fp32 order: rank r's interval lies strictly above rank r+1's
-    const int next_sel = __shfl_down_sync(0xffffffffu, my_sel, 1);
-    const bool pair_ok = lane + 1 >= k || (lv[my_sel] - dv[my_sel] > lv[next_sel] + dv[next_sel]);
-    bool ok = __all_sync(0xffffffffu, pair_ok);
-    const int sel_k = __shfl_sync(0xffffffffu, my_sel, k - 1);
-    const float lower_k = lv[sel_k] - dv[sel_k];
-    // candidates: every expert whose interval reaches the k-th one's lower end,
-    // listed in ascending index order (reusing the bound array, no longer needed)
-    int* cand = reinterpret_cast<int*>(dv);
+    // certification: consecutive ranks' intervals disjoint and no other candidate
+    const float nl = __shfl_down_sync(0xffffffffu, my_l, 1), nd = __shfl_down_sync(0xffffffffu, my_d, 1);
+    const bool pair_ok = lane + 1 >= k || (my_l - my_d > nl + nd);
+    bool ok = __all_sync(0xffffffffu, pair_ok) && !nan_seen && !isnan(lo_min);
+    int* cand = reinterpret_cast<int*>(dv);  // the bounds are no longer needed after this pass
     int n_cand = 0;
     for (int e0 = 0; e0 < E; e0 += 32) {
         const int e = e0 + lane;
-        const bool is_c = e < E && (isnan(lower_k) || isnan(lv[e]) || lv[e] + dv[e] >= lower_k);
-        const uint32_t m = __ballot_sync(0xffffffffu, is_c);
+        const bool is_c = e < E && (nan_seen || isnan(lv[e]) || lv[e] + dv[e] >= lo_min);
+        const uint32_t bm = __ballot_sync(0xffffffffu, is_c);
         __syncwarp();  // every lane has read dv[e0 .. e0+31] before it is overwritten
-        if (is_c) cand[n_cand + __popc(m & ((1u << lane) - 1u))] = e;
-        n_cand += __popc(m);
+        if (is_c) cand[n_cand + __popc(bm & ((1u << lane) - 1u))] = e;
+        n_cand += __popc(bm);
     }
     __syncwarp();
     if (n_cand != k) ok = false;
-    if (isnan(lower_k)) ok = false;
 
     float my_w = 0.f;  // lane r < k: logit of rank r
     if (ok) {
-        if (lane < k) my_w = lv[my_sel];
+        if (lane < k) my_w = my_l;
     } else {
         // fp64 logits of the candidates (sums of exact bf16 products), 8 products
         // per lane per 256-wide chunk, four candidates per pass (more loads in flight)
@@ -231,34 +265,59 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
             }
         }
         __syncwarp();
-        // exact ranking among the candidates: k rounds of warp argmax on (fp64 logit, index)
-        uint32_t tk = 0;  // bit j <-> candidate lane + 32 j (n_cand <= E <= 1024, so j < 32)
-        for (int r = 0; r < k; ++r) {
-            double bv = -INFINITY;
-            int bi = 0x7fffffff, bc = -1;
-            for (int j = 0, ci = lane; ci < n_cand; ++j, ci += 32) {
-                if (!((tk >> j) & 1u) && (bi == 0x7fffffff || better64(lg64[ci], cand[ci], bv, bi))) {
-                    bv = lg64[ci];
-                    bi = cand[ci];
-                    bc = ci;
+        if (n_cand <= 32) {
+            // exact rank of each candidate (lane c): how many candidates beat it
+            double v = -INFINITY;
+            int e = 0x7fffffff;
+            if (lane < n_cand) {
+                v = lg64[lane];
+                e = cand[lane];
+            }
+            int rank = 0;
+            for (int j = 0; j < n_cand; ++j) {
+                const double vj = __shfl_sync(0xffffffffu, v, j);
+                const int ej = __shfl_sync(0xffffffffu, e, j);
+                if (j != lane && better64(vj, ej, v, e)) ++rank;
+            }
+            for (int r = 0; r < k; ++r) {
+                const int src = __ffs(__ballot_sync(0xffffffffu, lane < n_cand && rank == r)) - 1;
+                const double vr = __shfl_sync(0xffffffffu, v, src);
+                const int er = __shfl_sync(0xffffffffu, e, src);
+                if (lane == r) {
+                    my_sel = er;
+                    my_w = (float)vr;
                 }
             }
+        } else {
+            // many candidates (ties or NaN): k rounds of warp argmax on (fp64 logit, index)
+            uint32_t tk = 0;  // bit j <-> candidate lane + 32 j (n_cand <= E <= 1024, so j < 32)
+            for (int r = 0; r < k; ++r) {
+                double bv = -INFINITY;
+                int bi = 0x7fffffff, bc = -1;
+                for (int j = 0, ci = lane; ci < n_cand; ++j, ci += 32) {
+                    if (!((tk >> j) & 1u) && (bi == 0x7fffffff || better64(lg64[ci], cand[ci], bv, bi))) {
+                        bv = lg64[ci];
+                        bi = cand[ci];
+                        bc = ci;
+                    }
+                }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                double ov = __shfl_xor_sync(0xffffffffu, bv, o);
-                int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-                int oc = __shfl_xor_sync(0xffffffffu, bc, o);
-                if (oi != 0x7fffffff && (bi == 0x7fffffff || better64(ov, oi, bv, bi))) {
-                    bv = ov;
-                    bi = oi;
-                    bc = oc;
+                for (int o = 16; o > 0; o >>= 1) {
+                    double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                    int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                    int oc = __shfl_xor_sync(0xffffffffu, bc, o);
+                    if (oi != 0x7fffffff && (bi == 0x7fffffff || better64(ov, oi, bv, bi))) {
+                        bv = ov;
+                        bi = oi;
+                        bc = oc;
+                    }
                 }
+                if (lane == r) {
+                    my_sel = bi;
+                    my_w = (float)bv;
+                }
+                if (bc >= 0 && (bc & 31) == lane) tk |= 1u << (bc >> 5);
             }
-            if (lane == r) {
-                my_sel = bi;
-                my_w = (float)bv;
-            }
-            if (bc >= 0 && (bc & 31) == lane) tk |= 1u << (bc >> 5);
         }
         if (lane == 0) atomicAdd(&meta->n_fixup, 1);
     }
@@ -296,12 +355,14 @@ cudaError_t launch_router_logits(const RouteArgs& a, cudaStream_t s) {
 
 cudaError_t launch_topk(const RouteArgs& a, cudaStream_t s) {
     const size_t smem_t = (size_t)kTopkWarps * a.E * (sizeof(double) + 2 * sizeof(float));
+    auto kern = a.E <= 512 ? topk_kernel<16> : topk_kernel<32>;
+    if (a.E > 1024) return cudaErrorInvalidValue;
     if (smem_t > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_t);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_t);
         if (e != cudaSuccess) return e;
     }
     const float depth = a.depth > 0.f ? a.depth : (float)(a.d / 32 + 6);
-    topk_kernel<<<(a.T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, smem_t, s>>>(
+    kern<<<(a.T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, smem_t, s>>>(
         a.logits, static_cast<const __nv_bfloat16*>(a.x), a.T, a.d, a.E, a.k,
         static_cast<const __nv_bfloat16*>(a.wr), a.bias, a.wnorm, depth, a.ids, a.w, a.meta);
     return cudaGetLastError();

@@ -135,3 +135,68 @@ def test_expert_split_full_shape_decode(torch_cuda, T):
         _run_split(torch_cuda, h, sh, L, xb, 8, 0, REL_L2_FP32, "ep full-shape")
     finally:
         h.close()
+
+
+# ---------------------------------------------------------------- all-to-all dispatch and combine
+def _segments(rows, counts):
+    out, off = [], 0
+    for n in counts:
+        out.append(rows[off:off + n])
+        off += n
+    return out
+
+
+@pytest.mark.parametrize("world,tokens", [(2, (3, 20)), (4, (1, 9, 40, 5))])
+def test_all_to_all_virtual_ranks(torch_cuda, small, world, tokens):
+    """Tokens data-parallel over `world` virtual ranks on the one GPU, experts split: each rank's tokens
+    are dispatched to the ranks holding their experts, the library computes each rank's partial outputs on
+    the rows it received (its expert range, no shared expert), and the partials return and are combined
+    with the shared expert's output.  Run phase by phase in one process (the exchange is a list
+    transposition; the gloo test covers torch.distributed's); every rank's layer output must match the
+    oracle."""
+    import bit_expert_ffn_gemv_b200 as moe
+    from bit_expert_ffn_gemv_b200.expert_parallel import combine_rows, dispatch_plan, pack_rows
+    torch = torch_cuda
+    L, h = small
+    sh = SMALL
+    xbs = [synth.x_host(sh, 4243, 500 + r, tokens[r]) for r in range(world)]
+    xs = [x_to_device(xb) for xb in xbs]
+    try:
+        plans, sends = [], []
+        for r in range(world):
+            ids, _ = h.route(0, xs[r])
+            plan = dispatch_plan(ids, sh.E, world)
+            plans.append(plan)
+            sends.append(pack_rows(xs[r], plan))
+        # exchange: rank R receives, source by source, the rows each rank packed for it
+        recv = [torch.cat([_segments(*sends[r])[R] for r in range(world)]) for R in range(world)]
+        recv_counts = [[sends[r][1][R] for r in range(world)] for R in range(world)]
+        parts = []
+        for R in range(world):
+            b, e, _ = expert_shard(sh.E, R, world)
+            h.set_expert_range(b, e, False)
+            parts.append(h.forward(0, recv[R], flags=moe.MOE_OUT_FP32))
+        back = [torch.cat([_segments(parts[R], recv_counts[R])[r] for R in range(world)]) for r in range(world)]
+        h.set_expert_range(0, 0, True)
+        for r in range(world):
+            y = h.forward(0, xs[r], flags=moe.MOE_OUT_FP32)
+            combine_rows(y, plans[r], back[r])
+            torch.cuda.synchronize()
+            assert h.check_status() == 0
+            full, _, _ = oracle.layer(sh, xbs[r], L["router_w"], L["bias"], L["codes"], L["scales"])
+            err = np.linalg.norm(y_to_f64(y) - full) / np.linalg.norm(full)
+            print(f"a2a world={world} rank {r} T={tokens[r]}: rel_l2 {err:.3e}")
+            assert err <= REL_L2_FP32_TC, (world, r, err)
+    finally:
+        h.set_expert_range(0, sh.E, True)
+
+
+def test_all_to_all_layer_single_rank(torch_cuda, small):
+    """a2a_layer without a process group (one rank) is the layer."""
+    from bit_expert_ffn_gemv_b200.expert_parallel import a2a_layer
+    L, h = small
+    xb = synth.x_host(SMALL, 4243, 77, 33)
+    y = a2a_layer(h, 0, x_to_device(xb))
+    torch_cuda.cuda.synchronize()
+    full, _, _ = oracle.layer(SMALL, xb, L["router_w"], L["bias"], L["codes"], L["scales"])
+    assert np.linalg.norm(y_to_f64(y) - full) / np.linalg.norm(full) <= REL_L2_FP32_TC
