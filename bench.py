@@ -51,6 +51,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-graph", action="store_true", help="time eager launches instead of a CUDA graph")
     p.add_argument("--no-sub", action="store_true", help="skip the decode T=1 and prefill sub-measurements")
+    p.add_argument("--chain-two-calls", action="store_true", help="chain48: a norm launch, then the layer (default: "
+                   "one call per layer with MOE_NORM_INPUT)")
     return p.parse_args()
 
 
@@ -401,12 +403,16 @@ def measure_decode(moe, h, sh, xs, layers, T, flags, args, steps, warmup, clock_
 
     def step(i, stream=None):
         if chain:
-            # residual chain: u_l = rmsnorm(x_l), x_{l+1} = x_l + layer_l(u_l) in place
+            # residual chain x_{l+1} = x_l + layer_l(rmsnorm(x_l)), in place; one call per layer
+            # (MOE_NORM_INPUT), or the norm kernel then the layer with --chain-two-calls
             r = resid[i & 1]
             r.copy_(xs[i % n_x])
             for l in range(layers):
-                moe.rms_normalize(r, normed, stream=stream)
-                h.forward(l, normed, r, flags=flags | moe.MOE_ACCUMULATE, stream=stream)
+                if args.chain_two_calls:
+                    moe.rms_normalize(r, normed, stream=stream)
+                    h.forward(l, normed, r, flags=flags | moe.MOE_ACCUMULATE, stream=stream)
+                else:
+                    h.forward(l, r, r, flags=flags | moe.MOE_ACCUMULATE | moe.MOE_NORM_INPUT, stream=stream)
             return r
         return h.forward(i % layers, xs[i % n_x], ys[i & 1], flags=flags, stream=stream)
 

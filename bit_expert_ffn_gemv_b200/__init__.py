@@ -18,7 +18,7 @@ import threading
 
 __all__ = ["MoeError", "MoeConfig", "MoeLayerWeights", "MoeLayer", "lib", "library_path", "MOE_OUT_FP32",
            "MOE_ACCUMULATE", "MOE_FORCE_GEMV", "MOE_FORCE_GEMM", "MOE_FORCE_UNFUSED", "MOE_ROUTE_TAIL_SKIP",
-           "MOE_TAIL_SKIP_RANK", "STATUS", "moe_layer_init", "moe_load_layer",
+           "MOE_TAIL_SKIP_RANK", "MOE_NORM_INPUT", "STATUS", "moe_layer_init", "moe_load_layer",
            "moe_route", "moe_route_noalloc", "moe_forward", "moe_forward_host", "moe_destroy", "moe_debug_dequant", "moe_debug_last_routing", "moe_debug_bucket", "moe_check_status",
            "moe_get_stats", "moe_status_string", "moe_profile", "moe_profile_read", "moe_kernel_name", "MoeStats",
            "moe_debug_router_logits", "moe_router_error_depth", "moe_rms_normalize", "rms_normalize",
@@ -34,6 +34,7 @@ MOE_FORCE_GEMM = 0x8
 MOE_FORCE_UNFUSED = 0x10
 MOE_ROUTE_TAIL_SKIP = 0x20  # drop experts that every selecting token ranks >= MOE_TAIL_SKIP_RANK
 MOE_TAIL_SKIP_RANK = 6
+MOE_NORM_INPUT = 0x40  # the layer reads rmsnorm(x); with MOE_ACCUMULATE and y == x: x += layer(rmsnorm(x))
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_CUDA", 3: "MOE_ERR_OOM", 4: "MOE_ERR_NOT_LOADED",
           5: "MOE_ERR_TIMEOUT", 6: "MOE_ERR_BOUNDS", 7: "MOE_ERR_RANGE"}
 
@@ -55,7 +56,7 @@ class MoeStats(ctypes.Structure):
                 ("launches", ctypes.c_int64), ("cuda_error", ctypes.c_int64)]
 
 
-MOE_KERNEL_COUNT = 12
+MOE_KERNEL_COUNT = 13
 
 
 class MoeLayerWeights(ctypes.Structure):

@@ -16,7 +16,7 @@
 
 static const char* const kKernelNames[MOE_KERNEL_COUNT] = {
     "router_logits", "topk", "bucket", "gemv_gateup", "gemv_down", "combine", "gemm_gateup", "gemm_down",
-    "router_gemm", "decode_fused", "gather_f16", "tile_list"};
+    "router_gemm", "decode_fused", "gather_f16", "tile_list", "rms_norm"};
 
 struct moe_layer_state {
     const uint8_t* codes = nullptr;
@@ -57,6 +57,7 @@ struct moe_handle {
     int withhold = -1;                   // test hook: a CTA that never announces its router rows
     void* x_stage = nullptr;
     void* y_stage = nullptr;
+    void* x_norm = nullptr;      // rmsnorm(x) for MOE_NORM_INPUT outside the clustered decode kernel
     void* xg = nullptr;          // fp16 x rows in group order (tensor-core path)
     moe::GemmMaps gu_maps{};     // TMA maps of xg (gate/up B) and h (down B); the
     moe::GemmMaps dn_maps{};     // codes/scales maps come from the layer
@@ -80,8 +81,9 @@ struct moe_handle {
 namespace {
 
 
-constexpr uint32_t kAllFlags =
-    MOE_OUT_FP32 | MOE_ACCUMULATE | MOE_FORCE_GEMV | MOE_FORCE_GEMM | MOE_FORCE_UNFUSED | MOE_ROUTE_TAIL_SKIP;
+constexpr uint32_t kAllFlags = MOE_OUT_FP32 | MOE_ACCUMULATE | MOE_FORCE_GEMV | MOE_FORCE_GEMM | MOE_FORCE_UNFUSED |
+                               MOE_ROUTE_TAIL_SKIP | MOE_NORM_INPUT;
+constexpr float kNormEps = 1e-6f;  // the pre-norm of MOE_NORM_INPUT and moe_rms_normalize
 
 // Shared experts this handle computes (0 when another rank owns the shared expert).
 int eff_shared(const moe_handle* h) { return h->ep_shared ? h->cfg.n_shared : 0; }
@@ -241,10 +243,19 @@ bool try_decode(moe_handle* h, int32_t layer, const void* x, int32_t T, void* y,
     d.down_codes_map = &L.pair_dc;
     d.down_scales_map = &L.pair_ds;
     if (T <= moe::kPairMaxTokens && moe::pair_decode_supported(d)) {
+        d.norm_input = (flags & MOE_NORM_INPUT) ? 1 : 0;  // normalised inside the launch
         *st = cuda_status(run(h, MOE_K_DECODE, s, [&] { return moe::launch_decode_pair(d, s); }));
         return true;
     }
     if (T <= moe::kDecodeMaxTokens && !mixed_widths(c)) {
+        if (flags & MOE_NORM_INPUT) {
+            if (run(h, MOE_K_RMS_NORM, s,
+                    [&] { return moe::launch_rms_normalize(x, T, c.d, h->x_norm, kNormEps, s); }) != cudaSuccess) {
+                *st = MOE_ERR_CUDA;
+                return true;
+            }
+            d.x = h->x_norm;
+        }
         *st = cuda_status(run(h, MOE_K_DECODE, s, [&] { return moe::launch_decode(d, s); }));
         return true;
     }
@@ -256,6 +267,12 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     const moe_config& c = h->cfg;
     moe_status dst = MOE_OK;
     if (try_decode(h, layer, x, T, y, flags, s, &dst)) return dst;
+    if (flags & MOE_NORM_INPUT) {  // the unfused and tensor-core paths read the normalised copy
+        if (run(h, MOE_K_RMS_NORM, s, [&] { return moe::launch_rms_normalize(x, T, c.d, h->x_norm, kNormEps, s); }) !=
+            cudaSuccess)
+            return MOE_ERR_CUDA;
+        x = h->x_norm;
+    }
     const bool tc = use_tensor_cores(c, T, flags);
     cudaError_t e;
     moe_status st = do_route(h, layer, x, T, h->ids, h->w, tc, s);
@@ -413,6 +430,7 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     const size_t o_h = take(sizeof(__half) * rows * (size_t)c.f);
     const size_t o_obuf = take(sizeof(float) * rows * (size_t)c.d);
     const size_t o_xs = take(sizeof(uint16_t) * T * (size_t)c.d);
+    const size_t o_xn = take(sizeof(uint16_t) * T * (size_t)c.d);
     const size_t o_ys = take(sizeof(float) * T * (size_t)c.d);
     const size_t o_norms = take(sizeof(float) * E * (size_t)c.n_layers);
     const size_t o_l64 = take(sizeof(double) * std::min<size_t>(T, moe::kDecodeMaxTokens) * E);
@@ -452,6 +470,7 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     h->part = reinterpret_cast<float*>(base + o_part);
     h->ctr = reinterpret_cast<unsigned long long*>(base + o_ctr);
     h->x_stage = base + o_xs;
+    h->x_norm = base + o_xn;
     h->y_stage = base + o_ys;
     h->xg = base + o_xg;
     h->desc_gu = reinterpret_cast<int4*>(base + o_dgu);
@@ -571,7 +590,7 @@ moe_status moe_rms_normalize(const void* x, int32_t T, int32_t d, void* out, voi
     if (T < 0 || d <= 0 || d % 8) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x || !out || !aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-    return cuda_status(moe::launch_rms_normalize(x, T, d, out, 1e-6f, static_cast<cudaStream_t>(stream)));
+    return cuda_status(moe::launch_rms_normalize(x, T, d, out, kNormEps, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_set_expert_range(moe_handle* h, int32_t begin, int32_t end, int32_t with_shared) {

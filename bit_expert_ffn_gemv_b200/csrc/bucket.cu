@@ -151,6 +151,9 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
 //            match-any, as in the single-CTA kernel) and writes them at
 //            base[c][e] + rank.
 constexpr int kChunks = 128;
+constexpr int kScanCols = 256;  // experts per shared-memory tile of the scan (kChunks x 256 x 4 B = 128 KB)
+constexpr int kScanThreads = 1024;
+constexpr int kScanLoads = kChunks * kScanCols / kScanThreads;
 constexpr int kChunkWarps = 8;
 
 __global__ void __launch_bounds__(kChunkWarps * 32)
@@ -181,31 +184,56 @@ __global__ void __launch_bounds__(kChunkWarps * 32)
     }
 }
 
-__global__ void __launch_bounds__(1024) bucket_scan_kernel(int32_t* __restrict__ cnt, int32_t* __restrict__ best,
+__global__ void __launch_bounds__(kScanThreads) bucket_scan_kernel(int32_t* __restrict__ cnt, int32_t* __restrict__ best,
                                                            int R, int e0, int e1, int nchunks, int E,
                                                            int32_t* __restrict__ offsets,
                                                            int32_t* __restrict__ active, Meta* __restrict__ meta) {
-    extern __shared__ int32_t tot[];  // [E]
+    extern __shared__ int32_t sm_scan[];
+    int32_t* tot = sm_scan;                       // [E]
+    int32_t* tile = sm_scan + ((E + 31) & ~31);   // [nchunks][kScanCols] column tile of cnt
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // per expert: exclusive prefix over the chunks (in place), total; with
     // R > 0, the lowest rank over the chunks goes to best[e] (row 0) and an
-    // expert with none below R gets no group
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = 0;
-#pragma unroll 8
-        for (int c = 0; c < nchunks; ++c) {
-            const int v = cnt[(int64_t)c * E + e];
-            cnt[(int64_t)c * E + e] = run;
-            run += v;
+    // expert with none below R gets no group.  The counts are staged in
+    // column tiles of kScanCols experts (coalesced row loads and stores), and
+    // a thread scans one expert's column in shared memory.
+    for (int c0 = 0; c0 < E; c0 += kScanCols) {
+        const int ncol = min(kScanCols, E - c0);
+        {
+            // every load of the tile in flight at once (1024 threads x 32 values)
+            int v[kScanLoads];
+#pragma unroll
+            for (int j = 0; j < kScanLoads; ++j) {
+                const int idx = threadIdx.x + j * kScanThreads, c = idx / kScanCols, ee = idx - c * kScanCols;
+                v[j] = (c < nchunks && ee < ncol) ? cnt[(int64_t)c * E + c0 + ee] : 0;
+            }
+#pragma unroll
+            for (int j = 0; j < kScanLoads; ++j) tile[threadIdx.x + j * kScanThreads] = v[j];
         }
-        if (R > 0) {
-            int b = best[e];
-            for (int c = 1; c < nchunks; ++c) b = min(b, best[(int64_t)c * E + e]);
-            best[e] = b;
-            if (b >= R) run = 0;
+        __syncthreads();
+        for (int ee = threadIdx.x; ee < ncol; ee += blockDim.x) {
+            const int e = c0 + ee;
+            int run = 0;
+            for (int c = 0; c < nchunks; ++c) {
+                const int v = tile[c * kScanCols + ee];
+                tile[c * kScanCols + ee] = run;
+                run += v;
+            }
+            if (R > 0) {
+                int b = best[e];
+                for (int c = 1; c < nchunks; ++c) b = min(b, best[(int64_t)c * E + e]);
+                best[e] = b;
+                if (b >= R) run = 0;
+            }
+            if (e < e0 || e >= e1) run = 0;
+            tot[e] = run;
         }
-        if (e < e0 || e >= e1) run = 0;
-        tot[e] = run;
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < nchunks * kScanCols; idx += blockDim.x) {
+            const int c = idx / kScanCols, ee = idx - c * kScanCols;
+            if (ee < ncol) cnt[(int64_t)c * E + c0 + ee] = tile[idx];
+        }
+        __syncthreads();  // the tile is refilled next
     }
     __syncthreads();
     if (warp == 0) {
@@ -302,8 +330,12 @@ cudaError_t launch_bucket(const BucketArgs& a, cudaStream_t s) {
         bucket_count_kernel<<<kChunks, kChunkWarps * 32, 2 * sizeof(int32_t) * a.E, s>>>(a.ids, n_pairs, a.k, a.E,
                                                                                          chunk, a.cnt, best, R,
                                                                                          a.status);
-        bucket_scan_kernel<<<1, 1024, sizeof(int32_t) * a.E, s>>>(a.cnt, best, R, e0, e1, kChunks, a.E, a.offsets,
-                                                                   a.active, a.meta);
+        const size_t scan_smem = sizeof(int32_t) * (((size_t)a.E + 31) / 32 * 32 + (size_t)kChunks * kScanCols);
+        cudaError_t es = cudaFuncSetAttribute(bucket_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              (int)scan_smem);
+        if (es != cudaSuccess) return es;
+        bucket_scan_kernel<<<1, kScanThreads, scan_smem, s>>>(a.cnt, best, R, e0, e1, kChunks, a.E, a.offsets, a.active,
+                                                       a.meta);
         const size_t smem = sizeof(int32_t) * (size_t)kChunkWarps * a.E;
         if (smem > 48 * 1024) {
             cudaError_t e = cudaFuncSetAttribute(bucket_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -141,6 +141,7 @@ struct Args {
     int nc;                // clusters in the grid
     uint32_t spin_limit;   // polls before a wait gives up
     int withhold;          // test only: this CTA never announces its router rows (-1: off)
+    int norm_input;        // normalise x (rmsnorm, as launch_rms_normalize) before the router
     // shared memory layout (bytes from the dynamic base)
     int ng, nd;            // ring slots
     int g_bytes, d_bytes;  // item sizes
@@ -487,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t fullG[kMaxSlots], emptyG[kMaxSlots], fullD[kMaxSlots], emptyD[kMaxSlots];
     __shared__ __align__(8) uint64_t hfull[3], hempty[3], barX, sched;
-    __shared__ int s_nslots, s_nunits, s_wcnt[kCWarps];
+    __shared__ int s_nslots, s_nunits, s_stride, s_wcnt[kCWarps];
     __shared__ float s_w[2][16];
     __shared__ uint32_t s_mask[2];
     __shared__ int s_slot[2];
@@ -542,13 +543,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         emask[e] = 0u;
         ebest[e] = k;
     }
+    if (tid == 0) s_stride = nc;
     __syncthreads();
     cluster_arrive();  // the peer's barriers are initialised once this completes (waited below)
 
-    // ---- work units of this cluster: u = q + i * nc -> (slot u / FC, chunk u % FC)
+    // ---- work units of this cluster: u = q + i * stride -> (slot u / FC, chunk u % FC).
+    // The stride is nc until the schedule is known (the shared-expert units, slot
+    // 0, are units 0 .. FC*ns - 1 of clusters 0 ..); the schedule may then keep
+    // the routed units off the clusters that ran shared-expert units (stride
+    // nc - FC*ns), which reach the routing step late.
     const int n_pre = (q < FC * ns) ? (FC * ns - 1 - q) / nc + 1 : 0;  // shared-expert units
     auto unit_expert = [&](int i, int& e, int& j, int& s) {
-        const int u = q + i * nc;
+        const int u = q + i * s_stride;
         s = u / FC;
         j = u - s * FC;
         e = s < ns ? E : slot_e[s];
@@ -556,13 +562,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kProducer) {
         // ================================================================ producer
-        if (lane == 0) {
-            mbar_arrive_expect_tx(&barX, (uint32_t)T * d * 2);
-            for (int t = 0; t < T; ++t) bulk_g2s(xs + t * xstride, a.x + (int64_t)t * d, d * 2, &barX);
-        }
         int item = 0;
-        auto issue_until = [&](int n_units) {
-            for (; item < 6 * n_units; ++item) {
+        auto issue_items = [&](int end) {
+            for (; item < end; ++item) {
                 const int i = item / 6, r6 = item - 6 * i;
                 int e, j, s;
                 unit_expert(i, e, j, s);
@@ -596,6 +598,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
             }
         };
+        auto issue_until = [&](int n_units) { issue_items(6 * n_units); };
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&barX, (uint32_t)T * d * 2);
+            for (int t = 0; t < T; ++t) bulk_g2s(xs + t * xstride, a.x + (int64_t)t * d, d * 2, &barX);
+        }
+        __syncwarp();
         issue_until(n_pre);
         slot_wait(&sched, 0u, a);  // the consumers published the schedule
         issue_until(s_nunits);
@@ -603,6 +611,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ================================================================ consumers
         const unsigned long long c_start = cyc();
+        // ---- 0. pre-norm (MOE_NORM_INPUT): x <- bf16(x / sqrt(mean(x^2) + 1e-6)) in
+        // shared memory, token by token, with the same 256 threads, the same
+        // order of fp32 operations and the same rounding as the stand-alone
+        // norm kernel, so the result is bit-identical to it
+        if (a.norm_input) {
+            copy_wait(&barX, 0u, a);
+            float* red = gus;
+            for (int t = 0; t < T; ++t) {
+                uint16_t* xr = xs + t * xstride;
+                float ss = 0.f;
+                for (int i = tid * 8; i < d; i += kConsumers * 8) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(xr + i);
+                    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        const float lo = __uint_as_float(u[qq] << 16), hi = __uint_as_float(u[qq] & 0xFFFF0000u);
+                        ss = fmaf(lo, lo, ss);
+                        ss = fmaf(hi, hi, ss);
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                if (lane == 0) red[warp] = ss;
+                consumer_sync();
+                float tot = 0.f;
+#pragma unroll
+                for (int w = 0; w < kCWarps; ++w) tot += red[w];
+                const float inv = rsqrtf(tot / (float)d + 1e-6f);
+                for (int i = tid * 8; i < d; i += kConsumers * 8) {
+                    uint4* p4 = reinterpret_cast<uint4*>(xr + i);
+                    const uint4 v = *p4;
+                    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+                    uint32_t o4[4];
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        const __nv_bfloat162 r2 = __floats2bfloat162_rn(__uint_as_float(u[qq] << 16) * inv,
+                                                                        __uint_as_float(u[qq] & 0xFFFF0000u) * inv);
+                        o4[qq] = *reinterpret_cast<const uint32_t*>(&r2);
+                    }
+                    *p4 = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+                }
+                consumer_sync();  // red is reused by the next token; the router reads the normalised rows
+            }
+        }
+
         // ---- 1. router rows [r0, r1): exact logits.  Warp task = (row, 4
         // tokens, half of the input dimension): a lane holds 8 of every 256
         // inputs of its half (all its weight loads issued at once) and sums
@@ -1025,8 +1078,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 big = (int)__reduce_max_sync(0xffffffffu, (unsigned)big);
                 if (lane == 0) {
-                    const int U = n_slots * FC;
-                    const int nu = U > q ? (U - 1 - q) / nc + 1 : 0;
+                    // Routed units on the clusters without shared-expert units only,
+                    // when that takes no more rounds than spreading them over all.
+                    const int U = n_slots * FC, S = FC * ns;
+                    const bool apart = S > 0 && S < nc && (U - S + nc - S - 1) / (nc - S) <= (U + nc - 1) / nc;
+                    int nu;
+                    if (!apart) {
+                        nu = U > q ? (U - 1 - q) / nc + 1 : 0;
+                    } else if (q < S) {
+                        nu = 1;  // its shared-expert unit, u = q
+                    } else {
+                        nu = U > q ? (U - 1 - q) / (nc - S) + 1 : 0;
+                        s_stride = nc - S;
+                    }
                     s_nunits = max(nu, n_pre);
                     if (b == 0) {
                         a.meta->n_active = n_slots - ns;
@@ -1286,6 +1350,7 @@ static cudaError_t launch_t(const DecodeLaunch& L, cudaStream_t st) {
     a.nc = clusters;
     a.spin_limit = L.spin_limit;
     a.withhold = L.withhold;
+    a.norm_input = L.norm_input;
     a.ng = lay.ng;
     a.nd = lay.nd;
     a.g_bytes = lay.g_bytes;

@@ -103,6 +103,7 @@ struct DecodeLaunch {
     unsigned long long* ctr = nullptr;  // [kPairCounters] monotonic counters, zero once
     uint32_t spin_limit = 1u << 21;   // polls before a bounded wait gives up
     int withhold = -1;                // test only: this CTA never announces its router rows
+    int norm_input = 0;               // the layer reads rmsnorm(x) (bit-identical to launch_rms_normalize)
     const CUtensorMap* down_codes_map = nullptr;   // make_pair_down_maps of the layer
     const CUtensorMap* down_scales_map = nullptr;
 };

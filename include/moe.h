@@ -124,6 +124,18 @@ typedef struct {
  */
 #define MOE_ROUTE_TAIL_SKIP 0x20u
 #define MOE_TAIL_SKIP_RANK 6
+/*
+ * Pre-norm input: the layer reads u = rmsnorm(x) instead of x, with u exactly
+ * as moe_rms_normalize writes it (bf16(x / sqrt(mean(x^2) + 1e-6)), no gain):
+ * the model family the pages describe normalises the residual stream before
+ * each MoE layer (tech.okbari.net guide, "Strata, Qwen and GSQ-RCO are
+ * different components").  With MOE_ACCUMULATE and y == x, one call is a
+ * whole residual step x += layer(rmsnorm(x)).  The clustered decode kernel
+ * normalises inside its launch; the other paths run the norm first into the
+ * handle's scratch.  The output is bit-identical to moe_rms_normalize
+ * followed by moe_forward without the flag.
+ */
+#define MOE_NORM_INPUT 0x40u
 
 /*
  * Create a handle on the current CUDA device.  Checks the configuration and
@@ -349,7 +361,8 @@ enum {
     MOE_K_DECODE = 9,
     MOE_K_GATHER_F16 = 10,
     MOE_K_TILE_LIST = 11,
-    MOE_KERNEL_COUNT = 12
+    MOE_K_RMS_NORM = 12,
+    MOE_KERNEL_COUNT = 13
 };
 
 /*

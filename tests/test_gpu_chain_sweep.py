@@ -196,3 +196,65 @@ def test_coder_shape_layer(torch_cuda, coder, T):
     assert np.array_equal(ids.cpu().numpy(), ids_ref), f"E=256 T={T}: expert selection differs"
     _compare(sh, L, xb, y32, y16, label=f"E=256 T={T}", rows=rows,
              fp32_tol=REL_L2_FP32 if T <= 16 else REL_L2_FP32_TC)
+
+
+# ------------------------------------------------------------------ pre-norm input (MOE_NORM_INPUT)
+@pytest.fixture(scope="module")
+def decode_layer(torch_cuda):
+    from synth import gpu as sgpu
+    import bit_expert_ffn_gemv_b200 as moe
+    wl = WORKLOADS["decode"]
+    sh = wl.shape
+    h = moe.MoeLayer(sh.d, sh.f, sh.E, sh.k, sh.n_shared, 1, sh.bits, 512)
+    w = sgpu.layer_device(sh, wl.master, 0, wl.zipf)
+    h.load_layer(0, *w)
+    yield wl, h, w
+    h.close()
+
+
+@pytest.mark.parametrize("T,path", [(1, "default"), (4, "default"), (16, "default"), (4, "unfused"),
+                                    (40, "gemv"), (40, "default"), (300, "default")])
+def test_norm_input_is_the_two_call_sequence(torch_cuda, decode_layer, T, path):
+    """forward(x, MOE_NORM_INPUT) is bit for bit moe_rms_normalize then forward, on every path (the
+    clustered decode kernel normalises inside its launch, the others run the norm kernel first), and
+    with MOE_ACCUMULATE in place it is one residual step."""
+    import bit_expert_ffn_gemv_b200 as moe
+    torch = torch_cuda
+    wl, h, _ = decode_layer
+    sh = wl.shape
+    pf = {"default": 0, "unfused": moe.MOE_FORCE_UNFUSED, "gemv": moe.MOE_FORCE_GEMV}[path]
+    x = x_to_device(synth.x_host(sh, wl.master, 900 + T, T)) * 3
+    u = moe.rms_normalize(x)
+    for out in (0, moe.MOE_OUT_FP32):
+        ref = h.forward(0, u, flags=pf | out)
+        got = h.forward(0, x, flags=pf | out | moe.MOE_NORM_INPUT)
+        torch.cuda.synchronize()
+        assert h.check_status() == 0
+        assert torch.equal(got.view(torch.int16 if got.dtype != torch.float32 else torch.int32),
+                           ref.view(torch.int16 if ref.dtype != torch.float32 else torch.int32)), (T, path, out)
+    r = x.clone()
+    h.forward(0, r, r, flags=pf | moe.MOE_ACCUMULATE | moe.MOE_NORM_INPUT)
+    y32 = h.forward(0, u, flags=pf | moe.MOE_OUT_FP32)
+    torch.cuda.synchronize()
+    assert torch.equal(r, (x.float() + y32).to(torch.bfloat16)), (T, path)
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_chain48_with_norm_input_equals_two_calls(torch_cuda, chain, T):
+    """The 48-layer chain as one call per layer (MOE_NORM_INPUT | MOE_ACCUMULATE, in place) ends bit for
+    bit where the two-call chain (norm, then layer) ends."""
+    import bit_expert_ffn_gemv_b200 as moe
+    torch = torch_cuda
+    wl, h = chain
+    sh = wl.shape
+    x0 = x_to_device(synth.x_host(sh, wl.master, 2, T))
+    r1, r2 = x0.clone(), x0.clone()
+    u = torch.empty_like(x0)
+    for l in range(wl.layers):
+        moe.rms_normalize(r1, u)
+        h.forward(l, u, r1, flags=moe.MOE_ACCUMULATE)
+        h.forward(l, r2, r2, flags=moe.MOE_ACCUMULATE | moe.MOE_NORM_INPUT)
+    torch.cuda.synchronize()
+    assert h.check_status() == 0
+    assert torch.isfinite(r2.float()).all()
+    assert torch.equal(r1, r2)
