@@ -61,10 +61,10 @@ _KERNEL_SOURCE = {"gemm_gateup": "gemm_sm100.cu", "gemm_down": "gemm_sm100.cu", 
                   "decode_fused": "decode_pair.cu", "gemv_gateup": "gemv.cu", "gemv_down": "gemv.cu"}
 
 
-def profile_traffic(kernel: str):
+def profile_traffic(kernel: str, tokens=None):
     """DRAM bytes per launch of `kernel` from a committed ncu summary (profiles/*.md lines
-    `traffic: kernel=K source_sha256_16=H dram_bytes_per_launch=B`), or None when no capture exists or
-    the kernel's source changed since it was taken."""
+    `traffic: kernel=K source_sha256_16=H tokens=T dram_bytes_per_launch=B`), or None when no capture of
+    this workload size exists or the kernel's source changed since it was taken."""
     import glob
     import hashlib
     src = _KERNEL_SOURCE.get(kernel)
@@ -80,7 +80,8 @@ def profile_traffic(kernel: str):
             if not line.startswith("traffic:"):
                 continue
             kv = dict(t.split("=", 1) for t in line.split()[1:] if "=" in t)
-            if kv.get("kernel") == kernel and kv.get("source_sha256_16") == cur:
+            if kv.get("kernel") == kernel and kv.get("source_sha256_16") == cur and \
+                    (tokens is None or kv.get("tokens") == str(tokens)):
                 return int(kv["dram_bytes_per_launch"])
     return None
 
@@ -360,7 +361,7 @@ def kernel_profile(h, step, first, n):
     return prof
 
 
-def roofline_of(prof, alg_bytes, flops, nprof):
+def roofline_of(prof, alg_bytes, flops, nprof, tokens=None):
     """Roofline entry of the dominant kernel of a per-kernel profile."""
     hbm, tc_burst, tc_sus, peak_kind = measured_peaks()
     if not prof:
@@ -369,15 +370,26 @@ def roofline_of(prof, alg_bytes, flops, nprof):
     if dom in flops:
         dom_ms = prof[dom][0] / prof[dom][1]
         ach = flops[dom] / (dom_ms / 1000.0) / 1e12
-        return {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": tc_burst, "unit": "TFLOP/s",
-                "frac": ach / tc_burst, "traffic": profile_traffic(dom),
-                "peak_kind": peak_kind + " bf16 dense (burst)", "flops_per_launch": flops[dom],
-                "avg_launch_us": 1000.0 * dom_ms}
+        r = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": tc_burst, "unit": "TFLOP/s",
+             "frac": ach / tc_burst, "traffic": profile_traffic(dom, tokens),
+             "peak_kind": peak_kind + " bf16 dense (burst)", "flops_per_launch": flops[dom],
+             "avg_launch_us": 1000.0 * dom_ms}
+        if alg_bytes.get(dom):
+            # a grouped GEMM over small expert groups is bound by its weight bytes, not its FLOPs:
+            # report against whichever bound takes longer
+            bpl = alg_bytes[dom] / max(1, prof[dom][1])
+            ach_b = bpl / (dom_ms / 1000.0) / 1e9
+            r["hbm_frac"] = ach_b / hbm
+            r["bytes_per_launch"] = bpl
+            if bpl / (hbm * 1e9) > flops[dom] / (tc_burst * 1e12):
+                r.update({"bound": "hbm", "achieved": ach_b, "peak": hbm, "unit": "GB/s", "frac": ach_b / hbm,
+                          "peak_kind": peak_kind, "tensor_frac": ach / tc_burst})
+        return r
     if dom in alg_bytes:
         dom_ms = prof[dom][0]
         ach = alg_bytes[dom] / (dom_ms / 1000.0) / 1e9
         r = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-             "traffic": profile_traffic(dom), "peak_kind": peak_kind,
+             "traffic": profile_traffic(dom, tokens), "peak_kind": peak_kind,
              "bytes_per_launch": alg_bytes[dom] / max(1, prof[dom][1]),
              "avg_launch_us": 1000.0 * dom_ms / max(1, prof[dom][1])}
         if dom == "decode_fused":
@@ -422,13 +434,16 @@ def measure_decode(moe, h, sh, xs, layers, T, flags, args, steps, warmup, clock_
     # per-kernel device time and the algorithmic bytes of the same steps
     nl = layers if chain else 1
     nprof = min(steps, 64)
-    alg = {"gemv_gateup": 0.0, "gemv_down": 0.0, "decode_fused": 0.0, "layer": 0.0}
+    alg = {"gemv_gateup": 0.0, "gemv_down": 0.0, "gemm_gateup": 0.0, "gemm_down": 0.0, "decode_fused": 0.0,
+           "layer": 0.0}
     for i in range(nprof):
         step(warmup + i)
         D = h.stats()["active_experts"]
         lb = nl * layer_bytes(sh, D, T)
         alg["gemv_gateup"] += nl * (D + sh.n_shared) * 2 * mat_bytes(sh, 0)
         alg["gemv_down"] += nl * (D + sh.n_shared) * mat_bytes(sh, 2)
+        alg["gemm_gateup"] += nl * (D + sh.n_shared) * 2 * mat_bytes(sh, 0)
+        alg["gemm_down"] += nl * (D + sh.n_shared) * mat_bytes(sh, 2)
         alg["decode_fused"] += lb
         alg["layer"] += lb
     prof = kernel_profile(h, step, warmup, nprof)
@@ -436,7 +451,7 @@ def measure_decode(moe, h, sh, xs, layers, T, flags, args, steps, warmup, clock_
     flops = {"gemm_gateup": 2.0 * rows * 2 * sh.f * sh.d, "gemm_down": 2.0 * rows * sh.d * sh.f}
     layer_time = sum(v[0] for v in prof.values())
     return {"ms": ms, "clocks": clocks, "launches": launches, "step": step,
-            "roofline": roofline_of(prof, alg, flops, nprof),
+            "roofline": roofline_of(prof, alg, flops, nprof, T),
             "layer_hbm_gbs": alg["layer"] / (layer_time / 1000.0) / 1e9 if layer_time else None,
             "kernels_ms_per_step": {k: v[0] / nprof for k, v in prof.items()}}
 
