@@ -111,7 +111,7 @@ def lib() -> ctypes.CDLL:
             L.moe_debug_router_logits.restype = st
             L.moe_debug_router_logits.argtypes = [vp, i32, vp, i32, vp, i32, vp]
             L.moe_router_error_depth.restype = ctypes.c_float
-            L.moe_router_error_depth.argtypes = [i32, i32]
+            L.moe_router_error_depth.argtypes = [i32, i32, i32]
             L.moe_rms_normalize.restype = st
             L.moe_rms_normalize.argtypes = [vp, i32, i32, vp, vp]
             L.moe_set_expert_range.restype = st
@@ -199,8 +199,8 @@ def moe_debug_router_logits(handle: int, layer: int, x_ptr: int, T: int, logits_
            "moe_debug_router_logits")
 
 
-def moe_router_error_depth(d: int, tensor_cores: bool) -> float:
-    return float(lib().moe_router_error_depth(d, 1 if tensor_cores else 0))
+def moe_router_error_depth(d: int, tensor_cores: bool, T: int = 0) -> float:
+    return float(lib().moe_router_error_depth(d, T, 1 if tensor_cores else 0))
 
 
 def moe_rms_normalize(x_ptr: int, T: int, d: int, out_ptr: int, stream: int) -> None:

@@ -184,7 +184,7 @@ moe_status do_route(moe_handle* h, int32_t layer, const void* x, int32_t T, int3
     ra.w = w;
     ra.meta = h->meta;
     if (tc) {
-        ra.depth = moe::router_gemm_depth(ra.d);
+        ra.depth = moe::router_gemm_depth(ra.d, moe::router_gemm_chunks(T, ra.d));
         e = run(h, MOE_K_ROUTER_GEMM, s, [&] { return moe::launch_router_gemm(ra, h->status, s); });
     } else {
         e = run(h, MOE_K_ROUTER_LOGITS, s, [&] { return moe::launch_router_logits(ra, s); });
@@ -555,9 +555,11 @@ moe_status moe_debug_router_logits(moe_handle* h, int32_t layer, const void* x, 
     return cuda_status(e);
 }
 
-float moe_router_error_depth(int32_t d, int32_t tensor_cores) {
+float moe_router_error_depth(int32_t d, int32_t T, int32_t tensor_cores) {
     if (d <= 0) return 0.0f;
-    return tensor_cores ? moe::router_gemm_depth(d) : (float)(d / 32 + 6);
+    if (!tensor_cores) return (float)(d / 32 + 6);
+    // T <= 0: the bound for any batch (full 128-token tiles have the fewest chunks)
+    return moe::router_gemm_depth(d, moe::router_gemm_chunks(T > 0 ? T : (1 << 20), d));
 }
 
 moe_status moe_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, void* y, uint32_t flags,

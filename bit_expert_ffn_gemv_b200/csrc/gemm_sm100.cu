@@ -560,13 +560,18 @@ __global__ void __launch_bounds__(kExpertThreads, 1)
 
 // ---------------------------------------------------------------- router GEMM
 // logits[t][e] = W_r[e] . x_t + bias_e for 128-expert x 128-token tiles, bf16
-// operands copied straight into the SW128 tiles.
+// operands copied straight into the SW128 tiles.  The contraction is split
+// into `chunks` consecutive K ranges, each accumulated in its own tensor-memory
+// columns; the epilogue adds the chunk sums in chunk order.  A chunk's rounding
+// error grows with its own length, so the logits' error bound is that many
+// times tighter than one running sum over all of d (router_gemm_depth).
 constexpr int kRouterStages = 4;
 constexpr int kRouterStage = kTileM * 128 + kRouterTileN * 128;
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
     router_gemm_kernel(const uint16_t* __restrict__ x, int T, int d, const uint16_t* __restrict__ wr,
-                       const float* __restrict__ bias, int E, float* __restrict__ logits, uint32_t* status) {
+                       const float* __restrict__ bias, int E, float* __restrict__ logits, int chunks,
+                       uint32_t* status) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t mma_bar[kRouterStages];
     __shared__ uint32_t tmem_slot;
@@ -578,11 +583,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int i = 0; i < kRouterStages; ++i) mbar_init(&mma_bar[i], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) tc::tmem_alloc(&tmem_slot, kRouterTileN);
+    if (warp == 0) tc::tmem_alloc(&tmem_slot, 512);
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = tmem_slot;
+    const int csteps = KS / chunks;          // K steps per chunk
+    const uint32_t ccols = 512u / chunks;    // tensor-memory columns per chunk (>= the tile's width)
     uint32_t gstep = 0;
     bool ok = true, all_ok = true;
     for (int tile = blockIdx.x; tile < MT * NT && all_ok; tile += gridDim.x) {
@@ -626,10 +633,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             if (tid == 0) {
                 tc::fence_after();
                 const uint32_t a_addr = smem_addr(smem + st * kRouterStage), b_addr = a_addr + kTileM * 128;
+                const int ch = s / csteps;  // this step's chunk
 #pragma unroll
                 for (int kk = 0; kk < kStepK / 16; ++kk)
-                    tc::mma(tmem, tc::sdesc(a_addr + kk * 32), tc::sdesc(b_addr + kk * 32), idesc,
-                            (s > 0 || kk > 0) ? 1u : 0u);
+                    tc::mma(tmem + ch * ccols, tc::sdesc(a_addr + kk * 32), tc::sdesc(b_addr + kk * 32), idesc,
+                            (s > ch * csteps || kk > 0) ? 1u : 0u);
                 tc::commit(&mma_bar[st]);
             }
         }
@@ -643,11 +651,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int e = e0 + 32 * (warp & 3) + lane;
         const float b = (bias && e < E) ? bias[e] : 0.0f;
         for (int c0 = 16 * (warp >> 2); c0 < nmma && all_ok; c0 += 32) {
-            uint32_t r0[16];
-            tc::ld16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c0, r0);
+            const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c0;
+            float v[16];
+            for (int ch0 = 0; ch0 < chunks; ch0 += 4) {  // chunk sums in chunk order, 4 loads in flight
+                uint32_t r[4][16];
+                const int nc = min(4, chunks - ch0);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (j < nc) tc::ld16_nowait(ta + (ch0 + j) * ccols, r[j]);
+                tc::ld_wait();
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (j < nc) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            v[i] = (ch0 + j == 0) ? __uint_as_float(r[j][i]) : v[i] + __uint_as_float(r[j][i]);
+                    }
+            }
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-                if (c0 + i < n && e < E) logits[(int64_t)(t0 + c0 + i) * E + e] = __uint_as_float(r0[i]) + b;
+                if (c0 + i < n && e < E) logits[(int64_t)(t0 + c0 + i) * E + e] = v[i] + b;
         }
         tc::fence_before();
         __syncthreads();
@@ -655,7 +678,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc::cp_wait<0>();
     tc::fence_before();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, kRouterTileN);
+    if (warp == 0) tc::tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------- activation gather, combine
@@ -925,19 +948,33 @@ cudaError_t launch_router_gemm(const RouteArgs& a, uint32_t* status, cudaStream_
     const int tiles = ((a.E + kTileM - 1) / kTileM) * ((a.T + kRouterTileN - 1) / kRouterTileN);
     router_gemm_kernel<<<min(tiles, num_sms()), kGemmThreads, smem, s>>>(
         static_cast<const uint16_t*>(a.x), a.T, a.d, static_cast<const uint16_t*>(a.wr), a.bias, a.E, a.logits,
-        status);
+        router_gemm_chunks(a.T, a.d), status);
     return cudaGetLastError();
+}
+
+// K chunks of the router GEMM for T tokens: as many as the 512 tensor-memory
+// columns hold at the tile's width (16..128 columns), a power of two dividing
+// the d / 64 steps, at most 32 (4 for 128-token tiles, 8 at 64 tokens or fewer).
+int router_gemm_chunks(int T, int d) {
+    const int cols = T >= kRouterTileN ? kRouterTileN : ((T + 15) & ~15);
+    const int steps = d / kStepK;
+    int c = 1;
+    while (2 * c <= 512 / (cols > 16 ? cols : 16) && 2 * c <= 32 && steps % (2 * c) == 0) c *= 2;
+    return c;
 }
 
 // Error bound of the tensor-core logits, in the units of the top-k kernel's
 // certificate delta = 2 * depth * 2^-24 * (||W_r,e|| ||x|| + |bias_e|).
-// Model: each MMA adds 16 exact bf16 x bf16 products to the fp32 accumulator;
-// aligning the 17 terms to the largest exponent and truncating costs at most
-// one fp32 ulp of that largest term per term, and every term is at most
-// sum_i |w_i x_i| <= ||w|| ||x||.  So a K = 16 step errs by at most
-// 17 * 2^-23 * ||w|| ||x||; doubled for margin and summed over d / 16 steps,
-// plus the fp32 bias add: depth = 34 * (d / 16) + 2.
-float router_gemm_depth(int d) { return 34.0f * (float)(d / 16) + 2.0f; }
+// Model: each MMA adds 16 exact bf16 x bf16 products to its chunk's fp32
+// accumulator; aligning the 17 terms to the largest exponent and truncating
+// costs at most one fp32 ulp of that largest term per term, and every term is
+// at most the chunk's sum_i |w_i x_i| <= ||w|| ||x||.  Summed over a chunk's
+// d / (16 c) steps (doubled for margin), the chunk errors together stay
+// within 34 * d / (16 c) units of the whole sum; then c - 1 fp32 adds of the
+// chunk sums and the bias add, one unit each.
+float router_gemm_depth(int d, int chunks) {
+    return 34.0f * (float)(d / 16 / chunks) + (float)(chunks - 1) + 2.0f;
+}
 
 cudaError_t launch_gather_f16(const void* x, int T, int d, int k, int n_shared, const int32_t* pairs,
                               const int32_t* n_pairs, void* xg, uint32_t* status, cudaStream_t s) {

@@ -128,7 +128,8 @@ cudaError_t launch_gemv_down(const ExpertArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 // tcgen05 path (T > kDecodeMaxTokens)
 cudaError_t launch_router_gemm(const RouteArgs& a, uint32_t* status, cudaStream_t s);
-float router_gemm_depth(int d);
+int router_gemm_chunks(int T, int d);
+float router_gemm_depth(int d, int chunks);
 size_t tile_desc_count(int T, int k, int E, int n_shared, int jt);
 cudaError_t launch_build_tiles(const ExpertArgs& a, int4* desc_gu, int4* desc_dn, int32_t* counts, cudaStream_t s);
 // TMA descriptors of one expert GEMM: its activation rows (two box heights)

@@ -286,15 +286,20 @@ moe_status moe_debug_last_routing(moe_handle* h, int32_t T, int32_t* ids, float*
  * them: tensor_cores != 0 the bf16 tcgen05 GEMM (a forward uses it above 16
  * tokens, moe_route above 64), else the CUDA-core kernel.  Each logit is within
  *   delta_e = 2 * depth * 2^-24 * (||W_r,e||_2 ||x||_2 + |bias_e|)
- * of the exact value, depth = moe_router_error_depth(d, tensor_cores); the
+ * of the exact value, depth = moe_router_error_depth(d, T, tensor_cores); the
  * top-k re-ranks every token whose order these intervals leave open.
  * Errors: INVALID_ARG, NOT_LOADED, CUDA.
  */
 moe_status moe_debug_router_logits(moe_handle* h, int32_t layer, const void* x, int32_t T, float* logits,
                                    int32_t tensor_cores, void* stream);
 
-/* The `depth` of the logits error bound above for hidden size d (0 if d <= 0). */
-float moe_router_error_depth(int32_t d, int32_t tensor_cores);
+/*
+ * The `depth` of the logits error bound above for hidden size d and a batch of
+ * T tokens (0 if d <= 0).  The tensor-core GEMM sums the contraction in K
+ * chunks, more of them for narrower token tiles, so its bound tightens for
+ * T < 128; T <= 0 gives the bound that holds for every T.
+ */
+float moe_router_error_depth(int32_t d, int32_t T, int32_t tensor_cores);
 
 /*
  * Synchronise the device and return the first device-side error recorded
