@@ -39,6 +39,7 @@ struct moe_handle {
     size_t arena_bytes = 0;
     // views into the arena
     float* logits = nullptr;
+    float* logit_parts = nullptr;  // chunk sums of the split router GEMM [32][min(T, 128)][E]
     int32_t* ids = nullptr;
     float* w = nullptr;
     int32_t* offsets = nullptr;
@@ -184,8 +185,23 @@ moe_status do_route(moe_handle* h, int32_t layer, const void* x, int32_t T, int3
     ra.w = w;
     ra.meta = h->meta;
     if (tc) {
-        ra.depth = moe::router_gemm_depth(ra.d, moe::router_gemm_chunks(T, ra.d));
-        e = run(h, MOE_K_ROUTER_GEMM, s, [&] { return moe::launch_router_gemm(ra, h->status, s); });
+        const int chunks = moe::router_gemm_chunks(T, ra.d);
+        ra.depth = moe::router_gemm_depth(ra.d, chunks);
+        if (moe::router_gemm_split(T)) {
+            // small batch: the GEMM's chunk sums over all SMs, then their fixed-order
+            // reduction into the logits (both counted as the router GEMM)
+            moe::RouteArgs rp = ra;
+            rp.logits = h->logit_parts;
+            rp.logit_parts = chunks;
+            e = run(h, MOE_K_ROUTER_GEMM, s, [&] {
+                cudaError_t r = moe::launch_router_gemm(rp, h->status, s);
+                if (r == cudaSuccess) r = moe::launch_router_reduce(rp.logits, chunks, T, ra.E, ra.bias, ra.logits, s);
+                return r;
+            });
+            h->launches++;
+        } else {
+            e = run(h, MOE_K_ROUTER_GEMM, s, [&] { return moe::launch_router_gemm(ra, h->status, s); });
+        }
     } else {
         e = run(h, MOE_K_ROUTER_LOGITS, s, [&] { return moe::launch_router_logits(ra, s); });
     }
@@ -419,6 +435,7 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
         return o;
     };
     const size_t o_logits = take(sizeof(float) * T * E);
+    const size_t o_lparts = take(sizeof(float) * 32 * std::min<size_t>(T, 128) * E);
     const size_t o_ids = take(sizeof(int32_t) * T * k);
     const size_t o_w = take(sizeof(float) * T * k);
     const size_t o_off = take(sizeof(int32_t) * (E + 1));
@@ -455,6 +472,7 @@ moe_status moe_layer_init(const moe_config* cfg, moe_handle** out) {
     }
     char* base = static_cast<char*>(h->arena);
     h->logits = reinterpret_cast<float*>(base + o_logits);
+    h->logit_parts = reinterpret_cast<float*>(base + o_lparts);
     h->ids = reinterpret_cast<int32_t*>(base + o_ids);
     h->w = reinterpret_cast<float*>(base + o_w);
     h->offsets = reinterpret_cast<int32_t*>(base + o_off);
@@ -551,6 +569,13 @@ moe_status moe_debug_router_logits(moe_handle* h, int32_t layer, const void* x, 
     ra.ids = nullptr;
     ra.w = nullptr;
     ra.meta = h->meta;
+    if (tensor_cores && moe::router_gemm_split(T)) {  // chunk sums, then their fixed-order reduction
+        ra.logits = h->logit_parts;
+        ra.logit_parts = moe::router_gemm_chunks(T, ra.d);
+        cudaError_t e = moe::launch_router_gemm(ra, h->status, s);
+        if (e == cudaSuccess) e = moe::launch_router_reduce(ra.logits, ra.logit_parts, T, ra.E, ra.bias, logits, s);
+        return cuda_status(e);
+    }
     cudaError_t e = tensor_cores ? moe::launch_router_gemm(ra, h->status, s) : moe::launch_router_logits(ra, s);
     return cuda_status(e);
 }

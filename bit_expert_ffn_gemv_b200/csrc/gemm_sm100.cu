@@ -565,12 +565,16 @@ __global__ void __launch_bounds__(kExpertThreads, 1)
 // columns; the epilogue adds the chunk sums in chunk order.  A chunk's rounding
 // error grows with its own length, so the logits' error bound is that many
 // times tighter than one running sum over all of d (router_gemm_depth).
+// split != 0 (small batches, whose few tiles would leave most SMs idle): every
+// (tile, chunk) is a work item of its own, and its raw chunk sums go to
+// logits[chunk][t][e]; the reader adds the chunks in chunk order, then the
+// bias -- the same operations, so the same logits, as the unsplit epilogue.
 constexpr int kRouterStages = 4;
 constexpr int kRouterStage = kTileM * 128 + kRouterTileN * 128;
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
     router_gemm_kernel(const uint16_t* __restrict__ x, int T, int d, const uint16_t* __restrict__ wr,
-                       const float* __restrict__ bias, int E, float* __restrict__ logits, int chunks,
+                       const float* __restrict__ bias, int E, float* __restrict__ logits, int chunks, int split,
                        uint32_t* status) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t mma_bar[kRouterStages];
@@ -592,9 +596,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t ccols = 512u / chunks;    // tensor-memory columns per chunk (>= the tile's width)
     uint32_t gstep = 0;
     bool ok = true, all_ok = true;
-    for (int tile = blockIdx.x; tile < MT * NT && all_ok; tile += gridDim.x) {
+    const int items = MT * NT * (split ? chunks : 1);
+    for (int item = blockIdx.x; item < items && all_ok; item += gridDim.x) {
+        const int tile = item % (MT * NT), ich = item / (MT * NT);  // ich: the item's chunk (split)
         const int mt = tile % MT, nt = tile / MT;
         const int e0 = mt * kTileM, t0 = nt * kRouterTileN;
+        const int s0 = split ? ich * csteps : 0, ns = split ? csteps : KS;  // the item's K steps
         const int n = min(kRouterTileN, T - t0), nmma = (n + 15) & ~15;
         const uint32_t idesc = tc::idesc_f16(kTileM, nmma, true);
         auto load_step = [&](int s, int st) {
@@ -613,27 +620,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         };
         const int P = kRouterStages - 1;
         for (int s = 0; s < P; ++s) {
-            if (s < KS) load_step(s, (gstep + s) % kRouterStages);
+            if (s < ns) load_step(s0 + s, (gstep + s) % kRouterStages);
             tc::cp_commit();
         }
-        for (int s = 0; s < KS; ++s) {
+        for (int s = 0; s < ns; ++s) {
             const uint32_t cur = gstep + s;
             const int st = cur % kRouterStages;
             tc::cp_wait<kRouterStages - 2>();
             fence_proxy_async_smem();
-            if (s + P < KS) {
+            if (s + P < ns) {
                 if (cur >= 1 && ok) {
                     const uint32_t prev = cur - 1;
                     ok = tc::bar_wait(&mma_bar[prev % kRouterStages], (prev / kRouterStages) & 1, status);
                 }
-                load_step(s + P, (cur + P) % kRouterStages);
+                load_step(s0 + s + P, (cur + P) % kRouterStages);
             }
             tc::cp_commit();
             __syncthreads();
             if (tid == 0) {
                 tc::fence_after();
                 const uint32_t a_addr = smem_addr(smem + st * kRouterStage), b_addr = a_addr + kTileM * 128;
-                const int ch = s / csteps;  // this step's chunk
+                const int ch = split ? 0 : s / csteps;  // this step's accumulator
 #pragma unroll
                 for (int kk = 0; kk < kStepK / 16; ++kk)
                     tc::mma(tmem + ch * ccols, tc::sdesc(a_addr + kk * 32), tc::sdesc(b_addr + kk * 32), idesc,
@@ -642,15 +649,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
         }
         if (ok) {
-            const uint32_t last = gstep + KS - 1;
+            const uint32_t last = gstep + ns - 1;
             ok = tc::bar_wait(&mma_bar[last % kRouterStages], (last / kRouterStages) & 1, status);
         }
-        gstep += KS;
+        gstep += ns;
         all_ok = __syncthreads_and(ok) != 0;
         tc::fence_after();
         const int e = e0 + 32 * (warp & 3) + lane;
         const float b = (bias && e < E) ? bias[e] : 0.0f;
-        for (int c0 = 16 * (warp >> 2); c0 < nmma && all_ok; c0 += 32) {
+        for (int c0 = 16 * (warp >> 2); c0 < nmma && all_ok && split; c0 += 32) {
+            // the item's raw chunk sums
+            uint32_t r0[16];
+            tc::ld16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c0, r0);
+            float* lp = logits + (int64_t)ich * T * E;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                if (c0 + i < n && e < E) lp[(int64_t)(t0 + c0 + i) * E + e] = __uint_as_float(r0[i]);
+        }
+        for (int c0 = 16 * (warp >> 2); c0 < nmma && all_ok && !split; c0 += 32) {
             const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c0;
             float v[16];
             for (int ch0 = 0; ch0 < chunks; ch0 += 4) {  // chunk sums in chunk order, 4 loads in flight
@@ -946,21 +962,47 @@ cudaError_t launch_router_gemm(const RouteArgs& a, uint32_t* status, cudaStream_
     cudaError_t e = cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     const int tiles = ((a.E + kTileM - 1) / kTileM) * ((a.T + kRouterTileN - 1) / kRouterTileN);
-    router_gemm_kernel<<<min(tiles, num_sms()), kGemmThreads, smem, s>>>(
+    const int chunks = router_gemm_chunks(a.T, a.d), split = router_gemm_split(a.T) ? 1 : 0;
+    if (split && a.logit_parts != chunks) return cudaErrorInvalidValue;  // the caller sized logits for the chunks
+    const int items = tiles * (split ? chunks : 1);
+    router_gemm_kernel<<<min(items, num_sms()), kGemmThreads, smem, s>>>(
         static_cast<const uint16_t*>(a.x), a.T, a.d, static_cast<const uint16_t*>(a.wr), a.bias, a.E, a.logits,
-        router_gemm_chunks(a.T, a.d), status);
+        chunks, split, status);
     return cudaGetLastError();
 }
 
-// K chunks of the router GEMM for T tokens: as many as the 512 tensor-memory
-// columns hold at the tile's width (16..128 columns), a power of two dividing
-// the d / 64 steps, at most 32 (4 for 128-token tiles, 8 at 64 tokens or fewer).
+// Batches of at most one token tile are split by K chunk over the CTAs.
+bool router_gemm_split(int T) { return T <= kRouterTileN; }
+
+// K chunks of the router GEMM for T tokens, a power of two dividing the d / 64
+// steps, at most 32.  Split (T <= 128): 32, one step each at d = 2048.  Else as
+// many as the 512 tensor-memory columns hold at the tile's 128 columns: 4.
 int router_gemm_chunks(int T, int d) {
-    const int cols = T >= kRouterTileN ? kRouterTileN : ((T + 15) & ~15);
+    const int cols = router_gemm_split(T) ? 16 : kRouterTileN;  // split: one accumulator per CTA
     const int steps = d / kStepK;
     int c = 1;
-    while (2 * c <= 512 / (cols > 16 ? cols : 16) && 2 * c <= 32 && steps % (2 * c) == 0) c *= 2;
+    while (2 * c <= 512 / cols && 2 * c <= 32 && steps % (2 * c) == 0) c *= 2;
     return c;
+}
+
+// logits[t][e] = (sum over chunks c, in order, of parts[c][t][e]) + bias_e: the
+// split router GEMM's chunk sums reduced as its unsplit epilogue would.
+__global__ void router_reduce_kernel(const float* __restrict__ parts, int chunks, int T, int E,
+                                     const float* __restrict__ bias, float* __restrict__ logits) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x, n = (int64_t)T * E;
+    if (i >= n) return;
+    float v = parts[i];
+#pragma unroll 8
+    for (int c = 1; c < chunks; ++c) v += parts[(int64_t)c * n + i];
+    logits[i] = v + (bias ? bias[i % E] : 0.0f);
+}
+
+cudaError_t launch_router_reduce(const float* parts, int chunks, int T, int E, const float* bias, float* logits,
+                                 cudaStream_t s) {
+    const int64_t n = (int64_t)T * E;
+    if (n == 0) return cudaSuccess;
+    router_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(parts, chunks, T, E, bias, logits);
+    return cudaGetLastError();
 }
 
 // Error bound of the tensor-core logits, in the units of the top-k kernel's

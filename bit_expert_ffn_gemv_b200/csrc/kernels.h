@@ -14,7 +14,8 @@ struct RouteArgs {
     const void* wr;     // bf16 [E x d]
     const float* bias;  // [E] or null
     const float* wnorm; // [E] ||W_r,e||_2, rounded up
-    float* logits;      // scratch [T x E]
+    float* logits;      // scratch [T x E]; [logit_parts][T x E] raw chunk sums (split router GEMM)
+    int logit_parts = 1;  // > 1: the reader adds the parts in order, then the bias
     int32_t* ids;       // [T x k]
     float* w;           // [T x k]
     Meta* meta;
@@ -128,7 +129,10 @@ cudaError_t launch_gemv_down(const ExpertArgs& a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 // tcgen05 path (T > kDecodeMaxTokens)
 cudaError_t launch_router_gemm(const RouteArgs& a, uint32_t* status, cudaStream_t s);
+bool router_gemm_split(int T);
 int router_gemm_chunks(int T, int d);
+cudaError_t launch_router_reduce(const float* parts, int chunks, int T, int E, const float* bias, float* logits,
+                                 cudaStream_t s);
 float router_gemm_depth(int d, int chunks);
 size_t tile_desc_count(int T, int k, int E, int n_shared, int jt);
 cudaError_t launch_build_tiles(const ExpertArgs& a, int4* desc_gu, int4* desc_dn, int32_t* counts, cudaStream_t s);

@@ -99,6 +99,11 @@ MOE_DEV bool better64(double va, int ia, double vb, int ib) {
 }
 
 constexpr int kTopkWarps = 4;
+// Batches of up to this many tokens take a CTA of kTopkWideWarps warps per
+// token (the GPU is otherwise mostly idle there): every warp selects the same
+// k redundantly, and the fp64 candidate logits are split over the warps.
+constexpr int kTopkWideWarps = 8;
+constexpr int kTopkWideMaxT = 256;
 
 // order-preserving image of an fp32 logit (NaN as -inf): a larger key is a
 // larger value; 0 is below every key
@@ -109,9 +114,9 @@ MOE_DEV uint32_t fkey(float v) {
     return (b >> 31) ? ~b : (b | 0x80000000u);
 }
 
-// One warp per token.  Shared memory per warp: E doubles (fp64 logits of the
-// candidates), E floats (fp32 logits), E floats (their error bounds, later
-// the candidate list).
+// One warp per token (WIDE: one CTA per token, see kTopkWideWarps).  Shared
+// memory per warp: E doubles (fp64 logits of the candidates), E floats (fp32
+// logits), E floats (their error bounds, later the candidate list).
 //
 // Every fp32 logit l_e lies within d_e of the exact one.  k rounds of a warp
 // max-reduction over the logits' keys select S, the k largest fp32 logits (in
@@ -122,19 +127,21 @@ MOE_DEV uint32_t fkey(float v) {
 // intervals of consecutive ranks are disjoint, S in its fp32 order is the
 // exact selection; otherwise the candidates' logits are recomputed in fp64
 // (sums of exact bf16 products) and ranked exactly by (value desc, index asc).
-template <int KPL>
-__global__ void __launch_bounds__(kTopkWarps * 32)
+template <int KPL, bool WIDE>
+__global__ void __launch_bounds__((WIDE ? kTopkWideWarps : kTopkWarps) * 32)
     topk_kernel(const float* __restrict__ logits, const __nv_bfloat16* __restrict__ x, int T, int d, int E, int k,
                 const __nv_bfloat16* __restrict__ wr, const float* __restrict__ bias,
                 const float* __restrict__ wnorm, float depth, int32_t* __restrict__ ids_out,
                 float* __restrict__ w_out, Meta* __restrict__ meta) {
+    constexpr int NW = WIDE ? kTopkWideWarps : kTopkWarps;
     extern __shared__ unsigned char smem_raw[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * kTopkWarps + warp;
+    const int t = WIDE ? (int)blockIdx.x : (int)blockIdx.x * kTopkWarps + warp;
     double* lg64 = reinterpret_cast<double*>(smem_raw) + (size_t)warp * E;
-    float* lv = reinterpret_cast<float*>(smem_raw + sizeof(double) * (size_t)kTopkWarps * E) + (size_t)warp * 2 * E;
+    double* lg64_out = WIDE ? reinterpret_cast<double*>(smem_raw) : lg64;  // WIDE: warp 0's, shared by all
+    float* lv = reinterpret_cast<float*>(smem_raw + sizeof(double) * (size_t)NW * E) + (size_t)warp * 2 * E;
     float* dv = lv + E;
-    if (t >= T) return;
+    if (t >= T) return;  // WIDE: never (one CTA per token)
 
     // ||x_t||_2 (fp32, inflated to stay an upper bound); 8 values per lane per 256
     const __nv_bfloat16* xt = x + (int64_t)t * d;
@@ -229,8 +236,10 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
         if (lane < k) my_w = my_l;
     } else {
         // fp64 logits of the candidates (sums of exact bf16 products), 8 products
-        // per lane per 256-wide chunk, four candidates per pass (more loads in flight)
-        for (int ci = 0; ci < n_cand; ci += 4) {
+        // per lane per 256-wide chunk, four candidates per pass (more loads in
+        // flight); WIDE: the passes are dealt over the CTA's warps, which hold
+        // the same candidate list
+        for (int ci = WIDE ? 4 * warp : 0; ci < n_cand; ci += WIDE ? 4 * kTopkWideWarps : 4) {
             int ec[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) ec[u] = cand[min(ci + u, n_cand - 1)];
@@ -261,8 +270,12 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
             if (lane == 0) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                    if (ci + u < n_cand) lg64[ci + u] = acc[u] + (bias ? (double)bias[ec[u]] : 0.0);
+                    if (ci + u < n_cand) lg64_out[ci + u] = acc[u] + (bias ? (double)bias[ec[u]] : 0.0);
             }
+        }
+        if (WIDE) {
+            __syncthreads();  // every warp took the same branch: the certificate is computed alike
+            if (warp != 0) return;
         }
         __syncwarp();
         if (n_cand <= 32) {
@@ -322,6 +335,7 @@ __global__ void __launch_bounds__(kTopkWarps * 32)
         if (lane == 0) atomicAdd(&meta->n_fixup, 1);
     }
 
+    if (WIDE && warp != 0) return;  // warp 0 writes the token's result
     // renormalised weights = softmax over the k selected logits (lane r: rank r)
     const float m = __shfl_sync(0xffffffffu, my_w, 0);
     const float ex = lane < k ? expf(my_w - m) : 0.0f;
@@ -354,17 +368,21 @@ cudaError_t launch_router_logits(const RouteArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_topk(const RouteArgs& a, cudaStream_t s) {
-    const size_t smem_t = (size_t)kTopkWarps * a.E * (sizeof(double) + 2 * sizeof(float));
-    auto kern = a.E <= 512 ? topk_kernel<16> : topk_kernel<32>;
-    if (a.E > 1024) return cudaErrorInvalidValue;
+    if (a.E > 1024 || a.logit_parts != 1) return cudaErrorInvalidValue;  // reads reduced logits
+    const bool wide = a.T <= kTopkWideMaxT;
+    const int nw = wide ? kTopkWideWarps : kTopkWarps;
+    const size_t smem_t = (size_t)nw * a.E * (sizeof(double) + 2 * sizeof(float));
+    auto kern = wide ? (a.E <= 512 ? topk_kernel<16, true> : topk_kernel<32, true>)
+                     : (a.E <= 512 ? topk_kernel<16, false> : topk_kernel<32, false>);
     if (smem_t > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_t);
         if (e != cudaSuccess) return e;
     }
     const float depth = a.depth > 0.f ? a.depth : (float)(a.d / 32 + 6);
-    kern<<<(a.T + kTopkWarps - 1) / kTopkWarps, kTopkWarps * 32, smem_t, s>>>(
-        a.logits, static_cast<const __nv_bfloat16*>(a.x), a.T, a.d, a.E, a.k,
-        static_cast<const __nv_bfloat16*>(a.wr), a.bias, a.wnorm, depth, a.ids, a.w, a.meta);
+    const int grid = wide ? a.T : (a.T + kTopkWarps - 1) / kTopkWarps;
+    kern<<<grid, nw * 32, smem_t, s>>>(a.logits, static_cast<const __nv_bfloat16*>(a.x), a.T, a.d, a.E, a.k,
+                                      static_cast<const __nv_bfloat16*>(a.wr), a.bias, a.wnorm, depth, a.ids, a.w,
+                                      a.meta);
     return cudaGetLastError();
 }
 
