@@ -249,12 +249,20 @@ struct GemmArgs {
 //               acc_full[buffer]
 //   warps 8-11  epilogue: wait for a finished accumulator, tcgen05.ld, SwiGLU
 //               or weighting, fp16 stores; signal acc_empty[buffer]
+//
+// A pipeline step is kSK of K: 64 for gate/up (one SW128 atom; a step's codes
+// are half a 128-wide super-tile, so each super-tile is staged twice), 128
+// for down (two atoms side by side in A and in B; the whole super-tile once,
+// and half the steps, so half the per-step barriers, for the same K).
 template <int BITS, bool GATEUP>
 struct GemmCfg {
     static constexpr int kN = kExpertTileN;
-    static constexpr int kStages = GATEUP ? 3 : 4;
+    static constexpr int kSK = GATEUP ? 64 : 128;  // K per step
+    static constexpr int kAtoms = kSK / 64;         // SW128 atoms per row of a step's tile
+    static constexpr int kStages = GATEUP ? 3 : 2;
     static constexpr int kMats = GATEUP ? 2 : 1;
-    static constexpr int kA = kTileM * 128, kB = kN * 128;
+    static constexpr int kAtomA = kTileM * 128, kAtomB = kN * 128;  // one atom of A / of B
+    static constexpr int kA = kAtoms * kAtomA, kB = kAtoms * kAtomB;
     static constexpr int kCodeBytes = 8 * 256 * BITS;  // 8 row-tiles x one super-tile, in the A area
     static constexpr int kScaleBytes = 8 * 128;
     static_assert(kCodeBytes + kScaleBytes <= kA, "codes fit in the A area");
@@ -321,7 +329,7 @@ __global__ void __launch_bounds__(kExpertThreads, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     const int K = GATEUP ? a.d : a.f;  // contraction length
-    const int KS = K / kStepK;         // pipeline steps per tile
+    const int KS = K / C::kSK;         // pipeline steps per tile
 
     if (tid == 0) {
         for (int i = 0; i < C::kStages; ++i) {
@@ -350,40 +358,39 @@ __global__ void __launch_bounds__(kExpertThreads, 1)
         // ======================= dequant
         bool ok = true;
         const int rt = tid >> 5, ln = tid & 31, gg = ln >> 2, c = ln & 3;
+        constexpr int NKB = C::kSK / 32;  // 32-wide K blocks per step: 2 (half a super-tile) or 4
         for (int gs = 0; gs < total; ++gs) {
-            const int st = gs % C::kStages, hs = (gs % KS) & 1;
+            const int st = gs % C::kStages;
+            const int kbs = C::kSK == 64 ? 2 * ((gs % KS) & 1) : 0;  // first K block of the super-tile
             if (tid == 0 && ok) ok = tc::bar_wait(&load_bar[st], (gs / C::kStages) & 1, a.status);
             producer_sync();  // codes, scales and B rows of step gs have landed
             uint8_t* sb = smem + st * C::kStageBytes;
-            uint32_t lo[C::kMats][2], hi[C::kMats][2], sc[C::kMats][2];
+            uint32_t lo[C::kMats][NKB], hi[C::kMats][NKB], sc[C::kMats][NKB];
 #pragma unroll
             for (int m = 0; m < C::kMats; ++m) {
                 const uint8_t* cs = sb + m * C::kA + rt * (256 * BITS);
-                const uint2 w = *reinterpret_cast<const uint2*>(cs + 16 * ln + 8 * hs);
-                lo[m][0] = w.x;
-                lo[m][1] = w.y;
-                if (BITS == 3) {
-                    const uint32_t hv = *reinterpret_cast<const uint32_t*>(cs + 512 + 8 * ln + 4 * hs);
-                    hi[m][0] = hv & 0xFFFFu;
-                    hi[m][1] = hv >> 16;
-                } else if (BITS == 4) {
-                    const uint2 hv = *reinterpret_cast<const uint2*>(cs + 512 + 16 * ln + 8 * hs);
-                    hi[m][0] = hv.x;
-                    hi[m][1] = hv.y;
-                } else {
-                    hi[m][0] = hi[m][1] = 0;
+                const uint8_t* ss = sb + m * C::kA + C::kCodeBytes + rt * 128 + 16 * gg;
+#pragma unroll
+                for (int j = 0; j < NKB; ++j) {
+                    const int kb = kbs + j;
+                    lo[m][j] = *reinterpret_cast<const uint32_t*>(cs + 16 * ln + 4 * kb);
+                    if (BITS == 3) {
+                        const uint32_t hv = *reinterpret_cast<const uint32_t*>(cs + 512 + 8 * ln + 4 * (kb >> 1));
+                        hi[m][j] = (kb & 1) ? hv >> 16 : hv & 0xFFFFu;
+                    } else if (BITS == 4) {
+                        hi[m][j] = *reinterpret_cast<const uint32_t*>(cs + 512 + 16 * ln + 4 * kb);
+                    } else {
+                        hi[m][j] = 0;
+                    }
+                    sc[m][j] = *reinterpret_cast<const uint32_t*>(ss + 4 * kb);
                 }
-                const uint2 sv = *reinterpret_cast<const uint2*>(sb + m * C::kA + C::kCodeBytes + rt * 128 +
-                                                                 16 * gg + 8 * hs);
-                sc[m][0] = sv.x;
-                sc[m][1] = sv.y;
             }
             producer_sync();  // every read of the staged codes is done before A overwrites them
 #pragma unroll
             for (int m = 0; m < C::kMats; ++m) {
-                uint8_t* A = sb + m * C::kA;
 #pragma unroll
-                for (int kbl = 0; kbl < 2; ++kbl) {
+                for (int kbl = 0; kbl < NKB; ++kbl) {
+                    uint8_t* A = sb + m * C::kA + (kbl >> 1) * C::kAtomA;  // the block's atom
                     uint32_t q[8];
                     decode_block<true, BITS>(lo[m][kbl], hi[m][kbl], q);
                     const __half2 s_lo = __half2half2(__ushort_as_half((unsigned short)(sc[m][kbl] & 0xFFFFu)));
@@ -393,7 +400,7 @@ __global__ void __launch_bounds__(kExpertThreads, 1)
                         // pair p = 4 ks + 2 (m / 8) + r / 8 of the A-fragment layout
                         const int ks = p >> 2, hi8 = (p >> 1) & 1, half = p & 1;
                         const int r = rt * 16 + gg + 8 * half;
-                        const int kk = 32 * kbl + 16 * ks + 8 * hi8 + 2 * c;
+                        const int kk = 32 * (kbl & 1) + 16 * ks + 8 * hi8 + 2 * c;  // within the atom
                         const __half2 v = __hmul2(*reinterpret_cast<const __half2*>(&q[p]), half ? s_hi : s_lo);
                         *reinterpret_cast<__half2*>(A + tc::sw128(r, kk)) = v;
                     }
@@ -495,11 +502,12 @@ __global__ void __launch_bounds__(kExpertThreads, 1)
                     uint8_t* sb = smem + st * C::kStageBytes;
                     const uint32_t a_addr = smem_addr(sb), b_addr = smem_addr(sb + C::kMats * C::kA);
 #pragma unroll
-                    for (int kk = 0; kk < kStepK / 16; ++kk) {
-                        const uint64_t bd = tc::sdesc(b_addr + kk * 32);
+                    for (int kk = 0; kk < C::kSK / 16; ++kk) {
+                        const uint32_t ao = (kk >> 2) * C::kAtomA + (kk & 3) * 32;  // atom, then 16-wide K slice
+                        const uint64_t bd = tc::sdesc(b_addr + (kk >> 2) * C::kAtomB + (kk & 3) * 32);
                         const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-                        tc::mma(acc_addr, tc::sdesc(a_addr + kk * 32), bd, idesc, acc);
-                        if (GATEUP) tc::mma(acc_addr + C::kN, tc::sdesc(a_addr + C::kA + kk * 32), bd, idesc, acc);
+                        tc::mma(acc_addr, tc::sdesc(a_addr + ao), bd, idesc, acc);
+                        if (GATEUP) tc::mma(acc_addr + C::kN, tc::sdesc(a_addr + C::kA + ao), bd, idesc, acc);
                     }
                     tc::commit(&empty_bar[st]);
                 }
@@ -531,16 +539,20 @@ __global__ void __launch_bounds__(kExpertThreads, 1)
             uint8_t* Bs = sb + C::kMats * C::kA;
             const bool big = nmma > 2 * kBRowsSmall;
             const int nsmall = (nmma + kBRowsSmall - 1) / kBRowsSmall;
-            mbar_arrive_expect_tx(&load_bar[st],
-                                  C::kStageTxFixed + (uint32_t)(big ? kBRowsBig : nsmall * kBRowsSmall) * 128);
-            if (big) {
-                tma_load_2d(Bs, &bmap_b, s * kStepK, ds.y, &load_bar[st]);
-            } else {
-                for (int i = 0; i < nsmall; ++i)
-                    tma_load_2d(Bs + i * kBRowsSmall * 128, &bmap_s, s * kStepK, ds.y + i * kBRowsSmall,
-                                &load_bar[st]);
+            mbar_arrive_expect_tx(&load_bar[st], C::kStageTxFixed + (uint32_t)C::kAtoms *
+                                                                        (big ? kBRowsBig : nsmall * kBRowsSmall) * 128);
+#pragma unroll
+            for (int at = 0; at < C::kAtoms; ++at) {  // one 64-wide K atom of the B rows at a time
+                uint8_t* Ba = Bs + at * C::kAtomB;
+                const int kx = s * C::kSK + at * 64;
+                if (big) {
+                    tma_load_2d(Ba, &bmap_b, kx, ds.y, &load_bar[st]);
+                } else {
+                    for (int i = 0; i < nsmall; ++i)
+                        tma_load_2d(Ba + i * kBRowsSmall * 128, &bmap_s, kx, ds.y + i * kBRowsSmall, &load_bar[st]);
+                }
             }
-            const int expert = ds.x, jt = ds.z >> 16, kt = s >> 1;
+            const int expert = ds.x, jt = ds.z >> 16, kt = (s * C::kSK) / 128;  // the step's super-tile
 #pragma unroll
             for (int m = 0; m < C::kMats; ++m) {
                 uint8_t* A = sb + m * C::kA;
