@@ -7,7 +7,7 @@ These tests call it through the C ABI and compare each result with the
 handle-based moe_route on the same inputs, token by token on its CUDA-core
 router (at most 64 tokens per handle call): two calls in a row, the scratch's
 exact capacity (T * E = 65536), the widest expert count (E = 1024, whose top-k
-takes 64 KB of shared memory), and a call captured in a CUDA graph and
+takes 128 KB of shared memory at 64 tokens), and a call captured in a CUDA graph and
 replayed on new activations.  The file sorts last so
 that a run stopping at the first failure has already run everything else.
 """
