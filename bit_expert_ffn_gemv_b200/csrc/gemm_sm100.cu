@@ -118,7 +118,6 @@ MOE_DEV bool bar_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
 
 }  // namespace tc
 
-constexpr int kGemmThreads = 256;
 constexpr int kTileM = 128;  // weight rows per tile (the MMA's M)
 constexpr int kStepK = 64;   // K per pipeline step (one SW128 atom of 16-bit values)
 constexpr int kExpertTileN = 256;  // tokens per expert tile (at most; the MMA's N)
@@ -572,141 +571,178 @@ __global__ void __launch_bounds__(kExpertThreads, 1)
 
 // ---------------------------------------------------------------- router GEMM
 // logits[t][e] = W_r[e] . x_t + bias_e for 128-expert x 128-token tiles, bf16
-// operands copied straight into the SW128 tiles.  The contraction is split
-// into `chunks` consecutive K ranges, each accumulated in its own tensor-memory
-// columns; the epilogue adds the chunk sums in chunk order.  A chunk's rounding
-// error grows with its own length, so the logits' error bound is that many
-// times tighter than one running sum over all of d (router_gemm_depth).
-// split != 0 (small batches, whose few tiles would leave most SMs idle): every
-// (tile, chunk) is a work item of its own, and its raw chunk sums go to
-// logits[chunk][t][e]; the reader adds the chunks in chunk order, then the
-// bias -- the same operations, so the same logits, as the unsplit epilogue.
-constexpr int kRouterStages = 4;
+// operands loaded by TMA straight into the SW128 tiles.  The contraction is
+// split into `chunks` consecutive K ranges, each accumulated in its own
+// tensor-memory columns; the epilogue adds the chunk sums in chunk order.  A
+// chunk's rounding error grows with its own length, so the logits' error bound
+// is that many times tighter than one running sum over all of d
+// (router_gemm_depth).  split != 0 (small batches, whose few tiles would leave
+// most SMs idle): every (tile, chunk) is a work item of its own, and its raw
+// chunk sums go to logits[chunk][t][e]; the reader adds the chunks in chunk
+// order, then the bias -- the same operations, so the same logits, as the
+// unsplit epilogue.
+//
+// Warp roles (every role walks the same items blockIdx.x, + gridDim.x, ...):
+//   warp 0     loader (one thread): per K step, once the MMAs that last read
+//              the stage are done, one TMA box of router rows and one of x
+//              rows (rows past E or T read as zeros)
+//   warp 1     MMA issuer (one thread), after the epilogue has drained the
+//              previous item's accumulators
+//   warps 2-5  epilogue: tcgen05.ld of the chunk sums, in chunk order, then
+//              the bias; fp32 stores
+constexpr int kRouterStages = 6;
 constexpr int kRouterStage = kTileM * 128 + kRouterTileN * 128;
+constexpr int kRouterThreads = 6 * 32;
 
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    router_gemm_kernel(const uint16_t* __restrict__ x, int T, int d, const uint16_t* __restrict__ wr,
-                       const float* __restrict__ bias, int E, float* __restrict__ logits, int chunks, int split,
+__global__ void __launch_bounds__(kRouterThreads, 1)
+    router_gemm_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap xmap, int T,
+                       int d, const float* __restrict__ bias, int E, float* __restrict__ logits, int chunks, int split,
                        uint32_t* status) {
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t mma_bar[kRouterStages];
+    __shared__ __align__(8) uint64_t full_bar[kRouterStages], empty_bar[kRouterStages], accf_bar, acce_bar,
+        drain_bar;
     __shared__ uint32_t tmem_slot;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
     const int KS = d / kStepK;
     const int MT = (E + kTileM - 1) / kTileM, NT = (T + kRouterTileN - 1) / kRouterTileN;
     if (tid == 0) {
-        for (int i = 0; i < kRouterStages; ++i) mbar_init(&mma_bar[i], 1);
+        for (int i = 0; i < kRouterStages; ++i) {
+            mbar_init(&full_bar[i], 1);
+            mbar_init(&empty_bar[i], 1);
+        }
+        mbar_init(&accf_bar, 1);
+        mbar_init(&acce_bar, 128);
+        mbar_init(&drain_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) tc::tmem_alloc(&tmem_slot, 512);
+    if (warp == 1) tc::tmem_alloc(&tmem_slot, 512);
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = tmem_slot;
-    const int csteps = KS / chunks;          // K steps per chunk
-    const uint32_t ccols = 512u / chunks;    // tensor-memory columns per chunk (>= the tile's width)
-    uint32_t gstep = 0;
-    bool ok = true, all_ok = true;
+    const int csteps = KS / chunks;        // K steps per chunk
+    const uint32_t ccols = 512u / chunks;  // tensor-memory columns per chunk (>= the tile's width)
     const int items = MT * NT * (split ? chunks : 1);
-    for (int item = blockIdx.x; item < items && all_ok; item += gridDim.x) {
-        const int tile = item % (MT * NT), ich = item / (MT * NT);  // ich: the item's chunk (split)
-        const int mt = tile % MT, nt = tile / MT;
-        const int e0 = mt * kTileM, t0 = nt * kRouterTileN;
-        const int s0 = split ? ich * csteps : 0, ns = split ? csteps : KS;  // the item's K steps
-        const int n = min(kRouterTileN, T - t0), nmma = (n + 15) & ~15;
-        const uint32_t idesc = tc::idesc_f16(kTileM, nmma, true);
-        auto load_step = [&](int s, int st) {
-            uint8_t* As = smem + st * kRouterStage;
-            uint8_t* Bs = As + kTileM * 128;
-            for (int v = tid; v < kTileM * 8; v += kGemmThreads) {
-                const int r = v >> 3, c = v & 7;
-                const int e = min(e0 + r, E - 1);
-                tc::cp16(As + tc::sw128_chunk(r, c), wr + (int64_t)e * d + s * kStepK + c * 8);
-            }
-            for (int v = tid; v < nmma * 8; v += kGemmThreads) {
-                const int r = v >> 3, c = v & 7;
-                const int t = t0 + min(r, n - 1);
-                tc::cp16(Bs + tc::sw128_chunk(r, c), x + (int64_t)t * d + s * kStepK + c * 8);
-            }
-        };
-        const int P = kRouterStages - 1;
-        for (int s = 0; s < P; ++s) {
-            if (s < ns) load_step(s0 + s, (gstep + s) % kRouterStages);
-            tc::cp_commit();
-        }
-        for (int s = 0; s < ns; ++s) {
-            const uint32_t cur = gstep + s;
-            const int st = cur % kRouterStages;
-            tc::cp_wait<kRouterStages - 2>();
-            fence_proxy_async_smem();
-            if (s + P < ns) {
-                if (cur >= 1 && ok) {
-                    const uint32_t prev = cur - 1;
-                    ok = tc::bar_wait(&mma_bar[prev % kRouterStages], (prev / kRouterStages) & 1, status);
+    const int bid = (int)blockIdx.x, grid = (int)gridDim.x;
+    // item -> tile (mt, nt) and its K steps [s0, s0 + ns); ich: its chunk when split
+    auto item_of = [&](int item, int& mt, int& nt, int& ich, int& s0, int& ns) {
+        const int tile = item % (MT * NT);
+        ich = item / (MT * NT);
+        mt = tile % MT;
+        nt = tile / MT;
+        s0 = split ? ich * csteps : 0;
+        ns = split ? csteps : KS;
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ======================= loader
+            bool ok = true;
+            int j = 0;  // K steps issued
+            for (int item = bid; item < items && ok; item += grid) {
+                int mt, nt, ich, s0, ns;
+                item_of(item, mt, nt, ich, s0, ns);
+                for (int s = 0; s < ns; ++s, ++j) {
+                    const int st = j % kRouterStages;
+                    if (j >= kRouterStages)  // the MMAs of step j - S have read the stage
+                        ok = tc::bar_wait(&empty_bar[st], ((j / kRouterStages) - 1) & 1, status);
+                    if (!ok) break;
+                    uint8_t* As = smem + st * kRouterStage;
+                    mbar_arrive_expect_tx(&full_bar[st], (uint32_t)kRouterStage);
+                    tma_load_2d(As, &wmap, (s0 + s) * kStepK, mt * kTileM, &full_bar[st]);
+                    tma_load_2d(As + kTileM * 128, &xmap, (s0 + s) * kStepK, nt * kRouterTileN, &full_bar[st]);
                 }
-                load_step(s0 + s + P, (cur + P) % kRouterStages);
             }
-            tc::cp_commit();
-            __syncthreads();
-            if (tid == 0) {
+            // no copy may still be landing in shared memory when the CTA leaves
+            for (int jj = j > kRouterStages ? j - kRouterStages : 0; jj < j; ++jj)
+                tc::bar_wait(&full_bar[jj % kRouterStages], (jj / kRouterStages) & 1, status);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ======================= MMA issuer
+            bool ok = true;
+            int j = 0, it = 0;
+            for (int item = bid; item < items && ok; item += grid, ++it) {
+                int mt, nt, ich, s0, ns;
+                item_of(item, mt, nt, ich, s0, ns);
+                const int n = min(kRouterTileN, T - nt * kRouterTileN), nmma = (n + 15) & ~15;
+                const uint32_t idesc = tc::idesc_f16(kTileM, nmma, true);
+                if (it > 0) ok = tc::bar_wait(&acce_bar, (it - 1) & 1, status);  // accumulators drained
+                if (!ok) break;
                 tc::fence_after();
-                const uint32_t a_addr = smem_addr(smem + st * kRouterStage), b_addr = a_addr + kTileM * 128;
-                const int ch = split ? 0 : s / csteps;  // this step's accumulator
+                for (int s = 0; s < ns && ok; ++s, ++j) {
+                    const int st = j % kRouterStages;
+                    ok = tc::bar_wait(&full_bar[st], (j / kRouterStages) & 1, status);
+                    if (!ok) break;
+                    tc::fence_after();
+                    const uint32_t a_addr = smem_addr(smem + st * kRouterStage), b_addr = a_addr + kTileM * 128;
+                    const int ch = split ? 0 : s / csteps;  // this step's accumulator
 #pragma unroll
-                for (int kk = 0; kk < kStepK / 16; ++kk)
-                    tc::mma(tmem + ch * ccols, tc::sdesc(a_addr + kk * 32), tc::sdesc(b_addr + kk * 32), idesc,
-                            (s > ch * csteps || kk > 0) ? 1u : 0u);
-                tc::commit(&mma_bar[st]);
+                    for (int kk = 0; kk < kStepK / 16; ++kk)
+                        tc::mma(tmem + ch * ccols, tc::sdesc(a_addr + kk * 32), tc::sdesc(b_addr + kk * 32), idesc,
+                                (s > ch * csteps || kk > 0) ? 1u : 0u);
+                    tc::commit(&empty_bar[st]);
+                }
+                if (!ok) break;
+                tc::commit(&accf_bar);
             }
+            // every MMA issued has finished before tensor memory is released
+            tc::commit(&drain_bar);
+            tc::bar_wait(&drain_bar, 0, status);
         }
-        if (ok) {
-            const uint32_t last = gstep + ns - 1;
-            ok = tc::bar_wait(&mma_bar[last % kRouterStages], (last / kRouterStages) & 1, status);
-        }
-        gstep += ns;
-        all_ok = __syncthreads_and(ok) != 0;
-        tc::fence_after();
-        const int e = e0 + 32 * (warp & 3) + lane;
-        const float b = (bias && e < E) ? bias[e] : 0.0f;
-        for (int c0 = 16 * (warp >> 2); c0 < nmma && all_ok && split; c0 += 32) {
-            // the item's raw chunk sums
-            uint32_t r0[16];
-            tc::ld16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c0, r0);
-            float* lp = logits + (int64_t)ich * T * E;
+    } else {
+        // ======================= epilogue: warp w reads TMEM lanes 32 (w % 4) ..
+        const int q = warp & 3;
+        bool ok = true;
+        int it = 0;
+        for (int item = bid; item < items && ok; item += grid, ++it) {
+            int mt, nt, ich, s0, ns;
+            item_of(item, mt, nt, ich, s0, ns);
+            const int t0 = nt * kRouterTileN, n = min(kRouterTileN, T - t0), nmma = (n + 15) & ~15;
+            ok = warp_wait(&accf_bar, it & 1, status);
+            if (!ok) break;
+            tc::fence_after();
+            const int e = mt * kTileM + 32 * q + lane;
+            const float b = (bias && e < E) ? bias[e] : 0.0f;
+            const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
+            for (int c0 = 0; c0 < nmma; c0 += 16) {
+                float v[16];
+                if (split) {  // the item's raw chunk sums
+                    uint32_t r0[16];
+                    tc::ld16(tl + c0, r0);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (c0 + i < n && e < E) lp[(int64_t)(t0 + c0 + i) * E + e] = __uint_as_float(r0[i]);
-        }
-        for (int c0 = 16 * (warp >> 2); c0 < nmma && all_ok && !split; c0 += 32) {
-            const uint32_t ta = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c0;
-            float v[16];
-            for (int ch0 = 0; ch0 < chunks; ch0 += 4) {  // chunk sums in chunk order, 4 loads in flight
-                uint32_t r[4][16];
-                const int nc = min(4, chunks - ch0);
+                    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r0[i]);
+                } else {
+                    for (int ch0 = 0; ch0 < chunks; ch0 += 4) {  // chunk sums in chunk order, 4 loads in flight
+                        uint32_t r[4][16];
+                        const int nc = min(4, chunks - ch0);
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (j < nc) tc::ld16_nowait(ta + (ch0 + j) * ccols, r[j]);
-                tc::ld_wait();
+                        for (int jj = 0; jj < 4; ++jj)
+                            if (jj < nc) tc::ld16_nowait(tl + (ch0 + jj) * ccols + c0, r[jj]);
+                        tc::ld_wait();
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    if (j < nc) {
+                        for (int jj = 0; jj < 4; ++jj)
+                            if (jj < nc) {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            v[i] = (ch0 + j == 0) ? __uint_as_float(r[j][i]) : v[i] + __uint_as_float(r[j][i]);
+                                for (int i = 0; i < 16; ++i)
+                                    v[i] = (ch0 + jj == 0) ? __uint_as_float(r[jj][i]) : v[i] + __uint_as_float(r[jj][i]);
+                            }
                     }
-            }
+                }
+                float* lp = split ? logits + (int64_t)ich * T * E : logits;
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                if (c0 + i < n && e < E) logits[(int64_t)(t0 + c0 + i) * E + e] = v[i] + b;
+                for (int i = 0; i < 16; ++i)
+                    if (c0 + i < n && e < E) lp[(int64_t)(t0 + c0 + i) * E + e] = split ? v[i] : v[i] + b;
+            }
+            tc::fence_before();
+            mbar_arrive(&acce_bar);
         }
-        tc::fence_before();
-        __syncthreads();
     }
-    tc::cp_wait<0>();
     tc::fence_before();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, 512);
+    tc::fence_after();
+    if (warp == 1) tc::tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------- activation gather, combine
@@ -973,13 +1009,19 @@ cudaError_t launch_router_gemm(const RouteArgs& a, uint32_t* status, cudaStream_
     const int smem = kRouterStages * kRouterStage + 1024;
     cudaError_t e = cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    // row-major bf16 [E x d] and [T x d], boxes of 64 columns (128 B) x 128 rows, 128-byte swizzle
+    CUtensorMap wmap, xmap;
+    e = encode_2d(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.wr, a.E, a.d, 64, kTileM, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
+    e = encode_2d(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.x, a.T, a.d, 64, kRouterTileN,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess) return e;
     const int tiles = ((a.E + kTileM - 1) / kTileM) * ((a.T + kRouterTileN - 1) / kRouterTileN);
     const int chunks = router_gemm_chunks(a.T, a.d), split = router_gemm_split(a.T) ? 1 : 0;
     if (split && a.logit_parts != chunks) return cudaErrorInvalidValue;  // the caller sized logits for the chunks
     const int items = tiles * (split ? chunks : 1);
-    router_gemm_kernel<<<min(items, num_sms()), kGemmThreads, smem, s>>>(
-        static_cast<const uint16_t*>(a.x), a.T, a.d, static_cast<const uint16_t*>(a.wr), a.bias, a.E, a.logits,
-        chunks, split, status);
+    router_gemm_kernel<<<min(items, num_sms()), kRouterThreads, smem, s>>>(wmap, xmap, a.T, a.d, a.bias, a.E,
+                                                                          a.logits, chunks, split, status);
     return cudaGetLastError();
 }
 
