@@ -57,8 +57,34 @@ def parse():
 
 
 # ---------------------------------------------------------------- ncu traffic of the dominant kernel
-_KERNEL_SOURCE = {"gemm_gateup": "gemm_sm100.cu", "gemm_down": "gemm_sm100.cu", "router_gemm": "gemm_sm100.cu",
-                  "decode_fused": "decode_pair.cu", "gemv_gateup": "gemv.cu", "gemv_down": "gemv.cu"}
+# kernel -> (source file, first line of its section or None for the whole file, first line after it)
+_SEC = "// ---------------------------------------------------------------- "
+_KERNEL_SOURCE = {"gemm_gateup": ("gemm_sm100.cu", _SEC + "grouped expert GEMM", _SEC + "router GEMM"),
+                  "gemm_down": ("gemm_sm100.cu", _SEC + "grouped expert GEMM", _SEC + "router GEMM"),
+                  "router_gemm": ("gemm_sm100.cu", _SEC + "router GEMM", _SEC + "activation gather, combine"),
+                  "decode_fused": ("decode_pair.cu", None, None), "gemv_gateup": ("gemv.cu", None, None),
+                  "gemv_down": ("gemv.cu", None, None)}
+
+
+def kernel_source_hash(kernel: str):
+    """First 16 hex digits of the sha256 of the kernel's source section (its file when it has none)."""
+    import hashlib
+    src = _KERNEL_SOURCE.get(kernel)
+    if not src:
+        return None
+    path = os.path.join(ROOT, "bit_expert_ffn_gemv_b200", "csrc", src[0])
+    try:
+        text = open(path, "rb").read()
+    except OSError:
+        return None
+    if src[1] is not None:
+        a, b = src[1].encode(), src[2].encode()
+        i = text.find(a)
+        j = text.find(b, i + 1) if i >= 0 else -1
+        if i < 0 or j < 0:
+            return None
+        text = text[i:j]
+    return hashlib.sha256(text).hexdigest()[:16]
 
 
 def profile_traffic(kernel: str, tokens=None):
@@ -66,14 +92,8 @@ def profile_traffic(kernel: str, tokens=None):
     `traffic: kernel=K source_sha256_16=H tokens=T dram_bytes_per_launch=B`), or None when no capture of
     this workload size exists or the kernel's source changed since it was taken."""
     import glob
-    import hashlib
-    src = _KERNEL_SOURCE.get(kernel)
-    if not src:
-        return None
-    path = os.path.join(ROOT, "bit_expert_ffn_gemv_b200", "csrc", src)
-    try:
-        cur = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
-    except OSError:
+    cur = kernel_source_hash(kernel)
+    if cur is None:
         return None
     for f in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
         for line in open(f):
