@@ -748,22 +748,23 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
 // ---------------------------------------------------------------- activation gather, combine
 // xg[row] = fp16(x[token of row]) in group order: rows [0, offsets[E]) are
 // the routed pairs (token pairs[row] / k), rows T*k + t the shared expert's.
-// One warp per row (32 lanes x 16 bytes per step), kGatherRowsPerCta rows per
-// CTA, so the grid is a few thousand CTAs that each stream whole rows.
+// One warp per RPW rows (32 lanes x 16 bytes per step, eight steps in flight),
+// 8 warps per CTA: RPW = 4 for large batches (a few thousand CTAs that each
+// stream whole rows), 1 for small ones (more warps, each one round of loads).
 constexpr int kGatherWarps = 8;
-constexpr int kGatherRowsPerWarp = 4;
-constexpr int kGatherRowsPerCta = kGatherWarps * kGatherRowsPerWarp;
+constexpr int kGatherSmallRows = 148 * kGatherWarps * 16;  // below this many rows: one row per warp
 
+template <int RPW>
 __global__ void __launch_bounds__(kGatherWarps * 32)
     gather_f16_kernel(const __nv_bfloat16* __restrict__ x, int T, int d, int k, int n_shared,
                       const int32_t* __restrict__ pairs, const int32_t* __restrict__ n_pairs,
                       __half* __restrict__ xg, uint32_t* status) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rows = T * k + n_shared * T, np = *n_pairs;
-    const int r0 = (blockIdx.x * kGatherWarps + warp) * kGatherRowsPerWarp;
-    int tok[kGatherRowsPerWarp];
+    const int r0 = (blockIdx.x * kGatherWarps + warp) * RPW;
+    int tok[RPW];
 #pragma unroll
-    for (int i = 0; i < kGatherRowsPerWarp; ++i) {
+    for (int i = 0; i < RPW; ++i) {
         const int row = r0 + i;
         tok[i] = -1;
         if (row < T * k) {
@@ -774,10 +775,11 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
     }
     bool finite = true;
 #pragma unroll
-    for (int i = 0; i < kGatherRowsPerWarp; ++i) {
+    for (int i = 0; i < RPW; ++i) {
         if (tok[i] < 0) continue;
         const __nv_bfloat16* src = x + (int64_t)tok[i] * d;
         __half* dst = xg + (int64_t)(r0 + i) * d;
+#pragma unroll 8
         for (int c = lane * 8; c < d; c += 256) {
             const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + c));
             const uint32_t in[4] = {v.x, v.y, v.z, v.w};
@@ -812,9 +814,25 @@ __global__ void combine_f16_kernel(const CombineArgs a, const __half* __restrict
         }
     };
     if (a.n_shared) add_row((int64_t)a.T * a.k + t);
-    for (int r = 0; r < a.k; ++r) {
-        const int pos = a.inv[(int64_t)t * a.k + r];
-        if (pos >= 0) add_row(pos);
+    for (int r0 = 0; r0 < a.k; r0 += 4) {  // slots in order, four positions and rows in flight
+        int pos[4];
+        uint4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) pos[j] = r0 + j < a.k ? a.inv[(int64_t)t * a.k + r0 + j] : -1;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (pos[j] >= 0) v[j] = *reinterpret_cast<const uint4*>(o + (int64_t)pos[j] * a.d + n);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (pos[j] >= 0) {
+                const __half2* h2 = reinterpret_cast<const __half2*>(&v[j]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 f = __half22float2(h2[q]);
+                    acc[2 * q] += f.x;
+                    acc[2 * q + 1] += f.y;
+                }
+            }
     }
     if (a.out_fp32) {
         float* y = static_cast<float*>(a.y) + (int64_t)t * a.d + n;
@@ -1075,8 +1093,13 @@ float router_gemm_depth(int d, int chunks) {
 cudaError_t launch_gather_f16(const void* x, int T, int d, int k, int n_shared, const int32_t* pairs,
                               const int32_t* n_pairs, void* xg, uint32_t* status, cudaStream_t s) {
     const int rows = T * k + n_shared * T;
-    gather_f16_kernel<<<(rows + kGatherRowsPerCta - 1) / kGatherRowsPerCta, kGatherWarps * 32, 0, s>>>(static_cast<const __nv_bfloat16*>(x), T, d, k, n_shared, pairs, n_pairs,
-                                          static_cast<__half*>(xg), status);
+    const auto* xb = static_cast<const __nv_bfloat16*>(x);
+    if (rows < kGatherSmallRows)
+        gather_f16_kernel<1><<<(rows + kGatherWarps - 1) / kGatherWarps, kGatherWarps * 32, 0, s>>>(
+            xb, T, d, k, n_shared, pairs, n_pairs, static_cast<__half*>(xg), status);
+    else
+        gather_f16_kernel<4><<<(rows + 4 * kGatherWarps - 1) / (4 * kGatherWarps), kGatherWarps * 32, 0, s>>>(
+            xb, T, d, k, n_shared, pairs, n_pairs, static_cast<__half*>(xg), status);
     return cudaGetLastError();
 }
 
