@@ -312,6 +312,16 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
     ba.skip_rank = skip_rank(c, flags);
     ba.e_begin = h->ep_begin;
     ba.e_end = h->ep_end;
+    // the single-CTA bucketing also builds the tensor-core path's tile list (one launch fewer)
+    const bool tiles_in_bucket = tc && moe::bucket_builds_tiles(ba);
+    if (tiles_in_bucket) {
+        ba.desc_gu = h->desc_gu;
+        ba.desc_dn = h->desc_dn;
+        ba.tile_counts = h->n_tiles;
+        ba.n_shared = eff_shared(h);
+        ba.jt_gateup = c.f / 128;
+        ba.jt_down = c.d / 128;
+    }
     e = run(h, MOE_K_BUCKET, s, [&] { return moe::launch_bucket(ba, s); });
     h->launches += moe::bucket_kernel_count(ba) - 1;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -343,9 +353,11 @@ moe_status do_forward(moe_handle* h, int32_t layer, const void* x, int32_t T, vo
                                           h->status, s);
         });
         if (e != cudaSuccess) return MOE_ERR_CUDA;
-        e = run(h, MOE_K_TILE_LIST, s,
-                [&] { return moe::launch_build_tiles(ea, h->desc_gu, h->desc_dn, h->n_tiles, s); });
-        if (e != cudaSuccess) return MOE_ERR_CUDA;
+        if (!tiles_in_bucket) {
+            e = run(h, MOE_K_TILE_LIST, s,
+                    [&] { return moe::launch_build_tiles(ea, h->desc_gu, h->desc_dn, h->n_tiles, s); });
+            if (e != cudaSuccess) return MOE_ERR_CUDA;
+        }
         e = run(h, MOE_K_GEMM_GATEUP, s,
                 [&] {
                     moe::GemmMaps m = h->gu_maps;

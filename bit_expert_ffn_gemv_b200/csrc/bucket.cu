@@ -9,10 +9,12 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tiles.cuh"
 
 namespace moe {
 
 constexpr int kBucketWarps = 32;
+static_assert(kBucketWarps * 32 == kTileListThreads, "the bucketing CTA can build the tile list");
 int bucket_kernel_count(const BucketArgs& a);
 
 // Warp w owns the contiguous range of pair indices p = t*k + r in
@@ -22,8 +24,11 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
     bucket_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int32_t* __restrict__ offsets,
                   int32_t* __restrict__ pairs, int32_t* __restrict__ inv, int32_t* __restrict__ active,
                   Meta* __restrict__ meta, uint32_t* __restrict__ status, const float* __restrict__ w,
-                  float* __restrict__ wsorted, int R, int e0, int e1) {
+                  float* __restrict__ wsorted, int R, int e0, int e1, int4* __restrict__ desc_gu,
+                  int4* __restrict__ desc_dn, int32_t* __restrict__ tile_counts, int n_shared, int jt_gateup,
+                  int jt_down) {
     extern __shared__ int32_t sm[];
+    __shared__ int s_nact;
     int32_t* cnt = sm;                          // [kBucketWarps][E]
     int32_t* total = sm + kBucketWarps * E;     // [E]
     int32_t* off_s = total + E;                 // [E + 1]
@@ -99,6 +104,7 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
             off_s[E] = base;
             meta->n_active = nact;
             meta->max_count = mx;
+            s_nact = nact;
         }
     }
     __syncthreads();
@@ -137,6 +143,14 @@ __global__ void __launch_bounds__(kBucketWarps * 32)
                 inv[p] = -1;
             }
         }
+    }
+
+    // the expert GEMMs' tile list from the groups (active was written by warp 0
+    // before the barrier above; the builder synchronises the CTA first)
+    if (desc_gu) {
+        __shared__ TileListSmem tl;
+        build_tile_list(T, k, E, n_shared, s_nact, off_s, active, jt_gateup, jt_down, desc_gu, desc_dn, tile_counts,
+                        tl);
     }
 }
 
@@ -351,8 +365,10 @@ cudaError_t launch_bucket(const BucketArgs& a, cudaStream_t s) {
         cudaError_t e = cudaFuncSetAttribute(bucket_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
+    if (a.desc_gu && a.n_shared + a.E > kTileMaxSlots) return cudaErrorInvalidValue;
     bucket_kernel<<<1, kBucketWarps * 32, smem, s>>>(a.ids, a.T, a.k, a.E, a.offsets, a.pairs, a.inv, a.active,
-                                                     a.meta, a.status, a.w, a.wsorted, R, e0, e1);
+                                                     a.meta, a.status, a.w, a.wsorted, R, e0, e1, a.desc_gu,
+                                                     a.desc_dn, a.tile_counts, a.n_shared, a.jt_gateup, a.jt_down);
     return cudaGetLastError();
 }
 
@@ -361,4 +377,5 @@ cudaError_t launch_bucket(const BucketArgs& a, cudaStream_t s) {
 namespace moe {
 size_t bucket_scratch_words(int E) { return 2 * (size_t)kChunks * E; }
 int bucket_kernel_count(const BucketArgs& a) { return (a.cnt && a.T * a.k >= 8192) ? 3 : 1; }
+bool bucket_builds_tiles(const BucketArgs& a) { return bucket_kernel_count(a) == 1; }
 }  // namespace moe

@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tiles.cuh"
 
 namespace moe {
 namespace tc {
@@ -120,22 +121,10 @@ MOE_DEV bool bar_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
 
 constexpr int kTileM = 128;  // weight rows per tile (the MMA's M)
 constexpr int kStepK = 64;   // K per pipeline step (one SW128 atom of 16-bit values)
-constexpr int kExpertTileN = 256;  // tokens per expert tile (at most; the MMA's N)
 constexpr int kRouterTileN = 128;  // tokens per router tile
 
 // ---------------------------------------------------------------- tile list
-// Slots: the shared expert (if any), then the active routed experts in
-// ascending order.  A slot with c tokens holds ceil(c / kExpertTileN) token
-// tiles; token tile q of the layer times the JT row-tiles of a weight gives
-// tiles q * JT .. q * JT + JT - 1, so CTAs that take consecutive tiles read
-// the same activation rows.  One descriptor per tile:
-//   x = expert (E for the shared one), y = row0 (h / partial-output row of
-//   the tile's first token = its first pair position), z = n | jt << 16,
-//   w = first token for the shared expert, -1 for a routed one (whose rows'
-//   tokens are pairs[row0 + r] / k).
-constexpr int kTileListThreads = 1024;
-constexpr int kMaxSlots = 1024 + 1;
-
+// (tiles.cuh: the slots, token tiles and descriptors)
 static inline int max_token_tiles(int T, int k, int E, int n_shared) {
     return (T * k + kExpertTileN - 1) / kExpertTileN + E + n_shared * ((T + kExpertTileN - 1) / kExpertTileN) + 1;
 }
@@ -143,81 +132,9 @@ static inline int max_token_tiles(int T, int k, int E, int n_shared) {
 __global__ void __launch_bounds__(kTileListThreads)
     build_tiles_kernel(const ExpertArgs a, int jt_gateup, int jt_down, int4* __restrict__ desc_gu,
                        int4* __restrict__ desc_dn, int32_t* __restrict__ counts) {
-    __shared__ int pre[kMaxSlots + 1];
-    __shared__ int wsum[kTileListThreads / 32];
-    __shared__ int carry_s;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n_slots = a.n_shared + a.meta->n_active;
-    if (tid == 0) carry_s = 0;
-    __syncthreads();
-    for (int base = 0; base < n_slots; base += kTileListThreads) {
-        const int s = base + tid;
-        int tt = 0;
-        if (s < n_slots) {
-            int count;
-            if (s < a.n_shared) count = a.T;
-            else {
-                const int e = a.active[s - a.n_shared];
-                count = a.offsets[e + 1] - a.offsets[e];
-            }
-            tt = (count + kExpertTileN - 1) / kExpertTileN;
-        }
-        int inc = tt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += v;
-        }
-        if (lane == 31) wsum[warp] = inc;
-        __syncthreads();
-        if (warp == 0) {
-            int v = wsum[lane];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int u = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += u;
-            }
-            wsum[lane] = v;  // inclusive over warps
-        }
-        __syncthreads();
-        const int carry = carry_s;
-        if (s < n_slots) pre[s] = carry + (warp ? wsum[warp - 1] : 0) + inc - tt;
-        __syncthreads();
-        if (tid == 0) carry_s = carry + wsum[kTileListThreads / 32 - 1];
-        __syncthreads();
-    }
-    const int total_tt = carry_s;
-    if (tid == 0) {
-        pre[n_slots] = total_tt;
-        counts[0] = total_tt * jt_gateup;
-        counts[1] = total_tt * jt_down;
-    }
-    __syncthreads();
-    for (int q = tid; q < total_tt; q += kTileListThreads) {
-        int lo = 0, hi = n_slots - 1;  // last slot with pre[s] <= q
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (pre[mid] <= q) lo = mid;
-            else hi = mid - 1;
-        }
-        const int tt = q - pre[lo];
-        int expert, row0, count, tok0;
-        if (lo < a.n_shared) {
-            expert = a.E;
-            count = a.T;
-            row0 = a.T * a.k + tt * kExpertTileN;
-            tok0 = tt * kExpertTileN;
-        } else {
-            expert = a.active[lo - a.n_shared];
-            const int p0 = a.offsets[expert];
-            count = a.offsets[expert + 1] - p0;
-            row0 = p0 + tt * kExpertTileN;
-            tok0 = -1;
-        }
-        const int n = min(kExpertTileN, count - tt * kExpertTileN);
-        for (int jt = 0; jt < jt_gateup; ++jt) desc_gu[q * jt_gateup + jt] = make_int4(expert, row0, n | (jt << 16), tok0);
-        for (int jt = 0; jt < jt_down; ++jt) desc_dn[q * jt_down + jt] = make_int4(expert, row0, n | (jt << 16), tok0);
-    }
+    __shared__ TileListSmem sm;
+    build_tile_list(a.T, a.k, a.E, a.n_shared, a.meta->n_active, a.offsets, a.active, jt_gateup, jt_down, desc_gu,
+                    desc_dn, counts, sm);
 }
 
 struct GemmArgs {
@@ -878,7 +795,7 @@ size_t tile_desc_count(int T, int k, int E, int n_shared, int jt) {
 }
 
 cudaError_t launch_build_tiles(const ExpertArgs& a, int4* desc_gu, int4* desc_dn, int32_t* counts, cudaStream_t s) {
-    if (a.n_shared + a.E > kMaxSlots) return cudaErrorInvalidValue;
+    if (a.n_shared + a.E > kTileMaxSlots) return cudaErrorInvalidValue;
     build_tiles_kernel<<<1, kTileListThreads, 0, s>>>(a, a.f / kTileM, a.d / kTileM, desc_gu, desc_dn, counts);
     return cudaGetLastError();
 }

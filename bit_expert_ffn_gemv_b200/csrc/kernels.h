@@ -37,9 +37,15 @@ struct BucketArgs {
     int32_t* cnt = nullptr;    // scratch [2 x 128 x E] for the multi-CTA variant (large T), or null
     int skip_rank = 0;         // route-tail skip: drop experts whose best rank in the batch is >= this (0: off)
     int e_begin = 0, e_end = 1 << 30;  // experts outside [e_begin, e_end) are dropped (expert parallelism)
+    // the expert GEMMs' tile list, built at the end of the single-CTA variant (desc_gu null: not built)
+    int4* desc_gu = nullptr;
+    int4* desc_dn = nullptr;
+    int32_t* tile_counts = nullptr;
+    int n_shared = 0, jt_gateup = 0, jt_down = 0;
 };
 size_t bucket_scratch_words(int E);
 int bucket_kernel_count(const BucketArgs& a);  // kernels launch_bucket enqueues: 1, or 3 at large T
+bool bucket_builds_tiles(const BucketArgs& a);  // the single-CTA variant, which can build the tile list
 
 // Grouped GEMV/GEMM problem description shared by the expert kernels.
 struct ExpertArgs {
