@@ -90,3 +90,22 @@ def test_noalloc_route_rejects_bad_arguments_before_touching_the_gpu(L, bad):
     a.update(bad)
     s = L.moe_route_noalloc(a["x"], a["T"], a["d"], a["E"], a["k"], a["wr"], a["bias"], a["ids"], a["w"], None)
     assert s == 1  # MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("d,T,expect", [
+    # split router GEMM (T <= 128): one K chunk per 64-wide step, at most 32 chunks
+    (2048, 1, 34 * (2048 // 16 // 32) + 31 + 2), (2048, 16, 169.0), (2048, 64, 169.0), (2048, 128, 169.0),
+    # 128-token tiles: four chunks fill the 512 tensor-memory columns
+    (2048, 129, 34 * (2048 // 16 // 4) + 3 + 2), (2048, 8192, 1093.0), (2048, 0, 1093.0),
+    # few K steps cap the chunk count (a power of two dividing d / 64)
+    (128, 16, 34 * (128 // 16 // 2) + 1 + 2), (384, 16, 34 * (384 // 16 // 2) + 1 + 2),
+    (384, 8192, 34 * (384 // 16 // 2) + 1 + 2), (256, 8192, 34 * (256 // 16 // 4) + 3 + 2),
+])
+def test_router_error_depth_follows_the_chunk_count(L, d, T, expect):
+    """The tensor-core logits' depth is 34 per 16-wide step of one K chunk, plus one per chunk add and
+    two for the bias: the chunk count is what the GEMM uses at that batch size (host logic only)."""
+    import bit_expert_ffn_gemv_b200 as moe
+    assert moe.moe_router_error_depth(d, True, T) == pytest.approx(expect)
+    assert moe.moe_router_error_depth(d, True, T) <= moe.moe_router_error_depth(d, True)
+    assert moe.moe_router_error_depth(d, False, T) == pytest.approx(d // 32 + 6)
+    assert moe.moe_router_error_depth(0, True, T) == 0.0
