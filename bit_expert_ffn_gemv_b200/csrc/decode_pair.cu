@@ -386,8 +386,8 @@ MOE_DEV void topk_scan(const double* lg, int E, int k, int lane, int& sel, doubl
 // adjacent prefixes differ; where two selected keys share a prefix the k
 // entries are ranked again by (fp64 logit desc, index asc).  A tie of the
 // k-th and (k+1)-th prefixes (rare: equal fp32 images) takes the exact
-// scan.  Lane r < k returns id r and its weight w_r = softmax over the k
-// selected logits.
+// scan.  Lane r < k returns id r and l_r - l_0 (its logit less the top one),
+// from which w_r = softmax over the k selected logits is finished later.
 template <int KPL>
 MOE_DEV void topk_token(const double* lg, int E, int k, int lane, Cand* cand, int& id_out, float& w_out) {
     unsigned long long tc = cyc();
@@ -468,14 +468,10 @@ MOE_DEV void topk_token(const double* lg, int E, int k, int lane, Cand* cand, in
         cyc_add(15, tc);  // slow path taken
     }
     __syncwarp();  // cand is reused by the next token of this warp
-    tc = cyc();
-    const float ex = lane < k ? expf((float)(lsel - top)) : 0.0f;
-    float z = ex;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
     id_out = sel;
-    w_out = lane < k ? ex / z : 0.0f;
-    cyc_add(14, tc);  // weights
+    // the weight's logit less the top one; the softmax is finished after the
+    // schedule, which needs only the ids
+    w_out = lane < k ? (float)(lsel - top) : 0.0f;
 }
 
 MOE_DEV double bf16_to_f64(uint32_t bits16) { return (double)__uint_as_float(bits16 << 16); }
@@ -998,11 +994,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     topk_token<32>(lg, E, k, lane, cand + warp * 64, id, wt);
                 if (lane < k) {
                     sids[t * k + lane] = id;
-                    sw[t * k + lane] = wt;
-                    if (b == 0) {
-                        a.ids[(int64_t)t * k + lane] = id;
-                        a.w[(int64_t)t * k + lane] = wt;
-                    }
+                    sw[t * k + lane] = wt;  // l_r - l_0 until the weights are finished
+                    if (b == 0) a.ids[(int64_t)t * k + lane] = id;
                 }
             }
             cyc_add(6, ctk);
@@ -1104,6 +1097,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (tid == 0) mbar_arrive(&sched);  // the producer may issue the routed units
             cyc_add(7, ctk);
             trace(5);
+            // routing weights = softmax over each token's k selected logits, off the
+            // schedule's path: the producer is already issuing the routed units' copies
+            const unsigned long long cw = cyc();
+            for (int t = warp; t < T; t += kCWarps) {  // the warp that ranked token t
+                const float ex = lane < k ? expf(sw[t * k + lane]) : 0.0f;
+                float z = ex;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+                if (lane < k) {
+                    const float wv = ex / z;
+                    sw[t * k + lane] = wv;
+                    if (b == 0) a.w[(int64_t)t * k + lane] = wv;
+                }
+            }
+            consumer_sync();  // every token's weights are in sw before the units read them
+            cyc_add(14, cw);
             return s_nunits;
         };
 

@@ -33,7 +33,7 @@ BOUNDARIES = {0: "start", 1: "router done", 2: "routing starts (shared-expert ga
               40: "end"}
 BOUNDARIES.update({6 + 2 * i: f"gate/up of routed unit {i} done" for i in range(16)})
 CYCLES = {27: "router", 6: "top-k (own tokens)", 10: "top-k: loads + keys", 11: "top-k: extraction rounds",
-          13: "top-k: ranking", 15: "top-k: exact-scan fallback", 14: "top-k: weights",
+          13: "top-k: ranking", 15: "top-k: exact-scan fallback", 14: "weights (softmax, after the schedule)",
           16: "schedule: wait for other warps' top-k", 17: "schedule: masks + compaction",
           18: "schedule: slot places + meta", 7: "top-k + schedule", 1: "gate/up: wait for weights",
           2: "gate/up: compute", 3: "gate/up: h exchange", 4: "down: wait for weights", 5: "down: compute",
