@@ -206,7 +206,7 @@ MOE_DEV bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
     return __shfl_sync(0xffffffffu, okw ? 1 : 0, 0) != 0;
 }
 
-// 2-D TMA tile load (no multicast) completing on `bar`
+// 2-D TMA tile load into this CTA's shared memory, completing on `bar`
 MOE_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
@@ -215,7 +215,7 @@ MOE_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64
         : "memory");
 }
 
-// 3-D TMA tile load (no multicast) completing on `bar`
+// 3-D TMA tile load into this CTA's shared memory, completing on `bar`
 MOE_DEV void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
