@@ -33,3 +33,24 @@ def test_profile_traffic_matches_source_hash():
     # the prefill capture's kernel source is unchanged since the capture; an unknown kernel has none
     assert bench.profile_traffic("gemm_gateup") is None or bench.profile_traffic("gemm_gateup") > 0
     assert bench.profile_traffic("no_such_kernel") is None
+
+
+def test_kernel_source_sections_exist():
+    """Every kernel the bench hashes for its ncu traffic lines has its section markers in its source: a
+    renamed marker would otherwise turn the traffic silently null."""
+    sys.path.insert(0, ROOT)
+    import bench
+    for kernel, (src, start, end) in bench._KERNEL_SOURCE.items():
+        h = bench.kernel_source_hash(kernel)
+        assert h is not None and len(h) == 16, kernel
+        if start is not None:
+            text = open(os.path.join(ROOT, "bit_expert_ffn_gemv_b200", "csrc", src)).read()
+            i = text.find(start)
+            assert i >= 0 and text.find(end, i + 1) > i, kernel
+    # the gate/up and down kernels share one section; the router's is another
+    assert bench.kernel_source_hash("gemm_gateup") == bench.kernel_source_hash("gemm_down")
+    assert bench.kernel_source_hash("gemm_gateup") != bench.kernel_source_hash("router_gemm")
+    # the committed capture of the 8192-token chunk matches the current expert GEMM section
+    assert bench.profile_traffic("gemm_gateup", 8192) == 677046272
+    assert bench.profile_traffic("gemm_down", 8192) == 548585984
+    assert bench.profile_traffic("gemm_gateup", 64) is None
